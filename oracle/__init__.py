@@ -1,0 +1,322 @@
+"""Oracle for the DeepSeek-V3/R1 MoE FFN layer forward (CPU, plain, slow).
+
+TEST INFRASTRUCTURE ONLY: the test-suite, the package smoke check and the
+benchmark's CPU-baseline leg may use this package; the product path never
+imports, loads or calls it.  It shares no code with the CUDA library.
+
+What the layer computes, step by step, with the passage each step follows:
+
+ 1. Router logits l = x W_r^T (binary32, sequential fused multiply-add over
+    d_model) and affinity s = sigmoid(l); selection score s + b where b is a
+    per-expert bias used for routing only; top-k by (score desc, index asc);
+    gates g_j = s_j / sum_selected(s) * routed_scale.
+    ("DeepSeek v3 and R1 Model Architecture", section "Local Balanced Routing
+    to Experts": token-to-expert affinity plus a routing-only bias term;
+    "DeepSeek-R1" architecture card, "Every architecture field": 256 experts,
+    8 active.)  C core: moe_oracle.c.
+ 2. Permutation: expert e's segment holds, in ascending token order, the
+    tokens that selected e; segments are laid out in expert order; the shared
+    expert's segment follows them and holds every token in order.  (Same page,
+    "How is a token assigned to an expert"; card: 1 shared expert.)
+ 3. Blockwise e4m3 quantisation, 1x128 activation tiles and 128x128 weight
+    blocks with binary32 scales ("DeepSeek-R1", aguasto.com, "Quantization":
+    blockwise FP8).  C core.
+ 4. Gated experts (SwiGLU): H = silu(A W_gate^T) * (A W_up^T), Y = H W_down^T,
+    d_expert 2048, d_model 7168 (card, "ffns.moe.gated", "ffns.moe.d_expert";
+    "Architecture Overview" of the onlylabs page names SwiGLU).  In the FP8
+    scheme every product is the real-valued product of the dequantised
+    operands, evaluated in binary64 (numpy matmul); H is quantised 1x128 again
+    before the down projection; Y is stored as bf16.  In the bf16 scheme H is
+    rounded to bf16.
+ 5. Combine: out[t] = bf16( sum_j g[t,j] * Y[row(t,j)] + Y_shared[t] ) (the
+    shared expert is always active with weight 1: "v3 also inherits the
+    concept of the shared expert, i.e. an always-activated expert").
+
+The oracle mirrors every storage rounding of the layer (bf16 Y, bf16 or e4m3
+H, bf16 out) and otherwise computes in binary64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+__all__ = [
+    "lib", "bf16_to_f32", "bf16_from_f32", "e4m3_decode_table", "e4m3_encode", "sigmoid",
+    "router_logits", "route", "permute", "block_quant", "dequant", "expert_forward",
+    "moe_layer", "exp_cw",
+]
+
+_LIB = None
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        f32p = ctypes.POINTER(ctypes.c_float)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        L.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.oracle_bf16_to_f32.restype = ctypes.c_float
+        L.oracle_bf16_from_f32.argtypes = [ctypes.c_float]
+        L.oracle_bf16_from_f32.restype = ctypes.c_uint16
+        L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_decode.restype = ctypes.c_float
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_exp_cw.argtypes = [ctypes.c_float]
+        L.oracle_exp_cw.restype = ctypes.c_float
+        L.oracle_sigmoid.argtypes = [ctypes.c_float]
+        L.oracle_sigmoid.restype = ctypes.c_float
+        L.oracle_block_quant.argtypes = [f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, f32p]
+        L.oracle_block_quant.restype = None
+        L.oracle_router_logits.argtypes = [u16p, u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int, f32p]
+        L.oracle_router_logits.restype = None
+        L.oracle_route.argtypes = [f32p, f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_float, i32p, f32p, f32p]
+        L.oracle_route.restype = None
+        L.oracle_bf16_from_f32_array.argtypes = [f32p, ctypes.c_size_t, u16p]
+        L.oracle_e4m3_encode_array.argtypes = [f32p, ctypes.c_size_t, u8p]
+        L.oracle_sigmoid_array.argtypes = [f32p, ctypes.c_size_t, f32p]
+        _LIB = L
+    return _LIB
+
+
+def _p(a, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+# ------------------------------------------------------------------ codecs --
+
+def bf16_to_f32(h) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> float32 (exact widening)."""
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    return (h.astype(np.uint32) << 16).view(np.float32)
+
+
+def bf16_from_f32(f) -> np.ndarray:
+    """float32 -> bf16 bit patterns, round to nearest even (C core)."""
+    f = np.ascontiguousarray(f, dtype=np.float32)
+    out = np.empty(f.shape, dtype=np.uint16)
+    lib().oracle_bf16_from_f32_array(_p(f, ctypes.c_float), f.size, _p(out, ctypes.c_uint16))
+    return out
+
+
+def e4m3_decode_table() -> np.ndarray:
+    """binary64 value of each of the 256 e4m3 codes (NaN for S.1111.111)."""
+    L = lib()
+    return np.array([L.oracle_e4m3_decode(c) for c in range(256)], dtype=np.float64)
+
+
+def e4m3_encode(f) -> np.ndarray:
+    f = np.ascontiguousarray(f, dtype=np.float32)
+    out = np.empty(f.shape, dtype=np.uint8)
+    lib().oracle_e4m3_encode_array(_p(f, ctypes.c_float), f.size, _p(out, ctypes.c_uint8))
+    return out
+
+
+def sigmoid(l) -> np.ndarray:
+    l = np.ascontiguousarray(l, dtype=np.float32)
+    out = np.empty(l.shape, dtype=np.float32)
+    lib().oracle_sigmoid_array(_p(l, ctypes.c_float), l.size, _p(out, ctypes.c_float))
+    return out
+
+
+def exp_cw(y: float) -> float:
+    return lib().oracle_exp_cw(float(y))
+
+
+# ------------------------------------------------------------------ router --
+
+def router_logits(x_bf16, w_router_bf16) -> np.ndarray:
+    """[T, E] binary32 logits, sequential FMA over d_model (C core)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    w = np.ascontiguousarray(w_router_bf16, dtype=np.uint16)
+    T, d = x.shape
+    E = w.shape[0]
+    out = np.empty((T, E), dtype=np.float32)
+    lib().oracle_router_logits(_p(x, ctypes.c_uint16), _p(w, ctypes.c_uint16), T, d, E,
+                               _p(out, ctypes.c_float))
+    return out
+
+
+def route(logits, bias, k: int, routed_scale: float = 1.0):
+    """-> (idx int32 [T,k] rank order, gates fp32 [T,k], scores fp32 [T,E])."""
+    l = np.ascontiguousarray(logits, dtype=np.float32)
+    b = np.ascontiguousarray(bias, dtype=np.float32)
+    T, E = l.shape
+    idx = np.empty((T, k), dtype=np.int32)
+    g = np.empty((T, k), dtype=np.float32)
+    s = np.empty((T, E), dtype=np.float32)
+    lib().oracle_route(_p(l, ctypes.c_float), _p(b, ctypes.c_float), T, E, k,
+                       float(routed_scale), _p(idx, ctypes.c_int32), _p(g, ctypes.c_float),
+                       _p(s, ctypes.c_float))
+    return idx, g, s
+
+
+# ------------------------------------------------------------- permutation --
+
+def permute(idx, n_experts: int):
+    """Expert-major layout of the routed (token, slot) pairs.
+
+    counts[e]   tokens that selected e
+    offsets[e]  exclusive prefix sum of counts (E+1 entries, offsets[E] = T*k)
+    row_token[r] token of routed row r; within a segment tokens ascend
+    row_of[t,j]  routed row of (t, idx[t,j])
+    The shared segment (rows T*k .. T*k+T-1, token order) is implicit.
+    """
+    idx = np.asarray(idx, dtype=np.int64)
+    T, k = idx.shape
+    flat = idx.reshape(-1)                            # entry t*k + j
+    counts = np.bincount(flat, minlength=n_experts).astype(np.int32)
+    offsets = np.zeros(n_experts + 1, dtype=np.int32)
+    offsets[1:] = np.cumsum(counts)
+    order = np.argsort(flat, kind="stable")           # by expert, then entry (= token) order
+    row_token = (order // k).astype(np.int32)
+    row_of = np.empty(T * k, dtype=np.int32)
+    row_of[order] = np.arange(T * k, dtype=np.int32)
+    return counts, offsets, row_token, row_of.reshape(T, k)
+
+
+# ------------------------------------------------------------ quantisation --
+
+def block_quant(a, block_rows: int):
+    """e4m3 block quantisation of a [rows, cols] matrix (float32 or bf16 bits).
+
+    -> (codes uint8 [rows, cols], scales fp32 [ceil(rows/block_rows), cols/128])"""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        a = bf16_to_f32(a)
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    rows, cols = a.shape
+    if cols % 128:
+        raise ValueError("cols must be a multiple of 128")
+    q = np.empty((rows, cols), dtype=np.uint8)
+    s = np.empty(((rows + block_rows - 1) // block_rows, cols // 128), dtype=np.float32)
+    lib().oracle_block_quant(_p(a, ctypes.c_float), rows, cols, block_rows,
+                             _p(q, ctypes.c_uint8), _p(s, ctypes.c_float))
+    return q, s
+
+
+_DEC = None
+
+
+def dequant(q, scales, block_rows: int) -> np.ndarray:
+    """binary64 decode(q) * scale of each block."""
+    global _DEC
+    if _DEC is None:
+        _DEC = e4m3_decode_table()
+    q = np.asarray(q, dtype=np.uint8)
+    rows, cols = q.shape
+    s = np.asarray(scales, dtype=np.float64)
+    s_full = np.repeat(np.repeat(s, block_rows, axis=0)[:rows], 128, axis=1)
+    return _DEC[q] * s_full
+
+
+# ----------------------------------------------------------------- experts --
+
+def _silu_mul(g, u):
+    return g / (1.0 + np.exp(-g)) * u
+
+
+def _bf16_of_f64(v) -> np.ndarray:
+    # binary64 -> binary32 (round to nearest) -> bf16 (round to nearest even)
+    return bf16_from_f32(np.asarray(v, dtype=np.float64).astype(np.float32))
+
+
+def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=None,
+                   w2_scales=None, return_h: bool = False):
+    """One gated expert on a block of rows.
+
+    bf16:  a_rows uint16 [n, d], w13 uint16 [2*de, d], w2 uint16 [d, de].
+    fp8:   a_rows uint8 codes + a_scales [n, d/128]; w13 codes + w13_scales
+           [2*de/128, d/128]; w2 codes + w2_scales [d/128, de/128].
+    -> Y as bf16 bits [n, d] (and H: bf16 bits, or (codes, scales) for fp8)."""
+    n = a_rows.shape[0]
+    if precision == "bf16":
+        A = bf16_to_f32(a_rows).astype(np.float64)
+        W13 = bf16_to_f32(w13).astype(np.float64)
+        W2 = bf16_to_f32(w2).astype(np.float64)
+        de = W13.shape[0] // 2
+        G = A @ W13[:de].T
+        U = A @ W13[de:].T
+        H = _bf16_of_f64(_silu_mul(G, U))
+        Y = bf16_to_f32(H).astype(np.float64) @ W2.T
+        y = _bf16_of_f64(Y)
+        return (y, H) if return_h else y
+    if precision == "fp8":
+        A = dequant(a_rows, a_scales, 1)
+        W13 = dequant(w13, w13_scales, 128)
+        W2 = dequant(w2, w2_scales, 128)
+        de = W13.shape[0] // 2
+        G = A @ W13[:de].T
+        U = A @ W13[de:].T
+        H = _silu_mul(G, U).astype(np.float32)
+        hq, hs = block_quant(H, 1)
+        Y = dequant(hq, hs, 1) @ W2.T
+        y = _bf16_of_f64(Y)
+        return (y, (hq, hs)) if return_h else y
+    raise ValueError(precision)
+
+
+# ------------------------------------------------------------------- layer --
+
+def moe_layer(x, w_router, bias, expert, *, n_experts: int, top_k: int, n_shared: int,
+              precision: str, routed_scale: float = 1.0, tokens=None):
+    """Forward of one MoE FFN layer.
+
+    x uint16 [T, d] (bf16 bits); w_router uint16 [E, d]; bias fp32 [E];
+    expert(e) -> (w13, w2) as bf16 bits of expert e (e == n_experts is the
+    shared expert).  In the fp8 scheme the oracle quantises each expert it
+    touches itself (128x128 blocks).
+    tokens: indices of the output rows to evaluate (default: all).  Routing,
+    permutation and activation quantisation always cover every token.
+
+    Returns a dict: logits, scores, idx, gates, counts, offsets, row_token,
+    row_of, (fp8) xq, xs, out [len(tokens), d] bf16 bits, tokens."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    T, d = x.shape
+    E, k = n_experts, top_k
+    logits = router_logits(x, w_router)
+    idx, gates, scores = route(logits, bias, k, routed_scale)
+    counts, offsets, row_token, row_of = permute(idx, E)
+    res = dict(logits=logits, scores=scores, idx=idx, gates=gates, counts=counts,
+               offsets=offsets, row_token=row_token, row_of=row_of)
+    if precision == "fp8":
+        xq, xs = block_quant(x, 1)
+        res.update(xq=xq, xs=xs)
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    # rows needed per expert: (expert, token) pairs of the evaluated tokens
+    need = {}
+    for ti, t in enumerate(tokens):
+        for j in range(k):
+            need.setdefault(int(idx[t, j]), []).append((ti, j))
+        if n_shared:
+            need.setdefault(E, []).append((ti, k))
+    Yt = np.zeros((len(tokens), k + 1, d), dtype=np.float64)
+    for e in sorted(need):
+        w13, w2 = expert(e)
+        pairs = need[e]
+        rows = np.array([tokens[ti] for ti, _ in pairs])
+        if precision == "fp8":
+            w13q, w13s = block_quant(w13, 128)
+            w2q, w2s = block_quant(w2, 128)
+            y = expert_forward(res["xq"][rows], w13q, w2q, "fp8", res["xs"][rows], w13s, w2s)
+        else:
+            y = expert_forward(x[rows], w13, w2, "bf16")
+        yf = bf16_to_f32(y).astype(np.float64)
+        for n, (ti, j) in enumerate(pairs):
+            Yt[ti, j] = yf[n]
+    g = gates[tokens].astype(np.float64)
+    acc = np.einsum("tj,tjd->td", g, Yt[:, :k])
+    if n_shared:
+        acc = acc + Yt[:, k]
+    res["out"] = _bf16_of_f64(acc)
+    res["tokens"] = tokens
+    return res
