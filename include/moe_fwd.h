@@ -1,0 +1,181 @@
+/*
+ * moe_fwd.h — C ABI of the B200 (sm_100a) forward pass of one
+ * DeepSeek-V3/R1 Mixture-of-Experts FFN layer.
+ *
+ * The layer (sources are the pages' titles and sections):
+ *  - "DeepSeek-R1" architecture card (llm-architectures-explained.vercel.app),
+ *    table "Every architecture field": d_model 7168, 256 routed experts,
+ *    8 active per token, gated experts of width 2048, 1 shared expert.
+ *  - "DeepSeek v3 and R1 Model Architecture" (onlylabs.fyi), section "Local
+ *    Balanced Routing to Experts": tokens go to experts by token-to-expert
+ *    affinity; a per-expert bias is added for routing only.  Section
+ *    "Structural change": the shared expert is always active.
+ *  - "DeepSeek-R1" (aguasto.com), section "Quantization": blockwise FP8.
+ * Readings where the pages are silent: affinity s = sigmoid(l) on binary32
+ * logits accumulated by sequential fused multiply-adds over d_model; top-k
+ * by (s + bias) descending, lowest expert index first among equals; gates
+ * g = s / sum(selected s) * routed_scale; the shared expert has weight 1;
+ * FP8 is OCP e4m3 with 1x128 activation tiles and 128x128 weight blocks,
+ * each with a binary32 scale amax/448, and the expert GEMMs accumulate each
+ * 128-wide K block separately, then scale it and add it in binary32.
+ *
+ * Conventions for every call:
+ *  - Every pointer is caller-owned DEVICE memory unless stated otherwise; the
+ *    library never allocates or frees device memory.
+ *  - "bf16" buffers hold bfloat16 bit patterns (uint16_t); "e4m3" buffers
+ *    hold OCP FP8 E4M3 codes (uint8_t).  Matrices are row-major, contiguous.
+ *  - Device pointers must be 16-byte aligned; the workspace 256-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL: the legacy default stream).  Calls are
+ *    asynchronous: they only enqueue kernels.  Arguments are read by the
+ *    kernels when they run, so buffers must stay valid until then.
+ *  - Return value: MOE_OK, or a negative MOE_ERR_* code, in which case no
+ *    kernel was enqueued (except MOE_ERR_CUDA, raised when a launch failed).
+ *    moe_last_error() gives a message for the calling thread's last error.
+ *  - Errors found by the kernels themselves (an expert index out of range,
+ *    a duplicate expert for one token, a bounded device wait that ran out)
+ *    are recorded in a status word at the start of the workspace; read and
+ *    clear it with moe_check_status().  A kernel that records an error skips
+ *    the offending access and finishes, so the CUDA context stays usable.
+ *  - Shapes: d_model a multiple of 256, d_expert a multiple of 128;
+ *    1 <= top_k <= min(n_experts, 32); n_shared 0 or 1; n_experts + n_shared
+ *    <= 1024; T >= 0 (T = 0 enqueues nothing).
+ */
+#ifndef MOE_FWD_H
+#define MOE_FWD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1, /* null/misaligned pointer, bad shape value     */
+    MOE_ERR_UNSUPPORTED = -2, /* valid but not implemented (e.g. no sm_100a)  */
+    MOE_ERR_WORKSPACE = -3,   /* workspace smaller than moe_workspace_size()  */
+    MOE_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed         */
+    MOE_ERR_TIMEOUT = -5,     /* a bounded device-side wait ran out           */
+    MOE_ERR_DEVICE_INDEX = -6 /* kernel saw an expert index out of range or a
+                                 token that selected one expert twice        */
+};
+
+enum moe_precision {
+    MOE_BF16 = 0,      /* bf16 weights and activations, binary32 accumulate */
+    MOE_FP8_BLOCK = 1  /* e4m3 1x128 activations, 128x128 weights, fp32 scales */
+};
+
+/* Layer shape.  T tokens, d_model, n_experts routed experts (E), top_k (k),
+ * d_expert, n_shared (0 or 1 shared experts of width d_expert),
+ * routed_scale (multiplies every gate), precision (enum moe_precision). */
+typedef struct moe_shape {
+    int T;
+    int d_model;
+    int n_experts;
+    int top_k;
+    int d_expert;
+    int n_shared;
+    float routed_scale;
+    int precision;
+} moe_shape;
+
+/* Bytes of device workspace that moe_forward needs for this shape (the other
+ * calls need no more).  0 if the shape is invalid (see moe_last_error). */
+size_t moe_workspace_size(const moe_shape *shape);
+
+/* Router: logits l = x W_r^T in binary32 (sequential fused multiply-adds over
+ * d_model), affinity s = sigmoid(l), selection by s + bias (bias: routing
+ * only), top-k in rank order, gates g_j = s_j / sum_selected(s) *
+ * routed_scale ("Local Balanced Routing to Experts").
+ *   x        bf16 [T, d_model]
+ *   w_router bf16 [n_experts, d_model]
+ *   bias     fp32 [n_experts]
+ *   topk_idx int32 [T, top_k] out: expert ids, best first
+ *   topk_w   fp32 [T, top_k]  out: gates in the same order
+ *   ws       workspace (>= moe_workspace_size bytes): holds the [T, E] scores */
+int moe_route(const moe_shape *shape, const uint16_t *x, const uint16_t *w_router,
+              const float *bias, int32_t *topk_idx, float *topk_w,
+              void *ws, size_t ws_bytes, void *stream);
+
+/* Permutation into per-expert segments (expert order; tokens ascending inside
+ * a segment; deterministic).
+ *   topk_idx  int32 [T, top_k] in
+ *   counts    int32 [n_experts] out: tokens per expert
+ *   offsets   int32 [n_experts + 1] out: exclusive prefix sum, offsets[E] = T*k
+ *   row_token int32 [T*k] out: token of each routed row
+ *   row_of    int32 [T, top_k] out: routed row of (t, topk_idx[t, j])
+ * The shared segment is implicit: rows T*k .. T*k+T-1 hold tokens 0..T-1. */
+int moe_permute(const moe_shape *shape, const int32_t *topk_idx, int32_t *counts,
+                int32_t *offsets, int32_t *row_token, int32_t *row_of,
+                void *ws, size_t ws_bytes, void *stream);
+
+/* Blockwise e4m3 quantisation ("Quantization": blockwise FP8) of a bf16
+ * [rows, cols] matrix with leading dimension ld (elements, >= cols, multiple
+ * of 8).  Tiles are block_rows x 128 (block_rows 1 for activations, 128 for
+ * weights; a short last row block is allowed).  Per tile amax; scale =
+ * amax / 448, codes = e4m3_rn_satfinite(v * (448 / amax)); an all-zero tile
+ * gets scale 1 and +0 codes.
+ *   q      e4m3 [rows, cols] out (dense, leading dimension cols)
+ *   scales fp32 [ceil(rows / block_rows), cols / 128] out
+ * A stack of expert matrices [n, N, K] with N % 128 == 0 is one call with
+ * rows = n*N, cols = K. */
+int fp8_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
+                    uint8_t *q, float *scales, void *stream);
+
+/* Grouped gated expert MLP over the permuted rows (card: "experts are gated
+ * MLPs"): for every segment s (routed experts 0..E-1, then the shared expert
+ * at slot E when n_shared = 1)  H = silu(A_s W_gate,s^T) * (A_s W_up,s^T),
+ * Y_s = H W_down,s^T.  R_s = T*k + T*n_shared rows.
+ *   a          [R_s, d_model] bf16, or e4m3 codes in MOE_FP8_BLOCK
+ *   a_scales   fp32 [R_s, d_model/128] (MOE_FP8_BLOCK) or NULL
+ *   offsets    int32 [n_experts + 1] segment starts (as from moe_permute)
+ *   w13        [E + n_shared, 2*d_expert, d_model]: gate rows, then up rows
+ *   w13_scales fp32 [E + n_shared, 2*d_expert/128, d_model/128] or NULL
+ *   w2         [E + n_shared, d_model, d_expert]
+ *   w2_scales  fp32 [E + n_shared, d_model/128, d_expert/128] or NULL
+ *   y          bf16 [R_s, d_model] out
+ * In MOE_FP8_BLOCK, H is quantised 1x128 (e4m3) before the down GEMM; in
+ * MOE_BF16 it is rounded to bf16.  Accumulation is binary32. */
+int moe_grouped_swiglu(const moe_shape *shape, const void *a, const float *a_scales,
+                       const int32_t *offsets, const void *w13, const float *w13_scales,
+                       const void *w2, const float *w2_scales, uint16_t *y,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/* Weighted un-permute plus the always-on shared expert ("Structural change":
+ * an always-activated expert): out[t] = bf16( sum_j topk_w[t,j] *
+ * y[row_of[t,j]] + y[T*k + t] ), binary32 accumulation in rank order (the
+ * shared term only when n_shared = 1).
+ *   y bf16 [R_s, d_model]; row_of int32 [T, k]; topk_w fp32 [T, k];
+ *   out bf16 [T, d_model] */
+int moe_combine(const moe_shape *shape, const uint16_t *y, const int32_t *row_of,
+                const float *topk_w, uint16_t *out, void *stream);
+
+/* The whole layer: route, permute, quantise-and-scatter (or bf16 scatter),
+ * grouped gate/up GEMM + SwiGLU, grouped down GEMM, combine.
+ *   x [T, d_model] bf16 in; out [T, d_model] bf16 out.
+ *   w13/w2 and scales as for moe_grouped_swiglu (weights are quantised once,
+ *   ahead of time, with fp8_block_quant in MOE_FP8_BLOCK).
+ *   topk_idx_out int32 [T, k] or NULL: receives the routing decision. */
+int moe_forward(const moe_shape *shape, const uint16_t *x, const uint16_t *w_router,
+                const float *bias, const void *w13, const float *w13_scales,
+                const void *w2, const float *w2_scales, uint16_t *out,
+                int32_t *topk_idx_out, void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, returns the workspace status word (MOE_OK or the
+ * first device-recorded MOE_ERR_*), and resets it to MOE_OK.  A workspace must
+ * be zero-filled once before first use (or passed here once) so its status
+ * word starts clean. */
+int moe_check_status(void *ws, void *stream);
+
+/* Message for the calling thread's last failed call ("" if none). */
+const char *moe_last_error(void);
+
+/* Number of kernels the last successful call on this thread enqueued. */
+int moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_FWD_H */

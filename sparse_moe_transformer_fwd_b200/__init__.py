@@ -1,0 +1,91 @@
+"""B200 (sm_100a) forward pass of one DeepSeek-V3/R1 Mixture-of-Experts FFN
+layer: sigmoid-affinity router with a routing-only bias and top-k, per-expert
+permutation, blockwise e4m3 quantisation, grouped SwiGLU expert GEMMs on the
+tcgen05 tensor cores, and a weighted combine with the always-on shared
+expert.  The work happens in libmoe_fwd.so (include/moe_fwd.h); this package
+is its binding.
+
+    layer = MoELayer(w_router, bias, w13, w2, top_k=8, precision="fp8")
+    out = layer(x)          # x: bf16 [T, d_model] on the GPU
+"""
+from __future__ import annotations
+
+import torch
+
+from ._native import (EXPORTS, MOE_BF16, MOE_FP8_BLOCK, MoeError, MoeShape, alloc_workspace,
+                      fp8_block_quant, lib, make_shape, moe_check_status, moe_combine,
+                      moe_forward, moe_grouped_swiglu, moe_last_error, moe_last_launch_count,
+                      moe_permute, moe_route, moe_workspace_size)
+
+__all__ = [
+    "MoELayer", "MoeError", "MoeShape", "make_shape", "alloc_workspace", "lib", "EXPORTS",
+    "moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
+    "moe_combine", "moe_forward", "moe_check_status", "moe_last_error", "moe_last_launch_count",
+    "quantize_weights", "MOE_BF16", "MOE_FP8_BLOCK",
+]
+
+
+def quantize_weights(w13: torch.Tensor, w2: torch.Tensor, stream=None):
+    """128x128 e4m3 block quantisation of the stacked expert weights (done
+    once, ahead of the forward passes).  Returns (w13q, w13s, w2q, w2s)."""
+    S, n13, d = w13.shape
+    _, d2, de = w2.shape
+    w13q = torch.empty(S, n13, d, dtype=torch.uint8, device=w13.device)
+    w13s = torch.empty(S, n13 // 128, d // 128, dtype=torch.float32, device=w13.device)
+    w2q = torch.empty(S, d2, de, dtype=torch.uint8, device=w2.device)
+    w2s = torch.empty(S, d2 // 128, de // 128, dtype=torch.float32, device=w2.device)
+    fp8_block_quant(w13, 128, w13q, w13s, stream=stream)
+    fp8_block_quant(w2, 128, w2q, w2s, stream=stream)
+    return w13q, w13s, w2q, w2s
+
+
+class MoELayer:
+    """One MoE FFN layer with resident weights.
+
+    w_router bf16 [E, d]; bias fp32 [E]; w13 bf16 [E + n_shared, 2*d_expert, d]
+    (gate rows then up rows); w2 bf16 [E + n_shared, d, d_expert]; the shared
+    expert, if any, is the last slot.  precision "fp8" quantises the expert
+    weights once at construction (the bf16 copies are then not needed)."""
+
+    def __init__(self, w_router, bias, w13, w2, *, top_k: int, n_shared: int = 1,
+                 routed_scale: float = 1.0, precision: str = "fp8", keep_bf16: bool = False):
+        lib()  # fail loudly now if the CUDA library is missing
+        self.E, self.d = w_router.shape
+        self.de = w2.shape[2]
+        self.top_k, self.n_shared, self.routed_scale = top_k, n_shared, routed_scale
+        self.precision = precision
+        self.w_router, self.bias = w_router.contiguous(), bias.contiguous()
+        if precision == "fp8":
+            self.w13, self.w13s, self.w2, self.w2s = quantize_weights(w13.contiguous(),
+                                                                      w2.contiguous())
+            self.w13_bf16 = w13 if keep_bf16 else None
+            self.w2_bf16 = w2 if keep_bf16 else None
+        elif precision == "bf16":
+            self.w13, self.w2 = w13.contiguous(), w2.contiguous()
+            self.w13s = self.w2s = None
+        else:
+            raise ValueError(precision)
+        self._ws = {}
+
+    def shape(self, T: int) -> MoeShape:
+        return make_shape(T, self.d, self.E, self.top_k, self.de, self.n_shared,
+                          self.routed_scale, self.precision)
+
+    def workspace(self, T: int) -> torch.Tensor:
+        ws = self._ws.get(T)
+        if ws is None:
+            ws = alloc_workspace(self.shape(T), self.w13.device)
+            self._ws[T] = ws
+        return ws
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None,
+                 topk_idx_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty(T, self.d, dtype=torch.bfloat16, device=x.device)
+        moe_forward(self.shape(T), x, self.w_router, self.bias, self.w13, self.w13s, self.w2,
+                    self.w2s, out, self.workspace(T), topk_idx_out=topk_idx_out, stream=stream)
+        return out
+
+    def check_status(self, T: int) -> int:
+        return moe_check_status(self.workspace(T))

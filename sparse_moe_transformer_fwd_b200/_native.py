@@ -1,0 +1,192 @@
+"""ctypes binding of libmoe_fwd.so (include/moe_fwd.h): argument marshalling
+only.  Every computation of the layer runs in the library's CUDA kernels;
+torch supplies device memory and the current stream.  There is no fallback:
+if the library is missing or fails to load, every call raises."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_fwd.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED = -2
+MOE_ERR_WORKSPACE = -3
+MOE_ERR_CUDA = -4
+MOE_ERR_TIMEOUT = -5
+MOE_ERR_DEVICE_INDEX = -6
+MOE_BF16 = 0
+MOE_FP8_BLOCK = 1
+
+# every symbol include/moe_fwd.h declares
+EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant",
+           "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_check_status",
+           "moe_last_error", "moe_last_launch_count")
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("d_model", ctypes.c_int), ("n_experts", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("d_expert", ctypes.c_int), ("n_shared", ctypes.c_int),
+                ("routed_scale", ctypes.c_float), ("precision", ctypes.c_int)]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"moe_fwd error {code}: {msg}")
+        self.code = code
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library (built in-tree by build.py)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} not built: run sparse_moe_transformer_fwd_b200/build.py "
+                              "(or __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, ci, cf = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+        sp = ctypes.POINTER(MoeShape)
+        L.moe_workspace_size.argtypes = [sp]
+        L.moe_workspace_size.restype = sz
+        L.moe_route.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_permute.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.fp8_block_quant.argtypes = [vp, ci, ci, ci, ci, vp, vp, vp]
+        L.moe_grouped_swiglu.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_combine.argtypes = [sp, vp, vp, vp, vp, vp]
+        L.moe_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_check_status.argtypes = [vp, vp]
+        L.moe_last_error.argtypes = []
+        L.moe_last_error.restype = ctypes.c_char_p
+        L.moe_last_launch_count.argtypes = []
+        for name in ("moe_route", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
+                     "moe_combine", "moe_forward", "moe_check_status", "moe_last_launch_count"):
+            getattr(L, name).restype = ci
+        _LIB = L
+    return _LIB
+
+
+def _check(rc: int) -> None:
+    if rc != MOE_OK:
+        raise MoeError(rc, lib().moe_last_error().decode())
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_shape(T, d_model, n_experts, top_k, d_expert, n_shared=1, routed_scale=1.0,
+               precision="fp8") -> MoeShape:
+    prec = {"bf16": MOE_BF16, "fp8": MOE_FP8_BLOCK}[precision] if isinstance(precision, str) \
+        else int(precision)
+    return MoeShape(int(T), int(d_model), int(n_experts), int(top_k), int(d_expert),
+                    int(n_shared), float(routed_scale), prec)
+
+
+_BF16 = torch.bfloat16
+_FP8 = (torch.uint8, torch.float8_e4m3fn)
+
+
+def moe_workspace_size(shape: MoeShape) -> int:
+    n = lib().moe_workspace_size(ctypes.byref(shape))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, lib().moe_last_error().decode())
+    return n
+
+
+def alloc_workspace(shape: MoeShape, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace (zero status word) of moe_workspace_size bytes."""
+    return torch.zeros(moe_workspace_size(shape), dtype=torch.uint8, device=device)
+
+
+def moe_route(shape, x, w_router, bias, topk_idx, topk_w, ws, stream=None):
+    _check(lib().moe_route(ctypes.byref(shape), _ptr(x, _BF16, "x"),
+                           _ptr(w_router, _BF16, "w_router"), _ptr(bias, torch.float32, "bias"),
+                           _ptr(topk_idx, torch.int32, "topk_idx"),
+                           _ptr(topk_w, torch.float32, "topk_w"), _ptr(ws, torch.uint8, "ws"),
+                           ws.numel(), _stream(stream)))
+
+
+def moe_permute(shape, topk_idx, counts, offsets, row_token, row_of, ws, stream=None):
+    i32 = torch.int32
+    _check(lib().moe_permute(ctypes.byref(shape), _ptr(topk_idx, i32, "topk_idx"),
+                             _ptr(counts, i32, "counts"), _ptr(offsets, i32, "offsets"),
+                             _ptr(row_token, i32, "row_token"), _ptr(row_of, i32, "row_of"),
+                             _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def fp8_block_quant(inp, block_rows, q, scales, rows=None, cols=None, ld=None, stream=None):
+    """e4m3 block quantisation of a bf16 matrix (2-D, or a stack flattened to 2-D)."""
+    cols = inp.shape[-1] if cols is None else cols
+    rows = inp.numel() // inp.shape[-1] if rows is None else rows
+    ld = inp.shape[-1] if ld is None else ld
+    _check(lib().fp8_block_quant(_ptr(inp, _BF16, "in"), rows, cols, ld, block_rows,
+                                 _ptr(q, _FP8, "q"), _ptr(scales, torch.float32, "scales"),
+                                 _stream(stream)))
+
+
+def moe_grouped_swiglu(shape, a, a_scales, offsets, w13, w13_scales, w2, w2_scales, y, ws,
+                       stream=None):
+    fp8 = shape.precision == MOE_FP8_BLOCK
+    wt = _FP8 if fp8 else _BF16
+    _check(lib().moe_grouped_swiglu(
+        ctypes.byref(shape), _ptr(a, wt, "a"), _ptr(a_scales, torch.float32, "a_scales"),
+        _ptr(offsets, torch.int32, "offsets"), _ptr(w13, wt, "w13"),
+        _ptr(w13_scales, torch.float32, "w13_scales"), _ptr(w2, wt, "w2"),
+        _ptr(w2_scales, torch.float32, "w2_scales"), _ptr(y, _BF16, "y"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def moe_combine(shape, y, row_of, topk_w, out, stream=None):
+    _check(lib().moe_combine(ctypes.byref(shape), _ptr(y, _BF16, "y"),
+                             _ptr(row_of, torch.int32, "row_of"),
+                             _ptr(topk_w, torch.float32, "topk_w"), _ptr(out, _BF16, "out"),
+                             _stream(stream)))
+
+
+def moe_forward(shape, x, w_router, bias, w13, w13_scales, w2, w2_scales, out, ws,
+                topk_idx_out=None, stream=None):
+    fp8 = shape.precision == MOE_FP8_BLOCK
+    wt = _FP8 if fp8 else _BF16
+    _check(lib().moe_forward(
+        ctypes.byref(shape), _ptr(x, _BF16, "x"), _ptr(w_router, _BF16, "w_router"),
+        _ptr(bias, torch.float32, "bias"), _ptr(w13, wt, "w13"),
+        _ptr(w13_scales, torch.float32, "w13_scales"), _ptr(w2, wt, "w2"),
+        _ptr(w2_scales, torch.float32, "w2_scales"), _ptr(out, _BF16, "out"),
+        _ptr(topk_idx_out, torch.int32, "topk_idx_out"), _ptr(ws, torch.uint8, "ws"),
+        ws.numel(), _stream(stream)))
+
+
+def moe_check_status(ws, stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the workspace status word."""
+    return lib().moe_check_status(_ptr(ws, torch.uint8, "ws"), _stream(stream))
+
+
+def moe_last_error() -> str:
+    return lib().moe_last_error().decode()
+
+
+def moe_last_launch_count() -> int:
+    return lib().moe_last_launch_count()

@@ -1,0 +1,416 @@
+// C ABI of the MoE layer library: argument checks, workspace layout and the
+// launch order of the forward pass.  See include/moe_fwd.h for the contract.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <cstdarg>
+#include <cstdlib>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+namespace moe {
+
+int num_sms() {
+    int dev = 0, n = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+namespace {
+
+thread_local std::string g_err;
+thread_local int g_launches = 0;
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *where) {
+    return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Fault injection for tests of the bounded device waits, read per call from
+// the environment: MOE_FAULT_INJECT=gemm_tx makes the first grouped GEMM of
+// the call arm one pipeline stage for bytes that never arrive, so its
+// consumer's wait runs out and the call reports MOE_ERR_TIMEOUT through the
+// status word (the kernel then drains and exits normally).
+bool inject_gemm_fault() {
+    const char *v = getenv("MOE_FAULT_INJECT");
+    return v && strcmp(v, "gemm_tx") == 0;
+}
+
+int check_device() {
+    int dev = 0, major = 0, minor = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0)
+        return fail(MOE_ERR_UNSUPPORTED, "needs an sm_100 device (found sm_%d%d)", major, minor);
+    return MOE_OK;
+}
+
+int check_shape(const moe_shape *s) {
+    if (!s) return fail(MOE_ERR_INVALID_ARG, "shape is NULL");
+    if (s->T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+    if (s->d_model <= 0 || s->d_model % 256)
+        return fail(MOE_ERR_INVALID_ARG, "d_model must be a positive multiple of 256");
+    if (s->d_expert <= 0 || s->d_expert % 128)
+        return fail(MOE_ERR_INVALID_ARG, "d_expert must be a positive multiple of 128");
+    if (s->n_experts < 1 || s->n_shared < 0 || s->n_shared > 1 ||
+        s->n_experts + s->n_shared > 1024)
+        return fail(MOE_ERR_INVALID_ARG, "need 1 <= n_experts, n_shared in {0,1}, "
+                                         "n_experts + n_shared <= 1024");
+    if (s->top_k < 1 || s->top_k > 32 || s->top_k > s->n_experts)
+        return fail(MOE_ERR_INVALID_ARG, "need 1 <= top_k <= min(n_experts, 32)");
+    if (s->precision != MOE_BF16 && s->precision != MOE_FP8_BLOCK)
+        return fail(MOE_ERR_INVALID_ARG, "unknown precision %d", s->precision);
+    const long long R_s = static_cast<long long>(s->T) * (s->top_k + s->n_shared);
+    if (R_s * s->d_model > (1LL << 40) || R_s > (1LL << 30))
+        return fail(MOE_ERR_INVALID_ARG, "T too large");
+    return MOE_OK;
+}
+
+// ---------------------------------------------------------- workspace ---
+struct Layout {
+    size_t status, scores, idx, gates, counts, offsets, row_token, row_of;
+    size_t masks, hist, blkoff, seg_start, seg_rows, tile_start;
+    size_t a, a_scales, h, h_scales, y;
+    size_t total;
+};
+
+Layout layout(const moe_shape *s) {
+    const size_t T = s->T, E = s->n_experts, k = s->top_k, d = s->d_model, de = s->d_expert;
+    const size_t Rs = T * (k + s->n_shared);
+    const size_t nblk = (T + 255) / 256;
+    const bool fp8 = s->precision == MOE_FP8_BLOCK;
+    const size_t es = fp8 ? 1 : 2;
+    Layout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += (bytes + 255) & ~static_cast<size_t>(255);
+        return at;
+    };
+    L.status = take(256);
+    L.scores = take(T * E * 4);
+    L.idx = take(T * k * 4);
+    L.gates = take(T * k * 4);
+    L.counts = take(E * 4);
+    L.offsets = take((E + 1) * 4);
+    L.row_token = take(T * k * 4);
+    L.row_of = take(T * k * 4);
+    L.masks = take(nblk * E * 8 * 4);
+    L.hist = take(nblk * E * 4);
+    L.blkoff = take(nblk * E * 4);
+    L.seg_start = take((E + 1) * 4);
+    L.seg_rows = take((E + 1) * 4);
+    L.tile_start = take((E + 2) * 4);
+    L.a = take(Rs * d * es);
+    L.a_scales = take(fp8 ? Rs * (d / 128) * 4 : 0);
+    L.h = take(Rs * de * es);
+    L.h_scales = take(fp8 ? Rs * (de / 128) * 4 : 0);
+    L.y = take(Rs * d * 2);
+    L.total = off;
+    return L;
+}
+
+template <class T>
+T *at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+int check_ws(const moe_shape *s, void *ws, size_t ws_bytes, Layout *L) {
+    *L = layout(s);
+    if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+    if (reinterpret_cast<uintptr_t>(ws) & 255)
+        return fail(MOE_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (ws_bytes < L->total)
+        return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L->total);
+    return MOE_OK;
+}
+
+#define CHECK_PTR(p)                                                                   \
+    do {                                                                               \
+        if (!(p)) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", #p);                  \
+        if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+    } while (0)
+
+#define RETURN_IF(call)            \
+    do {                           \
+        const int rc_ = (call);    \
+        if (rc_ != MOE_OK) return rc_; \
+    } while (0)
+
+#define LAUNCH(call, what)                                   \
+    do {                                                     \
+        const cudaError_t e_ = (call);                       \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what);   \
+    } while (0)
+
+PermScratch perm_scratch(void *ws, const Layout &L) {
+    PermScratch p;
+    p.masks = at<uint32_t>(ws, L.masks);
+    p.hist = at<int32_t>(ws, L.hist);
+    p.blkoff = at<int32_t>(ws, L.blkoff);
+    p.seg_start = at<int32_t>(ws, L.seg_start);
+    p.seg_rows = at<int32_t>(ws, L.seg_rows);
+    p.tile_start = at<int32_t>(ws, L.tile_start);
+    return p;
+}
+
+int grouped(const moe_shape *s, const void *a, const float *a_scales, const void *w13,
+            const float *w13_scales, const void *w2, const float *w2_scales, uint16_t *y,
+            void *ws, const Layout &L, cudaStream_t st, int *launches) {
+    const bool fp8 = s->precision == MOE_FP8_BLOCK;
+    const PermScratch ps = perm_scratch(ws, L);
+    const int Rs = s->T * (s->top_k + s->n_shared);
+    GemmArgs g{};
+    g.fp8 = fp8;
+    g.rows_total = Rs;
+    g.n_slots = s->n_experts + s->n_shared;
+    g.n_segments = s->n_experts + s->n_shared;
+    g.E = s->n_experts;
+    g.seg_start = ps.seg_start;
+    g.seg_rows = ps.seg_rows;
+    g.tile_start = ps.tile_start;
+    g.status = at<int>(ws, L.status);
+    g.inject_fault = inject_gemm_fault() ? 1 : 0;
+    // gate/up GEMM + SwiGLU
+    g.gate_up = true;
+    g.a = a;
+    g.a_scales = a_scales;
+    g.b = w13;
+    g.b_scales = w13_scales;
+    g.out = at<uint8_t>(ws, L.h);
+    g.out_scales = fp8 ? at<float>(ws, L.h_scales) : nullptr;
+    g.K = s->d_model;
+    g.N_out = s->d_expert;
+    LAUNCH(launch_grouped_gemm(g, st, launches), "grouped gate/up GEMM");
+    // down GEMM
+    g.inject_fault = 0;
+    g.gate_up = false;
+    g.a = at<uint8_t>(ws, L.h);
+    g.a_scales = fp8 ? at<float>(ws, L.h_scales) : nullptr;
+    g.b = w2;
+    g.b_scales = w2_scales;
+    g.out = y;
+    g.out_scales = nullptr;
+    g.K = s->d_expert;
+    g.N_out = s->d_model;
+    LAUNCH(launch_grouped_gemm(g, st, launches), "grouped down GEMM");
+    return MOE_OK;
+}
+
+int check_weights(const moe_shape *s, const void *w13, const float *w13s, const void *w2,
+                  const float *w2s) {
+    CHECK_PTR(w13);
+    CHECK_PTR(w2);
+    if (s->precision == MOE_FP8_BLOCK) {
+        CHECK_PTR(w13s);
+        CHECK_PTR(w2s);
+    }
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_shape *shape) {
+    if (check_shape(shape) != MOE_OK) return 0;
+    return layout(shape).total;
+}
+
+int moe_route(const moe_shape *s, const uint16_t *x, const uint16_t *w_router, const float *bias,
+              int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream) {
+    RETURN_IF(check_shape(s));
+    Layout L;
+    RETURN_IF(check_ws(s, ws, ws_bytes, &L));
+    if (s->T == 0) return g_launches = 0, MOE_OK;
+    CHECK_PTR(x);
+    CHECK_PTR(w_router);
+    CHECK_PTR(bias);
+    CHECK_PTR(topk_idx);
+    CHECK_PTR(topk_w);
+    RETURN_IF(check_device());
+    int n = 0;
+    LAUNCH(launch_router(x, w_router, bias, s->T, s->d_model, s->n_experts, s->top_k,
+                         s->routed_scale, at<float>(ws, L.scores), topk_idx, topk_w,
+                         static_cast<cudaStream_t>(stream), &n),
+           "router");
+    g_launches = n;
+    return MOE_OK;
+}
+
+int moe_permute(const moe_shape *s, const int32_t *topk_idx, int32_t *counts, int32_t *offsets,
+                int32_t *row_token, int32_t *row_of, void *ws, size_t ws_bytes, void *stream) {
+    RETURN_IF(check_shape(s));
+    Layout L;
+    RETURN_IF(check_ws(s, ws, ws_bytes, &L));
+    CHECK_PTR(counts);
+    CHECK_PTR(offsets);
+    if (s->T == 0) {
+        // empty input: zero counts and offsets, nothing else to write
+        LAUNCH(cudaMemsetAsync(counts, 0, sizeof(int32_t) * s->n_experts,
+                               static_cast<cudaStream_t>(stream)), "memset");
+        LAUNCH(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (s->n_experts + 1),
+                               static_cast<cudaStream_t>(stream)), "memset");
+        g_launches = 0;
+        return MOE_OK;
+    }
+    CHECK_PTR(topk_idx);
+    CHECK_PTR(row_token);
+    CHECK_PTR(row_of);
+    RETURN_IF(check_device());
+    int n = 0;
+    LAUNCH(launch_permute(topk_idx, s->T, s->top_k, s->n_experts, s->n_shared,
+                          perm_scratch(ws, L), counts, offsets, row_token, row_of,
+                          at<int>(ws, L.status), static_cast<cudaStream_t>(stream), &n),
+           "permute");
+    g_launches = n;
+    return MOE_OK;
+}
+
+int fp8_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows, uint8_t *q,
+                    float *scales, void *stream) {
+    if (rows < 0 || cols <= 0 || cols % 128 || ld < cols || ld % 8)
+        return fail(MOE_ERR_INVALID_ARG, "need rows >= 0, cols a positive multiple of 128, "
+                                         "ld >= cols, ld % 8 == 0");
+    if (block_rows != 1 && block_rows != 128)
+        return fail(MOE_ERR_INVALID_ARG, "block_rows must be 1 or 128");
+    if (rows == 0) return g_launches = 0, MOE_OK;
+    CHECK_PTR(in);
+    CHECK_PTR(q);
+    CHECK_PTR(scales);
+    RETURN_IF(check_device());
+    int n = 0;
+    LAUNCH(launch_block_quant(in, rows, cols, ld, block_rows, q, scales,
+                              static_cast<cudaStream_t>(stream), &n),
+           "fp8_block_quant");
+    g_launches = n;
+    return MOE_OK;
+}
+
+int moe_grouped_swiglu(const moe_shape *s, const void *a, const float *a_scales,
+                       const int32_t *offsets, const void *w13, const float *w13_scales,
+                       const void *w2, const float *w2_scales, uint16_t *y, void *ws,
+                       size_t ws_bytes, void *stream) {
+    RETURN_IF(check_shape(s));
+    Layout L;
+    RETURN_IF(check_ws(s, ws, ws_bytes, &L));
+    if (s->T == 0) return g_launches = 0, MOE_OK;
+    CHECK_PTR(a);
+    if (s->precision == MOE_FP8_BLOCK) CHECK_PTR(a_scales);
+    CHECK_PTR(offsets);
+    CHECK_PTR(y);
+    RETURN_IF(check_weights(s, w13, w13_scales, w2, w2_scales));
+    RETURN_IF(check_device());
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int n = 0;
+    LAUNCH(launch_tile_table(offsets, s->n_experts, s->T, s->top_k, s->n_shared,
+                             perm_scratch(ws, L), at<int>(ws, L.status), st, &n),
+           "tile table");
+    RETURN_IF(grouped(s, a, a_scales, w13, w13_scales, w2, w2_scales, y, ws, L, st, &n));
+    g_launches = n;
+    return MOE_OK;
+}
+
+int moe_combine(const moe_shape *s, const uint16_t *y, const int32_t *row_of,
+                const float *topk_w, uint16_t *out, void *stream) {
+    RETURN_IF(check_shape(s));
+    if (s->T == 0) return g_launches = 0, MOE_OK;
+    CHECK_PTR(y);
+    CHECK_PTR(row_of);
+    CHECK_PTR(topk_w);
+    CHECK_PTR(out);
+    RETURN_IF(check_device());
+    int n = 0;
+    LAUNCH(launch_combine(y, row_of, topk_w, s->T, s->d_model, s->top_k, s->n_shared, out,
+                          static_cast<cudaStream_t>(stream), &n),
+           "combine");
+    g_launches = n;
+    return MOE_OK;
+}
+
+int moe_forward(const moe_shape *s, const uint16_t *x, const uint16_t *w_router,
+                const float *bias, const void *w13, const float *w13_scales, const void *w2,
+                const float *w2_scales, uint16_t *out, int32_t *topk_idx_out, void *ws,
+                size_t ws_bytes, void *stream) {
+    RETURN_IF(check_shape(s));
+    Layout L;
+    RETURN_IF(check_ws(s, ws, ws_bytes, &L));
+    if (s->T == 0) return g_launches = 0, MOE_OK;
+    CHECK_PTR(x);
+    CHECK_PTR(w_router);
+    CHECK_PTR(bias);
+    CHECK_PTR(out);
+    if (topk_idx_out && !aligned16(topk_idx_out))
+        return fail(MOE_ERR_INVALID_ARG, "topk_idx_out is not 16-byte aligned");
+    RETURN_IF(check_weights(s, w13, w13_scales, w2, w2_scales));
+    RETURN_IF(check_device());
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool fp8 = s->precision == MOE_FP8_BLOCK;
+    int32_t *idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
+    float *gates = at<float>(ws, L.gates);
+    int32_t *row_of = at<int32_t>(ws, L.row_of);
+    int n = 0;
+    LAUNCH(launch_router(x, w_router, bias, s->T, s->d_model, s->n_experts, s->top_k,
+                         s->routed_scale, at<float>(ws, L.scores), idx, gates, st, &n),
+           "router");
+    LAUNCH(launch_permute(idx, s->T, s->top_k, s->n_experts, s->n_shared, perm_scratch(ws, L),
+                          at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
+                          at<int32_t>(ws, L.row_token), row_of, at<int>(ws, L.status), st, &n),
+           "permute");
+    if (fp8)
+        LAUNCH(launch_quant_scatter(x, s->T, s->d_model, s->top_k, s->n_shared, row_of,
+                                    at<uint8_t>(ws, L.a), at<float>(ws, L.a_scales), st, &n),
+               "quant_scatter");
+    else
+        LAUNCH(launch_scatter_bf16(x, s->T, s->d_model, s->top_k, s->n_shared, row_of,
+                                   at<uint16_t>(ws, L.a), st, &n),
+               "scatter");
+    uint16_t *y = at<uint16_t>(ws, L.y);
+    RETURN_IF(grouped(s, at<uint8_t>(ws, L.a), fp8 ? at<float>(ws, L.a_scales) : nullptr, w13,
+                      w13_scales, w2, w2_scales, y, ws, L, st, &n));
+    LAUNCH(launch_combine(y, row_of, gates, s->T, s->d_model, s->top_k, s->n_shared, out, st, &n),
+           "combine");
+    g_launches = n;
+    return MOE_OK;
+}
+
+int moe_check_status(void *ws, void *stream) {
+    if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int h = 0;
+    cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_check_status");
+    if (h != MOE_OK) {
+        const int zero = 0;
+        e = cudaMemcpyAsync(ws, &zero, sizeof(int), cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e, "moe_check_status reset");
+        return fail(h, "device status %d", h);
+    }
+    return MOE_OK;
+}
+
+const char *moe_last_error(void) { return g_err.c_str(); }
+
+int moe_last_launch_count(void) { return g_launches; }
+
+}  // extern "C"

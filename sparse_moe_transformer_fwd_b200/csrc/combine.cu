@@ -1,0 +1,68 @@
+// Weighted un-permute and shared-expert add ("DeepSeek v3 and R1 Model
+// Architecture", "Structural change": one always-activated shared expert):
+//   out[t] = bf16( sum_j g[t,j] * Y[row_of[t,j]]  (rank order, binary32 fma)
+//                  + Y[T*k + t] )                 (shared, weight 1)
+// One CTA per token, 16-byte vector loads of the k + 1 source rows.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+__global__ void __launch_bounds__(128)
+combine_kernel(const uint16_t *__restrict__ y, const int32_t *__restrict__ row_of,
+               const float *__restrict__ gates, int T, int d, int k, int n_shared,
+               uint16_t *__restrict__ out) {
+    __shared__ int rows_sh[32];
+    __shared__ float g_sh[32];
+    const int t = blockIdx.x;
+    if (threadIdx.x < k) {
+        rows_sh[threadIdx.x] = row_of[static_cast<size_t>(t) * k + threadIdx.x];
+        g_sh[threadIdx.x] = gates[static_cast<size_t>(t) * k + threadIdx.x];
+    }
+    __syncthreads();
+    const size_t shared_row = static_cast<size_t>(T) * k + t;
+    for (int v = threadIdx.x; v < d / 8; v += blockDim.x) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const uint4 raw =
+                reinterpret_cast<const uint4 *>(y + static_cast<size_t>(rows_sh[j]) * d)[v];
+            const uint32_t r[4] = {raw.x, raw.y, raw.z, raw.w};
+            const float g = g_sh[j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[2 * i] = __fmaf_rn(g, bf16_lo(r[i]), acc[2 * i]);
+                acc[2 * i + 1] = __fmaf_rn(g, bf16_hi(r[i]), acc[2 * i + 1]);
+            }
+        }
+        if (n_shared) {
+            const uint4 raw = reinterpret_cast<const uint4 *>(y + shared_row * d)[v];
+            const uint32_t r[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[2 * i] = __fadd_rn(acc[2 * i], bf16_lo(r[i]));
+                acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], bf16_hi(r[i]));
+            }
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        reinterpret_cast<uint4 *>(out + static_cast<size_t>(t) * d)[v] = o;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const uint16_t *y, const int32_t *row_of, const float *gates, int T,
+                           int d, int k, int n_shared, uint16_t *out, cudaStream_t st,
+                           int *launches) {
+    combine_kernel<<<T, 128, 0, st>>>(y, row_of, gates, T, d, k, n_shared, out);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,546 @@
+// Grouped expert GEMMs of the MoE layer on the 5th-generation tensor cores
+// (tcgen05, sm_100a).  "DeepSeek-R1" architecture card: experts are gated
+// MLPs (d_expert 2048, d_model 7168); "DeepSeek v3 and R1 Model
+// Architecture", "First ever FP8 Precision...": FP8 tensor-core math;
+// "DeepSeek-R1" (aguasto.com), "Quantization": blockwise FP8.
+//
+// One persistent kernel per GEMM, one CTA per SM, cluster size 1.
+// Work item = (segment, 128-row tile of the segment, 256-column tile of B).
+// Tiles are ordered m-major, n-minor, so the CTAs running at one time share
+// A tiles and the same expert's weights through L2.
+//   warp 0      TMA producer: A tile 128 x 128 B and two B tiles 128 x 128 B
+//               (gate/up rows, or two halves of the output columns) per
+//               stage, 128-byte swizzle, 4 stages.
+//   warp 1      TMEM allocator (512 columns) and MMA issuer (one thread):
+//               tcgen05.mma M=128 N=256, K=32 (e4m3) or K=16 (bf16), four per
+//               stage.
+//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (tile rows);
+//               warps 2-5 take columns [0,64) and [128,192), warps 6-9 take
+//               [64,128) and [192,256).
+// FP8: every 128-wide K block is accumulated by the tensor core into one of
+//   two TMEM buffers (fresh each block); the epilogue loads it and adds it
+//   into binary32 registers times s_a[row, kb] * s_w[nblock, kb] (the
+//   per-128-K promotion), while the tensor core fills the other buffer.
+// BF16: the tile accumulates over all K in TMEM; two accumulators alternate
+//   between tiles so the epilogue of one overlaps the main loop of the next.
+// Epilogue: gate/up GEMM -> H = silu(G) * U, then (FP8) 1x128 e4m3
+//   quantisation of H (one 128-feature tile per row per work item; the two
+//   column halves exchange their amax through shared memory) or (BF16) bf16
+//   rounding; down GEMM -> Y in bf16.  Rows past the segment end are computed
+//   from neighbouring rows and never stored.
+// Every wait is bounded; on expiry the block records MOE_ERR_TIMEOUT, drains
+// its own TMA loads and MMAs, frees its TMEM and exits.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <cstdio>
+#include <mutex>
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;                  // tile rows
+constexpr int BN = 256;                  // tile columns (TMEM columns per buffer)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * 128;        // 16 KB per stage
+constexpr int B_BYTES = BN * 128;        // 32 KB per stage
+constexpr int STAGE_TX = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_THREADS = 256;
+constexpr int TMEM_COLS = 512;
+constexpr int MAX_SEG = 1025;
+
+struct __align__(1024) GemmSmem {
+    uint8_t a[STAGES][A_BYTES];
+    uint8_t b[STAGES][B_BYTES];
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t xchg[2];        // amax exchange between the two column halves
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort;
+    float amax_x[2][2][BM];  // [iteration parity][column half][row]
+    int32_t seg_start[MAX_SEG];
+    int32_t seg_rows[MAX_SEG];
+    int32_t tile_start[MAX_SEG + 1];
+};
+
+static_assert(sizeof(GemmSmem) + 1024 <= 227 * 1024, "shared memory budget of one CTA");
+
+struct KParams {
+    const float *a_scales;
+    const float *b_scales;
+    void *out;
+    float *out_scales;
+    const int32_t *seg_start, *seg_rows, *tile_start;
+    int *status;
+    int K, N_out, n_segments, b_rows, n_tiles_n;
+    int inject_fault;  // 1: block 0 arms its first stage for 16 bytes that never arrive
+};
+
+__device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int tile, int n_tiles_n,
+                                            int &seg, int &row0, int &rows_valid, int &nt) {
+    const int mt = tile / n_tiles_n;
+    nt = tile - mt * n_tiles_n;
+    int lo = 0, hi = n_seg - 1;  // last segment whose first tile is <= mt
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s.tile_start[mid] <= mt) lo = mid;
+        else hi = mid - 1;
+    }
+    seg = lo;
+    const int mloc = mt - s.tile_start[seg];
+    row0 = s.seg_start[seg] + mloc * BM;
+    rows_valid = min(BM, s.seg_rows[seg] - mloc * BM);
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+template <bool FP8, bool GATE_UP>
+__global__ void __maxnreg__(200)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                    const __grid_constant__ CUtensorMap tmap_b, const KParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    GemmSmem &s = *reinterpret_cast<GemmSmem *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KB = FP8 ? p.K / 128 : p.K / 64;  // stages per tile (128 bytes of K each)
+    const int n_seg = p.n_segments;
+
+    // ---------------------------------------------------------------- setup
+    for (int i = threadIdx.x; i < n_seg; i += NUM_THREADS) {
+        s.seg_start[i] = p.seg_start[i];
+        s.seg_rows[i] = p.seg_rows[i];
+        s.tile_start[i] = p.tile_start[i];
+    }
+    if (threadIdx.x == 0) {
+        s.tile_start[n_seg] = p.tile_start[n_seg];
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.tfull[i], 1);
+            mbar_init(&s.tempty[i], EPI_THREADS / 32);
+            mbar_init(&s.xchg[i], EPI_THREADS);
+        }
+        mbar_init(&s.mma_done, 1);
+        s.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(&s.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = s.tmem_base;
+    const int total_tiles = s.tile_start[n_seg] * p.n_tiles_n;
+    volatile int *abort = &s.abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------------- producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int armed = 0;  // bit s: stage s has been armed at least once
+            uint32_t armed_phase[STAGES] = {0, 0, 0, 0};
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+                int seg, row0, rows_valid, nt;
+                decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
+                const int n_lo = GATE_UP ? nt * 128 : nt * 256;
+                const int n_hi = GATE_UP ? p.N_out + nt * 128 : nt * 256 + 128;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const bool inject = p.inject_fault && blockIdx.x == 0 && armed == 0;
+                    mbar_arrive_expect_tx(&s.full[stage], STAGE_TX + (inject ? 16 : 0));
+                    const int kc = FP8 ? kb * 128 : kb * 64;
+                    tma_load_2d(s.a[stage], &tmap_a, kc, row0, &s.full[stage]);
+                    tma_load_3d(s.b[stage], &tmap_b, kc, n_lo, seg, &s.full[stage]);
+                    tma_load_3d(s.b[stage] + B_BYTES / 2, &tmap_b, kc, n_hi, seg, &s.full[stage]);
+                    armed |= 1 << stage;
+                    armed_phase[stage] = phase;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            // drain: every load this thread issued has landed before the block exits
+            for (int i = 0; i < STAGES; ++i)
+                if (armed & (1 << i)) {
+                    long long t0 = clock64();
+                    while (!mbar_try_wait(&s.full[i], armed_phase[i])) {
+                        if (clock64() - t0 > kWaitBudgetCycles) {
+                            set_status(p.status, MOE_ERR_TIMEOUT);
+                            break;
+                        }
+                    }
+                }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA
+        if (lane == 0) {
+            constexpr uint32_t idesc = instr_desc<FP8>(BM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int tb = 0;
+            uint32_t tphase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+                if (!FP8) {
+                    if (!mbar_wait(&s.tempty[tb], tphase ^ 1, abort, p.status)) break;
+                    tc_fence_after();
+                }
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (FP8) {
+                        if (!mbar_wait(&s.tempty[tb], tphase ^ 1, abort, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!mbar_wait(&s.full[stage], phase, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + tb * BN;
+                    const uint64_t adesc = smem_desc_sw128(smem_u32(s.a[stage]));
+                    const uint64_t bdesc = smem_desc_sw128(smem_u32(s.b[stage]));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        // +32 bytes of K per instruction: +2 in the >>4 address field
+                        const uint32_t acc = FP8 ? (kk > 0) : ((kb | kk) > 0);
+                        tc_mma<FP8>(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc);
+                    }
+                    tc_commit(&s.empty[stage]);
+                    if (FP8) {
+                        tc_commit(&s.tfull[tb]);
+                        tb ^= 1;
+                        if (tb == 0) tphase ^= 1;
+                    }
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!FP8 && ok) {
+                    tc_commit(&s.tfull[tb]);
+                    tb ^= 1;
+                    if (tb == 0) tphase ^= 1;
+                }
+            }
+            // all MMAs issued by this thread are complete before TMEM is freed
+            tc_commit(&s.mma_done);
+            long long t0 = clock64();
+            while (!mbar_try_wait(&s.mma_done, 0)) {
+                if (clock64() - t0 > kWaitBudgetCycles) {
+                    set_status(p.status, MOE_ERR_TIMEOUT);
+                    break;
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------- epilogue
+        const int q = warp & 3;            // TMEM lane quadrant = tile rows 32q..32q+31
+        const int half = (warp - 2) >> 2;  // column half
+        const int r_in = q * 32 + lane;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+        const int KB128 = p.K / 128;
+        const int NB = p.b_rows / 128;
+        int tb = 0;
+        uint32_t tphase = 0;
+        int iter = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++iter) {
+            int seg, row0, rows_valid, nt;
+            decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
+            const bool warp_active = q * 32 < rows_valid;
+            const bool valid = r_in < rows_valid;
+            const size_t row = static_cast<size_t>(row0) + r_in;
+            const int col_lo = half * 64, col_hi = 128 + half * 64;
+            if constexpr (FP8) {
+                float acc[128];
+#pragma unroll
+                for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+                const int nb_lo = GATE_UP ? nt : 2 * nt;
+                const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
+                const float *sw_lo_p = p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * KB128;
+                const float *sw_hi_p = p.b_scales + (static_cast<size_t>(seg) * NB + nb_hi) * KB128;
+                const float *sa_p = p.a_scales + row * KB128;
+                for (int kb = 0; kb < KB; ++kb) {
+                    float sa = 0.0f, swl = 0.0f, swh = 0.0f;
+                    if (warp_active) {
+                        sa = valid ? __ldg(sa_p + kb) : 0.0f;
+                        swl = __ldg(sw_lo_p + kb);
+                        swh = __ldg(sw_hi_p + kb);
+                    }
+                    if (!mbar_wait(&s.tfull[tb], tphase, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (warp_active) {
+                        const float sc_lo = sa * swl, sc_hi = sa * swh;
+                        const uint32_t base = lane_base + tb * BN;
+#pragma unroll
+                        for (int ch = 0; ch < 4; ++ch) {
+                            const int col = (ch < 2 ? col_lo : col_hi) + 32 * (ch & 1);
+                            const float sc = ch < 2 ? sc_lo : sc_hi;
+                            float v[32];
+                            tmem_ld32(base + col, v);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                acc[32 * ch + i] = __fmaf_rn(v[i], sc, acc[32 * ch + i]);
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.tempty[tb]);
+                    tb ^= 1;
+                    if (tb == 0) tphase ^= 1;
+                }
+                if (!ok) break;
+                if constexpr (GATE_UP) {
+                    // H = silu(G) * U for features nt*128 + half*64 + c, c < 64
+                    float m = 0.0f;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) {
+                        acc[c] = silu(acc[c]) * acc[64 + c];
+                        m = fmaxf(m, fabsf(acc[c]));
+                    }
+                    const int par = iter & 1;
+                    s.amax_x[par][half][r_in] = m;
+                    mbar_arrive(&s.xchg[par]);
+                    if (!mbar_wait(&s.xchg[par], (iter >> 1) & 1, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const float amax = fmaxf(m, s.amax_x[par][half ^ 1][r_in]);
+                    if (valid) {
+                        float sc = 1.0f, inv = 0.0f;
+                        if (amax != 0.0f) {
+                            sc = __fdiv_rn(amax, 448.0f);
+                            inv = __fdiv_rn(448.0f, amax);
+                        }
+                        uint8_t *hq = static_cast<uint8_t *>(p.out) + row * p.N_out + nt * 128 +
+                                      half * 64;
+#pragma unroll
+                        for (int c = 0; c < 64; c += 16) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int b = c + 4 * i;
+                                const uint32_t lo = e4m3x2(__fmul_rn(acc[b], inv), __fmul_rn(acc[b + 1], inv));
+                                const uint32_t hi = e4m3x2(__fmul_rn(acc[b + 2], inv), __fmul_rn(acc[b + 3], inv));
+                                w[i] = amax != 0.0f ? (lo | (hi << 16)) : 0u;
+                            }
+                            *reinterpret_cast<uint4 *>(hq + c) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                        if (half == 0) p.out_scales[row * (p.N_out / 128) + nt] = sc;
+                    }
+                } else {
+                    if (valid) {
+                        uint16_t *y = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 256;
+#pragma unroll
+                        for (int c = 0; c < 64; c += 8) {
+                            uint4 o;
+                            o.x = pack_bf16x2(acc[c], acc[c + 1]);
+                            o.y = pack_bf16x2(acc[c + 2], acc[c + 3]);
+                            o.z = pack_bf16x2(acc[c + 4], acc[c + 5]);
+                            o.w = pack_bf16x2(acc[c + 6], acc[c + 7]);
+                            *reinterpret_cast<uint4 *>(y + col_lo + c) = o;
+                            o.x = pack_bf16x2(acc[64 + c], acc[64 + c + 1]);
+                            o.y = pack_bf16x2(acc[64 + c + 2], acc[64 + c + 3]);
+                            o.z = pack_bf16x2(acc[64 + c + 4], acc[64 + c + 5]);
+                            o.w = pack_bf16x2(acc[64 + c + 6], acc[64 + c + 7]);
+                            *reinterpret_cast<uint4 *>(y + col_hi + c) = o;
+                        }
+                    }
+                }
+            } else {
+                // BF16: whole-K accumulator in TMEM buffer tb
+                if (!mbar_wait(&s.tfull[tb], tphase, abort, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (warp_active) {
+                    const uint32_t base = lane_base + tb * BN;
+                    if constexpr (GATE_UP) {
+                        uint16_t *h = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 128 +
+                                      half * 64;
+#pragma unroll
+                        for (int ch = 0; ch < 2; ++ch) {
+                            float g[32], u[32];
+                            tmem_ld32(base + col_lo + 32 * ch, g);
+                            tmem_ld32(base + col_hi + 32 * ch, u);
+                            tmem_wait_ld();
+                            if (valid) {
+#pragma unroll
+                                for (int c = 0; c < 32; c += 8) {
+                                    uint4 o;
+                                    o.x = pack_bf16x2(silu(g[c]) * u[c], silu(g[c + 1]) * u[c + 1]);
+                                    o.y = pack_bf16x2(silu(g[c + 2]) * u[c + 2], silu(g[c + 3]) * u[c + 3]);
+                                    o.z = pack_bf16x2(silu(g[c + 4]) * u[c + 4], silu(g[c + 5]) * u[c + 5]);
+                                    o.w = pack_bf16x2(silu(g[c + 6]) * u[c + 6], silu(g[c + 7]) * u[c + 7]);
+                                    *reinterpret_cast<uint4 *>(h + 32 * ch + c) = o;
+                                }
+                            }
+                        }
+                    } else {
+                        uint16_t *y = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 256;
+#pragma unroll
+                        for (int ch = 0; ch < 4; ++ch) {
+                            const int col = (ch < 2 ? col_lo : col_hi) + 32 * (ch & 1);
+                            float v[32];
+                            tmem_ld32(base + col, v);
+                            tmem_wait_ld();
+                            if (valid) {
+#pragma unroll
+                                for (int c = 0; c < 32; c += 8) {
+                                    uint4 o;
+                                    o.x = pack_bf16x2(v[c], v[c + 1]);
+                                    o.y = pack_bf16x2(v[c + 2], v[c + 3]);
+                                    o.z = pack_bf16x2(v[c + 4], v[c + 5]);
+                                    o.w = pack_bf16x2(v[c + 6], v[c + 7]);
+                                    *reinterpret_cast<uint4 *>(y + col + c) = o;
+                                }
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.tempty[tb]);
+                tb ^= 1;
+                if (tb == 0) tphase ^= 1;
+            }
+        }
+    }
+
+    // ------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ----------------------------------------------------------- host side ---
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+bool make_map_2d(CUtensorMap *m, const void *base, bool fp8, int K, int rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const int es = fp8 ? 1 : 2;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * es};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), 128};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_3d(CUtensorMap *m, const void *base, bool fp8, int K, int rows, int slots) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const int es = fp8 ? 1 : 2;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(slots)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * es,
+                             static_cast<cuuint64_t>(K) * es * static_cast<cuuint64_t>(rows)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool FP8, bool GATE_UP>
+cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams &kp, int grid,
+                     cudaStream_t st) {
+    const size_t smem = sizeof(GemmSmem) + 1024;
+    static bool configured = false;  // per template instance; attribute is per device function
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<FP8, GATE_UP>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    grouped_gemm_kernel<FP8, GATE_UP><<<grid, NUM_THREADS, smem, st>>>(ma, mb, kp);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launches) {
+    if (g.n_segments > MAX_SEG) return cudaErrorInvalidValue;
+    const int b_rows = g.gate_up ? 2 * g.N_out : g.N_out;
+    CUtensorMap ma, mb;
+    if (!make_map_2d(&ma, g.a, g.fp8, g.K, g.rows_total)) return cudaErrorInvalidValue;
+    if (!make_map_3d(&mb, g.b, g.fp8, g.K, b_rows, g.n_slots)) return cudaErrorInvalidValue;
+    KParams kp;
+    kp.a_scales = g.a_scales;
+    kp.b_scales = g.b_scales;
+    kp.out = g.out;
+    kp.out_scales = g.out_scales;
+    kp.seg_start = g.seg_start;
+    kp.seg_rows = g.seg_rows;
+    kp.tile_start = g.tile_start;
+    kp.status = g.status;
+    kp.K = g.K;
+    kp.N_out = g.N_out;
+    kp.n_segments = g.n_segments;
+    kp.b_rows = b_rows;
+    kp.n_tiles_n = g.gate_up ? g.N_out / 128 : g.N_out / 256;
+    kp.inject_fault = g.inject_fault;
+    // upper bound of work items: every segment's tiles, each at most one partial
+    const long long max_mtiles = g.rows_total / BM + g.n_segments;
+    const long long max_tiles = max_mtiles * kp.n_tiles_n;
+    const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
+    if (grid <= 0) return cudaSuccess;
+    cudaError_t e;
+    if (g.fp8) e = g.gate_up ? launch_t<true, true>(ma, mb, kp, grid, st)
+                             : launch_t<true, false>(ma, mb, kp, grid, st);
+    else e = g.gate_up ? launch_t<false, true>(ma, mb, kp, grid, st)
+                       : launch_t<false, false>(ma, mb, kp, grid, st);
+    ++*launches;
+    return e;
+}
+
+}  // namespace moe

@@ -1,0 +1,84 @@
+// Internal launchers of the MoE layer library (host side of each kernel
+// file).  Each returns the launch error, if any, and adds the number of
+// kernels it enqueued to *launches.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+constexpr int kTileM = 128;  // rows per grouped-GEMM tile (tcgen05 M)
+
+// Scratch of the permutation and of the grouped GEMM's tile table.
+struct PermScratch {
+    uint32_t *masks;     // [nblk][E][8] token bit matrix per 256-token block
+    int32_t *hist;       // [nblk][E]
+    int32_t *blkoff;     // [nblk][E]
+    int32_t *seg_start;  // [E + 1] first row of segment s (shared segment last)
+    int32_t *seg_rows;   // [E + 1] rows of segment s
+    int32_t *tile_start; // [E + 2] prefix of 128-row tiles per segment
+};
+
+cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bias, int T, int d,
+                          int E, int k, float routed_scale, float *scores, int32_t *idx,
+                          float *gates, cudaStream_t st, int *launches);
+
+cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int n_shared, PermScratch s,
+                           int32_t *counts, int32_t *offsets, int32_t *row_token, int32_t *row_of,
+                           int *status, cudaStream_t st, int *launches);
+
+cudaError_t launch_tile_table(const int32_t *offsets, int E, int T, int k, int n_shared,
+                              PermScratch s, int *status, cudaStream_t st, int *launches);
+
+// e4m3 quantisation of bf16 [rows, cols] (leading dimension ld) in tiles of
+// block_rows x 128.
+cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
+                               uint8_t *q, float *scales, cudaStream_t st, int *launches);
+
+// Quantise each token row of x once (1x128 tiles) and write its codes and
+// scales to its k routed rows (row_of) and, with n_shared, to row T*k + t.
+cudaError_t launch_quant_scatter(const uint16_t *x, int T, int d, int k, int n_shared,
+                                 const int32_t *row_of, uint8_t *a, float *a_scales,
+                                 cudaStream_t st, int *launches);
+
+// bf16 copy of each token row to its k routed rows and its shared row.
+cudaError_t launch_scatter_bf16(const uint16_t *x, int T, int d, int k, int n_shared,
+                                const int32_t *row_of, uint16_t *a, cudaStream_t st,
+                                int *launches);
+
+cudaError_t launch_combine(const uint16_t *y, const int32_t *row_of, const float *gates, int T,
+                           int d, int k, int n_shared, uint16_t *out, cudaStream_t st,
+                           int *launches);
+
+// Grouped GEMM over the segment table.
+//   gate_up = true : out = H [rows, N_out] = silu(A Wg^T) * (A Wu^T), B rows per
+//                    slot = 2*N_out (gate rows then up rows); fp8: H quantised
+//                    1x128 with scales h_scales [rows, N_out/128]; bf16: H bf16
+//   gate_up = false: out = Y [rows, N_out] bf16 = A W^T, B rows per slot N_out
+struct GemmArgs {
+    bool fp8;
+    bool gate_up;
+    const void *a;          // [rows_total, K]
+    const float *a_scales;  // [rows_total, K/128] (fp8)
+    const void *b;          // [n_slots, B rows, K]
+    const float *b_scales;  // [n_slots, B rows/128, K/128] (fp8)
+    void *out;              // H or Y
+    float *out_scales;      // H scales (fp8 gate_up)
+    int rows_total;         // R_s
+    int K;
+    int N_out;
+    int n_slots;
+    int n_segments;         // E + n_shared
+    int E;                  // segments 0..E-1 use slot s; segment E uses slot E
+    const int32_t *seg_start, *seg_rows, *tile_start;
+    int *status;
+    int inject_fault;       // test hook: make one bounded wait run out (see api.cu)
+};
+cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launches);
+
+int num_sms();
+
+}  // namespace moe

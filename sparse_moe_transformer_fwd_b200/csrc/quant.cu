@@ -1,0 +1,219 @@
+// Blockwise e4m3 quantisation ("DeepSeek-R1", aguasto.com, "Quantization":
+// the checkpoint is blockwise FP8).  Per tile: amax = max |v| (exact on the
+// bf16 inputs), scale = amax / 448 and inv = 448 / amax (correctly rounded
+// binary32 divisions), code = e4m3 round-to-nearest-even, saturating, of the
+// binary32 product v * inv (hardware cvt.rn.satfinite.e4m3x2.f32).  An
+// all-zero tile gets scale 1 and +0 codes.
+//
+// Activations use 1x128 tiles: 16 threads own one tile (8 elements each,
+// one 16-byte load), amax by shuffles inside the 16-lane group.  Weights use
+// 128x128 blocks: one CTA per block, 64 elements per thread in registers,
+// amax through shared memory.  The forward pass fuses activation
+// quantisation with the permutation: each token row is quantised once and
+// its codes and scales are written to its k routed rows and its shared row.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+struct Quant8 {
+    float v[8];
+};
+
+__device__ __forceinline__ Quant8 load8_bf16(const uint16_t *p) {
+    const uint4 raw = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t r[4] = {raw.x, raw.y, raw.z, raw.w};
+    Quant8 q;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        q.v[2 * i] = bf16_lo(r[i]);
+        q.v[2 * i + 1] = bf16_hi(r[i]);
+    }
+    return q;
+}
+
+__device__ __forceinline__ float amax8(const Quant8 &q) {
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(q.v[i]));
+    return m;
+}
+
+// codes of 8 values for a tile with the given amax; returns the scale
+__device__ __forceinline__ uint2 encode8(const Quant8 &q, float amax, float *scale) {
+    if (amax == 0.0f) {
+        *scale = 1.0f;
+        return make_uint2(0, 0);
+    }
+    *scale = __fdiv_rn(amax, 448.0f);
+    const float inv = __fdiv_rn(448.0f, amax);
+    uint16_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        c[i] = e4m3x2(__fmul_rn(q.v[2 * i], inv), __fmul_rn(q.v[2 * i + 1], inv));
+    return make_uint2(static_cast<uint32_t>(c[0]) | (static_cast<uint32_t>(c[1]) << 16),
+                      static_cast<uint32_t>(c[2]) | (static_cast<uint32_t>(c[3]) << 16));
+}
+
+__device__ __forceinline__ float group16_max(float m) {
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    return m;
+}
+
+// 1 x 128 tiles over a [rows, cols] matrix
+__global__ void __launch_bounds__(256)
+quant_1x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld,
+                   uint8_t *__restrict__ q, float *__restrict__ scales) {
+    const int vpr = cols / 8;  // 16-byte vectors per row
+    const long long total = static_cast<long long>(rows) * vpr;
+    const long long nthreads = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long base = static_cast<long long>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
+         base < total; base += nthreads) {
+        const long long v = base + (threadIdx.x & 31);
+        const bool ok = v < total;
+        const int r = ok ? static_cast<int>(v / vpr) : 0;
+        const int vc = ok ? static_cast<int>(v % vpr) : 0;
+        Quant8 x;
+        if (ok) x = load8_bf16(in + static_cast<size_t>(r) * ld + vc * 8);
+        else
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x.v[i] = 0.0f;
+        const float amax = group16_max(amax8(x));
+        float sc;
+        const uint2 codes = encode8(x, amax, &sc);
+        if (ok) {
+            *reinterpret_cast<uint2 *>(q + static_cast<size_t>(r) * cols + vc * 8) = codes;
+            if ((vc & 15) == 0) scales[static_cast<size_t>(r) * (cols / 128) + vc / 16] = sc;
+        }
+    }
+}
+
+// 128 x 128 blocks; one CTA (256 threads) per block, grid-stride over blocks
+__global__ void __launch_bounds__(256)
+quant_128x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld,
+                     uint8_t *__restrict__ q, float *__restrict__ scales) {
+    __shared__ float red[8];
+    const int nkb = cols / 128, nrb = (rows + 127) / 128;
+    const long long nblocks = static_cast<long long>(nkb) * nrb;
+    const int tr = threadIdx.x / 16, tc = (threadIdx.x % 16) * 8;
+    for (long long b = blockIdx.x; b < nblocks; b += gridDim.x) {
+        const int rb = static_cast<int>(b / nkb), kb = static_cast<int>(b % nkb);
+        Quant8 x[8];
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = rb * 128 + tr + 16 * i;
+            if (r < rows) x[i] = load8_bf16(in + static_cast<size_t>(r) * ld + kb * 128 + tc);
+            else
+#pragma unroll
+                for (int j = 0; j < 8; ++j) x[i].v[j] = 0.0f;
+            m = fmaxf(m, amax8(x[i]));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+        __syncthreads();
+        float amax = red[0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+        __syncthreads();
+        float sc = 1.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = rb * 128 + tr + 16 * i;
+            const uint2 codes = encode8(x[i], amax, &sc);
+            if (r < rows) *reinterpret_cast<uint2 *>(q + static_cast<size_t>(r) * cols + kb * 128 + tc) = codes;
+        }
+        if (threadIdx.x == 0) scales[static_cast<size_t>(rb) * nkb + kb] = sc;
+    }
+}
+
+// Forward pass: quantise token t's row once, write it to its k + n_shared rows.
+__global__ void __launch_bounds__(256)
+quant_scatter_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_shared,
+                     const int32_t *__restrict__ row_of, uint8_t *__restrict__ a,
+                     float *__restrict__ a_scales) {
+    __shared__ int rows_sh[33];
+    const int t = blockIdx.x;
+    const int ndst = k + n_shared;
+    if (threadIdx.x < k) rows_sh[threadIdx.x] = row_of[static_cast<size_t>(t) * k + threadIdx.x];
+    if (threadIdx.x == 0 && n_shared) rows_sh[k] = T * k + t;
+    __syncthreads();
+    const int ntiles = d / 128, nkb = d / 128;
+    const int g = threadIdx.x / 16, l16 = threadIdx.x % 16;
+    for (int p = 0; p * 16 < ntiles; ++p) {
+        const int tile = p * 16 + g;
+        const bool ok = tile < ntiles;
+        Quant8 v;
+        if (ok) v = load8_bf16(x + static_cast<size_t>(t) * d + tile * 128 + l16 * 8);
+        else
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v.v[i] = 0.0f;
+        const float amax = group16_max(amax8(v));
+        float sc;
+        const uint2 codes = encode8(v, amax, &sc);
+        if (!ok) continue;
+        for (int j = 0; j < ndst; ++j) {
+            const size_t row = static_cast<size_t>(rows_sh[j]);
+            *reinterpret_cast<uint2 *>(a + row * d + tile * 128 + l16 * 8) = codes;
+            if (l16 == 0) a_scales[row * nkb + tile] = sc;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256)
+scatter_bf16_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_shared,
+                    const int32_t *__restrict__ row_of, uint16_t *__restrict__ a) {
+    __shared__ int rows_sh[33];
+    const int t = blockIdx.x;
+    const int ndst = k + n_shared;
+    if (threadIdx.x < k) rows_sh[threadIdx.x] = row_of[static_cast<size_t>(t) * k + threadIdx.x];
+    if (threadIdx.x == 0 && n_shared) rows_sh[k] = T * k + t;
+    __syncthreads();
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t) * d);
+    for (int v = threadIdx.x; v < d / 8; v += blockDim.x) {
+        const uint4 val = src[v];
+        for (int j = 0; j < ndst; ++j)
+            reinterpret_cast<uint4 *>(a + static_cast<size_t>(rows_sh[j]) * d)[v] = val;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
+                               uint8_t *q, float *scales, cudaStream_t st, int *launches) {
+    if (rows == 0) return cudaSuccess;
+    const int sms = num_sms();
+    if (block_rows == 1) {
+        const long long total = static_cast<long long>(rows) * (cols / 8);
+        const long long want = (total + 255) / 256;
+        const int grid = static_cast<int>(want < sms * 16LL ? want : sms * 16LL);
+        quant_1x128_kernel<<<grid, 256, 0, st>>>(in, rows, cols, ld, q, scales);
+    } else {
+        const long long nblocks = static_cast<long long>(cols / 128) * ((rows + 127) / 128);
+        const int grid = static_cast<int>(nblocks < sms * 8LL ? nblocks : sms * 8LL);
+        quant_128x128_kernel<<<grid, 256, 0, st>>>(in, rows, cols, ld, q, scales);
+    }
+    ++*launches;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_scatter(const uint16_t *x, int T, int d, int k, int n_shared,
+                                 const int32_t *row_of, uint8_t *a, float *a_scales,
+                                 cudaStream_t st, int *launches) {
+    quant_scatter_kernel<<<T, 256, 0, st>>>(x, T, d, k, n_shared, row_of, a, a_scales);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_bf16(const uint16_t *x, int T, int d, int k, int n_shared,
+                                const int32_t *row_of, uint16_t *a, cudaStream_t st,
+                                int *launches) {
+    scatter_bf16_kernel<<<T, 256, 0, st>>>(x, T, d, k, n_shared, row_of, a);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,250 @@
+// Router of the MoE layer ("DeepSeek v3 and R1 Model Architecture", section
+// "Local Balanced Routing to Experts": token-to-expert affinity, plus a
+// per-expert bias used only to select experts).
+//
+// Kernel 1 (router_scores): l[t,e] = sum_i x[t,i] W_r[e,i] in binary32, one
+//   fused multiply-add per term in the order i = 0..d-1 (each output is owned
+//   by one thread walking d in order; no split over d, no tensor cores), then
+//   s = sigmoid(l) with exp evaluated by Cody-Waite range reduction and a
+//   degree-7 Taylor polynomial (W. J. Cody, W. Waite, "Software Manual for
+//   the Elementary Functions", 1980).  Every operation is a correctly rounded
+//   binary32 operation, so the results are reproducible bit for bit.
+//   Tiling: a CTA owns BT tokens x BE experts; each thread a TT x TE register
+//   tile.  x and W_r chunks of KC columns are staged in shared memory as
+//   binary32 (bf16 widening is exact).
+// Kernel 2 (router_topk): one warp per token.  sel = s + b; k rounds of a
+//   warp arg-max under (sel desc, expert asc); gates g_j = s_j / S *
+//   routed_scale with S the binary32 sum of the selected s in rank order.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+// ------------------------------------------------- exp / sigmoid (binary32)
+// Constants derived from their definitions: ln 2 split into a head with the
+// low 12 significand bits cleared (so n * head is exact for |n| < 2^12) and
+// a tail; Taylor coefficients 1/i! rounded to binary32.
+constexpr double kLn2 = 0.693147180559945309417232121458176568;
+constexpr double kLog2e = 1.442695040888963407359924681001892137;
+
+struct ExpConsts {
+    float log2e, ln2_hi, ln2_lo, c[8];
+};
+
+__device__ __forceinline__ ExpConsts exp_consts() {
+    ExpConsts k;
+    k.log2e = static_cast<float>(kLog2e);
+    k.ln2_hi = __uint_as_float(__float_as_uint(static_cast<float>(kLn2)) & 0xfffff000u);
+    k.ln2_lo = static_cast<float>(kLn2 - static_cast<double>(k.ln2_hi));
+    double f = 1.0;
+    for (int i = 0; i < 8; ++i) {
+        if (i) f *= i;
+        k.c[i] = static_cast<float>(1.0 / f);
+    }
+    return k;
+}
+
+__device__ __forceinline__ float sigmoid_cw(float l, const ExpConsts &k) {
+    float y = -l;
+    y = fminf(fmaxf(y, -87.0f), 87.0f);
+    float n = rintf(__fmul_rn(y, k.log2e));
+    float r = __fmaf_rn(-n, k.ln2_hi, y);
+    r = __fmaf_rn(-n, k.ln2_lo, r);
+    float p = k.c[7];
+#pragma unroll
+    for (int i = 6; i >= 0; --i) p = __fmaf_rn(p, r, k.c[i]);
+    // 2^n with n in [-126, 126]: exact scaling of a normal result
+    float e = __fmul_rn(p, __int_as_float((static_cast<int>(n) + 127) << 23));
+    return __fdiv_rn(1.0f, __fadd_rn(1.0f, e));
+}
+
+// ------------------------------------------------------- router_scores ---
+template <int BT, int BE, int TT, int TE, int KC>
+__global__ void __launch_bounds__((BT / TT) * (BE / TE))
+router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w, int T, int d,
+                     int E, float *__restrict__ scores) {
+    constexpr int NTX = BE / TE;                  // threads along experts
+    constexpr int NTHREADS = (BT / TT) * NTX;
+    __shared__ __align__(16) float xs[2][KC][BT];  // [k][token]
+    __shared__ __align__(16) float ws[2][KC][BE];  // [k][expert]
+
+    const int tid = threadIdx.x;
+    const int t0 = blockIdx.y * BT, e0 = blockIdx.x * BE;
+    const int tx = tid % NTX, ty = tid / NTX;
+
+    float acc[TT][TE];
+#pragma unroll
+    for (int a = 0; a < TT; ++a)
+#pragma unroll
+        for (int b = 0; b < TE; ++b) acc[a][b] = 0.0f;
+
+    // staging: chunk kc of KC columns; each loader thread moves 8 bf16 (16 B)
+    auto stage = [&](int buf, int kc) {
+        const int k0 = kc * KC;
+        constexpr int XV = BT * KC / 8, WV = BE * KC / 8;
+        for (int v = tid; v < XV + WV; v += NTHREADS) {
+            const bool isx = v < XV;
+            const int vv = isx ? v : v - XV;
+            const int row = vv / (KC / 8), col = (vv % (KC / 8)) * 8;
+            const int g = isx ? t0 + row : e0 + row;
+            const int lim = isx ? T : E;
+            uint4 raw = make_uint4(0, 0, 0, 0);
+            if (g < lim) {
+                const uint16_t *src = (isx ? x : w) + static_cast<size_t>(g) * d + k0 + col;
+                raw = *reinterpret_cast<const uint4 *>(src);
+            }
+            const uint32_t r4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (isx) {
+                    xs[buf][col + 2 * q][row] = bf16_lo(r4[q]);
+                    xs[buf][col + 2 * q + 1][row] = bf16_hi(r4[q]);
+                } else {
+                    ws[buf][col + 2 * q][row] = bf16_lo(r4[q]);
+                    ws[buf][col + 2 * q + 1][row] = bf16_hi(r4[q]);
+                }
+            }
+        }
+    };
+
+    const int nk = d / KC;
+    stage(0, 0);
+    __syncthreads();
+    for (int kc = 0; kc < nk; ++kc) {
+        const int buf = kc & 1;
+        if (kc + 1 < nk) stage(buf ^ 1, kc + 1);
+#pragma unroll 4
+        for (int kk = 0; kk < KC; ++kk) {
+            float xv[TT], wv[TE];
+#pragma unroll
+            for (int a = 0; a < TT; ++a) xv[a] = xs[buf][kk][ty * TT + a];
+#pragma unroll
+            for (int b = 0; b < TE; ++b) wv[b] = ws[buf][kk][tx + b * NTX];
+#pragma unroll
+            for (int a = 0; a < TT; ++a)
+#pragma unroll
+                for (int b = 0; b < TE; ++b) acc[a][b] = __fmaf_rn(xv[a], wv[b], acc[a][b]);
+        }
+        __syncthreads();
+    }
+
+    const ExpConsts k = exp_consts();
+#pragma unroll
+    for (int a = 0; a < TT; ++a) {
+        const int t = t0 + ty * TT + a;
+        if (t >= T) continue;
+#pragma unroll
+        for (int b = 0; b < TE; ++b) {
+            const int e = e0 + tx + b * NTX;
+            if (e < E) scores[static_cast<size_t>(t) * E + e] = sigmoid_cw(acc[a][b], k);
+        }
+    }
+}
+
+// --------------------------------------------------------- router_topk ---
+constexpr int kMaxPerLane = 32;  // E <= 1024
+
+template <int PER_LANE>
+__global__ void __launch_bounds__(256)
+router_topk_kernel(const float *__restrict__ scores, const float *__restrict__ bias, int T, int E,
+                   int k, float routed_scale, int32_t *__restrict__ idx_out,
+                   float *__restrict__ gates_out) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float *srow = scores + static_cast<size_t>(t) * E;
+    float s[PER_LANE], sel[PER_LANE];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int m = 0; m < PER_LANE; ++m) {
+        const int e = lane + 32 * m;
+        if (e < E) {
+            s[m] = srow[e];
+            sel[m] = __fadd_rn(s[m], bias[e]);
+        } else {
+            s[m] = 0.0f;
+            sel[m] = 0.0f;
+            taken |= 1u << m;
+        }
+    }
+    float my_s = 0.0f;  // lane j keeps the affinity of its rank-j choice
+    int my_e = 0;
+    for (int j = 0; j < k; ++j) {
+        // best untaken expert of this lane (lowest index among equals: e grows with m)
+        float bv = 0.0f;
+        int be = 0x7fffffff;
+        float bs = 0.0f;
+#pragma unroll
+        for (int m = 0; m < PER_LANE; ++m) {
+            if (taken & (1u << m)) continue;
+            const int e = lane + 32 * m;
+            if (be == 0x7fffffff || sel[m] > bv) {
+                bv = sel[m];
+                be = e;
+                bs = s[m];
+            }
+        }
+        // warp arg-max under (sel desc, expert asc); lanes without candidates carry e = INT_MAX
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+            const bool other_better =
+                (oe != 0x7fffffff) && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be));
+            if (other_better) {
+                bv = ov;
+                be = oe;
+                bs = os;
+            }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        if (lane == j) {
+            my_s = bs;
+            my_e = be;
+        }
+    }
+    // S in rank order, then the gates
+    float S = 0.0f;
+    for (int j = 0; j < k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, my_s, j));
+    if (lane < k) {
+        idx_out[static_cast<size_t>(t) * k + lane] = my_e;
+        gates_out[static_cast<size_t>(t) * k + lane] = __fmul_rn(__fdiv_rn(my_s, S), routed_scale);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bias, int T, int d,
+                          int E, int k, float routed_scale, float *scores, int32_t *idx,
+                          float *gates, cudaStream_t st, int *launches) {
+    constexpr int KC = 32;
+    if (T >= 512) {
+        constexpr int BT = 64, BE = 128, TT = 4, TE = 8;
+        dim3 grid((E + BE - 1) / BE, (T + BT - 1) / BT);
+        router_scores_kernel<BT, BE, TT, TE, KC>
+            <<<grid, (BT / TT) * (BE / TE), 0, st>>>(x, w, T, d, E, scores);
+    } else {
+        constexpr int BT = 4, BE = 32, TT = 1, TE = 1;
+        dim3 grid((E + BE - 1) / BE, (T + BT - 1) / BT);
+        router_scores_kernel<BT, BE, TT, TE, KC>
+            <<<grid, (BT / TT) * (BE / TE), 0, st>>>(x, w, T, d, E, scores);
+    }
+    ++*launches;
+    const int per_lane = (E + 31) / 32;
+    dim3 grid2((T + 7) / 8);
+    if (per_lane <= 1)
+        router_topk_kernel<1><<<grid2, 256, 0, st>>>(scores, bias, T, E, k, routed_scale, idx, gates);
+    else if (per_lane <= 4)
+        router_topk_kernel<4><<<grid2, 256, 0, st>>>(scores, bias, T, E, k, routed_scale, idx, gates);
+    else if (per_lane <= 8)
+        router_topk_kernel<8><<<grid2, 256, 0, st>>>(scores, bias, T, E, k, routed_scale, idx, gates);
+    else
+        router_topk_kernel<kMaxPerLane>
+            <<<grid2, 256, 0, st>>>(scores, bias, T, E, k, routed_scale, idx, gates);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,86 @@
+"""CPU checks of the C ABI: the library loads without a GPU, exports every
+function include/moe_fwd.h declares, and rejects bad arguments on the host
+(before touching CUDA) with the documented codes."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_moe_transformer_fwd_b200 as moe
+from sparse_moe_transformer_fwd_b200 import _native as N
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_fwd.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w \*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+def test_header_functions_exported():
+    names = _declared_functions()
+    assert len(names) >= 10, names
+    L = moe.lib()
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing
+    assert sorted(N.EXPORTS) == names
+
+
+def _shape(**kw):
+    s = dict(T=64, d_model=7168, n_experts=256, top_k=8, d_expert=2048, n_shared=1,
+             routed_scale=1.0, precision="fp8")
+    s.update(kw)
+    return moe.make_shape(**s)
+
+
+def test_workspace_size_and_bad_shapes():
+    assert moe.moe_workspace_size(_shape()) > 64 * 7168 * 9
+    for bad in (dict(d_model=7000), dict(d_model=384), dict(d_expert=100), dict(top_k=0),
+                dict(top_k=33), dict(top_k=300), dict(n_shared=2), dict(n_experts=1024),
+                dict(precision=7), dict(T=-1)):
+        assert moe.lib().moe_workspace_size(ctypes.byref(_shape(**bad))) == 0, bad
+        assert moe.moe_last_error()
+
+
+FAKE = ctypes.c_void_p(0x7F0000001000)       # never dereferenced on the host
+MISALIGNED = ctypes.c_void_p(0x7F0000001004)
+
+
+def _call_forward(shape, ws_bytes, x=FAKE, ws=FAKE):
+    L = moe.lib()
+    return L.moe_forward(ctypes.byref(shape), x, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                         ws, ws_bytes, None)
+
+
+def test_host_side_errors_return_codes():
+    s = _shape()
+    need = moe.moe_workspace_size(s)
+    assert _call_forward(_shape(d_model=100), need) == N.MOE_ERR_INVALID_ARG
+    assert _call_forward(s, need - 1) == N.MOE_ERR_WORKSPACE
+    assert "needs" in moe.moe_last_error()
+    assert _call_forward(s, need, ws=ctypes.c_void_p(0x7F0000001010)) == N.MOE_ERR_INVALID_ARG
+    assert _call_forward(s, need, x=MISALIGNED) == N.MOE_ERR_INVALID_ARG
+    assert "aligned" in moe.moe_last_error()
+    assert _call_forward(s, need, x=None) == N.MOE_ERR_INVALID_ARG
+    L = moe.lib()
+    assert L.fp8_block_quant(FAKE, 10, 100, 100, 1, FAKE, FAKE, None) == N.MOE_ERR_INVALID_ARG
+    assert L.fp8_block_quant(FAKE, 10, 128, 128, 64, FAKE, FAKE, None) == N.MOE_ERR_INVALID_ARG
+    assert L.fp8_block_quant(FAKE, 0, 128, 128, 1, FAKE, FAKE, None) == N.MOE_OK
+
+
+def test_empty_batch_enqueues_nothing():
+    s = _shape(T=0)
+    assert _call_forward(s, moe.moe_workspace_size(s)) == N.MOE_OK
+    assert moe.moe_last_launch_count() == 0
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    s = _shape(T=4, d_model=256, n_experts=16, top_k=4, d_expert=128)
+    x = torch.zeros(4, 256, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        moe.moe_route(s, x, x, x, x, x, torch.zeros(16, dtype=torch.uint8))

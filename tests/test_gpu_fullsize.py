@@ -1,0 +1,88 @@
+"""GPU parity at the full DeepSeek-V3 layer sizes (d_model 7168, 256 experts
+top-8 + 1 shared, d_expert 2048) for the decode (T=64), prefill (T=4096),
+skewed-routing (T=16384) and bf16 (T=8192) workloads, in the launch
+configuration the benchmark times.  Inputs are generated on the GPU by the
+seeded generators; the oracle evaluates sampled tokens one batch at a time
+(tokens of the layer are independent): routing bit-exact, outputs within
+tolerance.  Weight codes and scales of sampled experts and the whole
+permutation are compared bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_moe_transformer_fwd_b200 as moe
+from moe_inputs import CONFIGS, make_inputs
+
+from _gpu_util import assert_out_close, oracle_layer, u16
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0") if torch.cuda.is_available() else None
+
+
+@pytest.fixture(scope="module", params=["decode", "prefill", "skew", "bf16"])
+def run(request):
+    cfg = CONFIGS[request.param]
+    inp = make_inputs(cfg, seed=0, device=DEV)
+    layer = moe.MoELayer(inp["w_router"], inp["bias"], inp["w13"], inp["w2"], top_k=cfg.top_k,
+                         n_shared=cfg.n_shared, precision=cfg.precision)
+    idx = torch.empty(cfg.T, cfg.top_k, dtype=torch.int32, device=DEV)
+    out = layer(inp["x"], topk_idx_out=idx)
+    status = layer.check_status(cfg.T)
+    yield cfg, inp, layer, idx, out, status
+    del layer, inp, out
+    torch.cuda.empty_cache()
+
+
+def test_status_ok(run):
+    assert run[5] == 0, moe.moe_last_error()
+
+
+def test_weight_quant_bitexact(run):
+    cfg, inp, layer = run[:3]
+    if cfg.precision != "fp8":
+        pytest.skip("bf16 workload")
+    for e in (0, 137 % cfg.n_experts, cfg.n_experts):
+        q13, s13 = oracle.block_quant(u16(inp["w13"][e]), 128)
+        assert np.array_equal(layer.w13s[e].cpu().numpy().view(np.uint32), s13.view(np.uint32))
+        assert np.array_equal(layer.w13[e].cpu().numpy(), q13)
+        q2, s2 = oracle.block_quant(u16(inp["w2"][e]), 128)
+        assert np.array_equal(layer.w2s[e].cpu().numpy().view(np.uint32), s2.view(np.uint32))
+        assert np.array_equal(layer.w2[e].cpu().numpy(), q2)
+
+
+def test_permutation_bitexact(run):
+    cfg, inp, layer, idx = run[:4]
+    T, E, k = cfg.T, cfg.n_experts, cfg.top_k
+    shape = layer.shape(T)
+    ws = moe.alloc_workspace(shape, DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    row_token = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    row_of = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    moe.moe_permute(shape, idx, counts, offsets, row_token, row_of, ws)
+    assert moe.moe_check_status(ws) == 0
+    rc, ro, rt, rr = oracle.permute(idx.cpu().numpy(), E)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(row_token.cpu().numpy(), rt)
+    assert np.array_equal(row_of.cpu().numpy(), rr)
+    if cfg.name == "skew":   # the workload's hottest expert carries about 10x the mean load
+        ratio = rc.max() / (T * k / E)
+        assert 8.0 <= ratio <= 12.0, ratio
+
+
+def _sample(cfg, idx_np):
+    counts = np.bincount(idx_np.reshape(-1), minlength=cfg.n_experts)
+    hot = int(np.argmax(counts))
+    t_hot = int(np.nonzero((idx_np == hot).any(1))[0][-1])
+    return sorted({0, cfg.T // 2, cfg.T - 1, t_hot})
+
+
+def test_sampled_tokens_vs_oracle(run):
+    cfg, inp, layer, idx, out = run[:5]
+    idx_np = idx.cpu().numpy()
+    tokens = _sample(cfg, idx_np)
+    ref = oracle_layer(cfg, inp, tokens=tokens)
+    assert np.array_equal(idx_np[tokens], ref["idx"])
+    assert_out_close(out[tokens], ref["out"], cfg.name)
