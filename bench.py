@@ -1,0 +1,390 @@
+"""Benchmark of the MoE-layer forward (DeepSeek-V3 dims) on B200.
+
+One step = one forward pass of the whole layer (router, permutation,
+quantise-and-scatter, grouped gate/up GEMM + SwiGLU, grouped down GEMM,
+combine) over one batch of synthetic tokens.  Default workload: the decode
+batch (T=64 tokens, d_model 7168, 256 routed experts top-8 + 1 shared,
+d_expert 2048, e4m3 blockwise weights and activations, bf16 I/O).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|prefill|skew|bf16|tiny]
+
+N > 1 (launched by torch.distributed.run) runs N independent replicas, one
+per GPU (the layer has no exchange step on one node's replicas): value =
+tokens of all ranks / max-over-ranks time.  Rank 0 prints one JSON line.
+--impl reference times the oracle (plain CPU implementation) on the host
+cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from moe_inputs import CONFIGS, make_inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at DeepSeek-V3 dims"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return PEAKS_FALLBACK, "fallback"
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- our arm ---
+
+def kernel_names(cfg):
+    names = ["router_scores", "router_topk", "perm_hist", "perm_scan", "perm_scatter",
+             "quant_scatter" if cfg.precision == "fp8" else "scatter_bf16",
+             "grouped_gemm_gate_up", "grouped_gemm_down", "combine"]
+    return names
+
+
+def algorithmic_bytes_gemm1(cfg, touched: int) -> float:
+    """Bytes the gate/up GEMM must move once: the weights of every touched
+    expert (and the shared one), their scales, the permuted activations and
+    scales in, H and its scales out."""
+    d, de, Rs = cfg.d_model, cfg.d_expert, cfg.R_s
+    es = 1 if cfg.precision == "fp8" else 2
+    w = touched * (2 * de * d * es + (4 * (2 * de // 128) * (d // 128) if es == 1 else 0))
+    a = Rs * d * es + (Rs * (d // 128) * 4 if es == 1 else 0)
+    h = Rs * de * es + (Rs * (de // 128) * 4 if es == 1 else 0)
+    return float(w + a + h)
+
+
+def run_ours(args, world, rank, local):
+    import sparse_moe_transformer_fwd_b200 as moe
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = CONFIGS[args.workload]
+    inp = make_inputs(cfg, seed=args.seed + rank, device=dev)
+    layer = moe.MoELayer(inp["w_router"], inp["bias"], inp["w13"], inp["w2"], top_k=cfg.top_k,
+                         n_shared=cfg.n_shared, precision=cfg.precision)
+    del inp["w13"], inp["w2"]
+    torch.cuda.empty_cache()
+    x = inp["x"]
+    T = cfg.T
+    out = torch.empty(T, cfg.d_model, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(T, cfg.top_k, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        layer(x, out=out, topk_idx_out=idx)
+    torch.cuda.synchronize()
+    status = layer.check_status(T)
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {moe.moe_last_error()}")
+    n_launch = moe.moe_last_launch_count()
+    touched = int(torch.unique(idx).numel()) + cfg.n_shared
+    counts = torch.bincount(idx.reshape(-1).long(), minlength=cfg.n_experts)
+
+    # ---- device-timed region: K steps, inputs resident in HBM
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)]
+          for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            moe.moe_set_kernel_events(ev[k])
+            layer(x, out=out, topk_idx_out=idx)
+        moe.moe_set_kernel_events(None)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_total = max_over_ranks(start.elapsed_time(stop), world, dev)
+    ms_step = ms_total / args.steps
+    per_kernel = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(n_launch)]
+                           for k in range(args.steps)])
+    kmean = per_kernel.mean(0)
+
+    # ---- end to end through the public API with host buffers
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty(T, cfg.d_model, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer(x_dev, out=out)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer(x_dev, out=out)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    status = layer.check_status(T)
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {moe.moe_last_error()}")
+
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    names = kernel_names(cfg)
+    gi = names.index("grouped_gemm_gate_up")
+    g1_ms = float(kmean[gi])
+    g1_bytes = algorithmic_bytes_gemm1(cfg, touched)
+    achieved = g1_bytes / (g1_ms * 1e-3) / 1e9
+    tokens_total = T * world
+    value = tokens_total / (ms_step * 1e-3)
+    res = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3" if cfg.precision == "fp8" else "bf16",
+        "data": "synthetic (seeded; random-init weights of the DeepSeek-V3 MoE layer shape)",
+        "config": {
+            "workload": f"{cfg.name}: T={T}, d_model={cfg.d_model}, {cfg.n_experts} experts "
+                        f"top-{cfg.top_k} + {cfg.n_shared} shared, d_expert={cfg.d_expert}, "
+                        + ("e4m3 1x128/128x128 blockwise, bf16 I/O" if cfg.precision == "fp8"
+                           else "bf16"),
+            "tokens_per_gpu": T,
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "l2": f"inputs larger than L2: {touched} touched experts' weights "
+                  f"({g1_bytes / 1e9:.2f} GB in the gate/up GEMM alone) per step",
+            "expert_load_max_over_mean": round(float(counts.max()) / (T * cfg.top_k / cfg.n_experts), 2),
+        },
+        "roofline": {
+            "kernel": "grouped_gemm_gate_up",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"],
+            "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                           else "fallback",
+            "algorithmic_bytes": g1_bytes,
+            "kernel_ms": round(g1_ms, 4),
+            "traffic": None,
+        },
+        "kernels_ms": {n: round(float(v), 4) for n, v in zip(names, kmean)},
+        "e2e": {"value": round(tokens_total / (ms_e2e * 1e-3), 1), "unit": "tokens/s",
+                "ms_per_step": round(ms_e2e, 4),
+                "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                "d2h_bytes_per_step": int(out.numel() * out.element_size())},
+        "gpu_launches": n_launch * args.steps,
+        "clocks": clk.summary(),
+    }
+    return res, cfg
+
+
+# ----------------------------------------------------- oracle (CPU) arm ---
+
+def oracle_sample_time(cfg, dev, n_tokens: int, seed: int, reps: int = 1):
+    """Time the oracle's whole layer on a sample of n_tokens of the workload's
+    batch (tokens are independent), BLAS limited to one thread."""
+    import oracle
+    from threadpoolctl import threadpool_limits
+    inp = make_inputs(cfg, seed=seed, device=dev)
+    u16 = lambda t: t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    tokens = list(range(0, cfg.T, max(1, cfg.T // n_tokens)))[:n_tokens]
+    x = u16(inp["x"][tokens])
+    wr = u16(inp["w_router"])
+    b = inp["bias"].cpu().numpy()
+    # host copies of the experts the sample touches (inputs, copied before timing)
+    import oracle as _o
+    sel = set()
+    idx, _, _ = _o.route(_o.router_logits(x, wr), b, cfg.top_k)
+    sel.update(int(e) for e in idx.reshape(-1))
+    sel.add(cfg.n_experts)
+    experts = {e: (u16(inp["w13"][e]), u16(inp["w2"][e])) for e in sorted(sel)}
+    del inp
+    times = []
+    with threadpool_limits(limits=1):
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            oracle.moe_layer(x, wr, b, lambda e: experts[e], n_experts=cfg.n_experts,
+                             top_k=cfg.top_k, n_shared=cfg.n_shared, precision=cfg.precision)
+            times.append(time.perf_counter() - t0)
+    return times, len(tokens), len(sel)
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for l in f:
+                if l.startswith("model name"):
+                    return l.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def run_reference(args, world, rank, local):
+    if rank != 0:
+        return None
+    cfg = CONFIGS[args.workload]
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    n_tok = args.ref_tokens
+    step_times = []
+    warm, _, _ = oracle_sample_time(cfg, dev, n_tok, args.seed, reps=max(1, min(args.warmup, 1)))
+    times, ntok, nexp = oracle_sample_time(cfg, dev, n_tok, args.seed, reps=args.steps)
+    step_times = times
+    s_step = statistics.mean(step_times)
+    value = ntok / s_step
+    sample = (f"{ntok} tokens of the {cfg.name} batch per step through the oracle's whole layer "
+              f"(routing, permutation, quantisation incl. the {nexp} touched experts' weights, "
+              f"binary64 expert GEMMs, combine); C core and numpy on 1 thread")
+    return {
+        "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(s_step * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{cfg.name}: T={cfg.T}, d_model={cfg.d_model}, "
+                               f"{cfg.n_experts} experts top-{cfg.top_k} + {cfg.n_shared} shared"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": sample, "cpu": cpu_model()},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }, cfg
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(CONFIGS), default="decode")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--ref-tokens", type=int, default=1,
+                    help="tokens of the batch per oracle step (reference arm)")
+    ap.add_argument("--cpu-baseline-tokens", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            r = run_reference(args, world, rank, local)
+            if r is not None:
+                print(json.dumps(r[0]), flush=True)
+            return
+        r = run_ours(args, world, rank, local)
+        if r is not None:
+            res, cfg = r
+            if world == 1 and not args.no_cpu_baseline:
+                dev = torch.device("cuda", local)
+                times, ntok, nexp = oracle_sample_time(cfg, dev, args.cpu_baseline_tokens,
+                                                       args.seed)
+                res["cpu_baseline"] = {
+                    "value": round(ntok / times[0], 4), "unit": "tokens/s", "cores": 1,
+                    "kind": "oracle",
+                    "sample": f"{ntok} tokens of the {cfg.name} batch through the oracle's whole "
+                              f"layer ({nexp} experts incl. their weight quantisation), "
+                              f"{times[0]:.1f} s, 1 thread",
+                    "cpu": cpu_model()}
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

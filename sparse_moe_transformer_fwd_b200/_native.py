@@ -25,7 +25,7 @@ MOE_FP8_BLOCK = 1
 # every symbol include/moe_fwd.h declares
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant",
            "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_check_status",
-           "moe_last_error", "moe_last_launch_count")
+           "moe_last_error", "moe_last_launch_count", "moe_set_kernel_events")
 
 
 class MoeShape(ctypes.Structure):
@@ -65,8 +65,10 @@ def lib() -> ctypes.CDLL:
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         L.moe_last_launch_count.argtypes = []
+        L.moe_set_kernel_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ci]
         for name in ("moe_route", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
-                     "moe_combine", "moe_forward", "moe_check_status", "moe_last_launch_count"):
+                     "moe_combine", "moe_forward", "moe_check_status", "moe_last_launch_count",
+                     "moe_set_kernel_events"):
             getattr(L, name).restype = ci
         _LIB = L
     return _LIB
@@ -190,3 +192,15 @@ def moe_last_error() -> str:
 
 def moe_last_launch_count() -> int:
     return lib().moe_last_launch_count()
+
+
+def moe_set_kernel_events(events) -> None:
+    """Profiling hook: `events` is a list of torch.cuda.Event (created with
+    enable_timing=True) or None.  Later calls on this thread record events[i]
+    before their i-th kernel launch and events[launches] after the last."""
+    if events is None:
+        _check(lib().moe_set_kernel_events(None, 0))
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    moe_set_kernel_events._keep = arr  # the library keeps the pointer
+    _check(lib().moe_set_kernel_events(arr, len(events)))

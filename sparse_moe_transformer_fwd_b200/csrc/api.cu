@@ -19,6 +19,15 @@ int num_sms() {
 }
 
 namespace {
+thread_local cudaEvent_t *g_events = nullptr;  // profiling hook (moe_set_kernel_events)
+thread_local int g_n_events = 0;
+}  // namespace
+
+void mark_launch(cudaStream_t st, int index) {
+    if (g_events && index < g_n_events) cudaEventRecord(g_events[index], st);
+}
+
+namespace {
 
 thread_local std::string g_err;
 thread_local int g_launches = 0;
@@ -252,6 +261,7 @@ int moe_route(const moe_shape *s, const uint16_t *x, const uint16_t *w_router, c
                          s->routed_scale, at<float>(ws, L.scores), topk_idx, topk_w,
                          static_cast<cudaStream_t>(stream), &n),
            "router");
+    mark_launch(static_cast<cudaStream_t>(stream), n);
     g_launches = n;
     return MOE_OK;
 }
@@ -281,6 +291,7 @@ int moe_permute(const moe_shape *s, const int32_t *topk_idx, int32_t *counts, in
                           perm_scratch(ws, L), counts, offsets, row_token, row_of,
                           at<int>(ws, L.status), static_cast<cudaStream_t>(stream), &n),
            "permute");
+    mark_launch(static_cast<cudaStream_t>(stream), n);
     g_launches = n;
     return MOE_OK;
 }
@@ -301,6 +312,7 @@ int fp8_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_ro
     LAUNCH(launch_block_quant(in, rows, cols, ld, block_rows, q, scales,
                               static_cast<cudaStream_t>(stream), &n),
            "fp8_block_quant");
+    mark_launch(static_cast<cudaStream_t>(stream), n);
     g_launches = n;
     return MOE_OK;
 }
@@ -325,6 +337,7 @@ int moe_grouped_swiglu(const moe_shape *s, const void *a, const float *a_scales,
                              perm_scratch(ws, L), at<int>(ws, L.status), st, &n),
            "tile table");
     RETURN_IF(grouped(s, a, a_scales, w13, w13_scales, w2, w2_scales, y, ws, L, st, &n));
+    mark_launch(st, n);
     g_launches = n;
     return MOE_OK;
 }
@@ -342,6 +355,7 @@ int moe_combine(const moe_shape *s, const uint16_t *y, const int32_t *row_of,
     LAUNCH(launch_combine(y, row_of, topk_w, s->T, s->d_model, s->top_k, s->n_shared, out,
                           static_cast<cudaStream_t>(stream), &n),
            "combine");
+    mark_launch(static_cast<cudaStream_t>(stream), n);
     g_launches = n;
     return MOE_OK;
 }
@@ -388,6 +402,7 @@ int moe_forward(const moe_shape *s, const uint16_t *x, const uint16_t *w_router,
                       w13_scales, w2, w2_scales, y, ws, L, st, &n));
     LAUNCH(launch_combine(y, row_of, gates, s->T, s->d_model, s->top_k, s->n_shared, out, st, &n),
            "combine");
+    mark_launch(st, n);
     g_launches = n;
     return MOE_OK;
 }
@@ -412,5 +427,12 @@ int moe_check_status(void *ws, void *stream) {
 const char *moe_last_error(void) { return g_err.c_str(); }
 
 int moe_last_launch_count(void) { return g_launches; }
+
+int moe_set_kernel_events(void **events, int n_events) {
+    if (events && n_events <= 0) return fail(MOE_ERR_INVALID_ARG, "n_events must be positive");
+    g_events = reinterpret_cast<cudaEvent_t *>(events);
+    g_n_events = events ? n_events : 0;
+    return MOE_OK;
+}
 
 }  // extern "C"

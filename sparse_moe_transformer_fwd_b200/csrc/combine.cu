@@ -60,6 +60,7 @@ combine_kernel(const uint16_t *__restrict__ y, const int32_t *__restrict__ row_o
 cudaError_t launch_combine(const uint16_t *y, const int32_t *row_of, const float *gates, int T,
                            int d, int k, int n_shared, uint16_t *out, cudaStream_t st,
                            int *launches) {
+    mark_launch(st, *launches);
     combine_kernel<<<T, 128, 0, st>>>(y, row_of, gates, T, d, k, n_shared, out);
     ++*launches;
     return cudaGetLastError();

@@ -99,7 +99,7 @@ __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int ti
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
 template <bool FP8, bool GATE_UP>
-__global__ void __maxnreg__(200)
+__global__ void __maxnreg__(192)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const KParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -535,6 +535,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
     if (grid <= 0) return cudaSuccess;
     cudaError_t e;
+    mark_launch(st, *launches);
     if (g.fp8) e = g.gate_up ? launch_t<true, true>(ma, mb, kp, grid, st)
                              : launch_t<true, false>(ma, mb, kp, grid, st);
     else e = g.gate_up ? launch_t<false, true>(ma, mb, kp, grid, st)

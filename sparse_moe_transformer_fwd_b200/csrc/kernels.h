@@ -81,4 +81,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
 
 int num_sms();
 
+// Profiling hook: records the caller's event `index` on `st` when the
+// moe_set_kernel_events hook is active (call just before a kernel launch).
+void mark_launch(cudaStream_t st, int index);
+
 }  // namespace moe

@@ -184,17 +184,23 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int n_shared
                            int *status, cudaStream_t st, int *launches) {
     const int nblk = (T + kBT - 1) / kBT;
     const size_t smem = static_cast<size_t>(E) * kWords * sizeof(uint32_t);
+    mark_launch(st, *launches);
     perm_hist_kernel<<<nblk, 256, smem, st>>>(idx, T, k, E, s.masks, s.hist, status);
+    ++*launches;
+    mark_launch(st, *launches);
     perm_scan_kernel<<<1, 1024, 0, st>>>(s.hist, nblk, E, T, k, n_shared, s.blkoff, counts,
                                          offsets, s.seg_start, s.seg_rows, s.tile_start);
+    ++*launches;
+    mark_launch(st, *launches);
     perm_scatter_kernel<<<nblk, 256, smem, st>>>(idx, T, k, E, s.masks, s.blkoff, offsets,
                                                   row_token, row_of);
-    *launches += 3;
+    ++*launches;
     return cudaGetLastError();
 }
 
 cudaError_t launch_tile_table(const int32_t *offsets, int E, int T, int k, int n_shared,
                               PermScratch s, int *status, cudaStream_t st, int *launches) {
+    mark_launch(st, *launches);
     tile_table_kernel<<<1, 1024, 0, st>>>(offsets, E, T, k, n_shared, s.seg_start, s.seg_rows,
                                           s.tile_start, status);
     ++*launches;

@@ -186,6 +186,7 @@ cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, i
                                uint8_t *q, float *scales, cudaStream_t st, int *launches) {
     if (rows == 0) return cudaSuccess;
     const int sms = num_sms();
+    mark_launch(st, *launches);
     if (block_rows == 1) {
         const long long total = static_cast<long long>(rows) * (cols / 8);
         const long long want = (total + 255) / 256;
@@ -203,6 +204,7 @@ cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, i
 cudaError_t launch_quant_scatter(const uint16_t *x, int T, int d, int k, int n_shared,
                                  const int32_t *row_of, uint8_t *a, float *a_scales,
                                  cudaStream_t st, int *launches) {
+    mark_launch(st, *launches);
     quant_scatter_kernel<<<T, 256, 0, st>>>(x, T, d, k, n_shared, row_of, a, a_scales);
     ++*launches;
     return cudaGetLastError();
@@ -211,6 +213,7 @@ cudaError_t launch_quant_scatter(const uint16_t *x, int T, int d, int k, int n_s
 cudaError_t launch_scatter_bf16(const uint16_t *x, int T, int d, int k, int n_shared,
                                 const int32_t *row_of, uint16_t *a, cudaStream_t st,
                                 int *launches) {
+    mark_launch(st, *launches);
     scatter_bf16_kernel<<<T, 256, 0, st>>>(x, T, d, k, n_shared, row_of, a);
     ++*launches;
     return cudaGetLastError();

@@ -220,6 +220,7 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
                           int E, int k, float routed_scale, float *scores, int32_t *idx,
                           float *gates, cudaStream_t st, int *launches) {
     constexpr int KC = 32;
+    mark_launch(st, *launches);
     if (T >= 512) {
         constexpr int BT = 64, BE = 128, TT = 4, TE = 8;
         dim3 grid((E + BE - 1) / BE, (T + BT - 1) / BT);
@@ -234,6 +235,7 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
     ++*launches;
     const int per_lane = (E + 31) / 32;
     dim3 grid2((T + 7) / 8);
+    mark_launch(st, *launches);
     if (per_lane <= 1)
         router_topk_kernel<1><<<grid2, 256, 0, st>>>(scores, bias, T, E, k, routed_scale, idx, gates);
     else if (per_lane <= 4)

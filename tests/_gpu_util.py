@@ -1,7 +1,13 @@
 """Helpers shared by the GPU parity tests: tensor conversions, running the
-CUDA path through the C ABI, running the oracle on the same inputs, and the
-output tolerance (relative L2 <= 1e-3 and max |diff| <= 1e-2 * RMS of the
-oracle output)."""
+oracle on the same inputs, and the output tolerance.
+
+Tolerance of a bf16 output against the oracle's bf16-rounded output:
+relative L2 <= 1e-3, and max |diff| <= 1e-2 * RMS(oracle) beyond one bf16
+step of the oracle value.  The step allowance is the storage quantum: two
+correct evaluations whose binary32 / binary64 sums straddle a bf16 rounding
+boundary store values one step apart, and a step is |v|/256..|v|/128, which
+is larger than 1e-2 * RMS wherever |v| > 1.28 * RMS.  Without it no bf16
+output could meet the max-abs bound."""
 from __future__ import annotations
 
 import numpy as np
@@ -22,19 +28,28 @@ def from_u16(a: np.ndarray, device) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
 
 
+def bf16_step(v: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 values at |v| (8 significant bits)."""
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
 def out_error(got_bf16: torch.Tensor, want_u16: np.ndarray):
+    """-> (relative L2, max |diff| / RMS, max (|diff| - one bf16 step)+ / RMS)."""
     got = got_bf16.detach().float().cpu().numpy().astype(np.float64)
     want = oracle.bf16_to_f32(want_u16).astype(np.float64).reshape(got.shape)
+    diff = np.abs(got - want)
     rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300)
-    rms = np.sqrt(np.mean(want ** 2))
-    mx = np.abs(got - want).max() / max(rms, 1e-300)
-    return rel, mx
+    rms = max(np.sqrt(np.mean(want ** 2)), 1e-300)
+    excess = np.maximum(diff - bf16_step(want), 0.0)
+    return rel, diff.max() / rms, excess.max() / rms
 
 
 def assert_out_close(got_bf16, want_u16, what=""):
-    rel, mx = out_error(got_bf16, want_u16)
-    assert rel <= REL_L2 and mx <= MAX_ABS_RMS, f"{what}: rel_l2={rel:.3e} max/rms={mx:.3e}"
-    return rel, mx
+    rel, mx, ex = out_error(got_bf16, want_u16)
+    assert rel <= REL_L2 and ex <= MAX_ABS_RMS, \
+        f"{what}: rel_l2={rel:.3e} max/rms={mx:.3e} beyond-one-step/rms={ex:.3e}"
+    return rel, mx, ex
 
 
 def oracle_layer(cfg, inp, tokens=None, expert=None):
