@@ -14,9 +14,13 @@
 //   warp 1      TMEM allocator (512 columns) and MMA issuer (one thread):
 //               tcgen05.mma M=128 N=256, K=32 (e4m3) or K=16 (bf16), four per
 //               stage.
-//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (tile rows);
-//               warps 2-5 take columns [0,64) and [128,192), warps 6-9 take
+//   warps 2-3   idle (warpgroup 0 gives its registers to the epilogue)
+//   warps 4-11  epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (tile rows);
+//               warps 4-7 take columns [0,64) and [128,192), warps 8-11 take
 //               [64,128) and [192,256).
+// Registers: the register file is split over the SM's four sub-partitions
+// and a warpgroup puts one warp on each, so warpgroup 0 drops to 40
+// registers and the two epilogue warpgroups rise to 232 (setmaxnreg).
 // FP8: every 128-wide K block is accumulated by the tensor core into one of
 //   two TMEM buffers (fresh each block); the epilogue loads it and adds it
 //   into binary32 registers times s_a[row, kb] * s_w[nblock, kb] (the
@@ -45,7 +49,12 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * 128;        // 16 KB per stage
 constexpr int B_BYTES = BN * 128;        // 32 KB per stage
 constexpr int STAGE_TX = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_THREADS = 384;  // 3 warpgroups
+constexpr int LAUNCH_REGS = 168;   // 65536 / 384, multiple of 8
+constexpr int PRODUCER_REGS = 40;  // warpgroup 0 after setmaxnreg.dec
+constexpr int EPILOGUE_REGS = 232; // warpgroups 1-2 after setmaxnreg.inc
+static_assert(128 * PRODUCER_REGS + 256 * EPILOGUE_REGS <= NUM_THREADS * LAUNCH_REGS,
+              "register split must fit in the block's launch allocation");
 constexpr int EPI_THREADS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_SEG = 1025;
@@ -99,7 +108,7 @@ __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int ti
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
 template <bool FP8, bool GATE_UP>
-__global__ void __maxnreg__(192)
+__global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const KParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -145,6 +154,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const int total_tiles = s.tile_start[n_seg] * p.n_tiles_n;
     volatile int *abort = &s.abort;
 
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(PRODUCER_REGS));
+    }
     if (warp == 0) {
         // ------------------------------------------------------- producer
         if (lane == 0) {
@@ -251,10 +263,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
             }
         }
-    } else {
+    } else if (warp >= 4) {
         // ------------------------------------------------------- epilogue
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(EPILOGUE_REGS));
         const int q = warp & 3;            // TMEM lane quadrant = tile rows 32q..32q+31
-        const int half = (warp - 2) >> 2;  // column half
+        const int half = (warp - 4) >> 2;  // column half
         const int r_in = q * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
         const int KB128 = p.K / 128;
@@ -496,9 +509,16 @@ cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams
     const size_t smem = sizeof(GemmSmem) + 1024;
     static bool configured = false;  // per template instance; attribute is per device function
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<FP8, GATE_UP>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
+        // setmaxnreg redistributes exactly NUM_THREADS * LAUNCH_REGS registers:
+        // refuse to launch a build whose register count differs, as the
+        // epilogue's increase would then never be granted.
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, grouped_gemm_kernel<FP8, GATE_UP>);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(grouped_gemm_kernel<FP8, GATE_UP>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         configured = true;
     }
