@@ -201,6 +201,9 @@ def moe_set_kernel_events(events) -> None:
     if events is None:
         _check(lib().moe_set_kernel_events(None, 0))
         return
+    for e in events:  # torch creates the CUDA event lazily, on its first record
+        if e.cuda_event == 0:
+            e.record()
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     moe_set_kernel_events._keep = arr  # the library keeps the pointer
     _check(lib().moe_set_kernel_events(arr, len(events)))

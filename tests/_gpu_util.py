@@ -10,6 +10,9 @@ is larger than 1e-2 * RMS wherever |v| > 1.28 * RMS.  Without it no bf16
 output could meet the max-abs bound."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -45,8 +48,18 @@ def out_error(got_bf16: torch.Tensor, want_u16: np.ndarray):
     return rel, diff.max() / rms, excess.max() / rms
 
 
+def _log(what, rel, mx, ex):
+    path = os.environ.get("MOE_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"test": os.environ.get("PYTEST_CURRENT_TEST", ""), "what": what,
+                                "rel_l2": rel, "max_over_rms": mx,
+                                "beyond_one_step_over_rms": ex}) + "\n")
+
+
 def assert_out_close(got_bf16, want_u16, what=""):
     rel, mx, ex = out_error(got_bf16, want_u16)
+    _log(what, rel, mx, ex)
     assert rel <= REL_L2 and ex <= MAX_ABS_RMS, \
         f"{what}: rel_l2={rel:.3e} max/rms={mx:.3e} beyond-one-step/rms={ex:.3e}"
     return rel, mx, ex
