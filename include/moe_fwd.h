@@ -98,6 +98,28 @@ int moe_route(const moe_shape *shape, const uint16_t *x, const uint16_t *w_route
               const float *bias, int32_t *topk_idx, float *topk_w,
               void *ws, size_t ws_bytes, void *stream);
 
+/* Router for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this call: it exists for callers that are not allowed to call
+ * cudaMalloc and have no workspace to pass, e.g. code inside a host
+ * framework's plugin interface that owns all device memory, or a serving loop
+ * that forbids allocation after start-up because cudaMalloc can synchronise
+ * the device and stall every other stream.  Same computation and outputs as
+ * moe_route, but its [T, E] score scratch is a fixed array inside the library
+ * (MOE_ROUTE_NOALLOC_MAX_SCORES floats, 4 MiB, held on every GPU that loads
+ * the library until the process exits).
+ *   - T * n_experts above MOE_ROUTE_NOALLOC_MAX_SCORES: MOE_ERR_INVALID_ARG,
+ *     nothing enqueued.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current), so make that first call before any stream capture.
+ *   - Every call shares the one array: calls whose kernels overlap on the GPU
+ *     (other streams, other host threads) race and must be serialised by the
+ *     caller.  The array keeps the last call's scores; nothing in it needs to
+ *     start at zero.
+ *   - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call). */
+#define MOE_ROUTE_NOALLOC_MAX_SCORES (1 << 20)
+int moe_route_noalloc(const moe_shape *shape, const uint16_t *x, const uint16_t *w_router,
+                      const float *bias, int32_t *topk_idx, float *topk_w, void *stream);
+
 /* Permutation into per-expert segments (expert order; tokens ascending inside
  * a segment; deterministic).
  *   topk_idx  int32 [T, top_k] in

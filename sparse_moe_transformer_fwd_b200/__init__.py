@@ -15,13 +15,15 @@ import torch
 from ._native import (EXPORTS, MOE_BF16, MOE_FP8_BLOCK, MoeError, MoeShape, alloc_workspace,
                       fp8_block_quant, lib, make_shape, moe_check_status, moe_combine,
                       moe_forward, moe_grouped_swiglu, moe_last_error, moe_last_launch_count,
-                      moe_permute, moe_route, moe_set_kernel_events, moe_workspace_size)
+                      moe_permute, moe_route, moe_route_noalloc, moe_set_kernel_events,
+                      moe_workspace_size, MOE_ROUTE_NOALLOC_MAX_SCORES)
 
 __all__ = [
     "MoELayer", "MoeError", "MoeShape", "make_shape", "alloc_workspace", "lib", "EXPORTS",
     "moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
     "moe_combine", "moe_forward", "moe_check_status", "moe_last_error", "moe_last_launch_count",
     "quantize_weights", "MOE_BF16", "MOE_FP8_BLOCK", "moe_set_kernel_events",
+    "moe_route_noalloc", "MOE_ROUTE_NOALLOC_MAX_SCORES",
 ]
 
 

@@ -25,7 +25,11 @@ MOE_FP8_BLOCK = 1
 # every symbol include/moe_fwd.h declares
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant",
            "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_check_status",
-           "moe_last_error", "moe_last_launch_count", "moe_set_kernel_events")
+           "moe_last_error", "moe_last_launch_count", "moe_set_kernel_events",
+           "moe_route_noalloc")
+
+# fixed score scratch of moe_route_noalloc, in floats (include/moe_fwd.h)
+MOE_ROUTE_NOALLOC_MAX_SCORES = 1 << 20
 
 
 class MoeShape(ctypes.Structure):
@@ -57,6 +61,7 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_size.restype = sz
         L.moe_route.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_permute.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_route_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp]
         L.fp8_block_quant.argtypes = [vp, ci, ci, ci, ci, vp, vp, vp]
         L.moe_grouped_swiglu.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_combine.argtypes = [sp, vp, vp, vp, vp, vp]
@@ -66,7 +71,7 @@ def lib() -> ctypes.CDLL:
         L.moe_last_error.restype = ctypes.c_char_p
         L.moe_last_launch_count.argtypes = []
         L.moe_set_kernel_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ci]
-        for name in ("moe_route", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
+        for name in ("moe_route", "moe_route_noalloc", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
                      "moe_combine", "moe_forward", "moe_check_status", "moe_last_launch_count",
                      "moe_set_kernel_events"):
             getattr(L, name).restype = ci
@@ -129,6 +134,17 @@ def moe_route(shape, x, w_router, bias, topk_idx, topk_w, ws, stream=None):
                            _ptr(topk_idx, torch.int32, "topk_idx"),
                            _ptr(topk_w, torch.float32, "topk_w"), _ptr(ws, torch.uint8, "ws"),
                            ws.numel(), _stream(stream)))
+
+
+def moe_route_noalloc(shape, x, w_router, bias, topk_idx, topk_w, stream=None):
+    """moe_route without a workspace: for callers that may not allocate device
+    memory.  The [T, E] score scratch is a fixed array inside the library
+    (T * E <= MOE_ROUTE_NOALLOC_MAX_SCORES); calls that overlap on the GPU race."""
+    _check(lib().moe_route_noalloc(ctypes.byref(shape), _ptr(x, _BF16, "x"),
+                                   _ptr(w_router, _BF16, "w_router"),
+                                   _ptr(bias, torch.float32, "bias"),
+                                   _ptr(topk_idx, torch.int32, "topk_idx"),
+                                   _ptr(topk_w, torch.float32, "topk_w"), _stream(stream)))
 
 
 def moe_permute(shape, topk_idx, counts, offsets, row_token, row_of, ws, stream=None):

@@ -8,6 +8,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "../../include/moe_fwd.h"
+
 namespace moe {
 
 constexpr int kTileM = 128;  // rows per grouped-GEMM tile (tcgen05 M)
@@ -80,6 +82,11 @@ struct GemmArgs {
 cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launches);
 
 int num_sms();
+
+// Error/launch bookkeeping shared by the C entry points (api.cu).
+int record_error(int code, const char *msg);  // sets moe_last_error, returns code
+void record_launches(int n);                   // sets moe_last_launch_count
+int validate_shape(const moe_shape *s);        // host-side shape checks
 
 // Profiling hook: records the caller's event `index` on `st` when the
 // moe_set_kernel_events hook is active (call just before a kernel launch).
