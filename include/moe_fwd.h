@@ -200,8 +200,8 @@ int moe_last_launch_count(void);
  * by the caller) or NULL to switch the hook off.  While set, every later
  * call on this thread records events[i] on its stream just before its i-th
  * kernel launch and events[launches] after the last one (the CUDA-event
- * timeline of each kernel); a call that would need more than n_events
- * events records none.  Returns MOE_OK or MOE_ERR_INVALID_ARG. */
+ * timeline of each kernel), for indices below n_events; a NULL entry is
+ * skipped.  Returns MOE_OK or MOE_ERR_INVALID_ARG. */
 int moe_set_kernel_events(void **events, int n_events);
 
 #ifdef __cplusplus

@@ -80,6 +80,10 @@ CONFIGS = {
     "prefill": MoEConfig("prefill", T=4096, precision="fp8", bias="zero", **_DS),
     "skew": MoEConfig("skew", T=16384, precision="fp8", bias="zipf", **_DS),
     "bf16": MoEConfig("bf16", T=8192, precision="bf16", bias="zero", **_DS),
+    # profiling-size stand-in for the decode batch: same per-expert shapes,
+    # 32 routed experts, so every buffer is a few GB at most
+    "decode_small": MoEConfig("decode_small", T=64, precision="fp8", bias="uniform",
+                              **{**_DS, "n_experts": 32}),
 }
 
 

@@ -212,14 +212,16 @@ def moe_last_launch_count() -> int:
 
 def moe_set_kernel_events(events) -> None:
     """Profiling hook: `events` is a list of torch.cuda.Event (created with
-    enable_timing=True) or None.  Later calls on this thread record events[i]
-    before their i-th kernel launch and events[launches] after the last."""
+    enable_timing=True; None entries are skipped) or None to switch it off.
+    Later calls on this thread record events[i] before their i-th kernel
+    launch and events[launches] after the last."""
     if events is None:
         _check(lib().moe_set_kernel_events(None, 0))
         return
     for e in events:  # torch creates the CUDA event lazily, on its first record
-        if e.cuda_event == 0:
+        if e is not None and e.cuda_event == 0:
             e.record()
-    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    arr = (ctypes.c_void_p * len(events))(
+        *[ctypes.c_void_p(e.cuda_event if e is not None else None) for e in events])
     moe_set_kernel_events._keep = arr  # the library keeps the pointer
     _check(lib().moe_set_kernel_events(arr, len(events)))

@@ -24,7 +24,7 @@ thread_local int g_n_events = 0;
 }  // namespace
 
 void mark_launch(cudaStream_t st, int index) {
-    if (g_events && index < g_n_events) cudaEventRecord(g_events[index], st);
+    if (g_events && index < g_n_events && g_events[index]) cudaEventRecord(g_events[index], st);
 }
 
 namespace {

@@ -79,22 +79,37 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
 #pragma unroll
         for (int b = 0; b < TE; ++b) acc[a][b] = 0.0f;
 
-    // staging: chunk kc of KC columns; each loader thread moves 8 bf16 (16 B)
-    auto stage = [&](int buf, int kc) {
+    // staging of chunk kc (KC columns of x and W_r) through registers: the
+    // global loads of chunk kc+1 are issued before chunk kc is computed and
+    // land in shared memory after it, so L2 latency hides behind the FMAs.
+    constexpr int XV = BT * KC / 8, WV = BE * KC / 8;   // 16-byte vectors
+    constexpr int NV = (XV + WV + NTHREADS - 1) / NTHREADS;
+    uint4 pre[NV];
+    auto load = [&](int kc) {
         const int k0 = kc * KC;
-        constexpr int XV = BT * KC / 8, WV = BE * KC / 8;
-        for (int v = tid; v < XV + WV; v += NTHREADS) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int v = tid + j * NTHREADS;
+            pre[j] = make_uint4(0, 0, 0, 0);
+            if (v < XV + WV) {
+                const bool isx = v < XV;
+                const int vv = isx ? v : v - XV;
+                const int row = vv / (KC / 8), col = (vv % (KC / 8)) * 8;
+                const int g = isx ? t0 + row : e0 + row;
+                if (g < (isx ? T : E))
+                    pre[j] = *reinterpret_cast<const uint4 *>((isx ? x : w) + static_cast<size_t>(g) * d + k0 + col);
+            }
+        }
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int v = tid + j * NTHREADS;
+            if (v >= XV + WV) continue;
             const bool isx = v < XV;
             const int vv = isx ? v : v - XV;
             const int row = vv / (KC / 8), col = (vv % (KC / 8)) * 8;
-            const int g = isx ? t0 + row : e0 + row;
-            const int lim = isx ? T : E;
-            uint4 raw = make_uint4(0, 0, 0, 0);
-            if (g < lim) {
-                const uint16_t *src = (isx ? x : w) + static_cast<size_t>(g) * d + k0 + col;
-                raw = *reinterpret_cast<const uint4 *>(src);
-            }
-            const uint32_t r4[4] = {raw.x, raw.y, raw.z, raw.w};
+            const uint32_t r4[4] = {pre[j].x, pre[j].y, pre[j].z, pre[j].w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 if (isx) {
@@ -109,11 +124,12 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
     };
 
     const int nk = d / KC;
-    stage(0, 0);
+    load(0);
+    store(0);
     __syncthreads();
     for (int kc = 0; kc < nk; ++kc) {
         const int buf = kc & 1;
-        if (kc + 1 < nk) stage(buf ^ 1, kc + 1);
+        if (kc + 1 < nk) load(kc + 1);
 #pragma unroll 4
         for (int kk = 0; kk < KC; ++kk) {
             float xv[TT], wv[TE];
@@ -126,6 +142,7 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
 #pragma unroll
                 for (int b = 0; b < TE; ++b) acc[a][b] = __fmaf_rn(xv[a], wv[b], acc[a][b]);
         }
+        if (kc + 1 < nk) store(buf ^ 1);
         __syncthreads();
     }
 
@@ -219,15 +236,14 @@ router_topk_kernel(const float *__restrict__ scores, const float *__restrict__ b
 cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bias, int T, int d,
                           int E, int k, float routed_scale, float *scores, int32_t *idx,
                           float *gates, cudaStream_t st, int *launches) {
-    constexpr int KC = 32;
     mark_launch(st, *launches);
     if (T >= 512) {
-        constexpr int BT = 64, BE = 128, TT = 4, TE = 8;
+        constexpr int BT = 64, BE = 128, TT = 4, TE = 8, KC = 32;
         dim3 grid((E + BE - 1) / BE, (T + BT - 1) / BT);
         router_scores_kernel<BT, BE, TT, TE, KC>
             <<<grid, (BT / TT) * (BE / TE), 0, st>>>(x, w, T, d, E, scores);
     } else {
-        constexpr int BT = 4, BE = 32, TT = 1, TE = 1;
+        constexpr int BT = 4, BE = 32, TT = 1, TE = 1, KC = 128;
         dim3 grid((E + BE - 1) / BE, (T + BT - 1) / BT);
         router_scores_kernel<BT, BE, TT, TE, KC>
             <<<grid, (BT / TT) * (BE / TE), 0, st>>>(x, w, T, d, E, scores);
