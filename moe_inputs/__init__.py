@@ -84,6 +84,9 @@ CONFIGS = {
     # 32 routed experts, so every buffer is a few GB at most
     "decode_small": MoEConfig("decode_small", T=64, precision="fp8", bias="uniform",
                               **{**_DS, "n_experts": 32}),
+    # profiling-size stand-in for the large batches: ~1000 rows per expert
+    "prefill_small": MoEConfig("prefill_small", T=4096, precision="fp8", bias="zero",
+                               **{**_DS, "n_experts": 32}),
 }
 
 

@@ -109,6 +109,13 @@ __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int ti
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
+// acc + partial * scale (FP8 promotion) or acc + partial (BF16 chunk sum)
+template <bool FP8>
+__device__ __forceinline__ float promote(float acc, float v, float sc) {
+    if constexpr (FP8) return __fmaf_rn(v, sc, acc);
+    else return __fadd_rn(acc, v);
+}
+
 template <bool FP8, bool GATE_UP>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
@@ -287,12 +294,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             const float *sw_lo_p = FP8 ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * NCH : nullptr;
             const float *sw_hi_p = FP8 ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_hi) * NCH : nullptr;
             const float *sa_p = FP8 ? p.a_scales + row * NCH : nullptr;
+            // scales of chunk c are loaded one chunk ahead (global latency)
+            float nsa = 0.0f, nswl = 1.0f, nswh = 1.0f;
+            if (FP8 && warp_active) {
+                nsa = valid ? __ldg(sa_p) : 0.0f;
+                nswl = __ldg(sw_lo_p);
+                nswh = __ldg(sw_hi_p);
+            }
             for (int c = 0; c < NCH; ++c) {
-                float sc_lo = 1.0f, sc_hi = 1.0f;
-                if (FP8 && warp_active) {
-                    const float sa = valid ? __ldg(sa_p + c) : 0.0f;
-                    sc_lo = sa * __ldg(sw_lo_p + c);
-                    sc_hi = sa * __ldg(sw_hi_p + c);
+                const float sc_lo = FP8 ? nsa * nswl : 1.0f, sc_hi = FP8 ? nsa * nswh : 1.0f;
+                if (FP8 && warp_active && c + 1 < NCH) {
+                    nsa = valid ? __ldg(sa_p + c + 1) : 0.0f;
+                    nswl = __ldg(sw_lo_p + c + 1);
+                    nswh = __ldg(sw_hi_p + c + 1);
                 }
                 if (!mbar_wait(&s.tfull[tb], tphase, abort, p.status)) {
                     ok = false;
@@ -300,20 +314,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
                 tc_fence_after();
                 if (warp_active) {
+                    // four 32-column pieces; the load of piece j+1 is in flight
+                    // while the FMAs of piece j issue
                     const uint32_t base = lane_base + tb * BN;
+                    float va[32], vb[32];
+                    tmem_ld32(base + col_lo, va);
+                    tmem_wait_ld(va);
+                    tmem_ld32(base + col_lo + 32, vb);
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const int col = (ch < 2 ? col_lo : col_hi) + 32 * (ch & 1);
-                        const float sc = ch < 2 ? sc_lo : sc_hi;
-                        float v[32];
-                        tmem_ld32(base + col, v);
-                        tmem_wait_ld();
+                    for (int i = 0; i < 32; ++i) acc[i] = promote<FP8>(acc[i], va[i], sc_lo);
+                    tmem_wait_ld(vb);
+                    tmem_ld32(base + col_hi, va);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            if constexpr (FP8) acc[32 * ch + i] = __fmaf_rn(v[i], sc, acc[32 * ch + i]);
-                            else acc[32 * ch + i] = __fadd_rn(acc[32 * ch + i], v[i]);
-                        }
-                    }
+                    for (int i = 0; i < 32; ++i) acc[32 + i] = promote<FP8>(acc[32 + i], vb[i], sc_lo);
+                    tmem_wait_ld(va);
+                    tmem_ld32(base + col_hi + 32, vb);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[64 + i] = promote<FP8>(acc[64 + i], va[i], sc_hi);
+                    tmem_wait_ld(vb);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[96 + i] = promote<FP8>(acc[96 + i], vb[i], sc_hi);
                 }
                 tc_fence_before();
                 __syncwarp();

@@ -159,6 +159,84 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
     }
 }
 
+// ------------------------------------------------- router_scores (small T)
+// Decode-sized batches: warp w of the CTA owns token t0 + w, lane l owns
+// expert e0 + l; one output per thread, so the kernel is bound by the length
+// of its d-long FMA chain.  x and W_r chunks sit k-contiguous in shared
+// memory (rows padded by 4 floats), read as 16-byte vectors: x by broadcast,
+// W_r in four conflict-free wavefronts per warp.  Staging goes through
+// registers one chunk ahead, as in the tiled kernel.
+template <int BT, int KC>
+__global__ void __launch_bounds__(BT * 32)
+router_scores_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w, int T,
+                           int d, int E, float *__restrict__ scores) {
+    constexpr int BE = 32, LD = KC + 4;
+    constexpr int NT = BT * 32;
+    constexpr int VPR = KC / 8;                  // 16-byte vectors per row per chunk
+    constexpr int NV = (BT + BE) * VPR;
+    constexpr int PER = (NV + NT - 1) / NT;
+    __shared__ __align__(16) float xs[2][BT][LD];
+    __shared__ __align__(16) float ws[2][BE][LD];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t0 = blockIdx.y * BT, e0 = blockIdx.x * BE;
+
+    uint4 pre[PER];
+    auto load = [&](int kc) {
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int v = tid + j * NT;
+            pre[j] = make_uint4(0, 0, 0, 0);
+            if (v < NV) {
+                const int row = v / VPR, col = (v % VPR) * 8;
+                const bool isx = row < BT;
+                const int g = isx ? t0 + row : e0 + row - BT;
+                if (g < (isx ? T : E))
+                    pre[j] = *reinterpret_cast<const uint4 *>((isx ? x : w) + static_cast<size_t>(g) * d +
+                                                              kc * KC + col);
+            }
+        }
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int v = tid + j * NT;
+            if (v >= NV) continue;
+            const int row = v / VPR, col = (v % VPR) * 8;
+            float *dst = row < BT ? &xs[buf][row][col] : &ws[buf][row - BT][col];
+            const uint32_t r4[4] = {pre[j].x, pre[j].y, pre[j].z, pre[j].w};
+            *reinterpret_cast<float4 *>(dst) =
+                make_float4(bf16_lo(r4[0]), bf16_hi(r4[0]), bf16_lo(r4[1]), bf16_hi(r4[1]));
+            *reinterpret_cast<float4 *>(dst + 4) =
+                make_float4(bf16_lo(r4[2]), bf16_hi(r4[2]), bf16_lo(r4[3]), bf16_hi(r4[3]));
+        }
+    };
+
+    float acc = 0.0f;
+    const int nk = d / KC;
+    load(0);
+    store(0);
+    __syncthreads();
+    for (int kc = 0; kc < nk; ++kc) {
+        const int buf = kc & 1;
+        if (kc + 1 < nk) load(kc + 1);
+        const float *xr = xs[buf][warp];
+        const float *wr = ws[buf][lane];
+#pragma unroll 8
+        for (int kk = 0; kk < KC; kk += 4) {
+            const float4 xa = *reinterpret_cast<const float4 *>(xr + kk);
+            const float4 wa = *reinterpret_cast<const float4 *>(wr + kk);
+            acc = __fmaf_rn(xa.x, wa.x, acc);
+            acc = __fmaf_rn(xa.y, wa.y, acc);
+            acc = __fmaf_rn(xa.z, wa.z, acc);
+            acc = __fmaf_rn(xa.w, wa.w, acc);
+        }
+        if (kc + 1 < nk) store(buf ^ 1);
+        __syncthreads();
+    }
+    const int t = t0 + warp, e = e0 + lane;
+    if (t < T && e < E) scores[static_cast<size_t>(t) * E + e] = sigmoid_cw(acc, exp_consts());
+}
+
 // --------------------------------------------------------- router_topk ---
 constexpr int kMaxPerLane = 32;  // E <= 1024
 
@@ -243,10 +321,9 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
         router_scores_kernel<BT, BE, TT, TE, KC>
             <<<grid, (BT / TT) * (BE / TE), 0, st>>>(x, w, T, d, E, scores);
     } else {
-        constexpr int BT = 4, BE = 32, TT = 1, TE = 1, KC = 128;
-        dim3 grid((E + BE - 1) / BE, (T + BT - 1) / BT);
-        router_scores_kernel<BT, BE, TT, TE, KC>
-            <<<grid, (BT / TT) * (BE / TE), 0, st>>>(x, w, T, d, E, scores);
+        constexpr int BT = 4, KC = 128;
+        dim3 grid((E + 31) / 32, (T + BT - 1) / BT);
+        router_scores_small_kernel<BT, KC><<<grid, BT * 32, 0, st>>>(x, w, T, d, E, scores);
     }
     ++*launches;
     const int per_lane = (E + 31) / 32;
