@@ -25,10 +25,11 @@
 //   one of two TMEM buffers (fresh each chunk); the epilogue loads it and adds
 //   it into binary32 registers (FP8: times s_a[row, kc] * s_w[nblock, kc], the
 //   per-128-K scale promotion), while the tensor core fills the other buffer.
-//   BF16 takes the same path without scales: the tensor core's internal sum
-//   over a long K is not IEEE binary32 (whole-K accumulation of K = 7168 put
-//   the layer output 1.25e-3 (relative L2) away from the binary64 oracle), and
-//   128-wide chunks added in binary32 registers bring it back.
+//   BF16 takes the same path without scales, in 256-wide chunks: the tensor
+//   core's internal sum over a long K is not IEEE binary32 (whole-K
+//   accumulation of K = 7168 put the layer output 1.25e-3 (relative L2) away
+//   from the binary64 oracle), and chunks added in binary32 registers bring
+//   it back.
 // Epilogue: gate/up GEMM -> H = silu(G) * U, then (FP8) 1x128 e4m3
 //   quantisation of H (one 128-feature tile per row per work item; the two
 //   column halves exchange their amax through shared memory) or (BF16) bf16
@@ -109,11 +110,19 @@ __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int ti
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
-// acc + partial * scale (FP8 promotion) or acc + partial (BF16 chunk sum)
+// acc[base..base+15] (column pairs) += partial * scale (FP8 promotion) or
+// += partial (BF16 chunk sum), with the paired binary32 FMA / add of sm_100
+// (two correctly rounded operations per instruction).
 template <bool FP8>
-__device__ __forceinline__ float promote(float acc, float v, float sc) {
-    if constexpr (FP8) return __fmaf_rn(v, sc, acc);
-    else return __fadd_rn(acc, v);
+__device__ __forceinline__ void promote32(float2 (&acc)[64], int base, const float (&v)[32],
+                                          float sc) {
+    const float2 s2 = make_float2(sc, sc);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const float2 p = make_float2(v[2 * j], v[2 * j + 1]);
+        if constexpr (FP8) acc[base + j] = __ffma2_rn(p, s2, acc[base + j]);
+        else acc[base + j] = __fadd2_rn(acc[base + j], p);
+    }
 }
 
 template <bool FP8, bool GATE_UP>
@@ -125,8 +134,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = FP8 ? p.K / 128 : p.K / 64;  // stages per tile (128 bytes of K each)
-    constexpr int SPC = FP8 ? 1 : 2;             // stages per 128-wide K chunk
-    const int NCH = p.K / 128;                   // K chunks per tile
+    // stages per promotion chunk: FP8 128 K (the scale block); BF16 256 K
+    constexpr int SPC = FP8 ? 1 : 4;
+    const int NCH = (KB + SPC - 1) / SPC;        // K chunks per tile (last may be short)
     const int n_seg = p.n_segments;
 
     // ---------------------------------------------------------------- setup
@@ -223,7 +233,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             bool ok = true;
             for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
                 for (int kb = 0; kb < KB; ++kb) {
-                    const bool chunk_first = (kb % SPC) == 0, chunk_last = (kb % SPC) == SPC - 1;
+                    const bool chunk_first = (kb % SPC) == 0;
+                    const bool chunk_last = (kb % SPC) == SPC - 1 || kb == KB - 1;
                     if (chunk_first) {
                         if (!mbar_wait(&s.tempty[tb], tphase ^ 1, abort, p.status)) {
                             ok = false;
@@ -286,9 +297,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             const bool valid = r_in < rows_valid;
             const size_t row = static_cast<size_t>(row0) + r_in;
             const int col_lo = half * 64, col_hi = 128 + half * 64;
-            float acc[128];
+            float2 acc2[64];  // columns (2j, 2j+1) of the thread's 128
 #pragma unroll
-            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
             const int nb_lo = GATE_UP ? nt : 2 * nt;
             const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
             const float *sw_lo_p = FP8 ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * NCH : nullptr;
@@ -321,19 +332,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     tmem_ld32(base + col_lo, va);
                     tmem_wait_ld(va);
                     tmem_ld32(base + col_lo + 32, vb);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[i] = promote<FP8>(acc[i], va[i], sc_lo);
+                    promote32<FP8>(acc2, 0, va, sc_lo);
                     tmem_wait_ld(vb);
                     tmem_ld32(base + col_hi, va);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[32 + i] = promote<FP8>(acc[32 + i], vb[i], sc_lo);
+                    promote32<FP8>(acc2, 16, vb, sc_lo);
                     tmem_wait_ld(va);
                     tmem_ld32(base + col_hi + 32, vb);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[64 + i] = promote<FP8>(acc[64 + i], va[i], sc_hi);
+                    promote32<FP8>(acc2, 32, va, sc_hi);
                     tmem_wait_ld(vb);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[96 + i] = promote<FP8>(acc[96 + i], vb[i], sc_hi);
+                    promote32<FP8>(acc2, 48, vb, sc_hi);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -342,13 +349,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 if (tb == 0) tphase ^= 1;
             }
             if (!ok) break;
+            // column c of the thread's 128 (in place, no copy)
+            auto acc = [&](int c) -> float & { return (c & 1) ? acc2[c >> 1].y : acc2[c >> 1].x; };
             if constexpr (GATE_UP) {
                 // H = silu(G) * U for features nt*128 + half*64 + c, c < 64
                 float m = 0.0f;
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
-                    acc[c] = silu(acc[c]) * acc[64 + c];
-                    m = fmaxf(m, fabsf(acc[c]));
+                    acc(c) = silu(acc(c)) * acc(64 + c);
+                    m = fmaxf(m, fabsf(acc(c)));
                 }
                 if constexpr (FP8) {
                     const int par = iter & 1;
@@ -373,8 +382,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
                                 const int b = c + 4 * i;
-                                const uint32_t lo = e4m3x2(__fmul_rn(acc[b], inv), __fmul_rn(acc[b + 1], inv));
-                                const uint32_t hi = e4m3x2(__fmul_rn(acc[b + 2], inv), __fmul_rn(acc[b + 3], inv));
+                                const uint32_t lo = e4m3x2(__fmul_rn(acc(b), inv), __fmul_rn(acc(b + 1), inv));
+                                const uint32_t hi = e4m3x2(__fmul_rn(acc(b + 2), inv), __fmul_rn(acc(b + 3), inv));
                                 w[i] = amax != 0.0f ? (lo | (hi << 16)) : 0u;
                             }
                             *reinterpret_cast<uint4 *>(hq + c) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -387,10 +396,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 #pragma unroll
                     for (int c = 0; c < 64; c += 8) {
                         uint4 o;
-                        o.x = pack_bf16x2(acc[c], acc[c + 1]);
-                        o.y = pack_bf16x2(acc[c + 2], acc[c + 3]);
-                        o.z = pack_bf16x2(acc[c + 4], acc[c + 5]);
-                        o.w = pack_bf16x2(acc[c + 6], acc[c + 7]);
+                        o.x = pack_bf16x2(acc(c), acc(c + 1));
+                        o.y = pack_bf16x2(acc(c + 2), acc(c + 3));
+                        o.z = pack_bf16x2(acc(c + 4), acc(c + 5));
+                        o.w = pack_bf16x2(acc(c + 6), acc(c + 7));
                         *reinterpret_cast<uint4 *>(h + c) = o;
                     }
                 }
@@ -399,15 +408,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 #pragma unroll
                 for (int c = 0; c < 64; c += 8) {
                     uint4 o;
-                    o.x = pack_bf16x2(acc[c], acc[c + 1]);
-                    o.y = pack_bf16x2(acc[c + 2], acc[c + 3]);
-                    o.z = pack_bf16x2(acc[c + 4], acc[c + 5]);
-                    o.w = pack_bf16x2(acc[c + 6], acc[c + 7]);
+                    o.x = pack_bf16x2(acc(c), acc(c + 1));
+                    o.y = pack_bf16x2(acc(c + 2), acc(c + 3));
+                    o.z = pack_bf16x2(acc(c + 4), acc(c + 5));
+                    o.w = pack_bf16x2(acc(c + 6), acc(c + 7));
                     *reinterpret_cast<uint4 *>(y + col_lo + c) = o;
-                    o.x = pack_bf16x2(acc[64 + c], acc[64 + c + 1]);
-                    o.y = pack_bf16x2(acc[64 + c + 2], acc[64 + c + 3]);
-                    o.z = pack_bf16x2(acc[64 + c + 4], acc[64 + c + 5]);
-                    o.w = pack_bf16x2(acc[64 + c + 6], acc[64 + c + 7]);
+                    o.x = pack_bf16x2(acc(64 + c), acc(64 + c + 1));
+                    o.y = pack_bf16x2(acc(64 + c + 2), acc(64 + c + 3));
+                    o.z = pack_bf16x2(acc(64 + c + 4), acc(64 + c + 5));
+                    o.w = pack_bf16x2(acc(64 + c + 6), acc(64 + c + 7));
                     *reinterpret_cast<uint4 *>(y + col_hi + c) = o;
                 }
             }
