@@ -66,6 +66,17 @@ enum moe_precision {
     MOE_FP8_BLOCK = 1  /* e4m3 1x128 activations, 128x128 weights, fp32 scales */
 };
 
+/* Weight storage.  The expert GEMMs read their weights in TILED layout: a
+ * row-major matrix of R rows x C bytes (R, C multiples of 128) stored as
+ * (R/128) x (C/128) tiles of 128 rows x 128 bytes, tile (i, j) at byte
+ * offset (i * (C/128) + j) * 16384, row r of a tile at r * 128 inside it.
+ * For a stack [n, N, K] of expert matrices, R = n*N.  Each tile is one
+ * contiguous 16 KB read (for e4m3 exactly one 128x128 scale block). */
+enum moe_layout {
+    MOE_LAYOUT_ROWMAJOR = 0,
+    MOE_LAYOUT_TILED = 1
+};
+
 /* Layer shape.  T tokens, d_model, n_experts routed experts (E), top_k (k),
  * d_expert, n_shared (0 or 1 shared experts of width d_expert),
  * routed_scale (multiplies every gate), precision (enum moe_precision). */
@@ -135,15 +146,23 @@ int moe_permute(const moe_shape *shape, const int32_t *topk_idx, int32_t *counts
 /* Blockwise e4m3 quantisation ("Quantization": blockwise FP8) of a bf16
  * [rows, cols] matrix with leading dimension ld (elements, >= cols, multiple
  * of 8).  Tiles are block_rows x 128 (block_rows 1 for activations, 128 for
- * weights; a short last row block is allowed).  Per tile amax; scale =
- * amax / 448, codes = e4m3_rn_satfinite(v * (448 / amax)); an all-zero tile
- * gets scale 1 and +0 codes.
- *   q      e4m3 [rows, cols] out (dense, leading dimension cols)
+ * weights; a short last row block is allowed in row-major output).  Per tile
+ * amax; scale = amax / 448, codes = e4m3_rn_satfinite(v * (448 / amax)); an
+ * all-zero tile gets scale 1 and +0 codes.
+ *   out_layout MOE_LAYOUT_ROWMAJOR: q is e4m3 [rows, cols] (leading dimension
+ *              cols); MOE_LAYOUT_TILED (block_rows 128, rows % 128 == 0):
+ *              q holds the same codes in the tiled layout the GEMMs read
  *   scales fp32 [ceil(rows / block_rows), cols / 128] out
  * A stack of expert matrices [n, N, K] with N % 128 == 0 is one call with
  * rows = n*N, cols = K. */
 int fp8_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
-                    uint8_t *q, float *scales, void *stream);
+                    int out_layout, uint8_t *q, float *scales, void *stream);
+
+/* Repacks a row-major matrix of `rows` rows x `row_bytes` bytes (both
+ * multiples of 128; src and dst 16-byte aligned, not overlapping) into the
+ * tiled layout (MOE_LAYOUT_TILED).  Used once, ahead of time, for bf16
+ * expert weights; pure data movement. */
+int moe_pack_tiles(const void *src, int rows, int row_bytes, void *dst, void *stream);
 
 /* Grouped gated expert MLP over the permuted rows (card: "experts are gated
  * MLPs"): for every segment s (routed experts 0..E-1, then the shared expert
@@ -152,9 +171,10 @@ int fp8_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_ro
  *   a          [R_s, d_model] bf16, or e4m3 codes in MOE_FP8_BLOCK
  *   a_scales   fp32 [R_s, d_model/128] (MOE_FP8_BLOCK) or NULL
  *   offsets    int32 [n_experts + 1] segment starts (as from moe_permute)
- *   w13        [E + n_shared, 2*d_expert, d_model]: gate rows, then up rows
+ *   w13        [E + n_shared, 2*d_expert, d_model]: gate rows, then up rows,
+ *              e4m3 or bf16, in MOE_LAYOUT_TILED
  *   w13_scales fp32 [E + n_shared, 2*d_expert/128, d_model/128] or NULL
- *   w2         [E + n_shared, d_model, d_expert]
+ *   w2         [E + n_shared, d_model, d_expert], MOE_LAYOUT_TILED
  *   w2_scales  fp32 [E + n_shared, d_model/128, d_expert/128] or NULL
  *   y          bf16 [R_s, d_model] out
  * In MOE_FP8_BLOCK, H is quantised 1x128 (e4m3) before the down GEMM; in
@@ -176,8 +196,9 @@ int moe_combine(const moe_shape *shape, const uint16_t *y, const int32_t *row_of
 /* The whole layer: route, permute, quantise-and-scatter (or bf16 scatter),
  * grouped gate/up GEMM + SwiGLU, grouped down GEMM, combine.
  *   x [T, d_model] bf16 in; out [T, d_model] bf16 out.
- *   w13/w2 and scales as for moe_grouped_swiglu (weights are quantised once,
- *   ahead of time, with fp8_block_quant in MOE_FP8_BLOCK).
+ *   w13/w2 and scales as for moe_grouped_swiglu (tiled; weights are quantised
+ *   once, ahead of time, with fp8_block_quant(..., MOE_LAYOUT_TILED, ...) in
+ *   MOE_FP8_BLOCK, or repacked with moe_pack_tiles in MOE_BF16).
  *   topk_idx_out int32 [T, k] or NULL: receives the routing decision. */
 int moe_forward(const moe_shape *shape, const uint16_t *x, const uint16_t *w_router,
                 const float *bias, const void *w13, const float *w13_scales,

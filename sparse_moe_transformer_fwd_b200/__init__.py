@@ -12,7 +12,8 @@ from __future__ import annotations
 
 import torch
 
-from ._native import (EXPORTS, MOE_BF16, MOE_FP8_BLOCK, MoeError, MoeShape, alloc_workspace,
+from ._native import (EXPORTS, MOE_BF16, MOE_FP8_BLOCK, MOE_LAYOUT_ROWMAJOR, MOE_LAYOUT_TILED,
+                      MoeError, moe_pack_tiles, MoeShape, alloc_workspace,
                       fp8_block_quant, lib, make_shape, moe_check_status, moe_combine,
                       moe_forward, moe_grouped_swiglu, moe_last_error, moe_last_launch_count,
                       moe_permute, moe_route, moe_route_noalloc, moe_set_kernel_events,
@@ -23,22 +24,32 @@ __all__ = [
     "moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
     "moe_combine", "moe_forward", "moe_check_status", "moe_last_error", "moe_last_launch_count",
     "quantize_weights", "MOE_BF16", "MOE_FP8_BLOCK", "moe_set_kernel_events",
-    "moe_route_noalloc", "MOE_ROUTE_NOALLOC_MAX_SCORES",
+    "moe_route_noalloc", "MOE_ROUTE_NOALLOC_MAX_SCORES", "moe_pack_tiles", "pack_weights",
+    "MOE_LAYOUT_ROWMAJOR", "MOE_LAYOUT_TILED",
 ]
 
 
 def quantize_weights(w13: torch.Tensor, w2: torch.Tensor, stream=None):
     """128x128 e4m3 block quantisation of the stacked expert weights (done
-    once, ahead of the forward passes).  Returns (w13q, w13s, w2q, w2s)."""
+    once, ahead of the forward passes), codes in the tiled layout the GEMMs
+    read.  Returns (w13q, w13s, w2q, w2s)."""
     S, n13, d = w13.shape
     _, d2, de = w2.shape
     w13q = torch.empty(S, n13, d, dtype=torch.uint8, device=w13.device)
     w13s = torch.empty(S, n13 // 128, d // 128, dtype=torch.float32, device=w13.device)
     w2q = torch.empty(S, d2, de, dtype=torch.uint8, device=w2.device)
     w2s = torch.empty(S, d2 // 128, de // 128, dtype=torch.float32, device=w2.device)
-    fp8_block_quant(w13, 128, w13q, w13s, stream=stream)
-    fp8_block_quant(w2, 128, w2q, w2s, stream=stream)
+    fp8_block_quant(w13, 128, w13q, w13s, layout=MOE_LAYOUT_TILED, stream=stream)
+    fp8_block_quant(w2, 128, w2q, w2s, layout=MOE_LAYOUT_TILED, stream=stream)
     return w13q, w13s, w2q, w2s
+
+
+def pack_weights(w13: torch.Tensor, w2: torch.Tensor, stream=None):
+    """bf16 expert weights repacked into the tiled layout the GEMMs read."""
+    a, b = torch.empty_like(w13), torch.empty_like(w2)
+    moe_pack_tiles(w13.contiguous(), a, stream=stream)
+    moe_pack_tiles(w2.contiguous(), b, stream=stream)
+    return a, b
 
 
 class MoELayer:
@@ -63,7 +74,7 @@ class MoELayer:
             self.w13_bf16 = w13 if keep_bf16 else None
             self.w2_bf16 = w2 if keep_bf16 else None
         elif precision == "bf16":
-            self.w13, self.w2 = w13.contiguous(), w2.contiguous()
+            self.w13, self.w2 = pack_weights(w13, w2)
             self.w13s = self.w2s = None
         else:
             raise ValueError(precision)

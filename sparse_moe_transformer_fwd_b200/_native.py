@@ -21,12 +21,14 @@ MOE_ERR_TIMEOUT = -5
 MOE_ERR_DEVICE_INDEX = -6
 MOE_BF16 = 0
 MOE_FP8_BLOCK = 1
+MOE_LAYOUT_ROWMAJOR = 0
+MOE_LAYOUT_TILED = 1
 
 # every symbol include/moe_fwd.h declares
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant",
            "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_check_status",
            "moe_last_error", "moe_last_launch_count", "moe_set_kernel_events",
-           "moe_route_noalloc")
+           "moe_route_noalloc", "moe_pack_tiles")
 
 # fixed score scratch of moe_route_noalloc, in floats (include/moe_fwd.h)
 MOE_ROUTE_NOALLOC_MAX_SCORES = 1 << 20
@@ -62,7 +64,8 @@ def lib() -> ctypes.CDLL:
         L.moe_route.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_permute.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_route_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp]
-        L.fp8_block_quant.argtypes = [vp, ci, ci, ci, ci, vp, vp, vp]
+        L.fp8_block_quant.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp]
+        L.moe_pack_tiles.argtypes = [vp, ci, ci, vp, vp]
         L.moe_grouped_swiglu.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_combine.argtypes = [sp, vp, vp, vp, vp, vp]
         L.moe_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -73,7 +76,7 @@ def lib() -> ctypes.CDLL:
         L.moe_set_kernel_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ci]
         for name in ("moe_route", "moe_route_noalloc", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
                      "moe_combine", "moe_forward", "moe_check_status", "moe_last_launch_count",
-                     "moe_set_kernel_events"):
+                     "moe_set_kernel_events", "moe_pack_tiles"):
             getattr(L, name).restype = ci
         _LIB = L
     return _LIB
@@ -155,14 +158,27 @@ def moe_permute(shape, topk_idx, counts, offsets, row_token, row_of, ws, stream=
                              _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
 
 
-def fp8_block_quant(inp, block_rows, q, scales, rows=None, cols=None, ld=None, stream=None):
-    """e4m3 block quantisation of a bf16 matrix (2-D, or a stack flattened to 2-D)."""
+def fp8_block_quant(inp, block_rows, q, scales, rows=None, cols=None, ld=None,
+                    layout=MOE_LAYOUT_ROWMAJOR, stream=None):
+    """e4m3 block quantisation of a bf16 matrix (2-D, or a stack flattened to
+    2-D); layout MOE_LAYOUT_TILED writes the codes in 128 x 128 tiles."""
     cols = inp.shape[-1] if cols is None else cols
     rows = inp.numel() // inp.shape[-1] if rows is None else rows
     ld = inp.shape[-1] if ld is None else ld
-    _check(lib().fp8_block_quant(_ptr(inp, _BF16, "in"), rows, cols, ld, block_rows,
+    _check(lib().fp8_block_quant(_ptr(inp, _BF16, "in"), rows, cols, ld, block_rows, int(layout),
                                  _ptr(q, _FP8, "q"), _ptr(scales, torch.float32, "scales"),
                                  _stream(stream)))
+
+
+def moe_pack_tiles(src, dst, stream=None):
+    """Row-major -> 128 x 128-byte tiles (MOE_LAYOUT_TILED) of a matrix, or a
+    stack of matrices flattened to rows x row_bytes; same shape and dtype."""
+    if src.shape != dst.shape or src.dtype != dst.dtype:
+        raise ValueError("src and dst must have the same shape and dtype")
+    row_bytes = src.shape[-1] * src.element_size()
+    rows = src.numel() // src.shape[-1]
+    _check(lib().moe_pack_tiles(_ptr(src, name="src"), rows, row_bytes, _ptr(dst, name="dst"),
+                                _stream(stream)))
 
 
 def moe_grouped_swiglu(shape, a, a_scales, offsets, w13, w13_scales, w2, w2_scales, y, ws,

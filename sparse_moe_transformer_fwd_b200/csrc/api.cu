@@ -302,22 +302,41 @@ int moe_permute(const moe_shape *s, const int32_t *topk_idx, int32_t *counts, in
     return MOE_OK;
 }
 
-int fp8_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows, uint8_t *q,
-                    float *scales, void *stream) {
+int fp8_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
+                    int out_layout, uint8_t *q, float *scales, void *stream) {
     if (rows < 0 || cols <= 0 || cols % 128 || ld < cols || ld % 8)
         return fail(MOE_ERR_INVALID_ARG, "need rows >= 0, cols a positive multiple of 128, "
                                          "ld >= cols, ld % 8 == 0");
     if (block_rows != 1 && block_rows != 128)
         return fail(MOE_ERR_INVALID_ARG, "block_rows must be 1 or 128");
+    if (out_layout != MOE_LAYOUT_ROWMAJOR && out_layout != MOE_LAYOUT_TILED)
+        return fail(MOE_ERR_INVALID_ARG, "unknown out_layout %d", out_layout);
+    if (out_layout == MOE_LAYOUT_TILED && (block_rows != 128 || rows % 128))
+        return fail(MOE_ERR_INVALID_ARG, "tiled output needs block_rows 128 and rows % 128 == 0");
     if (rows == 0) return g_launches = 0, MOE_OK;
     CHECK_PTR(in);
     CHECK_PTR(q);
     CHECK_PTR(scales);
     RETURN_IF(check_device());
     int n = 0;
-    LAUNCH(launch_block_quant(in, rows, cols, ld, block_rows, q, scales,
-                              static_cast<cudaStream_t>(stream), &n),
+    LAUNCH(launch_block_quant(in, rows, cols, ld, block_rows, out_layout == MOE_LAYOUT_TILED, q,
+                              scales, static_cast<cudaStream_t>(stream), &n),
            "fp8_block_quant");
+    mark_launch(static_cast<cudaStream_t>(stream), n);
+    g_launches = n;
+    return MOE_OK;
+}
+
+int moe_pack_tiles(const void *src, int rows, int row_bytes, void *dst, void *stream) {
+    if (rows < 0 || row_bytes <= 0 || rows % 128 || row_bytes % 128)
+        return fail(MOE_ERR_INVALID_ARG, "rows and row_bytes must be multiples of 128");
+    if (rows == 0) return g_launches = 0, MOE_OK;
+    CHECK_PTR(src);
+    CHECK_PTR(dst);
+    RETURN_IF(check_device());
+    int n = 0;
+    LAUNCH(launch_pack_tiles(src, rows, row_bytes, dst, static_cast<cudaStream_t>(stream), &n),
+           "moe_pack_tiles");
     mark_launch(static_cast<cudaStream_t>(stream), n);
     g_launches = n;
     return MOE_OK;

@@ -10,7 +10,9 @@
 // A tiles and the same expert's weights through L2.
 //   warp 0      TMA producer: A tile 128 x 128 B and two B tiles 128 x 128 B
 //               (gate/up rows, or two halves of the output columns) per
-//               stage, 128-byte swizzle, 4 stages.
+//               stage, 128-byte swizzle, 4 stages.  The weights are stored in
+//               128 x 128-byte tiles, so each B box is one contiguous 16 KB
+//               read from HBM.
 //   warp 1      TMEM allocator (512 columns) and MMA issuer (one thread):
 //               tcgen05.mma M=128 N=256, K=32 (e4m3) or K=16 (bf16), four per
 //               stage.
@@ -189,8 +191,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
                 int seg, row0, rows_valid, nt;
                 decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
-                const int n_lo = GATE_UP ? nt * 128 : nt * 256;
-                const int n_hi = GATE_UP ? p.N_out + nt * 128 : nt * 256 + 128;
+                // 128-row blocks of B (tile rows of the tiled weight layout)
+                const int nb_lo = GATE_UP ? nt : 2 * nt;
+                const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
+                const int NBq = p.b_rows / 128;
+                const long long t_lo = (static_cast<long long>(seg) * NBq + nb_lo) * KB;
+                const long long t_hi = (static_cast<long long>(seg) * NBq + nb_hi) * KB;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, p.status)) {
                         ok = false;
@@ -200,8 +206,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     mbar_arrive_expect_tx(&s.full[stage], STAGE_TX + (inject ? 16 : 0));
                     const int kc = FP8 ? kb * 128 : kb * 64;
                     tma_load_2d(s.a[stage], &tmap_a, kc, row0, &s.full[stage]);
-                    tma_load_3d(s.b[stage], &tmap_b, kc, n_lo, seg, &s.full[stage]);
-                    tma_load_3d(s.b[stage] + B_BYTES / 2, &tmap_b, kc, n_hi, seg, &s.full[stage]);
+                    // each B box is one contiguous 16 KB weight tile
+                    tma_load_2d(s.b[stage], &tmap_b, 0, static_cast<int>((t_lo + kb) * 128),
+                                &s.full[stage]);
+                    tma_load_2d(s.b[stage] + B_BYTES / 2, &tmap_b, 0,
+                                static_cast<int>((t_hi + kb) * 128), &s.full[stage]);
                     armed |= 1 << stage;
                     armed_phase[stage] = phase;
                     if (++stage == STAGES) {
@@ -466,21 +475,6 @@ bool make_map_2d(CUtensorMap *m, const void *base, bool fp8, int K, int rows) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_map_3d(CUtensorMap *m, const void *base, bool fp8, int K, int rows, int slots) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const int es = fp8 ? 1 : 2;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows),
-                          static_cast<cuuint64_t>(slots)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * es,
-                             static_cast<cuuint64_t>(K) * es * static_cast<cuuint64_t>(rows)};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), 128, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 template <bool FP8, bool GATE_UP>
 cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams &kp, int grid,
@@ -512,7 +506,11 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     const int b_rows = g.gate_up ? 2 * g.N_out : g.N_out;
     CUtensorMap ma, mb;
     if (!make_map_2d(&ma, g.a, g.fp8, g.K, g.rows_total)) return cudaErrorInvalidValue;
-    if (!make_map_3d(&mb, g.b, g.fp8, g.K, b_rows, g.n_slots)) return cudaErrorInvalidValue;
+    // B in the tiled layout: one row of 128 bytes per tile row, tiles stacked
+    const long long b_tile_rows = static_cast<long long>(g.n_slots) * b_rows * (g.K * (g.fp8 ? 1 : 2) / 128);
+    if (b_tile_rows >= (1LL << 31)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&mb, g.b, g.fp8, g.fp8 ? 128 : 64, static_cast<int>(b_tile_rows)))
+        return cudaErrorInvalidValue;
     KParams kp;
     kp.a_scales = g.a_scales;
     kp.b_scales = g.b_scales;

@@ -38,7 +38,12 @@ cudaError_t launch_tile_table(const int32_t *offsets, int E, int T, int k, int n
 // e4m3 quantisation of bf16 [rows, cols] (leading dimension ld) in tiles of
 // block_rows x 128.
 cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
-                               uint8_t *q, float *scales, cudaStream_t st, int *launches);
+                               int tiled, uint8_t *q, float *scales, cudaStream_t st,
+                               int *launches);
+
+// Row-major [rows, row_bytes] -> 128 x 128-byte tiles (MOE_LAYOUT_TILED).
+cudaError_t launch_pack_tiles(const void *src, int rows, int row_bytes, void *dst, cudaStream_t st,
+                              int *launches);
 
 // Quantise each token row of x once (1x128 tiles) and write its codes and
 // scales to its k routed rows (row_of) and, with n_shared, to row T*k + t.
@@ -65,7 +70,7 @@ struct GemmArgs {
     bool gate_up;
     const void *a;          // [rows_total, K]
     const float *a_scales;  // [rows_total, K/128] (fp8)
-    const void *b;          // [n_slots, B rows, K]
+    const void *b;          // [n_slots, B rows, K] in 128 x 128-byte tiles
     const float *b_scales;  // [n_slots, B rows/128, K/128] (fp8)
     void *out;              // H or Y
     float *out_scales;      // H scales (fp8 gate_up)

@@ -90,9 +90,11 @@ quant_1x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld,
     }
 }
 
-// 128 x 128 blocks; one CTA (256 threads) per block, grid-stride over blocks
+// 128 x 128 blocks; one CTA (256 threads) per block, grid-stride over blocks.
+// tiled: block (rb, kb) is written as one contiguous 16 KB tile (128 rows of
+// 128 codes) at tile index rb * (cols/128) + kb.
 __global__ void __launch_bounds__(256)
-quant_128x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld,
+quant_128x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld, int tiled,
                      uint8_t *__restrict__ q, float *__restrict__ scales) {
     __shared__ float red[8];
     const int nkb = cols / 128, nrb = (rows + 127) / 128;
@@ -124,7 +126,9 @@ quant_128x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld
         for (int i = 0; i < 8; ++i) {
             const int r = rb * 128 + tr + 16 * i;
             const uint2 codes = encode8(x[i], amax, &sc);
-            if (r < rows) *reinterpret_cast<uint2 *>(q + static_cast<size_t>(r) * cols + kb * 128 + tc) = codes;
+            const size_t at = tiled ? (static_cast<size_t>(b) << 14) + (tr + 16 * i) * 128 + tc
+                                    : static_cast<size_t>(r) * cols + kb * 128 + tc;
+            if (r < rows) *reinterpret_cast<uint2 *>(q + at) = codes;
         }
         if (threadIdx.x == 0) scales[static_cast<size_t>(rb) * nkb + kb] = sc;
     }
@@ -180,10 +184,40 @@ scatter_bf16_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_s
     }
 }
 
+// Row-major rows x row_bytes -> 128 x 128-byte tiles; one 16-byte vector per
+// thread and step, grid-stride.
+__global__ void __launch_bounds__(256)
+pack_tiles_kernel(const uint8_t *__restrict__ src, int rows, int row_bytes,
+                  uint8_t *__restrict__ dst) {
+    const int tpr = row_bytes / 128;                       // tiles per row band
+    const long long total = static_cast<long long>(rows) * (row_bytes / 16);
+    for (long long v = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; v < total;
+         v += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int r = static_cast<int>(v / (row_bytes / 16));
+        const int cb = static_cast<int>(v % (row_bytes / 16)) * 16;   // byte column
+        const size_t tile = static_cast<size_t>(r / 128) * tpr + cb / 128;
+        const uint4 val = *reinterpret_cast<const uint4 *>(src + static_cast<size_t>(r) * row_bytes + cb);
+        *reinterpret_cast<uint4 *>(dst + (tile << 14) + (r % 128) * 128 + (cb % 128)) = val;
+    }
+}
+
 }  // namespace
 
+cudaError_t launch_pack_tiles(const void *src, int rows, int row_bytes, void *dst, cudaStream_t st,
+                              int *launches) {
+    const long long total = static_cast<long long>(rows) * (row_bytes / 16);
+    const long long want = (total + 255) / 256;
+    const int grid = static_cast<int>(want < num_sms() * 16LL ? want : num_sms() * 16LL);
+    mark_launch(st, *launches);
+    pack_tiles_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(src), rows, row_bytes,
+                                            static_cast<uint8_t *>(dst));
+    ++*launches;
+    return cudaGetLastError();
+}
+
 cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
-                               uint8_t *q, float *scales, cudaStream_t st, int *launches) {
+                               int tiled, uint8_t *q, float *scales, cudaStream_t st,
+                               int *launches) {
     if (rows == 0) return cudaSuccess;
     const int sms = num_sms();
     mark_launch(st, *launches);
@@ -195,7 +229,7 @@ cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, i
     } else {
         const long long nblocks = static_cast<long long>(cols / 128) * ((rows + 127) / 128);
         const int grid = static_cast<int>(nblocks < sms * 8LL ? nblocks : sms * 8LL);
-        quant_128x128_kernel<<<grid, 256, 0, st>>>(in, rows, cols, ld, q, scales);
+        quant_128x128_kernel<<<grid, 256, 0, st>>>(in, rows, cols, ld, tiled, q, scales);
     }
     ++*launches;
     return cudaGetLastError();

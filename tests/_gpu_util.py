@@ -31,6 +31,13 @@ def from_u16(a: np.ndarray, device) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
 
 
+def untile(a: np.ndarray, rows: int, row_bytes: int) -> np.ndarray:
+    """Tiled layout (128 x 128-byte tiles, include/moe_fwd.h) -> row-major
+    uint8 [rows, row_bytes]."""
+    t = np.ascontiguousarray(a).view(np.uint8).reshape(rows // 128, row_bytes // 128, 128, 128)
+    return t.transpose(0, 2, 1, 3).reshape(rows, row_bytes)
+
+
 def bf16_step(v: np.ndarray) -> np.ndarray:
     """Spacing of bf16 values at |v| (8 significant bits)."""
     a = np.maximum(np.abs(v), 2.0 ** -126)

@@ -67,9 +67,13 @@ def test_host_side_errors_return_codes():
     assert "aligned" in moe.moe_last_error()
     assert _call_forward(s, need, x=None) == N.MOE_ERR_INVALID_ARG
     L = moe.lib()
-    assert L.fp8_block_quant(FAKE, 10, 100, 100, 1, FAKE, FAKE, None) == N.MOE_ERR_INVALID_ARG
-    assert L.fp8_block_quant(FAKE, 10, 128, 128, 64, FAKE, FAKE, None) == N.MOE_ERR_INVALID_ARG
-    assert L.fp8_block_quant(FAKE, 0, 128, 128, 1, FAKE, FAKE, None) == N.MOE_OK
+    assert L.fp8_block_quant(FAKE, 10, 100, 100, 1, 0, FAKE, FAKE, None) == N.MOE_ERR_INVALID_ARG
+    assert L.fp8_block_quant(FAKE, 10, 128, 128, 64, 0, FAKE, FAKE, None) == N.MOE_ERR_INVALID_ARG
+    assert L.fp8_block_quant(FAKE, 100, 128, 128, 128, 1, FAKE, FAKE, None) == N.MOE_ERR_INVALID_ARG
+    assert L.fp8_block_quant(FAKE, 128, 128, 128, 1, 1, FAKE, FAKE, None) == N.MOE_ERR_INVALID_ARG
+    assert L.fp8_block_quant(FAKE, 0, 128, 128, 1, 0, FAKE, FAKE, None) == N.MOE_OK
+    assert L.moe_pack_tiles(FAKE, 100, 128, FAKE, None) == N.MOE_ERR_INVALID_ARG
+    assert L.moe_pack_tiles(FAKE, 128, 96, FAKE, None) == N.MOE_ERR_INVALID_ARG
 
 
 def test_empty_batch_enqueues_nothing():

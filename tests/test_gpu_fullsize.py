@@ -14,7 +14,7 @@ import oracle
 import sparse_moe_transformer_fwd_b200 as moe
 from moe_inputs import CONFIGS, make_inputs
 
-from _gpu_util import assert_out_close, oracle_layer, u16
+from _gpu_util import assert_out_close, oracle_layer, u16, untile
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0") if torch.cuda.is_available() else None
@@ -45,10 +45,10 @@ def test_weight_quant_bitexact(run):
     for e in (0, 137 % cfg.n_experts, cfg.n_experts):
         q13, s13 = oracle.block_quant(u16(inp["w13"][e]), 128)
         assert np.array_equal(layer.w13s[e].cpu().numpy().view(np.uint32), s13.view(np.uint32))
-        assert np.array_equal(layer.w13[e].cpu().numpy(), q13)
+        assert np.array_equal(untile(layer.w13[e].cpu().numpy(), *q13.shape), q13)
         q2, s2 = oracle.block_quant(u16(inp["w2"][e]), 128)
         assert np.array_equal(layer.w2s[e].cpu().numpy().view(np.uint32), s2.view(np.uint32))
-        assert np.array_equal(layer.w2[e].cpu().numpy(), q2)
+        assert np.array_equal(untile(layer.w2[e].cpu().numpy(), *q2.shape), q2)
 
 
 def test_permutation_bitexact(run):

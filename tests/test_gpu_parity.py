@@ -11,7 +11,7 @@ import oracle
 import sparse_moe_transformer_fwd_b200 as moe
 from moe_inputs import CONFIGS, make_inputs
 
-from _gpu_util import assert_out_close, from_u16, oracle_layer, u16
+from _gpu_util import assert_out_close, from_u16, oracle_layer, u16, untile
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0") if torch.cuda.is_available() else None
@@ -153,6 +153,23 @@ def test_block_quant_bitexact(rows, cols, block_rows):
     rq, rs = oracle.block_quant(u16(a), block_rows)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
     assert np.array_equal(q.cpu().numpy(), rq)
+    if block_rows == 128 and rows % 128 == 0:
+        # tiled output: the same codes and scales, 128 x 128 tiles contiguous
+        qt = torch.empty_like(q)
+        st = torch.empty_like(s)
+        moe.fp8_block_quant(a.to(DEV), block_rows, qt, st, layout=moe.MOE_LAYOUT_TILED)
+        assert torch.equal(st, s)
+        assert np.array_equal(untile(qt.cpu().numpy(), rows, cols), rq)
+
+
+@pytest.mark.parametrize("rows,row_bytes,dtype", [(128, 256, torch.bfloat16), (384, 1024, torch.uint8)])
+def test_pack_tiles_is_the_tiled_permutation(rows, row_bytes, dtype):
+    es = 2 if dtype == torch.bfloat16 else 1
+    src = torch.randint(0, 255, (rows, row_bytes), dtype=torch.uint8).view(dtype)
+    dst = torch.empty_like(src, device=DEV)
+    moe.moe_pack_tiles(src.to(DEV), dst)
+    got = untile(dst.cpu().contiguous().view(torch.uint8).numpy(), rows, row_bytes)
+    assert np.array_equal(got, src.contiguous().view(torch.uint8).numpy().reshape(rows, row_bytes))
 
 
 # ------------------------------------------- grouped experts and combine ---
@@ -178,7 +195,8 @@ def test_grouped_swiglu_and_combine(precision, T):
         moe.moe_grouped_swiglu(shape, a, a_s, offsets, w13q, w13s, w2q, w2s, y, ws)
     else:
         a = from_u16(u16(inp["x"])[rows], DEV)
-        moe.moe_grouped_swiglu(shape, a, None, offsets, w13, None, w2, None, y, ws)
+        w13t, w2t = moe.pack_weights(w13, w2)
+        moe.moe_grouped_swiglu(shape, a, None, offsets, w13t, None, w2t, None, y, ws)
     assert moe.moe_check_status(ws) == 0
     # oracle expert outputs, row by row
     seg_of_row = np.concatenate([np.repeat(np.arange(E), ref["counts"]), np.full(T, E)])
