@@ -110,7 +110,12 @@ __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int ti
     rows_valid = min(BM, s.seg_rows[seg] - mloc * BM);
 }
 
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+// silu(g) = g * sigmoid(g) with the fast exponential and reciprocal: H is
+// rounded to e4m3 or bf16 right after, so their few-ulp error is invisible,
+// and the accurate versions made the end of every tile a long latency chain
+// that stalled the tensor core (the next tile's third chunk waits for it).
+// exp(-g) overflows to +inf for g < -88 and rcp(inf) = 0, so silu -> 0.
+__device__ __forceinline__ float silu(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
 
 // acc[base..base+15] (column pairs) += partial * scale (FP8 promotion) or
 // += partial (BF16 chunk sum), with the paired binary32 FMA / add of sm_100
@@ -362,11 +367,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             auto acc = [&](int c) -> float & { return (c & 1) ? acc2[c >> 1].y : acc2[c >> 1].x; };
             if constexpr (GATE_UP) {
                 // H = silu(G) * U for features nt*128 + half*64 + c, c < 64
+                // (warps without valid rows skip the math, not the exchange)
                 float m = 0.0f;
+                if (warp_active) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    acc(c) = silu(acc(c)) * acc(64 + c);
-                    m = fmaxf(m, fabsf(acc(c)));
+                    for (int c = 0; c < 64; ++c) {
+                        acc(c) = silu(acc(c)) * acc(64 + c);
+                        m = fmaxf(m, fabsf(acc(c)));
+                    }
                 }
                 if constexpr (FP8) {
                     const int par = iter & 1;
