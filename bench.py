@@ -46,6 +46,26 @@ def load_peaks():
         return PEAKS_FALLBACK, "fallback"
 
 
+def kernel_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu record in
+    profiles/roofline_traffic.json, or None when that record was taken on
+    another workload or on a different version of the kernel sources."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "roofline_traffic.json")) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for pth in rec["sources"]:
+            with open(os.path.join(ROOT, pth), "rb") as f:
+                h.update(f.read())
+        k = rec["kernels"][kernel]
+        if h.hexdigest() != rec["source_sha256"] or k["workload"] != workload:
+            return None
+        return float(k["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def dist_setup(n_gpus):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -291,7 +311,9 @@ def run_ours(args, world, rank, local):
                            else "fallback",
             "algorithmic_bytes": g1_bytes,
             "kernel_ms": round(g1_ms, 4),
-            "traffic": None,
+            "traffic": kernel_traffic("grouped_gemm_gate_up", cfg.name),
+            "traffic_source": "profiles/roofline_traffic.json (ncu dram__bytes_read+write, "
+                              "one capture of this workload)",
         },
         "kernels_ms": {n: round(float(v), 4) for n, v in zip(names, kmean)},
         "kernels_ms_note": "per-kernel means from a separate pass of the same call with every "
