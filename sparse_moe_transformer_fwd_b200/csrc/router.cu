@@ -9,9 +9,10 @@
 //   degree-7 Taylor polynomial (W. J. Cody, W. Waite, "Software Manual for
 //   the Elementary Functions", 1980).  Every operation is a correctly rounded
 //   binary32 operation, so the results are reproducible bit for bit.
-//   Tiling: a CTA owns BT tokens x BE experts; each thread a TT x TE register
-//   tile.  x and W_r chunks of KC columns are staged in shared memory as
-//   binary32 (bf16 widening is exact).
+//   Tiling (large batches): a CTA owns 64 tokens x 64 experts, each thread an
+//   8 x 8 register tile; decode-size batches use one output per thread (see
+//   router_scores_small_kernel).  x and W_r chunks are staged in shared memory
+//   as binary32 (bf16 widening is exact).
 // Kernel 2 (router_topk): one warp per token.  sel = s + b; k rounds of a
 //   warp arg-max under (sel desc, expert asc); gates g_j = s_j / S *
 //   routed_scale with S the binary32 sum of the selected s in rank order.
@@ -60,70 +61,62 @@ __device__ __forceinline__ float sigmoid_cw(float l, const ExpConsts &k) {
 }
 
 // ------------------------------------------------------- router_scores ---
-template <int BT, int BE, int TT, int TE, int KC>
-__global__ void __launch_bounds__((BT / TT) * (BE / TE))
+// Larger batches: a CTA of 64 threads owns 64 tokens x 64 experts; thread
+// (ty, tx) owns tokens {4ty..4ty+3, 32+4ty..32+4ty+3} x experts {4tx..4tx+3,
+// 32+4tx..32+4tx+3}, 64 accumulators, each still a sequential FMA chain over
+// d.  Per k step: four 16-byte shared loads (x by broadcast, W_r conflict-
+// free) feed 64 FMAs.  x and W_r chunks of 32 columns are staged transposed
+// ([k][row], binary32) through registers one chunk ahead.
+constexpr int RT_B = 64, RT_KC = 32, RT_THREADS = 64;
+
+__global__ void __launch_bounds__(RT_THREADS)
 router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w, int T, int d,
                      int E, float *__restrict__ scores) {
-    constexpr int NTX = BE / TE;                  // threads along experts
-    constexpr int NTHREADS = (BT / TT) * NTX;
-    __shared__ __align__(16) float xs[2][KC][BT];  // [k][token]
-    __shared__ __align__(16) float ws[2][KC][BE];  // [k][expert]
+    __shared__ __align__(16) float xs[2][RT_KC][RT_B];  // [k][token]
+    __shared__ __align__(16) float ws[2][RT_KC][RT_B];  // [k][expert]
+    const int tid = threadIdx.x, tx = tid & 7, ty = tid >> 3;
+    const int t0 = blockIdx.y * RT_B, e0 = blockIdx.x * RT_B;
 
-    const int tid = threadIdx.x;
-    const int t0 = blockIdx.y * BT, e0 = blockIdx.x * BE;
-    const int tx = tid % NTX, ty = tid / NTX;
-
-    float acc[TT][TE];
+    float acc[8][8];
 #pragma unroll
-    for (int a = 0; a < TT; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < TE; ++b) acc[a][b] = 0.0f;
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
 
-    // staging of chunk kc (KC columns of x and W_r) through registers: the
-    // global loads of chunk kc+1 are issued before chunk kc is computed and
-    // land in shared memory after it, so L2 latency hides behind the FMAs.
-    constexpr int XV = BT * KC / 8, WV = BE * KC / 8;   // 16-byte vectors
-    constexpr int NV = (XV + WV + NTHREADS - 1) / NTHREADS;
-    uint4 pre[NV];
+    constexpr int VPR = RT_KC / 8;                 // 16-byte vectors per row per chunk
+    constexpr int NV = 2 * RT_B * VPR;             // x rows then W_r rows
+    constexpr int PER = NV / RT_THREADS;
+    uint4 pre[PER];
     auto load = [&](int kc) {
-        const int k0 = kc * KC;
 #pragma unroll
-        for (int j = 0; j < NV; ++j) {
-            const int v = tid + j * NTHREADS;
+        for (int j = 0; j < PER; ++j) {
+            const int v = tid + j * RT_THREADS;
+            const int row = v / VPR, col = (v % VPR) * 8;
+            const bool isx = row < RT_B;
+            const int g = isx ? t0 + row : e0 + row - RT_B;
             pre[j] = make_uint4(0, 0, 0, 0);
-            if (v < XV + WV) {
-                const bool isx = v < XV;
-                const int vv = isx ? v : v - XV;
-                const int row = vv / (KC / 8), col = (vv % (KC / 8)) * 8;
-                const int g = isx ? t0 + row : e0 + row;
-                if (g < (isx ? T : E))
-                    pre[j] = *reinterpret_cast<const uint4 *>((isx ? x : w) + static_cast<size_t>(g) * d + k0 + col);
-            }
+            if (g < (isx ? T : E))
+                pre[j] = *reinterpret_cast<const uint4 *>((isx ? x : w) + static_cast<size_t>(g) * d +
+                                                          kc * RT_KC + col);
         }
     };
     auto store = [&](int buf) {
 #pragma unroll
-        for (int j = 0; j < NV; ++j) {
-            const int v = tid + j * NTHREADS;
-            if (v >= XV + WV) continue;
-            const bool isx = v < XV;
-            const int vv = isx ? v : v - XV;
-            const int row = vv / (KC / 8), col = (vv % (KC / 8)) * 8;
+        for (int j = 0; j < PER; ++j) {
+            const int v = tid + j * RT_THREADS;
+            const int row = v / VPR, col = (v % VPR) * 8;
+            float(*dst)[RT_B] = row < RT_B ? xs[buf] : ws[buf];
+            const int r = row < RT_B ? row : row - RT_B;
             const uint32_t r4[4] = {pre[j].x, pre[j].y, pre[j].z, pre[j].w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                if (isx) {
-                    xs[buf][col + 2 * q][row] = bf16_lo(r4[q]);
-                    xs[buf][col + 2 * q + 1][row] = bf16_hi(r4[q]);
-                } else {
-                    ws[buf][col + 2 * q][row] = bf16_lo(r4[q]);
-                    ws[buf][col + 2 * q + 1][row] = bf16_hi(r4[q]);
-                }
+                dst[col + 2 * q][r] = bf16_lo(r4[q]);
+                dst[col + 2 * q + 1][r] = bf16_hi(r4[q]);
             }
         }
     };
 
-    const int nk = d / KC;
+    const int nk = d / RT_KC;
     load(0);
     store(0);
     __syncthreads();
@@ -131,16 +124,17 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
         const int buf = kc & 1;
         if (kc + 1 < nk) load(kc + 1);
 #pragma unroll 4
-        for (int kk = 0; kk < KC; ++kk) {
-            float xv[TT], wv[TE];
+        for (int kk = 0; kk < RT_KC; ++kk) {
+            const float4 xa = *reinterpret_cast<const float4 *>(&xs[buf][kk][4 * ty]);
+            const float4 xb = *reinterpret_cast<const float4 *>(&xs[buf][kk][32 + 4 * ty]);
+            const float4 wa = *reinterpret_cast<const float4 *>(&ws[buf][kk][4 * tx]);
+            const float4 wb = *reinterpret_cast<const float4 *>(&ws[buf][kk][32 + 4 * tx]);
+            const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+            const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-            for (int a = 0; a < TT; ++a) xv[a] = xs[buf][kk][ty * TT + a];
+            for (int a = 0; a < 8; ++a)
 #pragma unroll
-            for (int b = 0; b < TE; ++b) wv[b] = ws[buf][kk][tx + b * NTX];
-#pragma unroll
-            for (int a = 0; a < TT; ++a)
-#pragma unroll
-                for (int b = 0; b < TE; ++b) acc[a][b] = __fmaf_rn(xv[a], wv[b], acc[a][b]);
+                for (int b = 0; b < 8; ++b) acc[a][b] = __fmaf_rn(xv[a], wv[b], acc[a][b]);
         }
         if (kc + 1 < nk) store(buf ^ 1);
         __syncthreads();
@@ -148,12 +142,12 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
 
     const ExpConsts k = exp_consts();
 #pragma unroll
-    for (int a = 0; a < TT; ++a) {
-        const int t = t0 + ty * TT + a;
+    for (int a = 0; a < 8; ++a) {
+        const int t = t0 + (a < 4 ? 4 * ty + a : 32 + 4 * ty + a - 4);
         if (t >= T) continue;
 #pragma unroll
-        for (int b = 0; b < TE; ++b) {
-            const int e = e0 + tx + b * NTX;
+        for (int b = 0; b < 8; ++b) {
+            const int e = e0 + (b < 4 ? 4 * tx + b : 32 + 4 * tx + b - 4);
             if (e < E) scores[static_cast<size_t>(t) * E + e] = sigmoid_cw(acc[a][b], k);
         }
     }
@@ -316,10 +310,8 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
                           float *gates, cudaStream_t st, int *launches) {
     mark_launch(st, *launches);
     if (T >= 512) {
-        constexpr int BT = 64, BE = 128, TT = 4, TE = 8, KC = 32;
-        dim3 grid((E + BE - 1) / BE, (T + BT - 1) / BT);
-        router_scores_kernel<BT, BE, TT, TE, KC>
-            <<<grid, (BT / TT) * (BE / TE), 0, st>>>(x, w, T, d, E, scores);
+        dim3 grid((E + RT_B - 1) / RT_B, (T + RT_B - 1) / RT_B);
+        router_scores_kernel<<<grid, RT_THREADS, 0, st>>>(x, w, T, d, E, scores);
     } else {
         constexpr int BT = 4, KC = 128;
         dim3 grid((E + 31) / 32, (T + BT - 1) / BT);
