@@ -16,6 +16,7 @@ combine_kernel(const uint16_t *__restrict__ y, const int32_t *__restrict__ row_o
     __shared__ int rows_sh[32];
     __shared__ float g_sh[32];
     const int t = blockIdx.x;
+    pdl_wait_and_trigger();
     if (threadIdx.x < k) {
         rows_sh[threadIdx.x] = row_of[static_cast<size_t>(t) * k + threadIdx.x];
         g_sh[threadIdx.x] = gates[static_cast<size_t>(t) * k + threadIdx.x];
@@ -61,7 +62,8 @@ cudaError_t launch_combine(const uint16_t *y, const int32_t *row_of, const float
                            int d, int k, int n_shared, uint16_t *out, cudaStream_t st,
                            int *launches) {
     mark_launch(st, *launches);
-    combine_kernel<<<T, 128, 0, st>>>(y, row_of, gates, T, d, k, n_shared, out);
+    LAUNCH_OR_RETURN(launch_pdl(combine_kernel, dim3(T), dim3(128), 0, st, y, row_of, gates, T, d, k, n_shared,
+                                out));
     ++*launches;
     return cudaGetLastError();
 }

@@ -147,13 +147,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const int n_seg = p.n_segments;
 
     // ---------------------------------------------------------------- setup
-    for (int i = threadIdx.x; i < n_seg; i += NUM_THREADS) {
-        s.seg_start[i] = p.seg_start[i];
-        s.seg_rows[i] = p.seg_rows[i];
-        s.tile_start[i] = p.tile_start[i];
-    }
     if (threadIdx.x == 0) {
-        s.tile_start[n_seg] = p.tile_start[n_seg];
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], 1);
@@ -175,6 +169,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         tmem_alloc(&s.tmem_base, TMEM_COLS);
         tmem_relinquish();
     }
+    // everything above overlaps the previous kernel; its outputs are read below
+    pdl_wait_and_trigger();
+    for (int i = threadIdx.x; i < n_seg; i += NUM_THREADS) {
+        s.seg_start[i] = p.seg_start[i];
+        s.seg_rows[i] = p.seg_rows[i];
+        s.tile_start[i] = p.tile_start[i];
+    }
+    if (threadIdx.x == 0) s.tile_start[n_seg] = p.tile_start[n_seg];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -503,8 +505,8 @@ cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    grouped_gemm_kernel<FP8, GATE_UP><<<grid, NUM_THREADS, smem, st>>>(ma, mb, kp);
-    return cudaGetLastError();
+    return launch_pdl(grouped_gemm_kernel<FP8, GATE_UP>, dim3(grid), dim3(NUM_THREADS), smem, st, ma, mb,
+                      kp);
 }
 
 }  // namespace

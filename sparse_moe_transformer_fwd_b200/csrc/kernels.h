@@ -10,7 +10,35 @@
 
 #include "../../include/moe_fwd.h"
 
+#include <utility>
+
 namespace moe {
+
+// Launch with programmatic dependent launch allowed: the kernel may start
+// while its predecessor on the stream finishes; every kernel of this library
+// calls pdl_wait() (griddepcontrol.wait) before it reads anything an earlier
+// launch wrote, so only its prologue overlaps the predecessor's tail.
+#define LAUNCH_OR_RETURN(call)                 \
+    do {                                       \
+        const cudaError_t e_l_ = (call);       \
+        if (e_l_ != cudaSuccess) return e_l_;  \
+    } while (0)
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 constexpr int kTileM = 128;  // rows per grouped-GEMM tile (tcgen05 M)
 

@@ -28,6 +28,7 @@ perm_hist_kernel(const int32_t *__restrict__ idx, int T, int k, int E, uint32_t 
                  int32_t *__restrict__ hist, int *status) {
     extern __shared__ uint32_t mask[];  // [E][kWords]
     const int blk = blockIdx.x;
+    pdl_wait_and_trigger();
     for (int i = threadIdx.x; i < E * kWords; i += blockDim.x) mask[i] = 0;
     __syncthreads();
     const int t0 = blk * kBT;
@@ -115,6 +116,7 @@ perm_scan_kernel(const int32_t *__restrict__ hist, int nblk, int E, int T, int k
                  int32_t *tile_start) {
     __shared__ int tmp[32];
     const int e = threadIdx.x;
+    pdl_wait_and_trigger();
     int run = 0;
     if (e < E) {
         for (int b = 0; b < nblk; ++b) {
@@ -137,6 +139,7 @@ perm_scatter_kernel(const int32_t *__restrict__ idx, int T, int k, int E,
                     int32_t *__restrict__ row_of) {
     extern __shared__ uint32_t mask[];  // [E][kWords]
     const int blk = blockIdx.x;
+    pdl_wait_and_trigger();
     const uint32_t *gm = masks + static_cast<size_t>(blk) * E * kWords;
     for (int i = threadIdx.x; i < E * kWords; i += blockDim.x) mask[i] = gm[i];
     __syncthreads();
@@ -164,6 +167,7 @@ tile_table_kernel(const int32_t *__restrict__ offsets, int E, int T, int k, int 
                   int32_t *seg_start, int32_t *seg_rows, int32_t *tile_start, int *status) {
     __shared__ int tmp[32];
     const int e = threadIdx.x;
+    pdl_wait_and_trigger();
     int count = 0, start = 0;
     if (e < E) {
         start = offsets[e];
@@ -185,15 +189,16 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int n_shared
     const int nblk = (T + kBT - 1) / kBT;
     const size_t smem = static_cast<size_t>(E) * kWords * sizeof(uint32_t);
     mark_launch(st, *launches);
-    perm_hist_kernel<<<nblk, 256, smem, st>>>(idx, T, k, E, s.masks, s.hist, status);
+    LAUNCH_OR_RETURN(launch_pdl(perm_hist_kernel, dim3(nblk), dim3(256), smem, st, idx, T, k, E, s.masks,
+                                s.hist, status));
     ++*launches;
     mark_launch(st, *launches);
-    perm_scan_kernel<<<1, 1024, 0, st>>>(s.hist, nblk, E, T, k, n_shared, s.blkoff, counts,
-                                         offsets, s.seg_start, s.seg_rows, s.tile_start);
+    LAUNCH_OR_RETURN(launch_pdl(perm_scan_kernel, dim3(1), dim3(1024), 0, st, s.hist, nblk, E, T, k, n_shared,
+                                s.blkoff, counts, offsets, s.seg_start, s.seg_rows, s.tile_start));
     ++*launches;
     mark_launch(st, *launches);
-    perm_scatter_kernel<<<nblk, 256, smem, st>>>(idx, T, k, E, s.masks, s.blkoff, offsets,
-                                                  row_token, row_of);
+    LAUNCH_OR_RETURN(launch_pdl(perm_scatter_kernel, dim3(nblk), dim3(256), smem, st, idx, T, k, E, s.masks,
+                                s.blkoff, offsets, row_token, row_of));
     ++*launches;
     return cudaGetLastError();
 }
@@ -201,8 +206,8 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int n_shared
 cudaError_t launch_tile_table(const int32_t *offsets, int E, int T, int k, int n_shared,
                               PermScratch s, int *status, cudaStream_t st, int *launches) {
     mark_launch(st, *launches);
-    tile_table_kernel<<<1, 1024, 0, st>>>(offsets, E, T, k, n_shared, s.seg_start, s.seg_rows,
-                                          s.tile_start, status);
+    LAUNCH_OR_RETURN(launch_pdl(tile_table_kernel, dim3(1), dim3(1024), 0, st, offsets, E, T, k, n_shared,
+                                s.seg_start, s.seg_rows, s.tile_start, status));
     ++*launches;
     return cudaGetLastError();
 }

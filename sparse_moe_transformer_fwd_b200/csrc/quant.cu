@@ -66,6 +66,7 @@ __device__ __forceinline__ float group16_max(float m) {
 __global__ void __launch_bounds__(256)
 quant_1x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld,
                    uint8_t *__restrict__ q, float *__restrict__ scales) {
+    pdl_wait_and_trigger();
     const int vpr = cols / 8;  // 16-byte vectors per row
     const long long total = static_cast<long long>(rows) * vpr;
     const long long nthreads = static_cast<long long>(gridDim.x) * blockDim.x;
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(256)
 quant_128x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld, int tiled,
                      uint8_t *__restrict__ q, float *__restrict__ scales) {
     __shared__ float red[8];
+    pdl_wait_and_trigger();
     const int nkb = cols / 128, nrb = (rows + 127) / 128;
     const long long nblocks = static_cast<long long>(nkb) * nrb;
     const int tr = threadIdx.x / 16, tc = (threadIdx.x % 16) * 8;
@@ -142,6 +144,7 @@ quant_scatter_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_
     __shared__ int rows_sh[33];
     const int t = blockIdx.x;
     const int ndst = k + n_shared;
+    pdl_wait_and_trigger();
     if (threadIdx.x < k) rows_sh[threadIdx.x] = row_of[static_cast<size_t>(t) * k + threadIdx.x];
     if (threadIdx.x == 0 && n_shared) rows_sh[k] = T * k + t;
     __syncthreads();
@@ -173,6 +176,7 @@ scatter_bf16_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_s
     __shared__ int rows_sh[33];
     const int t = blockIdx.x;
     const int ndst = k + n_shared;
+    pdl_wait_and_trigger();
     if (threadIdx.x < k) rows_sh[threadIdx.x] = row_of[static_cast<size_t>(t) * k + threadIdx.x];
     if (threadIdx.x == 0 && n_shared) rows_sh[k] = T * k + t;
     __syncthreads();
@@ -189,6 +193,7 @@ scatter_bf16_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_s
 __global__ void __launch_bounds__(256)
 pack_tiles_kernel(const uint8_t *__restrict__ src, int rows, int row_bytes,
                   uint8_t *__restrict__ dst) {
+    pdl_wait_and_trigger();
     const int tpr = row_bytes / 128;                       // tiles per row band
     const long long total = static_cast<long long>(rows) * (row_bytes / 16);
     for (long long v = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; v < total;
@@ -209,8 +214,9 @@ cudaError_t launch_pack_tiles(const void *src, int rows, int row_bytes, void *ds
     const long long want = (total + 255) / 256;
     const int grid = static_cast<int>(want < num_sms() * 16LL ? want : num_sms() * 16LL);
     mark_launch(st, *launches);
-    pack_tiles_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(src), rows, row_bytes,
-                                            static_cast<uint8_t *>(dst));
+    LAUNCH_OR_RETURN(launch_pdl(pack_tiles_kernel, dim3(grid), dim3(256), 0, st,
+                                static_cast<const uint8_t *>(src), rows, row_bytes,
+                                static_cast<uint8_t *>(dst)));
     ++*launches;
     return cudaGetLastError();
 }
@@ -225,11 +231,13 @@ cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, i
         const long long total = static_cast<long long>(rows) * (cols / 8);
         const long long want = (total + 255) / 256;
         const int grid = static_cast<int>(want < sms * 16LL ? want : sms * 16LL);
-        quant_1x128_kernel<<<grid, 256, 0, st>>>(in, rows, cols, ld, q, scales);
+        LAUNCH_OR_RETURN(launch_pdl(quant_1x128_kernel, dim3(grid), dim3(256), 0, st, in, rows, cols, ld, q,
+                                    scales));
     } else {
         const long long nblocks = static_cast<long long>(cols / 128) * ((rows + 127) / 128);
         const int grid = static_cast<int>(nblocks < sms * 8LL ? nblocks : sms * 8LL);
-        quant_128x128_kernel<<<grid, 256, 0, st>>>(in, rows, cols, ld, tiled, q, scales);
+        LAUNCH_OR_RETURN(launch_pdl(quant_128x128_kernel, dim3(grid), dim3(256), 0, st, in, rows, cols, ld,
+                                    tiled, q, scales));
     }
     ++*launches;
     return cudaGetLastError();
@@ -239,7 +247,8 @@ cudaError_t launch_quant_scatter(const uint16_t *x, int T, int d, int k, int n_s
                                  const int32_t *row_of, uint8_t *a, float *a_scales,
                                  cudaStream_t st, int *launches) {
     mark_launch(st, *launches);
-    quant_scatter_kernel<<<T, 256, 0, st>>>(x, T, d, k, n_shared, row_of, a, a_scales);
+    LAUNCH_OR_RETURN(launch_pdl(quant_scatter_kernel, dim3(T), dim3(256), 0, st, x, T, d, k, n_shared, row_of,
+                                a, a_scales));
     ++*launches;
     return cudaGetLastError();
 }
@@ -248,7 +257,8 @@ cudaError_t launch_scatter_bf16(const uint16_t *x, int T, int d, int k, int n_sh
                                 const int32_t *row_of, uint16_t *a, cudaStream_t st,
                                 int *launches) {
     mark_launch(st, *launches);
-    scatter_bf16_kernel<<<T, 256, 0, st>>>(x, T, d, k, n_shared, row_of, a);
+    LAUNCH_OR_RETURN(launch_pdl(scatter_bf16_kernel, dim3(T), dim3(256), 0, st, x, T, d, k, n_shared, row_of,
+                                a));
     ++*launches;
     return cudaGetLastError();
 }

@@ -76,12 +76,16 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
     __shared__ __align__(16) float ws[2][RT_KC][RT_B];  // [k][expert]
     const int tid = threadIdx.x, tx = tid & 7, ty = tid >> 3;
     const int t0 = blockIdx.y * RT_B, e0 = blockIdx.x * RT_B;
+    pdl_wait_and_trigger();
 
-    float acc[8][8];
+    // acc[a][j] holds experts (2j, 2j+1) of the thread's 8: the paired FMA of
+    // sm_100 does two independent correctly rounded FMAs per instruction, so
+    // every output is still its own sequential binary32 FMA chain
+    float2 acc[8][4];
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+        for (int b = 0; b < 4; ++b) acc[a][b] = make_float2(0.0f, 0.0f);
 
     constexpr int VPR = RT_KC / 8;                 // 16-byte vectors per row per chunk
     constexpr int NV = 2 * RT_B * VPR;             // x rows then W_r rows
@@ -130,11 +134,14 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
             const float4 wa = *reinterpret_cast<const float4 *>(&ws[buf][kk][4 * tx]);
             const float4 wb = *reinterpret_cast<const float4 *>(&ws[buf][kk][32 + 4 * tx]);
             const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-            const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+            const float2 wv[4] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w),
+                                  make_float2(wb.x, wb.y), make_float2(wb.z, wb.w)};
 #pragma unroll
-            for (int a = 0; a < 8; ++a)
+            for (int a = 0; a < 8; ++a) {
+                const float2 x2 = make_float2(xv[a], xv[a]);
 #pragma unroll
-                for (int b = 0; b < 8; ++b) acc[a][b] = __fmaf_rn(xv[a], wv[b], acc[a][b]);
+                for (int b = 0; b < 4; ++b) acc[a][b] = __ffma2_rn(x2, wv[b], acc[a][b]);
+            }
         }
         if (kc + 1 < nk) store(buf ^ 1);
         __syncthreads();
@@ -148,7 +155,8 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
 #pragma unroll
         for (int b = 0; b < 8; ++b) {
             const int e = e0 + (b < 4 ? 4 * tx + b : 32 + 4 * tx + b - 4);
-            if (e < E) scores[static_cast<size_t>(t) * E + e] = sigmoid_cw(acc[a][b], k);
+            const float l = (b & 1) ? acc[a][b >> 1].y : acc[a][b >> 1].x;
+            if (e < E) scores[static_cast<size_t>(t) * E + e] = sigmoid_cw(l, k);
         }
     }
 }
@@ -173,6 +181,7 @@ router_scores_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__res
     __shared__ __align__(16) float ws[2][BE][LD];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t0 = blockIdx.y * BT, e0 = blockIdx.x * BE;
+    pdl_wait_and_trigger();
 
     uint4 pre[PER];
     auto load = [&](int kc) {
@@ -239,6 +248,7 @@ __global__ void __launch_bounds__(256)
 router_topk_kernel(const float *__restrict__ scores, const float *__restrict__ bias, int T, int E,
                    int k, float routed_scale, int32_t *__restrict__ idx_out,
                    float *__restrict__ gates_out) {
+    pdl_wait_and_trigger();
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
@@ -311,25 +321,26 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
     mark_launch(st, *launches);
     if (T >= 512) {
         dim3 grid((E + RT_B - 1) / RT_B, (T + RT_B - 1) / RT_B);
-        router_scores_kernel<<<grid, RT_THREADS, 0, st>>>(x, w, T, d, E, scores);
+        LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel, grid, dim3(RT_THREADS), 0, st, x, w, T, d, E, scores));
     } else {
         constexpr int BT = 4, KC = 128;
         dim3 grid((E + 31) / 32, (T + BT - 1) / BT);
-        router_scores_small_kernel<BT, KC><<<grid, BT * 32, 0, st>>>(x, w, T, d, E, scores);
+        LAUNCH_OR_RETURN(launch_pdl(router_scores_small_kernel<BT, KC>, grid, dim3(BT * 32), 0, st, x, w, T, d,
+                                    E, scores));
     }
     ++*launches;
     const int per_lane = (E + 31) / 32;
     dim3 grid2((T + 7) / 8);
     mark_launch(st, *launches);
     if (per_lane <= 1)
-        router_topk_kernel<1><<<grid2, 256, 0, st>>>(scores, bias, T, E, k, routed_scale, idx, gates);
+        LAUNCH_OR_RETURN(launch_pdl(router_topk_kernel<1>, grid2, dim3(256), 0, st, scores, bias, T, E, k, routed_scale, idx, gates));
     else if (per_lane <= 4)
-        router_topk_kernel<4><<<grid2, 256, 0, st>>>(scores, bias, T, E, k, routed_scale, idx, gates);
+        LAUNCH_OR_RETURN(launch_pdl(router_topk_kernel<4>, grid2, dim3(256), 0, st, scores, bias, T, E, k, routed_scale, idx, gates));
     else if (per_lane <= 8)
-        router_topk_kernel<8><<<grid2, 256, 0, st>>>(scores, bias, T, E, k, routed_scale, idx, gates);
+        LAUNCH_OR_RETURN(launch_pdl(router_topk_kernel<8>, grid2, dim3(256), 0, st, scores, bias, T, E, k, routed_scale, idx, gates));
     else
-        router_topk_kernel<kMaxPerLane>
-            <<<grid2, 256, 0, st>>>(scores, bias, T, E, k, routed_scale, idx, gates);
+        LAUNCH_OR_RETURN(launch_pdl(router_topk_kernel<kMaxPerLane>, grid2, dim3(256), 0, st, scores, bias, T,
+                                    E, k, routed_scale, idx, gates));
     ++*launches;
     return cudaGetLastError();
 }
