@@ -30,7 +30,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from moe_inputs import CONFIGS, make_inputs  # noqa: E402
+from moe_inputs import CONFIGS, make_inputs, make_residual  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at DeepSeek-V3 dims"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -175,11 +175,11 @@ class ClockSampler:
 
 # --------------------------------------------------------------- our arm ---
 
-def kernel_names(cfg):
+def kernel_names(cfg, prenorm=False):
     names = ["router_scores", "router_topk", "perm_hist", "perm_scan", "perm_scatter",
              "quant_scatter" if cfg.precision == "fp8" else "scatter_bf16",
              "grouped_gemm_gate_up", "grouped_gemm_down", "combine"]
-    return names
+    return (["prenorm_rstd"] if prenorm else []) + names
 
 
 def algorithmic_bytes_gemm1(cfg, touched: int) -> float:
@@ -204,14 +204,21 @@ def run_ours(args, world, rank, local):
                          n_shared=cfg.n_shared, precision=cfg.precision)
     del inp["w13"], inp["w2"]
     torch.cuda.empty_cache()
-    x = inp["x"]
     T = cfg.T
+    if args.prenorm:
+        # the FFN block: residual stream h in, pre-norm fused, h + MoE(x) out
+        x, gamma = make_residual(cfg, seed=args.seed + rank, device=dev)
+        call = lambda xx, out, topk_idx_out=None: layer.forward_prenorm(
+            xx, gamma, 1e-6, out=out, topk_idx_out=topk_idx_out)
+    else:
+        x = inp["x"]
+        call = layer
     out = torch.empty(T, cfg.d_model, dtype=torch.bfloat16, device=dev)
     idx = torch.empty(T, cfg.top_k, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
     for _ in range(args.warmup):
-        layer(x, out=out, topk_idx_out=idx)
+        call(x, out=out, topk_idx_out=idx)
     torch.cuda.synchronize()
     status = layer.check_status(T)
     if status != 0:
@@ -222,7 +229,7 @@ def run_ours(args, world, rank, local):
 
     # ---- device-timed region: K steps, inputs resident in HBM; the dominant
     # kernel (gate/up GEMM) is bracketed by CUDA events inside the region
-    names = kernel_names(cfg)
+    names = kernel_names(cfg, args.prenorm)
     gi = names.index("grouped_gemm_gate_up")
     g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(args.steps)]
@@ -236,7 +243,7 @@ def run_ours(args, world, rank, local):
         start.record(stream)
         for k in range(args.steps):
             moe.moe_set_kernel_events([None] * gi + [g_ev[k][0], g_ev[k][1]])
-            layer(x, out=out, topk_idx_out=idx)
+            call(x, out=out, topk_idx_out=idx)
         moe.moe_set_kernel_events(None)
         stop.record(stream)
         torch.cuda.synchronize()
@@ -250,7 +257,7 @@ def run_ours(args, world, rank, local):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)] for _ in range(nb)]
     for k in range(nb):
         moe.moe_set_kernel_events(ev[k])
-        layer(x, out=out, topk_idx_out=idx)
+        call(x, out=out, topk_idx_out=idx)
     moe.moe_set_kernel_events(None)
     torch.cuda.synchronize()
     kmean = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(n_launch)]
@@ -262,7 +269,7 @@ def run_ours(args, world, rank, local):
     x_dev = torch.empty_like(x)
     for _ in range(2):
         x_dev.copy_(x_host, non_blocking=True)
-        layer(x_dev, out=out)
+        call(x_dev, out=out)
         out_host.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
     barrier(world)
@@ -270,7 +277,7 @@ def run_ours(args, world, rank, local):
     e0.record(stream)
     for _ in range(args.steps):
         x_dev.copy_(x_host, non_blocking=True)
-        layer(x_dev, out=out)
+        call(x_dev, out=out)
         out_host.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -301,7 +308,8 @@ def run_ours(args, world, rank, local):
         "dtype": "e4m3" if cfg.precision == "fp8" else "bf16",
         "data": "synthetic (seeded; random-init weights of the DeepSeek-V3 MoE layer shape)",
         "config": {
-            "workload": f"{cfg.name}: T={T}, d_model={cfg.d_model}, {cfg.n_experts} experts "
+            "workload": ("pre-norm block (h + MoE(RMSNorm(h)), fused) " if args.prenorm else "")
+                        + f"{cfg.name}: T={T}, d_model={cfg.d_model}, {cfg.n_experts} experts "
                         f"top-{cfg.top_k} + {cfg.n_shared} shared, d_expert={cfg.d_expert}, "
                         + ("e4m3 1x128/128x128 blockwise, bf16 I/O" if cfg.precision == "fp8"
                            else "bf16"),
@@ -422,6 +430,8 @@ def main():
                     help="tokens of the batch per oracle step (reference arm)")
     ap.add_argument("--cpu-baseline-tokens", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prenorm", action="store_true",
+                    help="time the FFN block with its fused pre-norm and residual")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

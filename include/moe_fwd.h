@@ -205,6 +205,22 @@ int moe_forward(const moe_shape *shape, const uint16_t *x, const uint16_t *w_rou
                 const void *w2, const float *w2_scales, uint16_t *out,
                 int32_t *topk_idx_out, void *ws, size_t ws_bytes, void *stream);
 
+/* The FFN block around the layer ("DeepSeek-R1" card, "Facts": pre-norm,
+ * RMSNorm before the MLP): out = h + MoE(x) with x = bf16((h * rstd) *
+ * gamma), rstd = 1 / sqrt(sum_i h_i^2 / d_model + eps).  x is never written:
+ * the router and the quantise/scatter step normalise h as they read it, and
+ * the combine adds h before its final rounding.  sum_i h_i^2 is binary32 in
+ * a fixed order (32 lane sums over i mod 32, fused multiply-add in ascending
+ * i, then xor-butterfly pairwise adds), so routing stays reproducible.
+ *   h     bf16 [T, d_model] (the residual stream)
+ *   gamma bf16 [d_model]; eps >= 0 (DeepSeek-V3 uses 1e-6)
+ *   other arguments as for moe_forward. */
+int moe_forward_prenorm(const moe_shape *shape, const uint16_t *h, const uint16_t *gamma,
+                        float eps, const uint16_t *w_router, const float *bias, const void *w13,
+                        const float *w13_scales, const void *w2, const float *w2_scales,
+                        uint16_t *out, int32_t *topk_idx_out, void *ws, size_t ws_bytes,
+                        void *stream);
+
 /* Synchronises `stream`, returns the workspace status word (MOE_OK or the
  * first device-recorded MOE_ERR_*), and resets it to MOE_OK.  A workspace must
  * be zero-filled once before first use (or passed here once) so its status

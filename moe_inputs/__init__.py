@@ -27,12 +27,13 @@ import os
 
 import torch
 
-__all__ = ["MoEConfig", "CONFIGS", "make_inputs", "expert_weights", "skew_bias_scale"]
+__all__ = ["MoEConfig", "CONFIGS", "make_inputs", "expert_weights", "skew_bias_scale",
+           "make_residual"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
 # tensor ids for seeding
-_TID_X, _TID_WR, _TID_BIAS, _TID_W13, _TID_W2, _TID_RANK = 1, 2, 3, 4, 5, 6
+_TID_X, _TID_WR, _TID_BIAS, _TID_W13, _TID_W2, _TID_RANK, _TID_H, _TID_G = 1, 2, 3, 4, 5, 6, 7, 8
 
 
 @dataclasses.dataclass(frozen=True)
@@ -127,6 +128,18 @@ def make_x(cfg: MoEConfig, seed: int = 0, device="cpu", T: int | None = None) ->
                     dtype=torch.float32)
     x = x / torch.sqrt((x * x).mean(dim=1, keepdim=True) + 1e-6)
     return x.to(torch.bfloat16)
+
+
+def make_residual(cfg: MoEConfig, seed: int = 0, device="cpu", T: int | None = None):
+    """Inputs of the pre-norm block: the residual stream h ~ N(0, 1) * s_t with
+    a per-token scale s_t ~ exp(U(-1, 2)) (rows of very different norms), and
+    the RMSNorm weight gamma ~ U(0.5, 1.5); both bf16."""
+    T = cfg.T if T is None else T
+    g = _gen(device, seed, _TID_H)
+    h = torch.randn(T, cfg.d_model, generator=g, device=device, dtype=torch.float32)
+    h = h * torch.exp(torch.rand(T, 1, generator=g, device=device) * 3.0 - 1.0)
+    gamma = torch.rand(cfg.d_model, generator=_gen(device, seed, _TID_G), device=device) + 0.5
+    return h.to(torch.bfloat16), gamma.to(torch.bfloat16)
 
 
 def make_router(cfg: MoEConfig, seed: int = 0, device="cpu"):

@@ -47,7 +47,7 @@ from . import build as _build
 __all__ = [
     "lib", "bf16_to_f32", "bf16_from_f32", "e4m3_decode_table", "e4m3_encode", "sigmoid",
     "router_logits", "route", "permute", "block_quant", "dequant", "expert_forward",
-    "moe_layer", "exp_cw",
+    "moe_layer", "exp_cw", "rmsnorm", "moe_layer_prenorm",
 ]
 
 _LIB = None
@@ -84,6 +84,10 @@ def lib():
         L.oracle_bf16_from_f32_array.argtypes = [f32p, ctypes.c_size_t, u16p]
         L.oracle_e4m3_encode_array.argtypes = [f32p, ctypes.c_size_t, u8p]
         L.oracle_sigmoid_array.argtypes = [f32p, ctypes.c_size_t, f32p]
+        L.oracle_rms_rstd.argtypes = [u16p, ctypes.c_int, ctypes.c_float]
+        L.oracle_rms_rstd.restype = ctypes.c_float
+        L.oracle_rmsnorm.argtypes = [u16p, u16p, ctypes.c_int, ctypes.c_int, ctypes.c_float, u16p, f32p]
+        L.oracle_rmsnorm.restype = None
         _LIB = L
     return _LIB
 
@@ -318,5 +322,38 @@ def moe_layer(x, w_router, bias, expert, *, n_experts: int, top_k: int, n_shared
     if n_shared:
         acc = acc + Yt[:, k]
     res["out"] = _bf16_of_f64(acc)
+    res["out_f64"] = acc
     res["tokens"] = tokens
+    return res
+
+
+# ---------------------------------------------------------------- pre-norm --
+
+def rmsnorm(h, gamma, eps: float = 1e-6):
+    """Pre-norm of the FFN input (RMSNorm with weight gamma), C core.
+    -> (x bf16 bits [T, d], rstd fp32 [T])."""
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    g = np.ascontiguousarray(gamma, dtype=np.uint16)
+    T, d = h.shape
+    x = np.empty((T, d), dtype=np.uint16)
+    r = np.empty(T, dtype=np.float32)
+    lib().oracle_rmsnorm(_p(h, ctypes.c_uint16), _p(g, ctypes.c_uint16), T, d, float(eps),
+                         _p(x, ctypes.c_uint16), _p(r, ctypes.c_float))
+    return x, r
+
+
+def moe_layer_prenorm(h, gamma, eps, w_router, bias, expert, **kw):
+    """out = h + MoE(RMSNorm(h) * gamma): the FFN block with its pre-norm and
+    residual ("DeepSeek-R1" card, "Facts": pre-norm RMSNorm before the MLP).
+    The residual is added to the unrounded combine sum in binary64 and the
+    block output rounded to bf16 once."""
+    x, rstd = rmsnorm(h, gamma, eps)
+    tokens = kw.get("tokens")
+    res = moe_layer(x, w_router, bias, expert, **kw)
+    rows = np.arange(x.shape[0]) if tokens is None else np.asarray(tokens)
+    hh = bf16_to_f32(np.asarray(h, dtype=np.uint16)[rows]).astype(np.float64)
+    res["moe_out"] = res["out"]
+    res["out"] = _bf16_of_f64(hh + res["out_f64"])
+    res["x"] = x
+    res["rstd"] = rstd
     return res

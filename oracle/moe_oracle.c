@@ -268,3 +268,49 @@ void oracle_sigmoid_array(const float *in, size_t n, float *out)
 {
     for (size_t i = 0; i < n; ++i) out[i] = oracle_sigmoid(in[i]);
 }
+
+/* --------------------------------------------------------- RMSNorm ----- */
+/*
+ * Pre-norm of the FFN input ("DeepSeek-R1" architecture card, "Facts": norm
+ * placement pre, norm type RMSNorm; the norm before the MLP produces the MoE
+ * input): x_i = bf16( (h_i * rstd) * gamma_i ),
+ * rstd = 1 / sqrt( S / d + eps ),  S = sum_i h_i^2.
+ * The pages fix no precision or order; both are taken as the kernel's, so
+ * the routing decision on x stays reproducible: 32 binary32 partial sums
+ * p_l = sum_j h_{l+32j}^2 (fused multiply-add, j ascending), then five
+ * pairwise rounds p_l = p_l + p_{l xor off} for off = 16, 8, 4, 2, 1 (all p_l
+ * end equal), S = p_0; S / d, the add of eps, the square root and the
+ * reciprocal are correctly rounded binary32 operations.
+ */
+float oracle_rms_rstd(const uint16_t *h, int d, float eps)
+{
+    float p[32], q[32];
+    for (int l = 0; l < 32; ++l) {
+        float acc = 0.0f;
+        for (int i = l; i < d; i += 32) {
+            float v = oracle_bf16_to_f32(h[i]);
+            acc = fmaf(v, v, acc);
+        }
+        p[l] = acc;
+    }
+    for (int off = 16; off >= 1; off >>= 1) {
+        for (int l = 0; l < 32; ++l) q[l] = p[l] + p[l ^ off];
+        for (int l = 0; l < 32; ++l) p[l] = q[l];
+    }
+    float mean = p[0] / (float)d;
+    return 1.0f / sqrtf(mean + eps);
+}
+
+void oracle_rmsnorm(const uint16_t *h, const uint16_t *gamma, int T, int d, float eps,
+                    uint16_t *x, float *rstd_out)
+{
+    for (int t = 0; t < T; ++t) {
+        const uint16_t *ht = h + (size_t)t * d;
+        float r = oracle_rms_rstd(ht, d, eps);
+        if (rstd_out) rstd_out[t] = r;
+        for (int i = 0; i < d; ++i) {
+            float v = (oracle_bf16_to_f32(ht[i]) * r) * oracle_bf16_to_f32(gamma[i]);
+            x[(size_t)t * d + i] = oracle_bf16_from_f32(v);
+        }
+    }
+}

@@ -13,7 +13,7 @@ from __future__ import annotations
 import torch
 
 from ._native import (EXPORTS, MOE_BF16, MOE_FP8_BLOCK, MOE_LAYOUT_ROWMAJOR, MOE_LAYOUT_TILED,
-                      MoeError, moe_pack_tiles, MoeShape, alloc_workspace,
+                      MoeError, moe_pack_tiles, moe_forward_prenorm, MoeShape, alloc_workspace,
                       fp8_block_quant, lib, make_shape, moe_check_status, moe_combine,
                       moe_forward, moe_grouped_swiglu, moe_last_error, moe_last_launch_count,
                       moe_permute, moe_route, moe_route_noalloc, moe_set_kernel_events,
@@ -25,7 +25,7 @@ __all__ = [
     "moe_combine", "moe_forward", "moe_check_status", "moe_last_error", "moe_last_launch_count",
     "quantize_weights", "MOE_BF16", "MOE_FP8_BLOCK", "moe_set_kernel_events",
     "moe_route_noalloc", "MOE_ROUTE_NOALLOC_MAX_SCORES", "moe_pack_tiles", "pack_weights",
-    "MOE_LAYOUT_ROWMAJOR", "MOE_LAYOUT_TILED",
+    "MOE_LAYOUT_ROWMAJOR", "MOE_LAYOUT_TILED", "moe_forward_prenorm",
 ]
 
 
@@ -98,6 +98,18 @@ class MoELayer:
             out = torch.empty(T, self.d, dtype=torch.bfloat16, device=x.device)
         moe_forward(self.shape(T), x, self.w_router, self.bias, self.w13, self.w13s, self.w2,
                     self.w2s, out, self.workspace(T), topk_idx_out=topk_idx_out, stream=stream)
+        return out
+
+    def forward_prenorm(self, h: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
+                        out: torch.Tensor | None = None,
+                        topk_idx_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """The FFN block: out = h + MoE(RMSNorm(h) * gamma) (pre-norm fused)."""
+        T = h.shape[0]
+        if out is None:
+            out = torch.empty(T, self.d, dtype=torch.bfloat16, device=h.device)
+        moe_forward_prenorm(self.shape(T), h, gamma, eps, self.w_router, self.bias, self.w13,
+                            self.w13s, self.w2, self.w2s, out, self.workspace(T),
+                            topk_idx_out=topk_idx_out, stream=stream)
         return out
 
     def check_status(self, T: int) -> int:

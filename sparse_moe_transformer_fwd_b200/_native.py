@@ -28,7 +28,7 @@ MOE_LAYOUT_TILED = 1
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant",
            "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_check_status",
            "moe_last_error", "moe_last_launch_count", "moe_set_kernel_events",
-           "moe_route_noalloc", "moe_pack_tiles")
+           "moe_route_noalloc", "moe_pack_tiles", "moe_forward_prenorm")
 
 # fixed score scratch of moe_route_noalloc, in floats (include/moe_fwd.h)
 MOE_ROUTE_NOALLOC_MAX_SCORES = 1 << 20
@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
         L.moe_grouped_swiglu.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_combine.argtypes = [sp, vp, vp, vp, vp, vp]
         L.moe_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_forward_prenorm.argtypes = [sp, vp, vp, cf, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_check_status.argtypes = [vp, vp]
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
@@ -76,7 +77,7 @@ def lib() -> ctypes.CDLL:
         L.moe_set_kernel_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ci]
         for name in ("moe_route", "moe_route_noalloc", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
                      "moe_combine", "moe_forward", "moe_check_status", "moe_last_launch_count",
-                     "moe_set_kernel_events", "moe_pack_tiles"):
+                     "moe_set_kernel_events", "moe_pack_tiles", "moe_forward_prenorm"):
             getattr(L, name).restype = ci
         _LIB = L
     return _LIB
@@ -207,6 +208,20 @@ def moe_forward(shape, x, w_router, bias, w13, w13_scales, w2, w2_scales, out, w
     _check(lib().moe_forward(
         ctypes.byref(shape), _ptr(x, _BF16, "x"), _ptr(w_router, _BF16, "w_router"),
         _ptr(bias, torch.float32, "bias"), _ptr(w13, wt, "w13"),
+        _ptr(w13_scales, torch.float32, "w13_scales"), _ptr(w2, wt, "w2"),
+        _ptr(w2_scales, torch.float32, "w2_scales"), _ptr(out, _BF16, "out"),
+        _ptr(topk_idx_out, torch.int32, "topk_idx_out"), _ptr(ws, torch.uint8, "ws"),
+        ws.numel(), _stream(stream)))
+
+
+def moe_forward_prenorm(shape, h, gamma, eps, w_router, bias, w13, w13_scales, w2, w2_scales, out,
+                        ws, topk_idx_out=None, stream=None):
+    """out = h + MoE(bf16(RMSNorm(h) * gamma)); x is never materialised."""
+    fp8 = shape.precision == MOE_FP8_BLOCK
+    wt = _FP8 if fp8 else _BF16
+    _check(lib().moe_forward_prenorm(
+        ctypes.byref(shape), _ptr(h, _BF16, "h"), _ptr(gamma, _BF16, "gamma"), float(eps),
+        _ptr(w_router, _BF16, "w_router"), _ptr(bias, torch.float32, "bias"), _ptr(w13, wt, "w13"),
         _ptr(w13_scales, torch.float32, "w13_scales"), _ptr(w2, wt, "w2"),
         _ptr(w2_scales, torch.float32, "w2_scales"), _ptr(out, _BF16, "out"),
         _ptr(topk_idx_out, torch.int32, "topk_idx_out"), _ptr(ws, torch.uint8, "ws"),

@@ -92,7 +92,7 @@ int check_shape(const moe_shape *s) {
 
 // ---------------------------------------------------------- workspace ---
 struct Layout {
-    size_t status, scores, idx, gates, counts, offsets, row_token, row_of;
+    size_t status, rstd, scores, idx, gates, counts, offsets, row_token, row_of;
     size_t masks, hist, blkoff, seg_start, seg_rows, tile_start;
     size_t a, a_scales, h, h_scales, y;
     size_t total;
@@ -112,6 +112,7 @@ Layout layout(const moe_shape *s) {
         return at;
     };
     L.status = take(256);
+    L.rstd = take(T * 4);
     L.scores = take(T * E * 4);
     L.idx = take(T * k * 4);
     L.gates = take(T * k * 4);
@@ -385,10 +386,17 @@ int moe_combine(const moe_shape *s, const uint16_t *y, const int32_t *row_of,
     return MOE_OK;
 }
 
-int moe_forward(const moe_shape *s, const uint16_t *x, const uint16_t *w_router,
-                const float *bias, const void *w13, const float *w13_scales, const void *w2,
-                const float *w2_scales, uint16_t *out, int32_t *topk_idx_out, void *ws,
-                size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+// The whole layer.  x is the FFN input, or with gamma set the residual stream
+// h, normalised on the fly (pre-norm) and added back in the combine.
+int forward_impl(const moe_shape *s, const uint16_t *x, const uint16_t *gamma, float eps,
+                 const uint16_t *w_router, const float *bias, const void *w13,
+                 const float *w13_scales, const void *w2, const float *w2_scales, uint16_t *out,
+                 int32_t *topk_idx_out, void *ws, size_t ws_bytes, void *stream) {
     RETURN_IF(check_shape(s));
     Layout L;
     RETURN_IF(check_ws(s, ws, ws_bytes, &L));
@@ -399,6 +407,7 @@ int moe_forward(const moe_shape *s, const uint16_t *x, const uint16_t *w_router,
     CHECK_PTR(out);
     if (topk_idx_out && !aligned16(topk_idx_out))
         return fail(MOE_ERR_INVALID_ARG, "topk_idx_out is not 16-byte aligned");
+    if (gamma && !(eps >= 0.0f)) return fail(MOE_ERR_INVALID_ARG, "eps must be >= 0");
     RETURN_IF(check_weights(s, w13, w13_scales, w2, w2_scales));
     RETURN_IF(check_device());
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -407,8 +416,15 @@ int moe_forward(const moe_shape *s, const uint16_t *x, const uint16_t *w_router,
     float *gates = at<float>(ws, L.gates);
     int32_t *row_of = at<int32_t>(ws, L.row_of);
     int n = 0;
+    PreNorm pn{};
+    if (gamma) {
+        float *rstd = at<float>(ws, L.rstd);
+        LAUNCH(launch_rstd(x, s->T, s->d_model, eps, rstd, st, &n), "pre-norm statistics");
+        pn.rstd = rstd;
+        pn.gamma = gamma;
+    }
     LAUNCH(launch_router(x, w_router, bias, s->T, s->d_model, s->n_experts, s->top_k,
-                         s->routed_scale, at<float>(ws, L.scores), idx, gates, st, &n),
+                         s->routed_scale, at<float>(ws, L.scores), idx, gates, st, &n, pn),
            "router");
     LAUNCH(launch_permute(idx, s->T, s->top_k, s->n_experts, s->n_shared, perm_scratch(ws, L),
                           at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
@@ -416,20 +432,45 @@ int moe_forward(const moe_shape *s, const uint16_t *x, const uint16_t *w_router,
            "permute");
     if (fp8)
         LAUNCH(launch_quant_scatter(x, s->T, s->d_model, s->top_k, s->n_shared, row_of,
-                                    at<uint8_t>(ws, L.a), at<float>(ws, L.a_scales), st, &n),
+                                    at<uint8_t>(ws, L.a), at<float>(ws, L.a_scales), st, &n, pn),
                "quant_scatter");
     else
         LAUNCH(launch_scatter_bf16(x, s->T, s->d_model, s->top_k, s->n_shared, row_of,
-                                   at<uint16_t>(ws, L.a), st, &n),
+                                   at<uint16_t>(ws, L.a), st, &n, pn),
                "scatter");
     uint16_t *y = at<uint16_t>(ws, L.y);
     RETURN_IF(grouped(s, at<uint8_t>(ws, L.a), fp8 ? at<float>(ws, L.a_scales) : nullptr, w13,
                       w13_scales, w2, w2_scales, y, ws, L, st, &n));
-    LAUNCH(launch_combine(y, row_of, gates, s->T, s->d_model, s->top_k, s->n_shared, out, st, &n),
+    LAUNCH(launch_combine(y, row_of, gates, s->T, s->d_model, s->top_k, s->n_shared, out, st, &n,
+                          gamma ? x : nullptr),
            "combine");
     mark_launch(st, n);
     g_launches = n;
     return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+int moe_forward(const moe_shape *s, const uint16_t *x, const uint16_t *w_router,
+                const float *bias, const void *w13, const float *w13_scales, const void *w2,
+                const float *w2_scales, uint16_t *out, int32_t *topk_idx_out, void *ws,
+                size_t ws_bytes, void *stream) {
+    return forward_impl(s, x, nullptr, 0.0f, w_router, bias, w13, w13_scales, w2, w2_scales, out,
+                        topk_idx_out, ws, ws_bytes, stream);
+}
+
+int moe_forward_prenorm(const moe_shape *s, const uint16_t *h, const uint16_t *gamma, float eps,
+                        const uint16_t *w_router, const float *bias, const void *w13,
+                        const float *w13_scales, const void *w2, const float *w2_scales,
+                        uint16_t *out, int32_t *topk_idx_out, void *ws, size_t ws_bytes,
+                        void *stream) {
+    if (!gamma) return fail(MOE_ERR_INVALID_ARG, "gamma is NULL");
+    if (!aligned16(gamma)) return fail(MOE_ERR_INVALID_ARG, "gamma is not 16-byte aligned");
+    return forward_impl(s, h, gamma, eps, w_router, bias, w13, w13_scales, w2, w2_scales, out,
+                        topk_idx_out, ws, ws_bytes, stream);
 }
 
 int moe_check_status(void *ws, void *stream) {

@@ -1,7 +1,8 @@
 // Weighted un-permute and shared-expert add ("DeepSeek v3 and R1 Model
 // Architecture", "Structural change": one always-activated shared expert):
 //   out[t] = bf16( sum_j g[t,j] * Y[row_of[t,j]]  (rank order, binary32 fma)
-//                  + Y[T*k + t] )                 (shared, weight 1)
+//                  + Y[T*k + t]                   (shared, weight 1)
+//                  [+ h[t]] )                     (residual of the pre-norm block)
 // One CTA per token, 16-byte vector loads of the k + 1 source rows.
 #include "common.cuh"
 #include "kernels.h"
@@ -12,7 +13,7 @@ namespace {
 __global__ void __launch_bounds__(128)
 combine_kernel(const uint16_t *__restrict__ y, const int32_t *__restrict__ row_of,
                const float *__restrict__ gates, int T, int d, int k, int n_shared,
-               uint16_t *__restrict__ out) {
+               uint16_t *__restrict__ out, const uint16_t *__restrict__ residual) {
     __shared__ int rows_sh[32];
     __shared__ float g_sh[32];
     const int t = blockIdx.x;
@@ -47,6 +48,15 @@ combine_kernel(const uint16_t *__restrict__ y, const int32_t *__restrict__ row_o
                 acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], bf16_hi(r[i]));
             }
         }
+        if (residual) {  // pre-norm block: out = h + MoE(x), one final rounding
+            const uint4 raw = reinterpret_cast<const uint4 *>(residual + static_cast<size_t>(t) * d)[v];
+            const uint32_t r[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[2 * i] = __fadd_rn(acc[2 * i], bf16_lo(r[i]));
+                acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], bf16_hi(r[i]));
+            }
+        }
         uint4 o;
         o.x = pack_bf16x2(acc[0], acc[1]);
         o.y = pack_bf16x2(acc[2], acc[3]);
@@ -60,10 +70,10 @@ combine_kernel(const uint16_t *__restrict__ y, const int32_t *__restrict__ row_o
 
 cudaError_t launch_combine(const uint16_t *y, const int32_t *row_of, const float *gates, int T,
                            int d, int k, int n_shared, uint16_t *out, cudaStream_t st,
-                           int *launches) {
+                           int *launches, const uint16_t *residual) {
     mark_launch(st, *launches);
     LAUNCH_OR_RETURN(launch_pdl(combine_kernel, dim3(T), dim3(128), 0, st, y, row_of, gates, T, d, k, n_shared,
-                                out));
+                                out, residual));
     ++*launches;
     return cudaGetLastError();
 }

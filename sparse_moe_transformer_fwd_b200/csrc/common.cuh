@@ -40,6 +40,12 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
     return r;
 }
 
+// Pre-norm of one element: bf16((h * rstd) * gamma) widened back to binary32.
+__device__ __forceinline__ float prenorm_elem(float h, float rstd, float gamma) {
+    const float v = __fmul_rn(__fmul_rn(h, rstd), gamma);
+    return __bfloat162float(__float2bfloat16_rn(v));
+}
+
 // ------------------------------------------------------------- mbarrier ---
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

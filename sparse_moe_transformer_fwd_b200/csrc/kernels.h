@@ -52,9 +52,20 @@ struct PermScratch {
     int32_t *tile_start; // [E + 2] prefix of 128-row tiles per segment
 };
 
+// Pre-norm of the FFN input applied on the fly by the kernels that read it:
+// x = bf16((h * rstd[t]) * gamma); rstd == nullptr means the input is x itself.
+struct PreNorm {
+    const float *rstd;      // [T], from launch_rstd
+    const uint16_t *gamma;  // [d] bf16
+};
+
+// rstd[t] = 1 / sqrt(sum_i h[t,i]^2 / d + eps), fixed summation order.
+cudaError_t launch_rstd(const uint16_t *h, int T, int d, float eps, float *rstd, cudaStream_t st,
+                        int *launches);
+
 cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bias, int T, int d,
                           int E, int k, float routed_scale, float *scores, int32_t *idx,
-                          float *gates, cudaStream_t st, int *launches);
+                          float *gates, cudaStream_t st, int *launches, PreNorm pn = {});
 
 cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int n_shared, PermScratch s,
                            int32_t *counts, int32_t *offsets, int32_t *row_token, int32_t *row_of,
@@ -77,16 +88,17 @@ cudaError_t launch_pack_tiles(const void *src, int rows, int row_bytes, void *ds
 // scales to its k routed rows (row_of) and, with n_shared, to row T*k + t.
 cudaError_t launch_quant_scatter(const uint16_t *x, int T, int d, int k, int n_shared,
                                  const int32_t *row_of, uint8_t *a, float *a_scales,
-                                 cudaStream_t st, int *launches);
+                                 cudaStream_t st, int *launches, PreNorm pn = {});
 
 // bf16 copy of each token row to its k routed rows and its shared row.
 cudaError_t launch_scatter_bf16(const uint16_t *x, int T, int d, int k, int n_shared,
                                 const int32_t *row_of, uint16_t *a, cudaStream_t st,
-                                int *launches);
+                                int *launches, PreNorm pn = {});
 
+// residual (nullable, bf16 [T, d]) is added before the final rounding.
 cudaError_t launch_combine(const uint16_t *y, const int32_t *row_of, const float *gates, int T,
                            int d, int k, int n_shared, uint16_t *out, cudaStream_t st,
-                           int *launches);
+                           int *launches, const uint16_t *residual = nullptr);
 
 // Grouped GEMM over the segment table.
 //   gate_up = true : out = H [rows, N_out] = silu(A Wg^T) * (A Wu^T), B rows per

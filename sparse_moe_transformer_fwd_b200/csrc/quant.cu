@@ -136,11 +136,49 @@ quant_128x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld
     }
 }
 
+// Pre-norm statistics ("DeepSeek-R1" card, "Facts": pre-norm RMSNorm before
+// the MLP): one warp per token; lane l sums h_i^2 over i = l (mod 32) with
+// fused multiply-adds in ascending i, five xor-butterfly rounds add the 32
+// partial sums (every lane ends with the same value), then
+// rstd = 1 / sqrt(S / d + eps), each step a correctly rounded binary32 op.
+__global__ void __launch_bounds__(256)
+rstd_kernel(const uint16_t *__restrict__ h, int T, int d, float eps, float *__restrict__ rstd) {
+    pdl_wait_and_trigger();
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const uint16_t *row = h + static_cast<size_t>(t) * d;
+    float acc = 0.0f;
+    for (int i = lane; i < d; i += 32) {
+        const float v = __uint_as_float(static_cast<uint32_t>(row[i]) << 16);
+        acc = __fmaf_rn(v, v, acc);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+    if (lane == 0) {
+        const float mean = __fdiv_rn(acc, static_cast<float>(d));
+        rstd[t] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
+    }
+}
+
+// x values of 8 consecutive columns c0.. of token t: bf16 inputs, or the
+// pre-norm of the residual stream h when rstd is set.
+__device__ __forceinline__ Quant8 load8_x(const uint16_t *row, int c0, float rstd,
+                                          const uint16_t *gamma) {
+    Quant8 v = load8_bf16(row + c0);
+    if (gamma) {
+        const Quant8 g = load8_bf16(gamma + c0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v.v[i] = prenorm_elem(v.v[i], rstd, g.v[i]);
+    }
+    return v;
+}
+
 // Forward pass: quantise token t's row once, write it to its k + n_shared rows.
 __global__ void __launch_bounds__(256)
 quant_scatter_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_shared,
                      const int32_t *__restrict__ row_of, uint8_t *__restrict__ a,
-                     float *__restrict__ a_scales) {
+                     float *__restrict__ a_scales, PreNorm pn) {
     __shared__ int rows_sh[33];
     const int t = blockIdx.x;
     const int ndst = k + n_shared;
@@ -150,11 +188,12 @@ quant_scatter_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_
     __syncthreads();
     const int ntiles = d / 128, nkb = d / 128;
     const int g = threadIdx.x / 16, l16 = threadIdx.x % 16;
+    const float rs = pn.rstd ? pn.rstd[t] : 1.0f;
     for (int p = 0; p * 16 < ntiles; ++p) {
         const int tile = p * 16 + g;
         const bool ok = tile < ntiles;
         Quant8 v;
-        if (ok) v = load8_bf16(x + static_cast<size_t>(t) * d + tile * 128 + l16 * 8);
+        if (ok) v = load8_x(x + static_cast<size_t>(t) * d, tile * 128 + l16 * 8, rs, pn.gamma);
         else
 #pragma unroll
             for (int i = 0; i < 8; ++i) v.v[i] = 0.0f;
@@ -172,7 +211,7 @@ quant_scatter_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_
 
 __global__ void __launch_bounds__(256)
 scatter_bf16_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_shared,
-                    const int32_t *__restrict__ row_of, uint16_t *__restrict__ a) {
+                    const int32_t *__restrict__ row_of, uint16_t *__restrict__ a, PreNorm pn) {
     __shared__ int rows_sh[33];
     const int t = blockIdx.x;
     const int ndst = k + n_shared;
@@ -181,8 +220,17 @@ scatter_bf16_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_s
     if (threadIdx.x == 0 && n_shared) rows_sh[k] = T * k + t;
     __syncthreads();
     const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t) * d);
+    const float rs = pn.rstd ? pn.rstd[t] : 1.0f;
     for (int v = threadIdx.x; v < d / 8; v += blockDim.x) {
-        const uint4 val = src[v];
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (!pn.gamma) val = src[v];
+        else {
+            const Quant8 xv = load8_x(x + static_cast<size_t>(t) * d, v * 8, rs, pn.gamma);
+            val.x = pack_bf16x2(xv.v[0], xv.v[1]);
+            val.y = pack_bf16x2(xv.v[2], xv.v[3]);
+            val.z = pack_bf16x2(xv.v[4], xv.v[5]);
+            val.w = pack_bf16x2(xv.v[6], xv.v[7]);
+        }
         for (int j = 0; j < ndst; ++j)
             reinterpret_cast<uint4 *>(a + static_cast<size_t>(rows_sh[j]) * d)[v] = val;
     }
@@ -243,22 +291,30 @@ cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, i
     return cudaGetLastError();
 }
 
+cudaError_t launch_rstd(const uint16_t *h, int T, int d, float eps, float *rstd, cudaStream_t st,
+                        int *launches) {
+    mark_launch(st, *launches);
+    LAUNCH_OR_RETURN(launch_pdl(rstd_kernel, dim3((T + 7) / 8), dim3(256), 0, st, h, T, d, eps, rstd));
+    ++*launches;
+    return cudaGetLastError();
+}
+
 cudaError_t launch_quant_scatter(const uint16_t *x, int T, int d, int k, int n_shared,
                                  const int32_t *row_of, uint8_t *a, float *a_scales,
-                                 cudaStream_t st, int *launches) {
+                                 cudaStream_t st, int *launches, PreNorm pn) {
     mark_launch(st, *launches);
     LAUNCH_OR_RETURN(launch_pdl(quant_scatter_kernel, dim3(T), dim3(256), 0, st, x, T, d, k, n_shared, row_of,
-                                a, a_scales));
+                                a, a_scales, pn));
     ++*launches;
     return cudaGetLastError();
 }
 
 cudaError_t launch_scatter_bf16(const uint16_t *x, int T, int d, int k, int n_shared,
                                 const int32_t *row_of, uint16_t *a, cudaStream_t st,
-                                int *launches) {
+                                int *launches, PreNorm pn) {
     mark_launch(st, *launches);
     LAUNCH_OR_RETURN(launch_pdl(scatter_bf16_kernel, dim3(T), dim3(256), 0, st, x, T, d, k, n_shared, row_of,
-                                a));
+                                a, pn));
     ++*launches;
     return cudaGetLastError();
 }

@@ -46,6 +46,21 @@ __device__ __forceinline__ ExpConsts exp_consts() {
     return k;
 }
 
+// 8 bf16 x values (one 16-byte vector) of token t at absolute column c0:
+// the input itself, or the pre-norm of the residual stream h.
+__device__ __forceinline__ uint4 x_vec(uint4 raw, const PreNorm &pn, int t, int c0) {
+    if (!pn.gamma) return raw;
+    const float r = pn.rstd[t];
+    const uint4 gr = *reinterpret_cast<const uint4 *>(pn.gamma + c0);
+    const uint32_t h4[4] = {raw.x, raw.y, raw.z, raw.w}, g4[4] = {gr.x, gr.y, gr.z, gr.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        o[i] = pack_bf16x2(prenorm_elem(bf16_lo(h4[i]), r, bf16_lo(g4[i])),
+                           prenorm_elem(bf16_hi(h4[i]), r, bf16_hi(g4[i])));
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 __device__ __forceinline__ float sigmoid_cw(float l, const ExpConsts &k) {
     float y = -l;
     y = fminf(fmaxf(y, -87.0f), 87.0f);
@@ -71,7 +86,7 @@ constexpr int RT_B = 64, RT_KC = 32, RT_THREADS = 64;
 
 __global__ void __launch_bounds__(RT_THREADS)
 router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w, int T, int d,
-                     int E, float *__restrict__ scores) {
+                     int E, float *__restrict__ scores, PreNorm pn) {
     __shared__ __align__(16) float xs[2][RT_KC][RT_B];  // [k][token]
     __shared__ __align__(16) float ws[2][RT_KC][RT_B];  // [k][expert]
     const int tid = threadIdx.x, tx = tid & 7, ty = tid >> 3;
@@ -99,9 +114,11 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
             const bool isx = row < RT_B;
             const int g = isx ? t0 + row : e0 + row - RT_B;
             pre[j] = make_uint4(0, 0, 0, 0);
-            if (g < (isx ? T : E))
+            if (g < (isx ? T : E)) {
                 pre[j] = *reinterpret_cast<const uint4 *>((isx ? x : w) + static_cast<size_t>(g) * d +
                                                           kc * RT_KC + col);
+                if (isx) pre[j] = x_vec(pre[j], pn, g, kc * RT_KC + col);
+            }
         }
     };
     auto store = [&](int buf) {
@@ -171,7 +188,7 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
 template <int BT, int KC>
 __global__ void __launch_bounds__(BT * 32)
 router_scores_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w, int T,
-                           int d, int E, float *__restrict__ scores) {
+                           int d, int E, float *__restrict__ scores, PreNorm pn) {
     constexpr int BE = 32, LD = KC + 4;
     constexpr int NT = BT * 32;
     constexpr int VPR = KC / 8;                  // 16-byte vectors per row per chunk
@@ -193,9 +210,11 @@ router_scores_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__res
                 const int row = v / VPR, col = (v % VPR) * 8;
                 const bool isx = row < BT;
                 const int g = isx ? t0 + row : e0 + row - BT;
-                if (g < (isx ? T : E))
+                if (g < (isx ? T : E)) {
                     pre[j] = *reinterpret_cast<const uint4 *>((isx ? x : w) + static_cast<size_t>(g) * d +
                                                               kc * KC + col);
+                    if (isx) pre[j] = x_vec(pre[j], pn, g, kc * KC + col);
+                }
             }
         }
     };
@@ -317,16 +336,17 @@ router_topk_kernel(const float *__restrict__ scores, const float *__restrict__ b
 
 cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bias, int T, int d,
                           int E, int k, float routed_scale, float *scores, int32_t *idx,
-                          float *gates, cudaStream_t st, int *launches) {
+                          float *gates, cudaStream_t st, int *launches, PreNorm pn) {
     mark_launch(st, *launches);
     if (T >= 512) {
         dim3 grid((E + RT_B - 1) / RT_B, (T + RT_B - 1) / RT_B);
-        LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel, grid, dim3(RT_THREADS), 0, st, x, w, T, d, E, scores));
+        LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel, grid, dim3(RT_THREADS), 0, st, x, w, T, d, E, scores,
+                                    pn));
     } else {
         constexpr int BT = 4, KC = 128;
         dim3 grid((E + 31) / 32, (T + BT - 1) / BT);
         LAUNCH_OR_RETURN(launch_pdl(router_scores_small_kernel<BT, KC>, grid, dim3(BT * 32), 0, st, x, w, T, d,
-                                    E, scores));
+                                    E, scores, pn));
     }
     ++*launches;
     const int per_lane = (E + 31) / 32;

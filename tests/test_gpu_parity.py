@@ -310,3 +310,59 @@ def test_bounded_wait_timeout_reports_status(monkeypatch):
     out = layer(d["x"])
     assert layer.check_status(cfg.T) == 0
     assert_out_close(out, oracle_layer(cfg, inp)["out"], "after timeout")
+
+
+# ----------------------------------------------- pre-norm block (fused) ---
+
+PRENORM_CASES = {
+    "tiny_bf16": CONFIGS["tiny"],
+    "tiny_fp8": CONFIGS["tiny"].with_(precision="fp8"),
+    "tiny_fp8_T600": CONFIGS["tiny"].with_(precision="fp8", T=600),
+    "tiny_bf16_T3": CONFIGS["tiny"].with_(T=3),
+}
+
+
+@pytest.mark.parametrize("name", list(PRENORM_CASES))
+def test_forward_prenorm_vs_oracle(name):
+    """out = h + MoE(bf16(RMSNorm(h) * gamma)) with x never materialised:
+    routing bit-exact against the oracle's pre-norm, output within tolerance."""
+    from moe_inputs import make_residual
+    cfg = PRENORM_CASES[name]
+    inp = make_inputs(cfg, seed=12)
+    h, g = make_residual(cfg, seed=12)
+    d = _dev(inp)
+    layer = moe.MoELayer(d["w_router"], d["bias"], d["w13"], d["w2"], top_k=cfg.top_k,
+                         precision=cfg.precision)
+    idx = torch.empty(cfg.T, cfg.top_k, dtype=torch.int32, device=DEV)
+    out = layer.forward_prenorm(h.to(DEV), g.to(DEV), 1e-6, topk_idx_out=idx)
+    assert layer.check_status(cfg.T) == 0
+    ref = oracle.moe_layer_prenorm(
+        u16(h), u16(g), 1e-6, u16(inp["w_router"]), inp["bias"].numpy(),
+        lambda e: (u16(inp["w13"][e]), u16(inp["w2"][e])), n_experts=cfg.n_experts,
+        top_k=cfg.top_k, n_shared=cfg.n_shared, precision=cfg.precision)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    assert_out_close(out, ref["out"], "prenorm " + name)
+
+
+def test_prenorm_router_decode_dims_bitexact():
+    """Decode-size routing on normalised-on-the-fly inputs (small-batch router
+    kernel) and a 600-token batch (tiled router kernel), DeepSeek dims."""
+    from moe_inputs import make_residual
+    for T in (64, 600):
+        cfg = CONFIGS["decode"].with_(T=T)
+        h, g = make_residual(cfg, seed=13)
+        from moe_inputs import make_router
+        w, b = make_router(cfg, seed=13)
+        x_ref, _ = oracle.rmsnorm(u16(h), u16(g), 1e-6)
+        logits = oracle.router_logits(x_ref, u16(w))
+        ridx, rg, _ = oracle.route(logits, b.numpy(), cfg.top_k)
+        # zero experts of width 128: only the routing and the residual are compared
+        w13 = torch.zeros(cfg.n_experts + 1, 256, cfg.d_model, dtype=torch.bfloat16, device=DEV)
+        w2 = torch.zeros(cfg.n_experts + 1, cfg.d_model, 128, dtype=torch.bfloat16, device=DEV)
+        layer = moe.MoELayer(w.to(DEV), b.to(DEV), w13, w2, top_k=cfg.top_k, precision="bf16")
+        idx = torch.empty(T, cfg.top_k, dtype=torch.int32, device=DEV)
+        out = layer.forward_prenorm(h.to(DEV), g.to(DEV), 1e-6, topk_idx_out=idx)
+        assert layer.check_status(T) == 0
+        assert np.array_equal(idx.cpu().numpy(), ridx)
+        # zero experts: the block returns the residual stream unchanged
+        assert torch.equal(out.cpu().view(torch.int16), h.view(torch.int16))
