@@ -175,13 +175,6 @@ class ClockSampler:
 
 # --------------------------------------------------------------- our arm ---
 
-def kernel_names(cfg, prenorm=False):
-    names = ["router_scores", "router_topk", "perm_hist", "perm_scan", "perm_scatter",
-             "quant_scatter" if cfg.precision == "fp8" else "scatter_bf16",
-             "grouped_gemm_gate_up", "grouped_gemm_down", "combine"]
-    return (["prenorm_rstd"] if prenorm else []) + names
-
-
 def algorithmic_bytes_gemm1(cfg, touched: int) -> float:
     """Bytes the gate/up GEMM must move once: the weights of every touched
     expert (and the shared one), their scales, the permuted activations and
@@ -224,12 +217,12 @@ def run_ours(args, world, rank, local):
     if status != 0:
         raise RuntimeError(f"device status {status}: {moe.moe_last_error()}")
     n_launch = moe.moe_last_launch_count()
+    names = moe.moe_last_launch_names()  # the library's own record of its launches
     touched = int(torch.unique(idx).numel()) + cfg.n_shared
     counts = torch.bincount(idx.reshape(-1).long(), minlength=cfg.n_experts)
 
     # ---- device-timed region: K steps, inputs resident in HBM; the dominant
     # kernel (gate/up GEMM) is bracketed by CUDA events inside the region
-    names = kernel_names(cfg, args.prenorm)
     gi = names.index("grouped_gemm_gate_up")
     g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(args.steps)]

@@ -233,6 +233,13 @@ const char *moe_last_error(void);
 /* Number of kernels the last successful call on this thread enqueued. */
 int moe_last_launch_count(void);
 
+/* Name of kernel i (0 <= i < moe_last_launch_count()) of the last successful
+ * call on this thread, in launch order (for example "router_scores",
+ * "perm_small", "grouped_gemm_gate_up"); NULL for any other i.  The string is
+ * static: the caller does not free it.  No counterpart in the pages: it lets
+ * a profiler attach the moe_set_kernel_events timeline to kernels. */
+const char *moe_last_launch_name(int i);
+
 /* Profiling hook.  events: n_events cudaEvent_t handles (host array, owned
  * by the caller) or NULL to switch the hook off.  While set, every later
  * call on this thread records events[i] on its stream just before its i-th

@@ -16,6 +16,7 @@ from ._native import (EXPORTS, MOE_BF16, MOE_FP8_BLOCK, MOE_LAYOUT_ROWMAJOR, MOE
                       MoeError, moe_pack_tiles, moe_forward_prenorm, MoeShape, alloc_workspace,
                       fp8_block_quant, lib, make_shape, moe_check_status, moe_combine,
                       moe_forward, moe_grouped_swiglu, moe_last_error, moe_last_launch_count,
+                      moe_last_launch_names,
                       moe_permute, moe_route, moe_route_noalloc, moe_set_kernel_events,
                       moe_workspace_size, MOE_ROUTE_NOALLOC_MAX_SCORES)
 
@@ -25,7 +26,7 @@ __all__ = [
     "moe_combine", "moe_forward", "moe_check_status", "moe_last_error", "moe_last_launch_count",
     "quantize_weights", "MOE_BF16", "MOE_FP8_BLOCK", "moe_set_kernel_events",
     "moe_route_noalloc", "MOE_ROUTE_NOALLOC_MAX_SCORES", "moe_pack_tiles", "pack_weights",
-    "MOE_LAYOUT_ROWMAJOR", "MOE_LAYOUT_TILED", "moe_forward_prenorm",
+    "MOE_LAYOUT_ROWMAJOR", "MOE_LAYOUT_TILED", "moe_forward_prenorm", "moe_last_launch_names",
 ]
 
 

@@ -28,7 +28,7 @@ MOE_LAYOUT_TILED = 1
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant",
            "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_check_status",
            "moe_last_error", "moe_last_launch_count", "moe_set_kernel_events",
-           "moe_route_noalloc", "moe_pack_tiles", "moe_forward_prenorm")
+           "moe_route_noalloc", "moe_pack_tiles", "moe_forward_prenorm", "moe_last_launch_name")
 
 # fixed score scratch of moe_route_noalloc, in floats (include/moe_fwd.h)
 MOE_ROUTE_NOALLOC_MAX_SCORES = 1 << 20
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         L.moe_last_launch_count.argtypes = []
+        L.moe_last_launch_name.argtypes = [ci]
+        L.moe_last_launch_name.restype = ctypes.c_char_p
         L.moe_set_kernel_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ci]
         for name in ("moe_route", "moe_route_noalloc", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
                      "moe_combine", "moe_forward", "moe_check_status", "moe_last_launch_count",
@@ -239,6 +241,12 @@ def moe_last_error() -> str:
 
 def moe_last_launch_count() -> int:
     return lib().moe_last_launch_count()
+
+
+def moe_last_launch_names() -> list:
+    """Kernel names of the last call on this thread, in launch order."""
+    L = lib()
+    return [L.moe_last_launch_name(i).decode() for i in range(L.moe_last_launch_count())]
 
 
 def moe_set_kernel_events(events) -> None:

@@ -21,10 +21,13 @@ int num_sms() {
 namespace {
 thread_local cudaEvent_t *g_events = nullptr;  // profiling hook (moe_set_kernel_events)
 thread_local int g_n_events = 0;
+constexpr int kMaxNamed = 64;
+thread_local const char *g_names[kMaxNamed];  // kernel of each launch of the last call
 }  // namespace
 
-void mark_launch(cudaStream_t st, int index) {
+void mark_launch(cudaStream_t st, int index, const char *name) {
     if (g_events && index < g_n_events && g_events[index]) cudaEventRecord(g_events[index], st);
+    if (name && index >= 0 && index < kMaxNamed) g_names[index] = name;
 }
 
 namespace {
@@ -493,6 +496,10 @@ int moe_check_status(void *ws, void *stream) {
 const char *moe_last_error(void) { return g_err.c_str(); }
 
 int moe_last_launch_count(void) { return g_launches; }
+
+const char *moe_last_launch_name(int i) {
+    return (i >= 0 && i < g_launches && i < kMaxNamed) ? g_names[i] : nullptr;
+}
 
 int moe_set_kernel_events(void **events, int n_events) {
     if (events && n_events <= 0) return fail(MOE_ERR_INVALID_ARG, "n_events must be positive");

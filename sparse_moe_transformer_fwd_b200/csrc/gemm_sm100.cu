@@ -226,17 +226,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     }
                 }
             }
-            // drain: every load this thread issued has landed before the block exits
-            for (int i = 0; i < STAGES; ++i)
-                if (armed & (1 << i)) {
-                    long long t0 = clock64();
-                    while (!mbar_try_wait(&s.full[i], armed_phase[i])) {
-                        if (clock64() - t0 > kWaitBudgetCycles) {
-                            set_status(p.status, MOE_ERR_TIMEOUT);
-                            break;
-                        }
+            // drain: every load this thread issued has landed before the block
+            // exits (one budget for all stages)
+            const long long t0 = clock64();
+            for (int i = 0; i < STAGES; ++i) {
+                if (!(armed & (1 << i))) continue;
+                bool late = false;
+                while (!mbar_try_wait(&s.full[i], armed_phase[i])) {
+                    if (clock64() - t0 > kWaitBudgetCycles) {
+                        set_status(p.status, MOE_ERR_TIMEOUT);
+                        late = true;
+                        break;
                     }
                 }
+                if (late) break;
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
@@ -542,7 +546,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
     if (grid <= 0) return cudaSuccess;
     cudaError_t e;
-    mark_launch(st, *launches);
+    mark_launch(st, *launches, g.gate_up ? "grouped_gemm_gate_up" : "grouped_gemm_down");
     if (g.fp8) e = g.gate_up ? launch_t<true, true>(ma, mb, kp, grid, st)
                              : launch_t<true, false>(ma, mb, kp, grid, st);
     else e = g.gate_up ? launch_t<false, true>(ma, mb, kp, grid, st)

@@ -133,8 +133,10 @@ int record_error(int code, const char *msg);  // sets moe_last_error, returns co
 void record_launches(int n);                   // sets moe_last_launch_count
 int validate_shape(const moe_shape *s);        // host-side shape checks
 
-// Profiling hook: records the caller's event `index` on `st` when the
-// moe_set_kernel_events hook is active (call just before a kernel launch).
-void mark_launch(cudaStream_t st, int index);
+// Called just before the call's kernel launch number `index` with that
+// kernel's name (and once more after the last launch, without a name):
+// records the caller's event `index` on `st` when the moe_set_kernel_events
+// hook is active, and the name for moe_last_launch_name.
+void mark_launch(cudaStream_t st, int index, const char *name = nullptr);
 
 }  // namespace moe

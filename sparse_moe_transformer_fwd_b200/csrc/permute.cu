@@ -13,7 +13,9 @@
 //     GEMM's segment/tile table (routed segments, then the shared segment).
 //  3. perm_scatter: rank of token t inside expert e's segment = popcount of
 //     mask[e] below t; row = offsets[e] + block prefix + rank.
-// Also build_tile_table: the segment/tile table from caller-given offsets.
+// A batch of at most 256 tokens takes all three steps in one CTA
+// (perm_small).  Also build_tile_table: the segment/tile table from
+// caller-given offsets.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -159,12 +161,70 @@ perm_scatter_kernel(const int32_t *__restrict__ idx, int T, int k, int E,
     }
 }
 
+// Batches of at most 256 tokens (one bit-matrix block): kernels 1-3 in one
+// CTA of 1024 threads, the bit matrix and the offsets in shared memory.
+__global__ void __launch_bounds__(1024)
+perm_small_kernel(const int32_t *__restrict__ idx, int T, int k, int E, int n_shared,
+                  int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                  int32_t *__restrict__ row_token, int32_t *__restrict__ row_of,
+                  int32_t *seg_start, int32_t *seg_rows, int32_t *tile_start,
+                  int *status) {
+    __shared__ uint32_t mask[1024 * kWords];  // [E][kWords], E <= 1024
+    __shared__ int32_t off_sh[1024];
+    __shared__ int tmp[32];
+    const int e = threadIdx.x;
+    pdl_wait_and_trigger();
+    for (int i = threadIdx.x; i < E * kWords; i += blockDim.x) mask[i] = 0;
+    __syncthreads();
+    const int np = T * k;
+    for (int i = threadIdx.x; i < np; i += blockDim.x) {
+        const int v = idx[i];
+        if (v < 0 || v >= E) {
+            set_status(status, MOE_ERR_DEVICE_INDEX);
+            continue;
+        }
+        const int tl = i / k;
+        const uint32_t bit = 1u << (tl & 31);
+        const uint32_t old = atomicOr(&mask[v * kWords + (tl >> 5)], bit);
+        if (old & bit) set_status(status, MOE_ERR_DEVICE_INDEX);
+    }
+    __syncthreads();
+    int run = 0;
+    if (e < E) {
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) run += __popc(mask[e * kWords + w]);
+        counts[e] = run;
+    }
+    int total;
+    const int off = block_exclusive_scan(e < E ? run : 0, tmp, &total);
+    if (e < E) {
+        offsets[e] = off;
+        off_sh[e] = off;
+    }
+    if (e == 0) offsets[E] = total;
+    write_tile_table(run, off, e, E, T, T * k, n_shared, tmp, seg_start, seg_rows, tile_start);
+    __syncthreads();
+    for (int i = threadIdx.x; i < np; i += blockDim.x) {
+        const int v = idx[i];
+        if (v < 0 || v >= E) continue;
+        const int tl = i / k;
+        const uint32_t *m = mask + v * kWords;
+        int rank = 0;
+        for (int w = 0; w < (tl >> 5); ++w) rank += __popc(m[w]);
+        rank += __popc(m[tl >> 5] & ((1u << (tl & 31)) - 1u));
+        const int row = off_sh[v] + rank;
+        row_token[row] = tl;
+        row_of[i] = row;
+    }
+}
+
 // Segment table from caller-given offsets.  A segment that is not inside
 // [0, T*k) or has a negative size is recorded in the status word and
 // treated as empty, so the GEMMs never touch rows outside the buffers.
 __global__ void __launch_bounds__(1024)
 tile_table_kernel(const int32_t *__restrict__ offsets, int E, int T, int k, int n_shared,
-                  int32_t *seg_start, int32_t *seg_rows, int32_t *tile_start, int *status) {
+                  int32_t *seg_start, int32_t *seg_rows, int32_t *tile_start,
+                  int *status) {
     __shared__ int tmp[32];
     const int e = threadIdx.x;
     pdl_wait_and_trigger();
@@ -188,15 +248,23 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int n_shared
                            int *status, cudaStream_t st, int *launches) {
     const int nblk = (T + kBT - 1) / kBT;
     const size_t smem = static_cast<size_t>(E) * kWords * sizeof(uint32_t);
-    mark_launch(st, *launches);
+    if (nblk == 1) {
+        mark_launch(st, *launches, "perm_small");
+        LAUNCH_OR_RETURN(launch_pdl(perm_small_kernel, dim3(1), dim3(1024), 0, st, idx, T, k, E,
+                                    n_shared, counts, offsets, row_token, row_of, s.seg_start,
+                                    s.seg_rows, s.tile_start, status));
+        ++*launches;
+        return cudaGetLastError();
+    }
+    mark_launch(st, *launches, "perm_hist");
     LAUNCH_OR_RETURN(launch_pdl(perm_hist_kernel, dim3(nblk), dim3(256), smem, st, idx, T, k, E, s.masks,
                                 s.hist, status));
     ++*launches;
-    mark_launch(st, *launches);
+    mark_launch(st, *launches, "perm_scan");
     LAUNCH_OR_RETURN(launch_pdl(perm_scan_kernel, dim3(1), dim3(1024), 0, st, s.hist, nblk, E, T, k, n_shared,
                                 s.blkoff, counts, offsets, s.seg_start, s.seg_rows, s.tile_start));
     ++*launches;
-    mark_launch(st, *launches);
+    mark_launch(st, *launches, "perm_scatter");
     LAUNCH_OR_RETURN(launch_pdl(perm_scatter_kernel, dim3(nblk), dim3(256), smem, st, idx, T, k, E, s.masks,
                                 s.blkoff, offsets, row_token, row_of));
     ++*launches;
@@ -205,7 +273,7 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int n_shared
 
 cudaError_t launch_tile_table(const int32_t *offsets, int E, int T, int k, int n_shared,
                               PermScratch s, int *status, cudaStream_t st, int *launches) {
-    mark_launch(st, *launches);
+    mark_launch(st, *launches, "tile_table");
     LAUNCH_OR_RETURN(launch_pdl(tile_table_kernel, dim3(1), dim3(1024), 0, st, offsets, E, T, k, n_shared,
                                 s.seg_start, s.seg_rows, s.tile_start, status));
     ++*launches;

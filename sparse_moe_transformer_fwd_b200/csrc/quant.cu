@@ -189,23 +189,22 @@ quant_scatter_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_
     const int ntiles = d / 128, nkb = d / 128;
     const int g = threadIdx.x / 16, l16 = threadIdx.x % 16;
     const float rs = pn.rstd ? pn.rstd[t] : 1.0f;
-    for (int p = 0; p * 16 < ntiles; ++p) {
-        const int tile = p * 16 + g;
-        const bool ok = tile < ntiles;
-        Quant8 v;
-        if (ok) v = load8_x(x + static_cast<size_t>(t) * d, tile * 128 + l16 * 8, rs, pn.gamma);
-        else
+    // CTA (t, y) quantises tiles 16y .. 16y+15 of the row (16 threads per tile)
+    const int tile = blockIdx.y * 16 + g;
+    const bool ok = tile < ntiles;
+    Quant8 v;
+    if (ok) v = load8_x(x + static_cast<size_t>(t) * d, tile * 128 + l16 * 8, rs, pn.gamma);
+    else
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v.v[i] = 0.0f;
-        const float amax = group16_max(amax8(v));
-        float sc;
-        const uint2 codes = encode8(v, amax, &sc);
-        if (!ok) continue;
-        for (int j = 0; j < ndst; ++j) {
-            const size_t row = static_cast<size_t>(rows_sh[j]);
-            *reinterpret_cast<uint2 *>(a + row * d + tile * 128 + l16 * 8) = codes;
-            if (l16 == 0) a_scales[row * nkb + tile] = sc;
-        }
+        for (int i = 0; i < 8; ++i) v.v[i] = 0.0f;
+    const float amax = group16_max(amax8(v));
+    float sc;
+    const uint2 codes = encode8(v, amax, &sc);
+    if (!ok) return;
+    for (int j = 0; j < ndst; ++j) {
+        const size_t row = static_cast<size_t>(rows_sh[j]);
+        *reinterpret_cast<uint2 *>(a + row * d + tile * 128 + l16 * 8) = codes;
+        if (l16 == 0) a_scales[row * nkb + tile] = sc;
     }
 }
 
@@ -221,7 +220,9 @@ scatter_bf16_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_s
     __syncthreads();
     const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t) * d);
     const float rs = pn.rstd ? pn.rstd[t] : 1.0f;
-    for (int v = threadIdx.x; v < d / 8; v += blockDim.x) {
+    // CTA (t, y) copies 16-byte vectors 256y .. 256y+255 of the row
+    for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < min(d / 8, (blockIdx.y + 1) * blockDim.x);
+         v += blockDim.x) {
         uint4 val = make_uint4(0, 0, 0, 0);
         if (!pn.gamma) val = src[v];
         else {
@@ -261,7 +262,7 @@ cudaError_t launch_pack_tiles(const void *src, int rows, int row_bytes, void *ds
     const long long total = static_cast<long long>(rows) * (row_bytes / 16);
     const long long want = (total + 255) / 256;
     const int grid = static_cast<int>(want < num_sms() * 16LL ? want : num_sms() * 16LL);
-    mark_launch(st, *launches);
+    mark_launch(st, *launches, "pack_tiles");
     LAUNCH_OR_RETURN(launch_pdl(pack_tiles_kernel, dim3(grid), dim3(256), 0, st,
                                 static_cast<const uint8_t *>(src), rows, row_bytes,
                                 static_cast<uint8_t *>(dst)));
@@ -274,7 +275,7 @@ cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, i
                                int *launches) {
     if (rows == 0) return cudaSuccess;
     const int sms = num_sms();
-    mark_launch(st, *launches);
+    mark_launch(st, *launches, block_rows == 1 ? "quant_1x128" : "quant_128x128");
     if (block_rows == 1) {
         const long long total = static_cast<long long>(rows) * (cols / 8);
         const long long want = (total + 255) / 256;
@@ -293,7 +294,7 @@ cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, i
 
 cudaError_t launch_rstd(const uint16_t *h, int T, int d, float eps, float *rstd, cudaStream_t st,
                         int *launches) {
-    mark_launch(st, *launches);
+    mark_launch(st, *launches, "prenorm_rstd");
     LAUNCH_OR_RETURN(launch_pdl(rstd_kernel, dim3((T + 7) / 8), dim3(256), 0, st, h, T, d, eps, rstd));
     ++*launches;
     return cudaGetLastError();
@@ -302,8 +303,8 @@ cudaError_t launch_rstd(const uint16_t *h, int T, int d, float eps, float *rstd,
 cudaError_t launch_quant_scatter(const uint16_t *x, int T, int d, int k, int n_shared,
                                  const int32_t *row_of, uint8_t *a, float *a_scales,
                                  cudaStream_t st, int *launches, PreNorm pn) {
-    mark_launch(st, *launches);
-    LAUNCH_OR_RETURN(launch_pdl(quant_scatter_kernel, dim3(T), dim3(256), 0, st, x, T, d, k, n_shared, row_of,
+    mark_launch(st, *launches, "quant_scatter");
+    LAUNCH_OR_RETURN(launch_pdl(quant_scatter_kernel, dim3(T, (d / 128 + 15) / 16), dim3(256), 0, st, x, T, d, k, n_shared, row_of,
                                 a, a_scales, pn));
     ++*launches;
     return cudaGetLastError();
@@ -312,8 +313,8 @@ cudaError_t launch_quant_scatter(const uint16_t *x, int T, int d, int k, int n_s
 cudaError_t launch_scatter_bf16(const uint16_t *x, int T, int d, int k, int n_shared,
                                 const int32_t *row_of, uint16_t *a, cudaStream_t st,
                                 int *launches, PreNorm pn) {
-    mark_launch(st, *launches);
-    LAUNCH_OR_RETURN(launch_pdl(scatter_bf16_kernel, dim3(T), dim3(256), 0, st, x, T, d, k, n_shared, row_of,
+    mark_launch(st, *launches, "scatter_bf16");
+    LAUNCH_OR_RETURN(launch_pdl(scatter_bf16_kernel, dim3(T, (d / 8 + 255) / 256), dim3(256), 0, st, x, T, d, k, n_shared, row_of,
                                 a, pn));
     ++*launches;
     return cudaGetLastError();

@@ -181,81 +181,110 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
 // ------------------------------------------------- router_scores (small T)
 // Decode-sized batches: warp w of the CTA owns token t0 + w, lane l owns
 // expert e0 + l; one output per thread, so the kernel is bound by the length
-// of its d-long FMA chain.  x and W_r chunks sit k-contiguous in shared
-// memory (rows padded by 4 floats), read as 16-byte vectors: x by broadcast,
-// W_r in four conflict-free wavefronts per warp.  Staging goes through
-// registers one chunk ahead, as in the tiled kernel.
-template <int BT, int KC>
+// of its d-long FMA chain.  Chunks of 256 columns of the CTA's 32 W_r rows
+// and BT x rows stream into a 4-stage shared-memory ring with cp.async (W_r
+// rows padded by 16 bytes, so the 32 lanes' 16-byte reads of one column
+// fall in distinct banks), three chunks ahead of the FMAs; each warp widens
+// its own token's chunk to binary32 (applying the pre-norm if any) and the
+// lanes widen W_r in registers.
+constexpr int RS_KC = 256;                 // columns per chunk
+constexpr int RS_WLD = RS_KC + 8;          // padded W_r row, bf16 elements
+constexpr int RS_STAGES = 4;
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+                 "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <int BT>
+constexpr size_t router_small_smem() {
+    return static_cast<size_t>(RS_STAGES) * (32 * RS_WLD + BT * RS_KC) * 2 +
+           static_cast<size_t>(BT) * RS_KC * 4;
+}
+
+template <int BT>
 __global__ void __launch_bounds__(BT * 32)
 router_scores_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w, int T,
                            int d, int E, float *__restrict__ scores, PreNorm pn) {
-    constexpr int BE = 32, LD = KC + 4;
     constexpr int NT = BT * 32;
-    constexpr int VPR = KC / 8;                  // 16-byte vectors per row per chunk
-    constexpr int NV = (BT + BE) * VPR;
-    constexpr int PER = (NV + NT - 1) / NT;
-    __shared__ __align__(16) float xs[2][BT][LD];
-    __shared__ __align__(16) float ws[2][BE][LD];
+    constexpr int VPR = RS_KC / 8;                    // 16-byte vectors per row per chunk
+    constexpr int W_ELEMS = 32 * RS_WLD, X_ELEMS = BT * RS_KC;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint16_t *ring = reinterpret_cast<uint16_t *>(smem_raw);            // [stage][W | x]
+    float *xf = reinterpret_cast<float *>(ring + RS_STAGES * (W_ELEMS + X_ELEMS));  // [BT][KC]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int t0 = blockIdx.y * BT, e0 = blockIdx.x * BE;
+    const int t0 = blockIdx.y * BT, e0 = blockIdx.x * 32;
+    const int t = t0 + warp, e = e0 + lane;
     pdl_wait_and_trigger();
 
-    uint4 pre[PER];
-    auto load = [&](int kc) {
-#pragma unroll
-        for (int j = 0; j < PER; ++j) {
-            const int v = tid + j * NT;
-            pre[j] = make_uint4(0, 0, 0, 0);
-            if (v < NV) {
-                const int row = v / VPR, col = (v % VPR) * 8;
-                const bool isx = row < BT;
-                const int g = isx ? t0 + row : e0 + row - BT;
-                if (g < (isx ? T : E)) {
-                    pre[j] = *reinterpret_cast<const uint4 *>((isx ? x : w) + static_cast<size_t>(g) * d +
-                                                              kc * KC + col);
-                    if (isx) pre[j] = x_vec(pre[j], pn, g, kc * KC + col);
-                }
+    const int nk = d / RS_KC;
+    auto issue = [&](int kc) {
+        uint16_t *ws = ring + (kc % RS_STAGES) * (W_ELEMS + X_ELEMS);
+        uint16_t *xs = ws + W_ELEMS;
+        for (int v = tid; v < (32 + BT) * VPR; v += NT) {
+            const int row = v / VPR, col = (v % VPR) * 8;
+            if (row < 32) {
+                const bool ok = e0 + row < E;
+                const uint16_t *src = w + static_cast<size_t>(ok ? e0 + row : 0) * d + kc * RS_KC + col;
+                cp_async16(ws + row * RS_WLD + col, src, ok);
+            } else {
+                const int r = row - 32;
+                const bool ok = t0 + r < T;
+                const uint16_t *src = x + static_cast<size_t>(ok ? t0 + r : 0) * d + kc * RS_KC + col;
+                cp_async16(xs + r * RS_KC + col, src, ok);
             }
         }
     };
-    auto store = [&](int buf) {
 #pragma unroll
-        for (int j = 0; j < PER; ++j) {
-            const int v = tid + j * NT;
-            if (v >= NV) continue;
-            const int row = v / VPR, col = (v % VPR) * 8;
-            float *dst = row < BT ? &xs[buf][row][col] : &ws[buf][row - BT][col];
-            const uint32_t r4[4] = {pre[j].x, pre[j].y, pre[j].z, pre[j].w};
-            *reinterpret_cast<float4 *>(dst) =
-                make_float4(bf16_lo(r4[0]), bf16_hi(r4[0]), bf16_lo(r4[1]), bf16_hi(r4[1]));
-            *reinterpret_cast<float4 *>(dst + 4) =
-                make_float4(bf16_lo(r4[2]), bf16_hi(r4[2]), bf16_lo(r4[3]), bf16_hi(r4[3]));
-        }
-    };
-
-    float acc = 0.0f;
-    const int nk = d / KC;
-    load(0);
-    store(0);
-    __syncthreads();
-    for (int kc = 0; kc < nk; ++kc) {
-        const int buf = kc & 1;
-        if (kc + 1 < nk) load(kc + 1);
-        const float *xr = xs[buf][warp];
-        const float *wr = ws[buf][lane];
-#pragma unroll 8
-        for (int kk = 0; kk < KC; kk += 4) {
-            const float4 xa = *reinterpret_cast<const float4 *>(xr + kk);
-            const float4 wa = *reinterpret_cast<const float4 *>(wr + kk);
-            acc = __fmaf_rn(xa.x, wa.x, acc);
-            acc = __fmaf_rn(xa.y, wa.y, acc);
-            acc = __fmaf_rn(xa.z, wa.z, acc);
-            acc = __fmaf_rn(xa.w, wa.w, acc);
-        }
-        if (kc + 1 < nk) store(buf ^ 1);
-        __syncthreads();
+    for (int s = 0; s < RS_STAGES - 1; ++s) {
+        if (s < nk) issue(s);
+        cp_async_commit();
     }
-    const int t = t0 + warp, e = e0 + lane;
+    float acc = 0.0f;
+    float *xw = xf + warp * RS_KC;
+    for (int kc = 0; kc < nk; ++kc) {
+        cp_async_wait<RS_STAGES - 2>();
+        __syncthreads();  // chunk kc landed; every warp is done with chunk kc - 1
+        if (kc + RS_STAGES - 1 < nk) issue(kc + RS_STAGES - 1);
+        cp_async_commit();
+        const uint16_t *ws = ring + (kc % RS_STAGES) * (W_ELEMS + X_ELEMS);
+        const uint16_t *xs = ws + W_ELEMS;
+        {   // this warp's token: 8 columns per lane, widened (and pre-normed)
+            const int c = lane * 8;
+            const uint4 raw = x_vec(*reinterpret_cast<const uint4 *>(xs + warp * RS_KC + c), pn,
+                                    t < T ? t : 0, kc * RS_KC + c);
+            *reinterpret_cast<float4 *>(xw + c) =
+                make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
+            *reinterpret_cast<float4 *>(xw + c + 4) =
+                make_float4(bf16_lo(raw.z), bf16_hi(raw.z), bf16_lo(raw.w), bf16_hi(raw.w));
+        }
+        __syncwarp();
+        const uint16_t *wr = ws + lane * RS_WLD;
+#pragma unroll 4
+        for (int kk = 0; kk < RS_KC; kk += 8) {
+            const uint4 wv = *reinterpret_cast<const uint4 *>(wr + kk);
+            const float4 xa = *reinterpret_cast<const float4 *>(xw + kk);
+            const float4 xb = *reinterpret_cast<const float4 *>(xw + kk + 4);
+            acc = __fmaf_rn(xa.x, bf16_lo(wv.x), acc);
+            acc = __fmaf_rn(xa.y, bf16_hi(wv.x), acc);
+            acc = __fmaf_rn(xa.z, bf16_lo(wv.y), acc);
+            acc = __fmaf_rn(xa.w, bf16_hi(wv.y), acc);
+            acc = __fmaf_rn(xb.x, bf16_lo(wv.z), acc);
+            acc = __fmaf_rn(xb.y, bf16_hi(wv.z), acc);
+            acc = __fmaf_rn(xb.z, bf16_lo(wv.w), acc);
+            acc = __fmaf_rn(xb.w, bf16_hi(wv.w), acc);
+        }
+        __syncwarp();  // xw is rewritten next chunk
+    }
+    cp_async_wait<0>();
     if (t < T && e < E) scores[static_cast<size_t>(t) * E + e] = sigmoid_cw(acc, exp_consts());
 }
 
@@ -337,21 +366,29 @@ router_topk_kernel(const float *__restrict__ scores, const float *__restrict__ b
 cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bias, int T, int d,
                           int E, int k, float routed_scale, float *scores, int32_t *idx,
                           float *gates, cudaStream_t st, int *launches, PreNorm pn) {
-    mark_launch(st, *launches);
+    mark_launch(st, *launches, "router_scores");
     if (T >= 512) {
         dim3 grid((E + RT_B - 1) / RT_B, (T + RT_B - 1) / RT_B);
         LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel, grid, dim3(RT_THREADS), 0, st, x, w, T, d, E, scores,
                                     pn));
     } else {
-        constexpr int BT = 4, KC = 128;
+        constexpr int BT = 4;
+        constexpr size_t smem = router_small_smem<BT>();
+        static bool configured = false;
+        if (!configured) {
+            LAUNCH_OR_RETURN(cudaFuncSetAttribute(router_scores_small_kernel<BT>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(smem)));
+            configured = true;
+        }
         dim3 grid((E + 31) / 32, (T + BT - 1) / BT);
-        LAUNCH_OR_RETURN(launch_pdl(router_scores_small_kernel<BT, KC>, grid, dim3(BT * 32), 0, st, x, w, T, d,
-                                    E, scores, pn));
+        LAUNCH_OR_RETURN(launch_pdl(router_scores_small_kernel<BT>, grid, dim3(BT * 32), smem, st, x, w, T,
+                                    d, E, scores, pn));
     }
     ++*launches;
     const int per_lane = (E + 31) / 32;
     dim3 grid2((T + 7) / 8);
-    mark_launch(st, *launches);
+    mark_launch(st, *launches, "router_topk");
     if (per_lane <= 1)
         LAUNCH_OR_RETURN(launch_pdl(router_topk_kernel<1>, grid2, dim3(256), 0, st, scores, bias, T, E, k, routed_scale, idx, gates));
     else if (per_lane <= 4)

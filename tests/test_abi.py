@@ -80,6 +80,8 @@ def test_empty_batch_enqueues_nothing():
     s = _shape(T=0)
     assert _call_forward(s, moe.moe_workspace_size(s)) == N.MOE_OK
     assert moe.moe_last_launch_count() == 0
+    assert moe.moe_last_launch_names() == []
+    assert moe.lib().moe_last_launch_name(0) is None
 
 
 def test_binding_rejects_cpu_tensors():

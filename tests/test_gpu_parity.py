@@ -94,7 +94,9 @@ def _rand_idx(rng, T, E, k, mode="uniform"):
 
 PERM_CASES = [(1, 16, 4, "uniform"), (3, 16, 4, "uniform"), (257, 16, 4, "uniform"),
               (1000, 256, 8, "uniform"), (1000, 256, 8, "one"), (4096, 256, 8, "skew"),
-              (600, 1023, 32, "uniform"), (64, 8, 8, "uniform")]
+              (600, 1023, 32, "uniform"), (64, 8, 8, "uniform"),
+              # one 256-token block: the single-CTA path, up to its limits
+              (256, 1023, 32, "uniform"), (256, 256, 8, "skew"), (255, 16, 16, "one")]
 
 
 @pytest.mark.parametrize("T,E,k,mode", PERM_CASES)
@@ -116,8 +118,9 @@ def test_permute_bitexact(T, E, k, mode):
     assert np.array_equal(row_of.cpu().numpy(), rr)
 
 
-def test_permute_bad_index_reports_status():
-    T, E, k = 300, 16, 4
+@pytest.mark.parametrize("T", [300, 250])
+def test_permute_bad_index_reports_status(T):
+    E, k = 16, 4
     rng = np.random.default_rng(5)
     idx = _rand_idx(rng, T, E, k)
     idx[7, 2] = E + 5          # out of range
