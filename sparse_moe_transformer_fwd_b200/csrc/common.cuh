@@ -40,6 +40,22 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
     return r;
 }
 
+// UE8M0 tile scale (power-of-two variant of the block quantisation): the
+// least 2^k, k >= -127, with amax / 2^k <= 448.  amax = m * 2^(E-127) with
+// m = 1.f in [1, 2) from its bits (normal) and 448 = 1.75 * 2^8, so
+// k = E - 127 - 8 + (m > 1.75); subnormal amax (below 2^-126) always takes
+// k = -127.  Returns 2^k (binary32, 2^-127 being subnormal) and sets
+// *inv = 2^-k; multiplying by inv is exact.  amax must be > 0.
+__device__ __forceinline__ float ue8m0_scale(float amax, float *inv) {
+    const uint32_t b = __float_as_uint(amax);
+    const int e = static_cast<int>(b >> 23);
+    int k = -127;
+    if (e > 0) k = max(e - 135 + ((b & 0x7fffffu) > 0x600000u ? 1 : 0), -127);
+    *inv = __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
+    return k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23)
+                     : __uint_as_float(1u << 22);
+}
+
 // Pre-norm of one element: bf16((h * rstd) * gamma) widened back to binary32.
 __device__ __forceinline__ float prenorm_elem(float h, float rstd, float gamma) {
     const float v = __fmul_rn(__fmul_rn(h, rstd), gamma);
@@ -194,6 +210,16 @@ __device__ __forceinline__ void tmem_wait_ld(float (&v)[32]) {
           "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
           "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
           "+r"(r[31])
+        :
+        : "memory");
+}
+
+// Same for two arrays loaded by two tcgen05.ld still in flight.
+__device__ __forceinline__ void tmem_wait_ld(float (&va)[32], float (&vb)[32]) {
+    uint32_t *a = reinterpret_cast<uint32_t *>(va), *b = reinterpret_cast<uint32_t *>(vb);
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]), "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]), "+r"(a[16]), "+r"(a[17]), "+r"(a[18]), "+r"(a[19]), "+r"(a[20]), "+r"(a[21]), "+r"(a[22]), "+r"(a[23]), "+r"(a[24]), "+r"(a[25]), "+r"(a[26]), "+r"(a[27]), "+r"(a[28]), "+r"(a[29]), "+r"(a[30]), "+r"(a[31]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15]), "+r"(b[16]), "+r"(b[17]), "+r"(b[18]), "+r"(b[19]), "+r"(b[20]), "+r"(b[21]), "+r"(b[22]), "+r"(b[23]), "+r"(b[24]), "+r"(b[25]), "+r"(b[26]), "+r"(b[27]), "+r"(b[28]), "+r"(b[29]), "+r"(b[30]), "+r"(b[31])
         :
         : "memory");
 }

@@ -344,27 +344,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     break;
                 }
                 tc_fence_after();
+                // four 32-column pieces, two loads in flight at a time; the
+                // buffer is released as soon as the last piece is in registers
+                // (before its FMAs), since the MMA two chunks ahead waits for it
+                float va[32], vb[32];
                 if (warp_active) {
-                    // four 32-column pieces; the load of piece j+1 is in flight
-                    // while the FMAs of piece j issue
                     const uint32_t base = lane_base + tb * BN;
-                    float va[32], vb[32];
                     tmem_ld32(base + col_lo, va);
-                    tmem_wait_ld(va);
                     tmem_ld32(base + col_lo + 32, vb);
+                    tmem_wait_ld(va, vb);
                     promote32<FP8>(acc2, 0, va, sc_lo);
-                    tmem_wait_ld(vb);
                     tmem_ld32(base + col_hi, va);
                     promote32<FP8>(acc2, 16, vb, sc_lo);
-                    tmem_wait_ld(va);
                     tmem_ld32(base + col_hi + 32, vb);
-                    promote32<FP8>(acc2, 32, va, sc_hi);
-                    tmem_wait_ld(vb);
-                    promote32<FP8>(acc2, 48, vb, sc_hi);
+                    tmem_wait_ld(va, vb);
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.tempty[tb]);
+                if (warp_active) {
+                    promote32<FP8>(acc2, 32, va, sc_hi);
+                    promote32<FP8>(acc2, 48, vb, sc_hi);
+                }
                 tb ^= 1;
                 if (tb == 0) tphase ^= 1;
             }

@@ -268,19 +268,35 @@ router_scores_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__res
         }
         __syncwarp();
         const uint16_t *wr = ws + lane * RS_WLD;
-#pragma unroll 4
-        for (int kk = 0; kk < RS_KC; kk += 8) {
-            const uint4 wv = *reinterpret_cast<const uint4 *>(wr + kk);
-            const float4 xa = *reinterpret_cast<const float4 *>(xw + kk);
-            const float4 xb = *reinterpret_cast<const float4 *>(xw + kk + 4);
-            acc = __fmaf_rn(xa.x, bf16_lo(wv.x), acc);
-            acc = __fmaf_rn(xa.y, bf16_hi(wv.x), acc);
-            acc = __fmaf_rn(xa.z, bf16_lo(wv.y), acc);
-            acc = __fmaf_rn(xa.w, bf16_hi(wv.y), acc);
-            acc = __fmaf_rn(xb.x, bf16_lo(wv.z), acc);
-            acc = __fmaf_rn(xb.y, bf16_hi(wv.z), acc);
-            acc = __fmaf_rn(xb.z, bf16_lo(wv.w), acc);
-            acc = __fmaf_rn(xb.w, bf16_hi(wv.w), acc);
+        // operands are read two 8-column groups ahead of the FMAs that use
+        // them (a 3-slot register ring, fully unrolled), so only the FMA
+        // chain itself is on the critical path
+        constexpr int NG = RS_KC / 8, PD = 2;
+        uint4 wv[PD + 1];
+        float4 xa[PD + 1], xb[PD + 1];
+#pragma unroll
+        for (int g = 0; g < PD; ++g) {
+            wv[g] = *reinterpret_cast<const uint4 *>(wr + 8 * g);
+            xa[g] = *reinterpret_cast<const float4 *>(xw + 8 * g);
+            xb[g] = *reinterpret_cast<const float4 *>(xw + 8 * g + 4);
+        }
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            if (g + PD < NG) {
+                const int sl = (g + PD) % (PD + 1);
+                wv[sl] = *reinterpret_cast<const uint4 *>(wr + 8 * (g + PD));
+                xa[sl] = *reinterpret_cast<const float4 *>(xw + 8 * (g + PD));
+                xb[sl] = *reinterpret_cast<const float4 *>(xw + 8 * (g + PD) + 4);
+            }
+            const int c = g % (PD + 1);
+            acc = __fmaf_rn(xa[c].x, bf16_lo(wv[c].x), acc);
+            acc = __fmaf_rn(xa[c].y, bf16_hi(wv[c].x), acc);
+            acc = __fmaf_rn(xa[c].z, bf16_lo(wv[c].y), acc);
+            acc = __fmaf_rn(xa[c].w, bf16_hi(wv[c].y), acc);
+            acc = __fmaf_rn(xb[c].x, bf16_lo(wv[c].z), acc);
+            acc = __fmaf_rn(xb[c].y, bf16_hi(wv[c].z), acc);
+            acc = __fmaf_rn(xb[c].z, bf16_lo(wv[c].w), acc);
+            acc = __fmaf_rn(xb[c].w, bf16_hi(wv[c].w), acc);
         }
         __syncwarp();  // xw is rewritten next chunk
     }
