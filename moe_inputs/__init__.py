@@ -45,7 +45,7 @@ class MoEConfig:
     top_k: int
     d_expert: int
     n_shared: int       # 0 or 1 shared experts (width d_expert)
-    precision: str      # "bf16" or "fp8"
+    precision: str      # "bf16", "fp8" (FP32 block scales) or "fp8_ue8m0" (power-of-two scales)
     w_std: float        # std of expert weights
     wr_std: float       # std of router weights
     bias: str           # "uniform" (U(-0.1, 0.1)), "zero", or "zipf"

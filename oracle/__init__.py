@@ -76,6 +76,9 @@ def lib():
         L.oracle_sigmoid.restype = ctypes.c_float
         L.oracle_block_quant.argtypes = [f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, f32p]
         L.oracle_block_quant.restype = None
+        L.oracle_block_quant_ue8m0.argtypes = [f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p,
+                                               f32p]
+        L.oracle_block_quant_ue8m0.restype = None
         L.oracle_router_logits.argtypes = [u16p, u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int, f32p]
         L.oracle_router_logits.restype = None
         L.oracle_route.argtypes = [f32p, f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -190,8 +193,9 @@ def permute(idx, n_experts: int):
 
 # ------------------------------------------------------------ quantisation --
 
-def block_quant(a, block_rows: int):
+def block_quant(a, block_rows: int, ue8m0: bool = False):
     """e4m3 block quantisation of a [rows, cols] matrix (float32 or bf16 bits).
+    ue8m0: power-of-two scales (the UE8M0 variant), else amax / 448.
 
     -> (codes uint8 [rows, cols], scales fp32 [ceil(rows/block_rows), cols/128])"""
     a = np.asarray(a)
@@ -203,8 +207,9 @@ def block_quant(a, block_rows: int):
         raise ValueError("cols must be a multiple of 128")
     q = np.empty((rows, cols), dtype=np.uint8)
     s = np.empty(((rows + block_rows - 1) // block_rows, cols // 128), dtype=np.float32)
-    lib().oracle_block_quant(_p(a, ctypes.c_float), rows, cols, block_rows,
-                             _p(q, ctypes.c_uint8), _p(s, ctypes.c_float))
+    fn = lib().oracle_block_quant_ue8m0 if ue8m0 else lib().oracle_block_quant
+    fn(_p(a, ctypes.c_float), rows, cols, block_rows, _p(q, ctypes.c_uint8),
+       _p(s, ctypes.c_float))
     return q, s
 
 
@@ -241,6 +246,7 @@ def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=No
     bf16:  a_rows uint16 [n, d], w13 uint16 [2*de, d], w2 uint16 [d, de].
     fp8:   a_rows uint8 codes + a_scales [n, d/128]; w13 codes + w13_scales
            [2*de/128, d/128]; w2 codes + w2_scales [d/128, de/128].
+    fp8_ue8m0: as fp8, every scale a power of two; H is requantised the same way.
     -> Y as bf16 bits [n, d] (and H: bf16 bits, or (codes, scales) for fp8)."""
     n = a_rows.shape[0]
     if precision == "bf16":
@@ -254,7 +260,7 @@ def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=No
         Y = bf16_to_f32(H).astype(np.float64) @ W2.T
         y = _bf16_of_f64(Y)
         return (y, H) if return_h else y
-    if precision == "fp8":
+    if precision in ("fp8", "fp8_ue8m0"):
         A = dequant(a_rows, a_scales, 1)
         W13 = dequant(w13, w13_scales, 128)
         W2 = dequant(w2, w2_scales, 128)
@@ -262,7 +268,7 @@ def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=No
         G = A @ W13[:de].T
         U = A @ W13[de:].T
         H = _silu_mul(G, U).astype(np.float32)
-        hq, hs = block_quant(H, 1)
+        hq, hs = block_quant(H, 1, ue8m0=precision == "fp8_ue8m0")
         Y = dequant(hq, hs, 1) @ W2.T
         y = _bf16_of_f64(Y)
         return (y, (hq, hs)) if return_h else y
@@ -292,8 +298,10 @@ def moe_layer(x, w_router, bias, expert, *, n_experts: int, top_k: int, n_shared
     counts, offsets, row_token, row_of = permute(idx, E)
     res = dict(logits=logits, scores=scores, idx=idx, gates=gates, counts=counts,
                offsets=offsets, row_token=row_token, row_of=row_of)
-    if precision == "fp8":
-        xq, xs = block_quant(x, 1)
+    fp8 = precision in ("fp8", "fp8_ue8m0")
+    ue = precision == "fp8_ue8m0"
+    if fp8:
+        xq, xs = block_quant(x, 1, ue8m0=ue)
         res.update(xq=xq, xs=xs)
     tokens = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
     # rows needed per expert: (expert, token) pairs of the evaluated tokens
@@ -308,10 +316,11 @@ def moe_layer(x, w_router, bias, expert, *, n_experts: int, top_k: int, n_shared
         w13, w2 = expert(e)
         pairs = need[e]
         rows = np.array([tokens[ti] for ti, _ in pairs])
-        if precision == "fp8":
-            w13q, w13s = block_quant(w13, 128)
-            w2q, w2s = block_quant(w2, 128)
-            y = expert_forward(res["xq"][rows], w13q, w2q, "fp8", res["xs"][rows], w13s, w2s)
+        if fp8:
+            w13q, w13s = block_quant(w13, 128, ue8m0=ue)
+            w2q, w2s = block_quant(w2, 128, ue8m0=ue)
+            y = expert_forward(res["xq"][rows], w13q, w2q, precision, res["xs"][rows], w13s,
+                               w2s)
         else:
             y = expert_forward(x[rows], w13, w2, "bf16")
         yf = bf16_to_f32(y).astype(np.float64)

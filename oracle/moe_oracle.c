@@ -132,6 +132,49 @@ void oracle_block_quant(const float *in, int rows, int cols, int block_rows,
     }
 }
 
+/*
+ * UE8M0 variant: the same tiles with power-of-two scales (an 8-bit exponent
+ * per tile, no mantissa).  The scale is rounded up to a power of two, so per
+ * tile scale = 2^k with k the least integer such that amax / 2^k <= 448.
+ * With amax = f * 2^E (frexp: f in [0.5, 1), exact) and 448 = 0.875 * 2^9,
+ * k = E - 9 when f <= 0.875 and E - 8 otherwise.  UE8M0 holds 2^-127 ..
+ * 2^127, so k is raised to -127 for tiles with amax < 448 * 2^-128 (bf16
+ * inputs never need k > 120).  q = e4m3(v * 2^-k): the power-of-two multiply
+ * is exact, so each code is the nearest e4m3 value (ties to even) of the
+ * exact quotient, and none saturates.  Zero tile: scale 1 (2^0), +0 codes.
+ */
+void oracle_block_quant_ue8m0(const float *in, int rows, int cols, int block_rows,
+                              uint8_t *q, float *scales)
+{
+    int nkb = cols / 128;
+    int nrb = (rows + block_rows - 1) / block_rows;
+    for (int rb = 0; rb < nrb; ++rb) {
+        int r0 = rb * block_rows;
+        int r1 = r0 + block_rows < rows ? r0 + block_rows : rows;
+        for (int kb = 0; kb < nkb; ++kb) {
+            float amax = 0.0f;
+            for (int r = r0; r < r1; ++r)
+                for (int c = kb * 128; c < kb * 128 + 128; ++c) {
+                    float a = fabsf(in[(size_t)r * cols + c]);
+                    if (a > amax) amax = a;
+                }
+            int k = 0;
+            if (amax != 0.0f) {
+                int E;
+                float f = frexpf(amax, &E);
+                k = f > 0.875f ? E - 8 : E - 9;
+                if (k < -127) k = -127;
+            }
+            scales[(size_t)rb * nkb + kb] = ldexpf(1.0f, k);
+            for (int r = r0; r < r1; ++r)
+                for (int c = kb * 128; c < kb * 128 + 128; ++c) {
+                    size_t i = (size_t)r * cols + c;
+                    q[i] = amax == 0.0f ? 0 : oracle_e4m3_encode(ldexpf(in[i], -k));
+                }
+        }
+    }
+}
+
 /* Same quantiser on bf16 storage. */
 void oracle_block_quant_bf16(const uint16_t *in, int rows, int cols, int block_rows,
                              uint8_t *q, float *scales)
