@@ -180,7 +180,7 @@ def algorithmic_bytes_gemm1(cfg, touched: int) -> float:
     expert (and the shared one), their scales, the permuted activations and
     scales in, H and its scales out."""
     d, de, Rs = cfg.d_model, cfg.d_expert, cfg.R_s
-    es = 1 if cfg.precision == "fp8" else 2
+    es = 2 if cfg.precision == "bf16" else 1
     w = touched * (2 * de * d * es + (4 * (2 * de // 128) * (d // 128) if es == 1 else 0))
     a = Rs * d * es + (Rs * (d // 128) * 4 if es == 1 else 0)
     h = Rs * de * es + (Rs * (de // 128) * 4 if es == 1 else 0)
@@ -298,14 +298,15 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e4m3" if cfg.precision == "fp8" else "bf16",
+        "dtype": "bf16" if cfg.precision == "bf16" else "e4m3",
         "data": "synthetic (seeded; random-init weights of the DeepSeek-V3 MoE layer shape)",
         "config": {
             "workload": ("pre-norm block (h + MoE(RMSNorm(h)), fused) " if args.prenorm else "")
                         + f"{cfg.name}: T={T}, d_model={cfg.d_model}, {cfg.n_experts} experts "
                         f"top-{cfg.top_k} + {cfg.n_shared} shared, d_expert={cfg.d_expert}, "
-                        + ("e4m3 1x128/128x128 blockwise, bf16 I/O" if cfg.precision == "fp8"
-                           else "bf16"),
+                        + ({"fp8": "e4m3 1x128/128x128 blockwise, fp32 scales, bf16 I/O",
+                            "fp8_ue8m0": "e4m3 1x128/128x128 blockwise, power-of-two (UE8M0) "
+                                         "scales, bf16 I/O"}.get(cfg.precision, "bf16")),
             "tokens_per_gpu": T,
             "parallelism": "replicas" if world > 1 else "single GPU",
             "l2": f"inputs larger than L2: {touched} touched experts' weights "

@@ -63,7 +63,9 @@ enum moe_status {
 
 enum moe_precision {
     MOE_BF16 = 0,      /* bf16 weights and activations, binary32 accumulate */
-    MOE_FP8_BLOCK = 1  /* e4m3 1x128 activations, 128x128 weights, fp32 scales */
+    MOE_FP8_BLOCK = 1, /* e4m3 1x128 activations, 128x128 weights, fp32 scales */
+    MOE_FP8_UE8M0 = 2  /* as MOE_FP8_BLOCK with power-of-two scales (UE8M0 values
+                          stored as fp32); see fp8_block_quant_ue8m0 */
 };
 
 /* Weight storage.  The expert GEMMs read their weights in TILED layout: a
@@ -158,6 +160,16 @@ int moe_permute(const moe_shape *shape, const int32_t *topk_idx, int32_t *counts
 int fp8_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
                     int out_layout, uint8_t *q, float *scales, void *stream);
 
+/* The same quantisation with power-of-two scales (the UE8M0 variant used by
+ * MOE_FP8_UE8M0; the pages give blockwise FP8 with per-block scales, the
+ * power-of-two rounding is this library's reading of the variant): per tile
+ * scale = 2^k for the least integer k >= -127 with amax / 2^k <= 448 (an
+ * all-zero tile: 2^0), codes = e4m3_rn(v * 2^-k), the multiply being exact
+ * and never saturating.  Arguments, layouts and errors as fp8_block_quant;
+ * the scales are written as fp32 values (each exactly 2^k). */
+int fp8_block_quant_ue8m0(const uint16_t *in, int rows, int cols, int ld, int block_rows,
+                          int out_layout, uint8_t *q, float *scales, void *stream);
+
 /* Repacks a row-major matrix of `rows` rows x `row_bytes` bytes (both
  * multiples of 128; src and dst 16-byte aligned, not overlapping) into the
  * tiled layout (MOE_LAYOUT_TILED).  Used once, ahead of time, for bf16
@@ -168,8 +180,8 @@ int moe_pack_tiles(const void *src, int rows, int row_bytes, void *dst, void *st
  * MLPs"): for every segment s (routed experts 0..E-1, then the shared expert
  * at slot E when n_shared = 1)  H = silu(A_s W_gate,s^T) * (A_s W_up,s^T),
  * Y_s = H W_down,s^T.  R_s = T*k + T*n_shared rows.
- *   a          [R_s, d_model] bf16, or e4m3 codes in MOE_FP8_BLOCK
- *   a_scales   fp32 [R_s, d_model/128] (MOE_FP8_BLOCK) or NULL
+ *   a          [R_s, d_model] bf16, or e4m3 codes in MOE_FP8_BLOCK / _UE8M0
+ *   a_scales   fp32 [R_s, d_model/128] (fp8 precisions) or NULL
  *   offsets    int32 [n_experts + 1] segment starts (as from moe_permute)
  *   w13        [E + n_shared, 2*d_expert, d_model]: gate rows, then up rows,
  *              e4m3 or bf16, in MOE_LAYOUT_TILED
@@ -177,8 +189,9 @@ int moe_pack_tiles(const void *src, int rows, int row_bytes, void *dst, void *st
  *   w2         [E + n_shared, d_model, d_expert], MOE_LAYOUT_TILED
  *   w2_scales  fp32 [E + n_shared, d_model/128, d_expert/128] or NULL
  *   y          bf16 [R_s, d_model] out
- * In MOE_FP8_BLOCK, H is quantised 1x128 (e4m3) before the down GEMM; in
- * MOE_BF16 it is rounded to bf16.  Accumulation is binary32. */
+ * In MOE_FP8_BLOCK, H is quantised 1x128 (e4m3) before the down GEMM (with
+ * power-of-two scales in MOE_FP8_UE8M0); in MOE_BF16 it is rounded to bf16.
+ * Accumulation is binary32. */
 int moe_grouped_swiglu(const moe_shape *shape, const void *a, const float *a_scales,
                        const int32_t *offsets, const void *w13, const float *w13_scales,
                        const void *w2, const float *w2_scales, uint16_t *y,
@@ -198,7 +211,8 @@ int moe_combine(const moe_shape *shape, const uint16_t *y, const int32_t *row_of
  *   x [T, d_model] bf16 in; out [T, d_model] bf16 out.
  *   w13/w2 and scales as for moe_grouped_swiglu (tiled; weights are quantised
  *   once, ahead of time, with fp8_block_quant(..., MOE_LAYOUT_TILED, ...) in
- *   MOE_FP8_BLOCK, or repacked with moe_pack_tiles in MOE_BF16).
+ *   MOE_FP8_BLOCK, fp8_block_quant_ue8m0 in MOE_FP8_UE8M0, or repacked with
+ *   moe_pack_tiles in MOE_BF16).
  *   topk_idx_out int32 [T, k] or NULL: receives the routing decision. */
 int moe_forward(const moe_shape *shape, const uint16_t *x, const uint16_t *w_router,
                 const float *bias, const void *w13, const float *w13_scales,

@@ -81,6 +81,9 @@ CONFIGS = {
     "prefill": MoEConfig("prefill", T=4096, precision="fp8", bias="zero", **_DS),
     "skew": MoEConfig("skew", T=16384, precision="fp8", bias="zipf", **_DS),
     "bf16": MoEConfig("bf16", T=8192, precision="bf16", bias="zero", **_DS),
+    # the decode and prefill batches with the UE8M0 (power-of-two) block scales
+    "decode_ue8m0": MoEConfig("decode_ue8m0", T=64, precision="fp8_ue8m0", bias="uniform", **_DS),
+    "prefill_ue8m0": MoEConfig("prefill_ue8m0", T=4096, precision="fp8_ue8m0", bias="zero", **_DS),
     # profiling-size stand-in for the decode batch: same per-expert shapes,
     # 32 routed experts, so every buffer is a few GB at most
     "decode_small": MoEConfig("decode_small", T=64, precision="fp8", bias="uniform",

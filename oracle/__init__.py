@@ -239,15 +239,70 @@ def _bf16_of_f64(v) -> np.ndarray:
     return bf16_from_f32(np.asarray(v, dtype=np.float64).astype(np.float32))
 
 
+# Two correct evaluations of G and U differ in their accumulation order, so an
+# element of H whose e4m3 quantiser input lies at a rounding boundary may take
+# either neighbouring code (and, with power-of-two scales, a tile whose amax
+# lies at 448 * 2^k either of two scales).  The oracle reports, per output,
+# how far such alternative codes could move it; H_FLIP_RHO is the relative
+# perturbation of the quantiser input considered.
+H_FLIP_RHO = 2.0 ** -14
+
+
+def _ue8m0_exponent(amax):
+    m, e = np.frexp(np.asarray(amax, dtype=np.float64))
+    return np.maximum(np.where(m > 0.875, e - 8, e - 9), -127)
+
+
+def h_code_ambiguity(H, hq, hs, ue8m0: bool, rho: float = H_FLIP_RHO) -> np.ndarray:
+    """[n, de] binary64: per element of the fp32 H, the largest change of its
+    dequantised value that a relative perturbation of at most rho of its
+    quantiser input could cause (0 unless the input lies within rho of an
+    e4m3 rounding boundary); with power-of-two scales also the change when a
+    tile's amax lies within rho of a scale boundary and the scale doubles or
+    halves."""
+    global _DEC
+    if _DEC is None:
+        _DEC = e4m3_decode_table()
+    H = np.ascontiguousarray(H, dtype=np.float32)
+    n, de = H.shape
+    base = dequant(hq, hs, 1)
+    sc = np.repeat(np.asarray(hs, dtype=np.float64), 128, axis=1)
+    amax = np.abs(H).reshape(n, de // 128, 128).max(2)
+    if ue8m0:
+        x = (H.astype(np.float64) / sc).astype(np.float32)          # exact
+    else:
+        with np.errstate(divide="ignore"):
+            inv = np.where(amax > 0, np.float32(448.0) / amax, np.float32(0.0)).astype(np.float32)
+        x = H * np.repeat(inv, 128, axis=1)                          # binary32, as quantised
+    delta = np.zeros((n, de))
+    for f in (1.0 + rho, 1.0 - rho):
+        q = e4m3_encode(x.astype(np.float64) * f)
+        delta = np.maximum(delta, np.abs(_DEC[q] * sc - base))
+    if ue8m0:
+        k = _ue8m0_exponent(amax)
+        for f in (1.0 + rho, 1.0 - rho):
+            ka = _ue8m0_exponent(amax * f)
+            alt = (ka != k) & (amax > 0)
+            if alt.any():
+                s_alt = np.repeat(np.ldexp(1.0, ka), 128, axis=1)
+                q = e4m3_encode(H.astype(np.float64) / s_alt)
+                d = np.abs(_DEC[q] * s_alt - base)
+                delta = np.where(np.repeat(alt, 128, axis=1), np.maximum(delta, d), delta)
+    return delta
+
+
 def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=None,
-                   w2_scales=None, return_h: bool = False):
+                   w2_scales=None, return_h: bool = False, return_allow: bool = False):
     """One gated expert on a block of rows.
 
     bf16:  a_rows uint16 [n, d], w13 uint16 [2*de, d], w2 uint16 [d, de].
     fp8:   a_rows uint8 codes + a_scales [n, d/128]; w13 codes + w13_scales
            [2*de/128, d/128]; w2 codes + w2_scales [d/128, de/128].
     fp8_ue8m0: as fp8, every scale a power of two; H is requantised the same way.
-    -> Y as bf16 bits [n, d] (and H: bf16 bits, or (codes, scales) for fp8)."""
+    -> Y as bf16 bits [n, d] (and H: bf16 bits, or (codes, scales) for fp8;
+    return_allow: and [n, d] binary64, how far alternative H codes at e4m3
+    rounding boundaries could move Y: sum_i h_code_ambiguity_i * |W2[:, i]|;
+    zero for bf16)."""
     n = a_rows.shape[0]
     if precision == "bf16":
         A = bf16_to_f32(a_rows).astype(np.float64)
@@ -259,6 +314,8 @@ def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=No
         H = _bf16_of_f64(_silu_mul(G, U))
         Y = bf16_to_f32(H).astype(np.float64) @ W2.T
         y = _bf16_of_f64(Y)
+        if return_allow:
+            return y, np.zeros(Y.shape)
         return (y, H) if return_h else y
     if precision in ("fp8", "fp8_ue8m0"):
         A = dequant(a_rows, a_scales, 1)
@@ -268,9 +325,12 @@ def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=No
         G = A @ W13[:de].T
         U = A @ W13[de:].T
         H = _silu_mul(G, U).astype(np.float32)
-        hq, hs = block_quant(H, 1, ue8m0=precision == "fp8_ue8m0")
+        ue = precision == "fp8_ue8m0"
+        hq, hs = block_quant(H, 1, ue8m0=ue)
         Y = dequant(hq, hs, 1) @ W2.T
         y = _bf16_of_f64(Y)
+        if return_allow:
+            return y, h_code_ambiguity(H, hq, hs, ue) @ np.abs(W2).T
         return (y, (hq, hs)) if return_h else y
     raise ValueError(precision)
 
@@ -312,6 +372,7 @@ def moe_layer(x, w_router, bias, expert, *, n_experts: int, top_k: int, n_shared
         if n_shared:
             need.setdefault(E, []).append((ti, k))
     Yt = np.zeros((len(tokens), k + 1, d), dtype=np.float64)
+    At = np.zeros((len(tokens), k + 1, d), dtype=np.float64)
     for e in sorted(need):
         w13, w2 = expert(e)
         pairs = need[e]
@@ -319,19 +380,24 @@ def moe_layer(x, w_router, bias, expert, *, n_experts: int, top_k: int, n_shared
         if fp8:
             w13q, w13s = block_quant(w13, 128, ue8m0=ue)
             w2q, w2s = block_quant(w2, 128, ue8m0=ue)
-            y = expert_forward(res["xq"][rows], w13q, w2q, precision, res["xs"][rows], w13s,
-                               w2s)
+            y, al = expert_forward(res["xq"][rows], w13q, w2q, precision, res["xs"][rows],
+                                   w13s, w2s, return_allow=True)
         else:
-            y = expert_forward(x[rows], w13, w2, "bf16")
+            y, al = expert_forward(x[rows], w13, w2, "bf16", return_allow=True)
         yf = bf16_to_f32(y).astype(np.float64)
         for n, (ti, j) in enumerate(pairs):
             Yt[ti, j] = yf[n]
+            At[ti, j] = al[n]
     g = gates[tokens].astype(np.float64)
     acc = np.einsum("tj,tjd->td", g, Yt[:, :k])
+    allow = np.einsum("tj,tjd->td", np.abs(g), At[:, :k])
     if n_shared:
         acc = acc + Yt[:, k]
+        allow = allow + At[:, k]
     res["out"] = _bf16_of_f64(acc)
     res["out_f64"] = acc
+    # how far alternative H codes at e4m3 rounding boundaries could move out
+    res["out_allow"] = allow
     res["tokens"] = tokens
     return res
 

@@ -12,7 +12,7 @@ from __future__ import annotations
 
 import torch
 
-from ._native import (EXPORTS, MOE_BF16, MOE_FP8_BLOCK, MOE_LAYOUT_ROWMAJOR, MOE_LAYOUT_TILED,
+from ._native import (EXPORTS, MOE_BF16, MOE_FP8_BLOCK, MOE_FP8_UE8M0, MOE_LAYOUT_ROWMAJOR, MOE_LAYOUT_TILED,
                       MoeError, moe_pack_tiles, moe_forward_prenorm, MoeShape, alloc_workspace,
                       fp8_block_quant, lib, make_shape, moe_check_status, moe_combine,
                       moe_forward, moe_grouped_swiglu, moe_last_error, moe_last_launch_count,
@@ -24,24 +24,24 @@ __all__ = [
     "MoELayer", "MoeError", "MoeShape", "make_shape", "alloc_workspace", "lib", "EXPORTS",
     "moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
     "moe_combine", "moe_forward", "moe_check_status", "moe_last_error", "moe_last_launch_count",
-    "quantize_weights", "MOE_BF16", "MOE_FP8_BLOCK", "moe_set_kernel_events",
+    "quantize_weights", "MOE_BF16", "MOE_FP8_BLOCK", "MOE_FP8_UE8M0", "moe_set_kernel_events",
     "moe_route_noalloc", "MOE_ROUTE_NOALLOC_MAX_SCORES", "moe_pack_tiles", "pack_weights",
     "MOE_LAYOUT_ROWMAJOR", "MOE_LAYOUT_TILED", "moe_forward_prenorm", "moe_last_launch_names",
 ]
 
 
-def quantize_weights(w13: torch.Tensor, w2: torch.Tensor, stream=None):
+def quantize_weights(w13: torch.Tensor, w2: torch.Tensor, stream=None, ue8m0: bool = False):
     """128x128 e4m3 block quantisation of the stacked expert weights (done
     once, ahead of the forward passes), codes in the tiled layout the GEMMs
-    read.  Returns (w13q, w13s, w2q, w2s)."""
+    read; ue8m0: power-of-two scales.  Returns (w13q, w13s, w2q, w2s)."""
     S, n13, d = w13.shape
     _, d2, de = w2.shape
     w13q = torch.empty(S, n13, d, dtype=torch.uint8, device=w13.device)
     w13s = torch.empty(S, n13 // 128, d // 128, dtype=torch.float32, device=w13.device)
     w2q = torch.empty(S, d2, de, dtype=torch.uint8, device=w2.device)
     w2s = torch.empty(S, d2 // 128, de // 128, dtype=torch.float32, device=w2.device)
-    fp8_block_quant(w13, 128, w13q, w13s, layout=MOE_LAYOUT_TILED, stream=stream)
-    fp8_block_quant(w2, 128, w2q, w2s, layout=MOE_LAYOUT_TILED, stream=stream)
+    fp8_block_quant(w13, 128, w13q, w13s, layout=MOE_LAYOUT_TILED, stream=stream, ue8m0=ue8m0)
+    fp8_block_quant(w2, 128, w2q, w2s, layout=MOE_LAYOUT_TILED, stream=stream, ue8m0=ue8m0)
     return w13q, w13s, w2q, w2s
 
 
@@ -58,8 +58,10 @@ class MoELayer:
 
     w_router bf16 [E, d]; bias fp32 [E]; w13 bf16 [E + n_shared, 2*d_expert, d]
     (gate rows then up rows); w2 bf16 [E + n_shared, d, d_expert]; the shared
-    expert, if any, is the last slot.  precision "fp8" quantises the expert
-    weights once at construction (the bf16 copies are then not needed)."""
+    expert, if any, is the last slot.  precision "fp8" (fp32 block scales) or
+    "fp8_ue8m0" (power-of-two block scales) quantises the expert weights once
+    at construction (the bf16 copies are then not needed); "bf16" repacks
+    them."""
 
     def __init__(self, w_router, bias, w13, w2, *, top_k: int, n_shared: int = 1,
                  routed_scale: float = 1.0, precision: str = "fp8", keep_bf16: bool = False):
@@ -69,9 +71,9 @@ class MoELayer:
         self.top_k, self.n_shared, self.routed_scale = top_k, n_shared, routed_scale
         self.precision = precision
         self.w_router, self.bias = w_router.contiguous(), bias.contiguous()
-        if precision == "fp8":
-            self.w13, self.w13s, self.w2, self.w2s = quantize_weights(w13.contiguous(),
-                                                                      w2.contiguous())
+        if precision in ("fp8", "fp8_ue8m0"):
+            self.w13, self.w13s, self.w2, self.w2s = quantize_weights(
+                w13.contiguous(), w2.contiguous(), ue8m0=precision == "fp8_ue8m0")
             self.w13_bf16 = w13 if keep_bf16 else None
             self.w2_bf16 = w2 if keep_bf16 else None
         elif precision == "bf16":

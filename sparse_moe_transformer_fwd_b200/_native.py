@@ -21,6 +21,7 @@ MOE_ERR_TIMEOUT = -5
 MOE_ERR_DEVICE_INDEX = -6
 MOE_BF16 = 0
 MOE_FP8_BLOCK = 1
+MOE_FP8_UE8M0 = 2
 MOE_LAYOUT_ROWMAJOR = 0
 MOE_LAYOUT_TILED = 1
 
@@ -28,7 +29,8 @@ MOE_LAYOUT_TILED = 1
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant",
            "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_check_status",
            "moe_last_error", "moe_last_launch_count", "moe_set_kernel_events",
-           "moe_route_noalloc", "moe_pack_tiles", "moe_forward_prenorm", "moe_last_launch_name")
+           "moe_route_noalloc", "moe_pack_tiles", "moe_forward_prenorm", "moe_last_launch_name",
+           "fp8_block_quant_ue8m0")
 
 # fixed score scratch of moe_route_noalloc, in floats (include/moe_fwd.h)
 MOE_ROUTE_NOALLOC_MAX_SCORES = 1 << 20
@@ -65,6 +67,7 @@ def lib() -> ctypes.CDLL:
         L.moe_permute.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_route_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp]
         L.fp8_block_quant.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp]
+        L.fp8_block_quant_ue8m0.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp]
         L.moe_pack_tiles.argtypes = [vp, ci, ci, vp, vp]
         L.moe_grouped_swiglu.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_combine.argtypes = [sp, vp, vp, vp, vp, vp]
@@ -77,7 +80,8 @@ def lib() -> ctypes.CDLL:
         L.moe_last_launch_name.argtypes = [ci]
         L.moe_last_launch_name.restype = ctypes.c_char_p
         L.moe_set_kernel_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ci]
-        for name in ("moe_route", "moe_route_noalloc", "moe_permute", "fp8_block_quant", "moe_grouped_swiglu",
+        for name in ("moe_route", "moe_route_noalloc", "moe_permute", "fp8_block_quant",
+                     "fp8_block_quant_ue8m0", "moe_grouped_swiglu",
                      "moe_combine", "moe_forward", "moe_check_status", "moe_last_launch_count",
                      "moe_set_kernel_events", "moe_pack_tiles", "moe_forward_prenorm"):
             getattr(L, name).restype = ci
@@ -112,7 +116,8 @@ def _stream(stream):
 
 def make_shape(T, d_model, n_experts, top_k, d_expert, n_shared=1, routed_scale=1.0,
                precision="fp8") -> MoeShape:
-    prec = {"bf16": MOE_BF16, "fp8": MOE_FP8_BLOCK}[precision] if isinstance(precision, str) \
+    prec = {"bf16": MOE_BF16, "fp8": MOE_FP8_BLOCK, "fp8_ue8m0": MOE_FP8_UE8M0}[precision] \
+        if isinstance(precision, str) \
         else int(precision)
     return MoeShape(int(T), int(d_model), int(n_experts), int(top_k), int(d_expert),
                     int(n_shared), float(routed_scale), prec)
@@ -162,15 +167,16 @@ def moe_permute(shape, topk_idx, counts, offsets, row_token, row_of, ws, stream=
 
 
 def fp8_block_quant(inp, block_rows, q, scales, rows=None, cols=None, ld=None,
-                    layout=MOE_LAYOUT_ROWMAJOR, stream=None):
+                    layout=MOE_LAYOUT_ROWMAJOR, stream=None, ue8m0=False):
     """e4m3 block quantisation of a bf16 matrix (2-D, or a stack flattened to
-    2-D); layout MOE_LAYOUT_TILED writes the codes in 128 x 128 tiles."""
+    2-D); layout MOE_LAYOUT_TILED writes the codes in 128 x 128 tiles;
+    ue8m0 selects power-of-two scales (fp8_block_quant_ue8m0)."""
     cols = inp.shape[-1] if cols is None else cols
     rows = inp.numel() // inp.shape[-1] if rows is None else rows
     ld = inp.shape[-1] if ld is None else ld
-    _check(lib().fp8_block_quant(_ptr(inp, _BF16, "in"), rows, cols, ld, block_rows, int(layout),
-                                 _ptr(q, _FP8, "q"), _ptr(scales, torch.float32, "scales"),
-                                 _stream(stream)))
+    fn = lib().fp8_block_quant_ue8m0 if ue8m0 else lib().fp8_block_quant
+    _check(fn(_ptr(inp, _BF16, "in"), rows, cols, ld, block_rows, int(layout),
+              _ptr(q, _FP8, "q"), _ptr(scales, torch.float32, "scales"), _stream(stream)))
 
 
 def moe_pack_tiles(src, dst, stream=None):
@@ -186,7 +192,7 @@ def moe_pack_tiles(src, dst, stream=None):
 
 def moe_grouped_swiglu(shape, a, a_scales, offsets, w13, w13_scales, w2, w2_scales, y, ws,
                        stream=None):
-    fp8 = shape.precision == MOE_FP8_BLOCK
+    fp8 = shape.precision in (MOE_FP8_BLOCK, MOE_FP8_UE8M0)
     wt = _FP8 if fp8 else _BF16
     _check(lib().moe_grouped_swiglu(
         ctypes.byref(shape), _ptr(a, wt, "a"), _ptr(a_scales, torch.float32, "a_scales"),
@@ -205,7 +211,7 @@ def moe_combine(shape, y, row_of, topk_w, out, stream=None):
 
 def moe_forward(shape, x, w_router, bias, w13, w13_scales, w2, w2_scales, out, ws,
                 topk_idx_out=None, stream=None):
-    fp8 = shape.precision == MOE_FP8_BLOCK
+    fp8 = shape.precision in (MOE_FP8_BLOCK, MOE_FP8_UE8M0)
     wt = _FP8 if fp8 else _BF16
     _check(lib().moe_forward(
         ctypes.byref(shape), _ptr(x, _BF16, "x"), _ptr(w_router, _BF16, "w_router"),
@@ -219,7 +225,7 @@ def moe_forward(shape, x, w_router, bias, w13, w13_scales, w2, w2_scales, out, w
 def moe_forward_prenorm(shape, h, gamma, eps, w_router, bias, w13, w13_scales, w2, w2_scales, out,
                         ws, topk_idx_out=None, stream=None):
     """out = h + MoE(bf16(RMSNorm(h) * gamma)); x is never materialised."""
-    fp8 = shape.precision == MOE_FP8_BLOCK
+    fp8 = shape.precision in (MOE_FP8_BLOCK, MOE_FP8_UE8M0)
     wt = _FP8 if fp8 else _BF16
     _check(lib().moe_forward_prenorm(
         ctypes.byref(shape), _ptr(h, _BF16, "h"), _ptr(gamma, _BF16, "gamma"), float(eps),

@@ -85,13 +85,20 @@ int check_shape(const moe_shape *s) {
                                          "n_experts + n_shared <= 1024");
     if (s->top_k < 1 || s->top_k > 32 || s->top_k > s->n_experts)
         return fail(MOE_ERR_INVALID_ARG, "need 1 <= top_k <= min(n_experts, 32)");
-    if (s->precision != MOE_BF16 && s->precision != MOE_FP8_BLOCK)
+    if (s->precision != MOE_BF16 && s->precision != MOE_FP8_BLOCK &&
+        s->precision != MOE_FP8_UE8M0)
         return fail(MOE_ERR_INVALID_ARG, "unknown precision %d", s->precision);
     const long long R_s = static_cast<long long>(s->T) * (s->top_k + s->n_shared);
     if (R_s * s->d_model > (1LL << 40) || R_s > (1LL << 30))
         return fail(MOE_ERR_INVALID_ARG, "T too large");
     return MOE_OK;
 }
+
+// e4m3 codes in either scale format (fp32 amax/448 or power-of-two UE8M0)
+bool is_fp8(const moe_shape *s) {
+    return s->precision == MOE_FP8_BLOCK || s->precision == MOE_FP8_UE8M0;
+}
+bool is_ue8m0(const moe_shape *s) { return s->precision == MOE_FP8_UE8M0; }
 
 // ---------------------------------------------------------- workspace ---
 struct Layout {
@@ -105,7 +112,7 @@ Layout layout(const moe_shape *s) {
     const size_t T = s->T, E = s->n_experts, k = s->top_k, d = s->d_model, de = s->d_expert;
     const size_t Rs = T * (k + s->n_shared);
     const size_t nblk = (T + 255) / 256;
-    const bool fp8 = s->precision == MOE_FP8_BLOCK;
+    const bool fp8 = is_fp8(s);
     const size_t es = fp8 ? 1 : 2;
     Layout L{};
     size_t off = 0;
@@ -185,7 +192,7 @@ PermScratch perm_scratch(void *ws, const Layout &L) {
 int grouped(const moe_shape *s, const void *a, const float *a_scales, const void *w13,
             const float *w13_scales, const void *w2, const float *w2_scales, uint16_t *y,
             void *ws, const Layout &L, cudaStream_t st, int *launches) {
-    const bool fp8 = s->precision == MOE_FP8_BLOCK;
+    const bool fp8 = is_fp8(s);
     const PermScratch ps = perm_scratch(ws, L);
     const int Rs = s->T * (s->top_k + s->n_shared);
     GemmArgs g{};
@@ -199,6 +206,7 @@ int grouped(const moe_shape *s, const void *a, const float *a_scales, const void
     g.tile_start = ps.tile_start;
     g.status = at<int>(ws, L.status);
     g.inject_fault = inject_gemm_fault() ? 1 : 0;
+    g.ue8m0 = is_ue8m0(s);
     // gate/up GEMM + SwiGLU
     g.gate_up = true;
     g.a = a;
@@ -229,7 +237,7 @@ int check_weights(const moe_shape *s, const void *w13, const float *w13s, const 
                   const float *w2s) {
     CHECK_PTR(w13);
     CHECK_PTR(w2);
-    if (s->precision == MOE_FP8_BLOCK) {
+    if (is_fp8(s)) {
         CHECK_PTR(w13s);
         CHECK_PTR(w2s);
     }
@@ -306,8 +314,8 @@ int moe_permute(const moe_shape *s, const int32_t *topk_idx, int32_t *counts, in
     return MOE_OK;
 }
 
-int fp8_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
-                    int out_layout, uint8_t *q, float *scales, void *stream) {
+static int block_quant_entry(const uint16_t *in, int rows, int cols, int ld, int block_rows,
+                      int out_layout, uint8_t *q, float *scales, void *stream, bool ue8m0) {
     if (rows < 0 || cols <= 0 || cols % 128 || ld < cols || ld % 8)
         return fail(MOE_ERR_INVALID_ARG, "need rows >= 0, cols a positive multiple of 128, "
                                          "ld >= cols, ld % 8 == 0");
@@ -324,11 +332,21 @@ int fp8_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_ro
     RETURN_IF(check_device());
     int n = 0;
     LAUNCH(launch_block_quant(in, rows, cols, ld, block_rows, out_layout == MOE_LAYOUT_TILED, q,
-                              scales, static_cast<cudaStream_t>(stream), &n),
+                              scales, static_cast<cudaStream_t>(stream), &n, ue8m0),
            "fp8_block_quant");
     mark_launch(static_cast<cudaStream_t>(stream), n);
     g_launches = n;
     return MOE_OK;
+}
+
+int fp8_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
+                    int out_layout, uint8_t *q, float *scales, void *stream) {
+    return block_quant_entry(in, rows, cols, ld, block_rows, out_layout, q, scales, stream, false);
+}
+
+int fp8_block_quant_ue8m0(const uint16_t *in, int rows, int cols, int ld, int block_rows,
+                          int out_layout, uint8_t *q, float *scales, void *stream) {
+    return block_quant_entry(in, rows, cols, ld, block_rows, out_layout, q, scales, stream, true);
 }
 
 int moe_pack_tiles(const void *src, int rows, int row_bytes, void *dst, void *stream) {
@@ -355,7 +373,7 @@ int moe_grouped_swiglu(const moe_shape *s, const void *a, const float *a_scales,
     RETURN_IF(check_ws(s, ws, ws_bytes, &L));
     if (s->T == 0) return g_launches = 0, MOE_OK;
     CHECK_PTR(a);
-    if (s->precision == MOE_FP8_BLOCK) CHECK_PTR(a_scales);
+    if (is_fp8(s)) CHECK_PTR(a_scales);
     CHECK_PTR(offsets);
     CHECK_PTR(y);
     RETURN_IF(check_weights(s, w13, w13_scales, w2, w2_scales));
@@ -414,7 +432,7 @@ int forward_impl(const moe_shape *s, const uint16_t *x, const uint16_t *gamma, f
     RETURN_IF(check_weights(s, w13, w13_scales, w2, w2_scales));
     RETURN_IF(check_device());
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool fp8 = s->precision == MOE_FP8_BLOCK;
+    const bool fp8 = is_fp8(s);
     int32_t *idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
     float *gates = at<float>(ws, L.gates);
     int32_t *row_of = at<int32_t>(ws, L.row_of);
@@ -435,7 +453,8 @@ int forward_impl(const moe_shape *s, const uint16_t *x, const uint16_t *gamma, f
            "permute");
     if (fp8)
         LAUNCH(launch_quant_scatter(x, s->T, s->d_model, s->top_k, s->n_shared, row_of,
-                                    at<uint8_t>(ws, L.a), at<float>(ws, L.a_scales), st, &n, pn),
+                                    at<uint8_t>(ws, L.a), at<float>(ws, L.a_scales), st, &n, pn,
+                                    is_ue8m0(s)),
                "quant_scatter");
     else
         LAUNCH(launch_scatter_bf16(x, s->T, s->d_model, s->top_k, s->n_shared, row_of,

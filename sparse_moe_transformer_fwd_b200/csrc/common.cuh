@@ -180,6 +180,32 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
             : "memory");
     }
 }
+// Block-scaled MMA (UE8M0 scale factors in TMEM, one per 32 K of each row of
+// A and of B): D[tmem] (+)= (A * 2^sfa) (B * 2^sfb)^T, e4m3 operands, one
+// CTA; the scale-factor id bits of idesc pick the byte of each TMEM column.
+__device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+        "r"(sfb_tmem)
+        : "memory");
+}
+// Shared -> TMEM copy of 32 rows x 128 bits (rows at 16-byte stride),
+// written to TMEM lanes 0-31 and repeated in the other three lane quadrants
+// (columns taddr .. taddr + 3).  Ordered with this thread's later MMAs.
+__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+// Makes this thread's generic-proxy shared-memory writes visible to the
+// async proxy (tcgen05.cp, TMA) once a barrier orders them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // 32 consecutive binary32 columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     uint32_t *r = reinterpret_cast<uint32_t *>(v);
@@ -235,6 +261,27 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t smem_addr) {
     d |= static_cast<uint64_t>(1) << 46;                             // descriptor version
     d |= static_cast<uint64_t>(2) << 61;                             // 128-byte swizzle
     return d;
+}
+
+// Shared-memory matrix descriptor without swizzle: core matrices of 8 rows x
+// 16 bytes stored contiguously (128 bytes), 8-row groups `sbo` bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t smem_addr, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3fff);
+    d |= static_cast<uint64_t>(128 >> 4) << 16;                     // leading byte offset
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3fff) << 32;          // stride byte offset
+    d |= static_cast<uint64_t>(1) << 46;                            // descriptor version
+    return d;                                                       // layout 0: no swizzle
+}
+
+// Instruction descriptor of the block-scaled MMA: e4m3 x e4m3, both K-major,
+// UE8M0 scale factors, dense K = 32, scale-factor ids 0 (byte 0 of each TMEM
+// column); the accumulator is fp32.
+__host__ __device__ constexpr uint32_t instr_desc_mx(int M, int N) {
+    return (0u << 7) | (0u << 10)                      // A, B: e4m3
+           | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+           | (1u << 23)                                // scale factors: UE8M0
+           | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
 // Instruction descriptor: dense, fp32 accumulator, both operands K-major.

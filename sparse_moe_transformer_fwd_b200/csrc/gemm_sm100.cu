@@ -34,7 +34,8 @@
 //   it back.
 // Epilogue: gate/up GEMM -> H = silu(G) * U, then (FP8) 1x128 e4m3
 //   quantisation of H (one 128-feature tile per row per work item; the two
-//   column halves exchange their amax through shared memory) or (BF16) bf16
+//   column halves exchange their amax through shared memory; power-of-two
+//   scales in the UE8M0 variant) or (BF16) bf16
 //   rounding; down GEMM -> Y in bf16.  Rows past the segment end are computed
 //   from neighbouring rows and never stored.
 // Every wait is bounded; on expiry the block records MOE_ERR_TIMEOUT, drains
@@ -56,17 +57,29 @@ constexpr int B_BYTES = BN * 128;        // 32 KB per stage
 constexpr int STAGE_TX = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 384;  // 3 warpgroups
 constexpr int LAUNCH_REGS = 168;   // 65536 / 384, multiple of 8
-constexpr int PRODUCER_REGS = 40;  // warpgroup 0 after setmaxnreg.dec
-constexpr int EPILOGUE_REGS = 232; // warpgroups 1-2 after setmaxnreg.inc
-static_assert(128 * PRODUCER_REGS + 256 * EPILOGUE_REGS <= NUM_THREADS * LAUNCH_REGS,
-              "register split must fit in the block's launch allocation");
 constexpr int EPI_THREADS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_SEG = 1025;
+constexpr int SF_BYTES = 3 * 512;  // block-scaled MMA: A, B-lo and B-hi scale blocks of a stage
+constexpr int SF_COL = 256;        // TMEM column of the scale factors (A: 4 columns, B: 8)
+
+// Per-variant roles.  MX (block-scaled MMA): one 256-column accumulator (the
+// scale factors take TMEM columns 256..267), so the epilogue drains it once
+// per promotion group; warp 2 prepares the scale factors and needs a few
+// more registers, taken from the epilogue.
+template <bool MX>
+struct Roles {
+    static constexpr int NBUF = MX ? 1 : 2;              // accumulator buffers in TMEM
+    static constexpr int PRODUCER_REGS = MX ? 56 : 40;   // warpgroup 0 after setmaxnreg.dec
+    static constexpr int EPILOGUE_REGS = MX ? 224 : 232; // warpgroups 1-2 after setmaxnreg.inc
+    static_assert(128 * PRODUCER_REGS + 256 * EPILOGUE_REGS <= NUM_THREADS * LAUNCH_REGS,
+                  "register split must fit in the block's launch allocation");
+};
 
 struct __align__(1024) GemmSmem {
     uint8_t a[STAGES][A_BYTES];
     uint8_t b[STAGES][B_BYTES];
+    uint8_t sf[STAGES][SF_BYTES];  // MX: UE8M0 scale factors in the tcgen05.cp source layout
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t tfull[2];
@@ -92,6 +105,9 @@ struct KParams {
     int *status;
     int K, N_out, n_segments, b_rows, n_tiles_n;
     int inject_fault;  // 1: block 0 arms its first stage for 16 bytes that never arrive
+    int ue8m0;         // H scales: power of two (UE8M0 variant) instead of amax / 448
+    int rows_total;
+    int mx_spc;        // MX: K blocks accumulated in TMEM per promotion into registers
 };
 
 __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int tile, int n_tiles_n,
@@ -132,24 +148,35 @@ __device__ __forceinline__ void promote32(float2 (&acc)[64], int base, const flo
     }
 }
 
-template <bool FP8, bool GATE_UP>
+// E8M0 byte of a power-of-two binary32 scale (2^-127 is the subnormal with
+// exponent field 0, matching E8M0 code 0), repeated in the four bytes.
+__device__ __forceinline__ uint32_t e8m0x4(float sc) {
+    return ((__float_as_uint(sc) >> 23) & 0xffu) * 0x01010101u;
+}
+
+template <bool FP8, bool GATE_UP, bool MX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const KParams p) {
+    static_assert(FP8 || !MX, "the block-scaled MMA takes e4m3 operands");
+    using R = Roles<MX>;
     extern __shared__ uint8_t smem_raw[];
     GemmSmem &s = *reinterpret_cast<GemmSmem *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = FP8 ? p.K / 128 : p.K / 64;  // stages per tile (128 bytes of K each)
-    // stages per promotion chunk: FP8 128 K (the scale block); BF16 256 K
-    constexpr int SPC = FP8 ? 1 : 4;
+    // stages per promotion chunk: FP8 128 K (the scale block); BF16 256 K;
+    // MX: the tensor core applies the scales, so chunks are mx_spc K blocks
+    const int SPC = MX ? p.mx_spc : (FP8 ? 1 : 4);
+    // the epilogue multiplies each chunk by s_a * s_w (software promotion)
+    constexpr bool SCALED = FP8 && !MX;
     const int NCH = (KB + SPC - 1) / SPC;        // K chunks per tile (last may be short)
     const int n_seg = p.n_segments;
 
     // ---------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&s.full[i], 1);
+            mbar_init(&s.full[i], MX ? 2 : 1);  // MX: TMA bytes + the scale-factor warp
             mbar_init(&s.empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -185,7 +212,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     volatile int *abort = &s.abort;
 
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(PRODUCER_REGS));
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(R::PRODUCER_REGS));
     }
     if (warp == 0) {
         // ------------------------------------------------------- producer
@@ -245,7 +272,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
-            constexpr uint32_t idesc = instr_desc<FP8>(BM, BN);
+            constexpr uint32_t idesc = MX ? instr_desc_mx(BM, BN) : instr_desc<FP8>(BM, BN);
             int stage = 0;
             uint32_t phase = 0;
             int tb = 0;
@@ -269,18 +296,32 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const uint32_t d_tmem = tmem_base + tb * BN;
                     const uint64_t adesc = smem_desc_sw128(smem_u32(s.a[stage]));
                     const uint64_t bdesc = smem_desc_sw128(smem_u32(s.b[stage]));
+                    if constexpr (MX) {
+                        // this stage's scale factors into TMEM, ordered before its MMAs
+                        // (and after the previous stage's, which read the same columns)
+                        const uint32_t sf = smem_u32(s.sf[stage]);
+                        tc_cp_32x128b_warpx4(tmem_base + SF_COL, smem_desc_plain(sf, 128));
+                        tc_cp_32x128b_warpx4(tmem_base + SF_COL + 4, smem_desc_plain(sf + 512, 128));
+                        tc_cp_32x128b_warpx4(tmem_base + SF_COL + 8, smem_desc_plain(sf + 1024, 128));
+                    }
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         // +32 bytes of K per instruction: +2 in the >>4 address field;
-                        // each 128-wide K chunk starts a fresh partial sum
+                        // each K chunk starts a fresh partial sum
                         const uint32_t acc = (chunk_first && kk == 0) ? 0u : 1u;
-                        tc_mma<FP8>(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc);
+                        if constexpr (MX)
+                            tc_mma_mx(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                                      tmem_base + SF_COL, tmem_base + SF_COL + 4, acc);
+                        else
+                            tc_mma<FP8>(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc);
                     }
                     tc_commit(&s.empty[stage]);
                     if (chunk_last) {
                         tc_commit(&s.tfull[tb]);
-                        tb ^= 1;
-                        if (tb == 0) tphase ^= 1;
+                        if (++tb == R::NBUF) {
+                            tb = 0;
+                            tphase ^= 1;
+                        }
                     }
                     if (++stage == STAGES) {
                         stage = 0;
@@ -298,9 +339,72 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
             }
         }
+    } else if (warp == 2) {
+        // ------------------------------------- scale factors (block-scaled MMA)
+        // For each stage, in the producer's order: the UE8M0 bytes of A's 128
+        // row scales and of the two B row blocks' scales, written in the
+        // tcgen05.cp source layout (lane l holds rows l, 32+l, 64+l, 96+l of A,
+        // one 32-bit column each, the byte repeated for the four 32-wide K
+        // steps), then an arrive on the stage's full barrier.  Scales are read
+        // from global memory two stages ahead.
+        if constexpr (MX) {
+            const int NB = p.b_rows / 128;
+            const int my_tiles = total_tiles > static_cast<int>(blockIdx.x)
+                                     ? (total_tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
+                                     : 0;
+            const int n_steps = my_tiles * KB;
+            auto load = [&](int i, float (&a)[4], float (&b)[2]) {
+                if (i >= n_steps) return;
+                const int tile = blockIdx.x + (i / KB) * gridDim.x, kb = i % KB;
+                int seg, row0, rows_valid, nt;
+                decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int r = row0 + lane + 32 * c;
+                    a[c] = r < p.rows_total ? __ldg(p.a_scales + static_cast<size_t>(r) * KB + kb) : 1.0f;
+                }
+                const int nb_lo = GATE_UP ? nt : 2 * nt;
+                const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
+                b[0] = __ldg(p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * KB + kb);
+                b[1] = __ldg(p.b_scales + (static_cast<size_t>(seg) * NB + nb_hi) * KB + kb);
+            };
+            float a0[4] = {}, a1[4] = {}, a2[4] = {}, b0[2] = {}, b1[2] = {}, b2[2] = {};
+            load(0, a0, b0);
+            load(1, a1, b1);
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int i = 0; i < n_steps; ++i) {
+                load(i + 2, a2, b2);
+                int go = 1;
+                if (lane == 0) go = mbar_wait(&s.empty[stage], phase ^ 1, abort, p.status) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, go, 0)) break;
+                uint8_t *sf = s.sf[stage];
+                *reinterpret_cast<uint4 *>(sf + 16 * lane) =
+                    make_uint4(e8m0x4(a0[0]), e8m0x4(a0[1]), e8m0x4(a0[2]), e8m0x4(a0[3]));
+                const uint32_t bl = e8m0x4(b0[0]), bh = e8m0x4(b0[1]);
+                *reinterpret_cast<uint4 *>(sf + 512 + 16 * lane) = make_uint4(bl, bl, bl, bl);
+                *reinterpret_cast<uint4 *>(sf + 1024 + 16 * lane) = make_uint4(bh, bh, bh, bh);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.full[stage]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    a0[c] = a1[c];
+                    a1[c] = a2[c];
+                }
+                b0[0] = b1[0];
+                b0[1] = b1[1];
+                b1[0] = b2[0];
+                b1[1] = b2[1];
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
     } else if (warp >= 4) {
         // ------------------------------------------------------- epilogue
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(EPILOGUE_REGS));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(R::EPILOGUE_REGS));
         const int q = warp & 3;            // TMEM lane quadrant = tile rows 32q..32q+31
         const int half = (warp - 4) >> 2;  // column half
         const int r_in = q * 32 + lane;
@@ -322,19 +426,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
             const int nb_lo = GATE_UP ? nt : 2 * nt;
             const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
-            const float *sw_lo_p = FP8 ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * NCH : nullptr;
-            const float *sw_hi_p = FP8 ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_hi) * NCH : nullptr;
-            const float *sa_p = FP8 ? p.a_scales + row * NCH : nullptr;
+            const float *sw_lo_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * NCH : nullptr;
+            const float *sw_hi_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_hi) * NCH : nullptr;
+            const float *sa_p = SCALED ? p.a_scales + row * NCH : nullptr;
             // scales of chunk c are loaded one chunk ahead (global latency)
             float nsa = 0.0f, nswl = 1.0f, nswh = 1.0f;
-            if (FP8 && warp_active) {
+            if (SCALED && warp_active) {
                 nsa = valid ? __ldg(sa_p) : 0.0f;
                 nswl = __ldg(sw_lo_p);
                 nswh = __ldg(sw_hi_p);
             }
             for (int c = 0; c < NCH; ++c) {
-                const float sc_lo = FP8 ? nsa * nswl : 1.0f, sc_hi = FP8 ? nsa * nswh : 1.0f;
-                if (FP8 && warp_active && c + 1 < NCH) {
+                const float sc_lo = SCALED ? nsa * nswl : 1.0f, sc_hi = SCALED ? nsa * nswh : 1.0f;
+                if (SCALED && warp_active && c + 1 < NCH) {
                     nsa = valid ? __ldg(sa_p + c + 1) : 0.0f;
                     nswl = __ldg(sw_lo_p + c + 1);
                     nswh = __ldg(sw_hi_p + c + 1);
@@ -353,9 +457,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     tmem_ld32(base + col_lo, va);
                     tmem_ld32(base + col_lo + 32, vb);
                     tmem_wait_ld(va, vb);
-                    promote32<FP8>(acc2, 0, va, sc_lo);
+                    promote32<SCALED>(acc2, 0, va, sc_lo);
                     tmem_ld32(base + col_hi, va);
-                    promote32<FP8>(acc2, 16, vb, sc_lo);
+                    promote32<SCALED>(acc2, 16, vb, sc_lo);
                     tmem_ld32(base + col_hi + 32, vb);
                     tmem_wait_ld(va, vb);
                 }
@@ -363,11 +467,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.tempty[tb]);
                 if (warp_active) {
-                    promote32<FP8>(acc2, 32, va, sc_hi);
-                    promote32<FP8>(acc2, 48, vb, sc_hi);
+                    promote32<SCALED>(acc2, 32, va, sc_hi);
+                    promote32<SCALED>(acc2, 48, vb, sc_hi);
                 }
-                tb ^= 1;
-                if (tb == 0) tphase ^= 1;
+                if (++tb == R::NBUF) {
+                    tb = 0;
+                    tphase ^= 1;
+                }
             }
             if (!ok) break;
             // column c of the thread's 128 (in place, no copy)
@@ -395,8 +501,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     if (valid) {
                         float sc = 1.0f, inv = 0.0f;
                         if (amax != 0.0f) {
-                            sc = __fdiv_rn(amax, 448.0f);
-                            inv = __fdiv_rn(448.0f, amax);
+                            if (p.ue8m0) {
+                                sc = ue8m0_scale(amax, &inv);
+                            } else {
+                                sc = __fdiv_rn(amax, 448.0f);
+                                inv = __fdiv_rn(448.0f, amax);
+                            }
                         }
                         uint8_t *hq = static_cast<uint8_t *>(p.out) + row * p.N_out + nt * 128 +
                                       half * 64;
@@ -491,7 +601,7 @@ bool make_map_2d(CUtensorMap *m, const void *base, bool fp8, int K, int rows) {
 }
 
 
-template <bool FP8, bool GATE_UP>
+template <bool FP8, bool GATE_UP, bool MX>
 cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams &kp, int grid,
                      cudaStream_t st) {
     const size_t smem = sizeof(GemmSmem) + 1024;
@@ -501,17 +611,17 @@ cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams
         // refuse to launch a build whose register count differs, as the
         // epilogue's increase would then never be granted.
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, grouped_gemm_kernel<FP8, GATE_UP>);
+        cudaError_t e = cudaFuncGetAttributes(&fa, grouped_gemm_kernel<FP8, GATE_UP, MX>);
         if (e != cudaSuccess) return e;
         if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(grouped_gemm_kernel<FP8, GATE_UP>,
+        e = cudaFuncSetAttribute(grouped_gemm_kernel<FP8, GATE_UP, MX>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    return launch_pdl(grouped_gemm_kernel<FP8, GATE_UP>, dim3(grid), dim3(NUM_THREADS), smem, st, ma, mb,
-                      kp);
+    return launch_pdl(grouped_gemm_kernel<FP8, GATE_UP, MX>, dim3(grid), dim3(NUM_THREADS), smem, st,
+                      ma, mb, kp);
 }
 
 }  // namespace
@@ -541,6 +651,10 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     kp.b_rows = b_rows;
     kp.n_tiles_n = g.gate_up ? g.N_out / 128 : g.N_out / 256;
     kp.inject_fault = g.inject_fault;
+    kp.ue8m0 = g.ue8m0 ? 1 : 0;
+    kp.rows_total = g.rows_total;
+    // block-scaled MMA (UE8M0 scales): all of K accumulates in TMEM
+    kp.mx_spc = g.K / 128;
     // upper bound of work items: every segment's tiles, each at most one partial
     const long long max_mtiles = g.rows_total / BM + g.n_segments;
     const long long max_tiles = max_mtiles * kp.n_tiles_n;
@@ -548,10 +662,15 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     if (grid <= 0) return cudaSuccess;
     cudaError_t e;
     mark_launch(st, *launches, g.gate_up ? "grouped_gemm_gate_up" : "grouped_gemm_down");
-    if (g.fp8) e = g.gate_up ? launch_t<true, true>(ma, mb, kp, grid, st)
-                             : launch_t<true, false>(ma, mb, kp, grid, st);
-    else e = g.gate_up ? launch_t<false, true>(ma, mb, kp, grid, st)
-                       : launch_t<false, false>(ma, mb, kp, grid, st);
+    if (g.fp8 && g.ue8m0)
+        e = g.gate_up ? launch_t<true, true, true>(ma, mb, kp, grid, st)
+                      : launch_t<true, false, true>(ma, mb, kp, grid, st);
+    else if (g.fp8)
+        e = g.gate_up ? launch_t<true, true, false>(ma, mb, kp, grid, st)
+                      : launch_t<true, false, false>(ma, mb, kp, grid, st);
+    else
+        e = g.gate_up ? launch_t<false, true, false>(ma, mb, kp, grid, st)
+                      : launch_t<false, false, false>(ma, mb, kp, grid, st);
     ++*launches;
     return e;
 }

@@ -76,9 +76,10 @@ cudaError_t launch_tile_table(const int32_t *offsets, int E, int T, int k, int n
 
 // e4m3 quantisation of bf16 [rows, cols] (leading dimension ld) in tiles of
 // block_rows x 128.
+// ue8m0: power-of-two scales (least 2^k with amax / 2^k <= 448)
 cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
                                int tiled, uint8_t *q, float *scales, cudaStream_t st,
-                               int *launches);
+                               int *launches, bool ue8m0 = false);
 
 // Row-major [rows, row_bytes] -> 128 x 128-byte tiles (MOE_LAYOUT_TILED).
 cudaError_t launch_pack_tiles(const void *src, int rows, int row_bytes, void *dst, cudaStream_t st,
@@ -88,7 +89,8 @@ cudaError_t launch_pack_tiles(const void *src, int rows, int row_bytes, void *ds
 // scales to its k routed rows (row_of) and, with n_shared, to row T*k + t.
 cudaError_t launch_quant_scatter(const uint16_t *x, int T, int d, int k, int n_shared,
                                  const int32_t *row_of, uint8_t *a, float *a_scales,
-                                 cudaStream_t st, int *launches, PreNorm pn = {});
+                                 cudaStream_t st, int *launches, PreNorm pn = {},
+                                 bool ue8m0 = false);
 
 // bf16 copy of each token row to its k routed rows and its shared row.
 cudaError_t launch_scatter_bf16(const uint16_t *x, int T, int d, int k, int n_shared,
@@ -123,6 +125,7 @@ struct GemmArgs {
     const int32_t *seg_start, *seg_rows, *tile_start;
     int *status;
     int inject_fault;       // test hook: make one bounded wait run out (see api.cu)
+    bool ue8m0;             // fp8 gate/up: H requantised with power-of-two scales
 };
 cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launches);
 

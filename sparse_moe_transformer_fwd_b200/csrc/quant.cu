@@ -3,7 +3,9 @@
 // bf16 inputs), scale = amax / 448 and inv = 448 / amax (correctly rounded
 // binary32 divisions), code = e4m3 round-to-nearest-even, saturating, of the
 // binary32 product v * inv (hardware cvt.rn.satfinite.e4m3x2.f32).  An
-// all-zero tile gets scale 1 and +0 codes.
+// all-zero tile gets scale 1 and +0 codes.  UE8M0 variant (flag ue): the
+// scale is the least power of two 2^k (k >= -127) with amax / 2^k <= 448 and
+// inv = 2^-k, so v * inv is exact and no code saturates.
 //
 // Activations use 1x128 tiles: 16 threads own one tile (8 elements each,
 // one 16-byte load), amax by shuffles inside the 16-lane group.  Weights use
@@ -41,13 +43,19 @@ __device__ __forceinline__ float amax8(const Quant8 &q) {
 }
 
 // codes of 8 values for a tile with the given amax; returns the scale
-__device__ __forceinline__ uint2 encode8(const Quant8 &q, float amax, float *scale) {
+// (ue: the power-of-two UE8M0 scale instead of amax / 448)
+__device__ __forceinline__ uint2 encode8(const Quant8 &q, float amax, float *scale, bool ue) {
     if (amax == 0.0f) {
         *scale = 1.0f;
         return make_uint2(0, 0);
     }
-    *scale = __fdiv_rn(amax, 448.0f);
-    const float inv = __fdiv_rn(448.0f, amax);
+    float inv;
+    if (ue) {
+        *scale = ue8m0_scale(amax, &inv);
+    } else {
+        *scale = __fdiv_rn(amax, 448.0f);
+        inv = __fdiv_rn(448.0f, amax);
+    }
     uint16_t c[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -65,7 +73,7 @@ __device__ __forceinline__ float group16_max(float m) {
 // 1 x 128 tiles over a [rows, cols] matrix
 __global__ void __launch_bounds__(256)
 quant_1x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld,
-                   uint8_t *__restrict__ q, float *__restrict__ scales) {
+                   uint8_t *__restrict__ q, float *__restrict__ scales, int ue) {
     pdl_wait_and_trigger();
     const int vpr = cols / 8;  // 16-byte vectors per row
     const long long total = static_cast<long long>(rows) * vpr;
@@ -83,7 +91,7 @@ quant_1x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld,
             for (int i = 0; i < 8; ++i) x.v[i] = 0.0f;
         const float amax = group16_max(amax8(x));
         float sc;
-        const uint2 codes = encode8(x, amax, &sc);
+        const uint2 codes = encode8(x, amax, &sc, ue);
         if (ok) {
             *reinterpret_cast<uint2 *>(q + static_cast<size_t>(r) * cols + vc * 8) = codes;
             if ((vc & 15) == 0) scales[static_cast<size_t>(r) * (cols / 128) + vc / 16] = sc;
@@ -96,7 +104,7 @@ quant_1x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld,
 // 128 codes) at tile index rb * (cols/128) + kb.
 __global__ void __launch_bounds__(256)
 quant_128x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld, int tiled,
-                     uint8_t *__restrict__ q, float *__restrict__ scales) {
+                     uint8_t *__restrict__ q, float *__restrict__ scales, int ue) {
     __shared__ float red[8];
     pdl_wait_and_trigger();
     const int nkb = cols / 128, nrb = (rows + 127) / 128;
@@ -127,7 +135,7 @@ quant_128x128_kernel(const uint16_t *__restrict__ in, int rows, int cols, int ld
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int r = rb * 128 + tr + 16 * i;
-            const uint2 codes = encode8(x[i], amax, &sc);
+            const uint2 codes = encode8(x[i], amax, &sc, ue);
             const size_t at = tiled ? (static_cast<size_t>(b) << 14) + (tr + 16 * i) * 128 + tc
                                     : static_cast<size_t>(r) * cols + kb * 128 + tc;
             if (r < rows) *reinterpret_cast<uint2 *>(q + at) = codes;
@@ -178,7 +186,7 @@ __device__ __forceinline__ Quant8 load8_x(const uint16_t *row, int c0, float rst
 __global__ void __launch_bounds__(256)
 quant_scatter_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_shared,
                      const int32_t *__restrict__ row_of, uint8_t *__restrict__ a,
-                     float *__restrict__ a_scales, PreNorm pn) {
+                     float *__restrict__ a_scales, PreNorm pn, int ue) {
     __shared__ int rows_sh[33];
     const int t = blockIdx.x;
     const int ndst = k + n_shared;
@@ -199,7 +207,7 @@ quant_scatter_kernel(const uint16_t *__restrict__ x, int T, int d, int k, int n_
         for (int i = 0; i < 8; ++i) v.v[i] = 0.0f;
     const float amax = group16_max(amax8(v));
     float sc;
-    const uint2 codes = encode8(v, amax, &sc);
+    const uint2 codes = encode8(v, amax, &sc, ue);
     if (!ok) return;
     for (int j = 0; j < ndst; ++j) {
         const size_t row = static_cast<size_t>(rows_sh[j]);
@@ -272,7 +280,7 @@ cudaError_t launch_pack_tiles(const void *src, int rows, int row_bytes, void *ds
 
 cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, int block_rows,
                                int tiled, uint8_t *q, float *scales, cudaStream_t st,
-                               int *launches) {
+                               int *launches, bool ue8m0) {
     if (rows == 0) return cudaSuccess;
     const int sms = num_sms();
     mark_launch(st, *launches, block_rows == 1 ? "quant_1x128" : "quant_128x128");
@@ -281,12 +289,12 @@ cudaError_t launch_block_quant(const uint16_t *in, int rows, int cols, int ld, i
         const long long want = (total + 255) / 256;
         const int grid = static_cast<int>(want < sms * 16LL ? want : sms * 16LL);
         LAUNCH_OR_RETURN(launch_pdl(quant_1x128_kernel, dim3(grid), dim3(256), 0, st, in, rows, cols, ld, q,
-                                    scales));
+                                    scales, ue8m0 ? 1 : 0));
     } else {
         const long long nblocks = static_cast<long long>(cols / 128) * ((rows + 127) / 128);
         const int grid = static_cast<int>(nblocks < sms * 8LL ? nblocks : sms * 8LL);
         LAUNCH_OR_RETURN(launch_pdl(quant_128x128_kernel, dim3(grid), dim3(256), 0, st, in, rows, cols, ld,
-                                    tiled, q, scales));
+                                    tiled, q, scales, ue8m0 ? 1 : 0));
     }
     ++*launches;
     return cudaGetLastError();
@@ -302,10 +310,10 @@ cudaError_t launch_rstd(const uint16_t *h, int T, int d, float eps, float *rstd,
 
 cudaError_t launch_quant_scatter(const uint16_t *x, int T, int d, int k, int n_shared,
                                  const int32_t *row_of, uint8_t *a, float *a_scales,
-                                 cudaStream_t st, int *launches, PreNorm pn) {
+                                 cudaStream_t st, int *launches, PreNorm pn, bool ue8m0) {
     mark_launch(st, *launches, "quant_scatter");
     LAUNCH_OR_RETURN(launch_pdl(quant_scatter_kernel, dim3(T, (d / 128 + 15) / 16), dim3(256), 0, st, x, T, d, k, n_shared, row_of,
-                                a, a_scales, pn));
+                                a, a_scales, pn, ue8m0 ? 1 : 0));
     ++*launches;
     return cudaGetLastError();
 }

@@ -7,7 +7,12 @@ step of the oracle value.  The step allowance is the storage quantum: two
 correct evaluations whose binary32 / binary64 sums straddle a bf16 rounding
 boundary store values one step apart, and a step is |v|/256..|v|/128, which
 is larger than 1e-2 * RMS wherever |v| > 1.28 * RMS.  Without it no bf16
-output could meet the max-abs bound."""
+output could meet the max-abs bound.  In the fp8 precisions the max bound also
+allows, per output, the oracle's bound on how far alternative e4m3 codes of H
+could move it (H elements whose quantiser input lies at a rounding boundary,
+oracle.h_code_ambiguity): two correct evaluations of G and U may round such
+an element either way, and one code step of a large H element moves every
+output of its row by up to one step times |W2|."""
 from __future__ import annotations
 
 import json
@@ -44,14 +49,17 @@ def bf16_step(v: np.ndarray) -> np.ndarray:
     return 2.0 ** (np.floor(np.log2(a)) - 7)
 
 
-def out_error(got_bf16: torch.Tensor, want_u16: np.ndarray):
-    """-> (relative L2, max |diff| / RMS, max (|diff| - one bf16 step)+ / RMS)."""
+def out_error(got_bf16: torch.Tensor, want_u16: np.ndarray, allow=None):
+    """-> (relative L2, max |diff| / RMS, max (|diff| - one bf16 step - allow)+ / RMS)."""
     got = got_bf16.detach().float().cpu().numpy().astype(np.float64)
     want = oracle.bf16_to_f32(want_u16).astype(np.float64).reshape(got.shape)
     diff = np.abs(got - want)
     rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300)
     rms = max(np.sqrt(np.mean(want ** 2)), 1e-300)
-    excess = np.maximum(diff - bf16_step(want), 0.0)
+    slack = bf16_step(want)
+    if allow is not None:
+        slack = slack + np.asarray(allow, dtype=np.float64).reshape(got.shape)
+    excess = np.maximum(diff - slack, 0.0)
     return rel, diff.max() / rms, excess.max() / rms
 
 
@@ -64,8 +72,8 @@ def _log(what, rel, mx, ex):
                                 "beyond_one_step_over_rms": ex}) + "\n")
 
 
-def assert_out_close(got_bf16, want_u16, what=""):
-    rel, mx, ex = out_error(got_bf16, want_u16)
+def assert_out_close(got_bf16, want_u16, what="", allow=None):
+    rel, mx, ex = out_error(got_bf16, want_u16, allow)
     _log(what, rel, mx, ex)
     assert rel <= REL_L2 and ex <= MAX_ABS_RMS, \
         f"{what}: rel_l2={rel:.3e} max/rms={mx:.3e} beyond-one-step/rms={ex:.3e}"

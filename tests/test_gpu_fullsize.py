@@ -20,7 +20,8 @@ pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0") if torch.cuda.is_available() else None
 
 
-@pytest.fixture(scope="module", params=["decode", "prefill", "skew", "bf16"])
+@pytest.fixture(scope="module", params=["decode", "prefill", "skew", "bf16", "decode_ue8m0",
+                                        "prefill_ue8m0"])
 def run(request):
     cfg = CONFIGS[request.param]
     inp = make_inputs(cfg, seed=0, device=DEV)
@@ -40,13 +41,14 @@ def test_status_ok(run):
 
 def test_weight_quant_bitexact(run):
     cfg, inp, layer = run[:3]
-    if cfg.precision != "fp8":
+    if cfg.precision == "bf16":
         pytest.skip("bf16 workload")
+    ue = cfg.precision == "fp8_ue8m0"
     for e in (0, 137 % cfg.n_experts, cfg.n_experts):
-        q13, s13 = oracle.block_quant(u16(inp["w13"][e]), 128)
+        q13, s13 = oracle.block_quant(u16(inp["w13"][e]), 128, ue8m0=ue)
         assert np.array_equal(layer.w13s[e].cpu().numpy().view(np.uint32), s13.view(np.uint32))
         assert np.array_equal(untile(layer.w13[e].cpu().numpy(), *q13.shape), q13)
-        q2, s2 = oracle.block_quant(u16(inp["w2"][e]), 128)
+        q2, s2 = oracle.block_quant(u16(inp["w2"][e]), 128, ue8m0=ue)
         assert np.array_equal(layer.w2s[e].cpu().numpy().view(np.uint32), s2.view(np.uint32))
         assert np.array_equal(untile(layer.w2[e].cpu().numpy(), *q2.shape), q2)
 
@@ -85,4 +87,4 @@ def test_sampled_tokens_vs_oracle(run):
     tokens = _sample(cfg, idx_np)
     ref = oracle_layer(cfg, inp, tokens=tokens)
     assert np.array_equal(idx_np[tokens], ref["idx"])
-    assert_out_close(out[tokens], ref["out"], cfg.name)
+    assert_out_close(out[tokens], ref["out"], cfg.name, ref["out_allow"])

@@ -140,8 +140,9 @@ QUANT_CASES = [(1, 128, 1), (1000, 7168, 1), (33, 384, 1), (256, 512, 128), (300
                (4096, 7168, 128), (129, 128, 128)]
 
 
+@pytest.mark.parametrize("ue8m0", [False, True])
 @pytest.mark.parametrize("rows,cols,block_rows", QUANT_CASES)
-def test_block_quant_bitexact(rows, cols, block_rows):
+def test_block_quant_bitexact(rows, cols, block_rows, ue8m0):
     g = torch.Generator().manual_seed(rows + cols)
     scale = torch.exp(torch.rand(rows, 1, generator=g) * 12 - 8)
     a = (torch.randn(rows, cols, generator=g) * scale).to(torch.bfloat16)
@@ -149,18 +150,23 @@ def test_block_quant_bitexact(rows, cols, block_rows):
     if rows > 2:
         a[2, 5] = -0.0
         a[2, 130 % cols] = 1e30 if cols > 130 else a[2, 130 % cols]
+    if ue8m0 and rows > 4:
+        a[3, :128] *= 2.0 ** -120             # below the exponent floor 448 * 2^-128
+        a[4, :128] = 0.0
+        a[4, 1] = 448.0 * 2.0 ** -5           # amax exactly 448 * 2^j: scale 2^j
     q = torch.empty(rows, cols, dtype=torch.uint8, device=DEV)
     nrb = (rows + block_rows - 1) // block_rows
     s = torch.empty(nrb, cols // 128, dtype=torch.float32, device=DEV)
-    moe.fp8_block_quant(a.to(DEV), block_rows, q, s)
-    rq, rs = oracle.block_quant(u16(a), block_rows)
+    moe.fp8_block_quant(a.to(DEV), block_rows, q, s, ue8m0=ue8m0)
+    rq, rs = oracle.block_quant(u16(a), block_rows, ue8m0=ue8m0)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
     assert np.array_equal(q.cpu().numpy(), rq)
     if block_rows == 128 and rows % 128 == 0:
         # tiled output: the same codes and scales, 128 x 128 tiles contiguous
         qt = torch.empty_like(q)
         st = torch.empty_like(s)
-        moe.fp8_block_quant(a.to(DEV), block_rows, qt, st, layout=moe.MOE_LAYOUT_TILED)
+        moe.fp8_block_quant(a.to(DEV), block_rows, qt, st, layout=moe.MOE_LAYOUT_TILED,
+                            ue8m0=ue8m0)
         assert torch.equal(st, s)
         assert np.array_equal(untile(qt.cpu().numpy(), rows, cols), rq)
 
@@ -177,7 +183,7 @@ def test_pack_tiles_is_the_tiled_permutation(rows, row_bytes, dtype):
 
 # ------------------------------------------- grouped experts and combine ---
 
-@pytest.mark.parametrize("precision", ["bf16", "fp8"])
+@pytest.mark.parametrize("precision", ["bf16", "fp8", "fp8_ue8m0"])
 @pytest.mark.parametrize("T", [128, 37])
 def test_grouped_swiglu_and_combine(precision, T):
     cfg = CONFIGS["tiny"].with_(precision=precision, T=T)
@@ -191,10 +197,11 @@ def test_grouped_swiglu_and_combine(precision, T):
     y = torch.empty(cfg.R_s, cfg.d_model, dtype=torch.bfloat16, device=DEV)
     offsets = torch.from_numpy(ref["offsets"]).to(DEV)
     w13, w2 = inp["w13"].to(DEV), inp["w2"].to(DEV)
-    if precision == "fp8":
+    ue = precision == "fp8_ue8m0"
+    if precision != "bf16":
         a = torch.from_numpy(ref["xq"][rows]).to(DEV)
         a_s = torch.from_numpy(ref["xs"][rows]).to(DEV)
-        w13q, w13s, w2q, w2s = moe.quantize_weights(w13, w2)
+        w13q, w13s, w2q, w2s = moe.quantize_weights(w13, w2, ue8m0=ue)
         moe.moe_grouped_swiglu(shape, a, a_s, offsets, w13q, w13s, w2q, w2s, y, ws)
     else:
         a = from_u16(u16(inp["x"])[rows], DEV)
@@ -204,19 +211,21 @@ def test_grouped_swiglu_and_combine(precision, T):
     # oracle expert outputs, row by row
     seg_of_row = np.concatenate([np.repeat(np.arange(E), ref["counts"]), np.full(T, E)])
     want = np.empty((cfg.R_s, cfg.d_model), np.uint16)
+    want_allow = np.zeros((cfg.R_s, cfg.d_model))
     for e in range(E + 1):
         sel = np.nonzero(seg_of_row == e)[0]
         if sel.size == 0:
             continue
         w13e, w2e = u16(inp["w13"][e]), u16(inp["w2"][e])
-        if precision == "fp8":
-            q13, s13 = oracle.block_quant(w13e, 128)
-            q2, s2 = oracle.block_quant(w2e, 128)
-            want[sel] = oracle.expert_forward(ref["xq"][rows[sel]], q13, q2, "fp8",
-                                              ref["xs"][rows[sel]], s13, s2)
+        if precision != "bf16":
+            q13, s13 = oracle.block_quant(w13e, 128, ue8m0=ue)
+            q2, s2 = oracle.block_quant(w2e, 128, ue8m0=ue)
+            want[sel], want_allow[sel] = oracle.expert_forward(
+                ref["xq"][rows[sel]], q13, q2, precision, ref["xs"][rows[sel]], s13, s2,
+                return_allow=True)
         else:
             want[sel] = oracle.expert_forward(u16(inp["x"])[rows[sel]], w13e, w2e, "bf16")
-    assert_out_close(y, want, "grouped experts")
+    assert_out_close(y, want, "grouped experts", want_allow)
     # combine
     out = torch.empty(T, cfg.d_model, dtype=torch.bfloat16, device=DEV)
     moe.moe_combine(shape, y, torch.from_numpy(ref["row_of"]).to(DEV),
@@ -225,7 +234,7 @@ def test_grouped_swiglu_and_combine(precision, T):
     out_ref = torch.empty_like(out)
     moe.moe_combine(shape, yo, torch.from_numpy(ref["row_of"]).to(DEV),
                     torch.from_numpy(ref["gates"]).to(DEV), out_ref)
-    assert_out_close(out, ref["out"], "combine")
+    assert_out_close(out, ref["out"], "combine", ref["out_allow"])
     # combine alone, fed the oracle's Y: same as the oracle's combine
     assert_out_close(out_ref, ref["out"], "combine of oracle Y")
 
@@ -246,7 +255,7 @@ FWD_CASES = {
 }
 
 
-@pytest.mark.parametrize("precision", ["bf16", "fp8"])
+@pytest.mark.parametrize("precision", ["bf16", "fp8", "fp8_ue8m0"])
 @pytest.mark.parametrize("name", list(FWD_CASES))
 def test_forward_vs_oracle(name, precision):
     cfg = CONFIGS["tiny"].with_(precision=precision, **FWD_CASES[name])
@@ -260,13 +269,13 @@ def test_forward_vs_oracle(name, precision):
     assert layer.check_status(cfg.T) == 0, moe.moe_last_error()
     ref = oracle_layer(cfg, inp)
     assert np.array_equal(idx.cpu().numpy(), ref["idx"])
-    assert_out_close(out, ref["out"], name)
+    assert_out_close(out, ref["out"], name, ref["out_allow"])
     # deterministic: a second run gives the same bits
     out2 = layer(d["x"])
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
 
 
-@pytest.mark.parametrize("precision", ["bf16", "fp8"])
+@pytest.mark.parametrize("precision", ["bf16", "fp8", "fp8_ue8m0"])
 def test_forward_all_tokens_on_few_experts(precision):
     """A large bias on experts 0..k-1 sends every token there: the other
     segments are empty and four segments hold T rows each (several tiles)."""
@@ -283,7 +292,7 @@ def test_forward_all_tokens_on_few_experts(precision):
     ref = oracle_layer(cfg, inp)
     assert (np.sort(ref["idx"], 1) == np.arange(cfg.top_k)).all()
     assert np.array_equal(idx.cpu().numpy(), ref["idx"])
-    assert_out_close(out, ref["out"], "few experts")
+    assert_out_close(out, ref["out"], "few experts", ref["out_allow"])
 
 
 def test_forward_empty_batch():
@@ -312,7 +321,8 @@ def test_bounded_wait_timeout_reports_status(monkeypatch):
     assert layer.check_status(cfg.T) == moe._native.MOE_ERR_TIMEOUT
     out = layer(d["x"])
     assert layer.check_status(cfg.T) == 0
-    assert_out_close(out, oracle_layer(cfg, inp)["out"], "after timeout")
+    ref = oracle_layer(cfg, inp)
+    assert_out_close(out, ref["out"], "after timeout", ref["out_allow"])
 
 
 # ----------------------------------------------- pre-norm block (fused) ---
@@ -344,7 +354,7 @@ def test_forward_prenorm_vs_oracle(name):
         lambda e: (u16(inp["w13"][e]), u16(inp["w2"][e])), n_experts=cfg.n_experts,
         top_k=cfg.top_k, n_shared=cfg.n_shared, precision=cfg.precision)
     assert np.array_equal(idx.cpu().numpy(), ref["idx"])
-    assert_out_close(out, ref["out"], "prenorm " + name)
+    assert_out_close(out, ref["out"], "prenorm " + name, ref["out_allow"])
 
 
 def test_prenorm_router_decode_dims_bitexact():

@@ -1,0 +1,76 @@
+"""Pins of the oracle's bound on alternative H codes (oracle.h_code_ambiguity),
+which widens the max-abs output tolerance of the fp8 precisions: checked on
+constructed tiles whose quantiser inputs are known exactly."""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def _tile(vals, amax_at=0, amax=448.0):
+    """One 1x128 row whose quantiser input equals `vals` exactly (scale 1)."""
+    h = np.zeros((1, 128), np.float32)
+    h[0, amax_at] = amax
+    h[0, 1:1 + len(vals)] = vals
+    return h
+
+
+@pytest.mark.parametrize("ue8m0", [False, True])
+def test_zero_away_from_boundaries(ue8m0):
+    # amax 448 gives scale 1 in both variants; codes exactly representable
+    h = _tile([1.0, -1.125, 3.5, 0.015625, -240.0])
+    q, s = oracle.block_quant(h, 1, ue8m0=ue8m0)
+    assert s[0, 0] == 1.0
+    d = oracle.h_code_ambiguity(h, q, s, ue8m0)
+    assert not d.any()
+
+
+@pytest.mark.parametrize("ue8m0", [False, True])
+def test_one_step_at_a_rounding_midpoint(ue8m0):
+    # 1.0625 lies half way between the e4m3 values 1.0 and 1.125 (ties to even
+    # gives 1.0); a perturbation either way reaches 1.125: one step of 0.125
+    h = _tile([1.0625, 1.03125])
+    q, s = oracle.block_quant(h, 1, ue8m0=ue8m0)
+    d = oracle.h_code_ambiguity(h, q, s, ue8m0)
+    assert d[0, 1] == 0.125
+    assert d[0, 2] == 0.0                       # a quarter step from the boundary
+    assert np.count_nonzero(d) == 1
+
+
+def test_scale_boundary_of_power_of_two_tiles():
+    # amax exactly 448 * 2^3: scale 2^3, and the next binary32 value up takes
+    # 2^4, so every element may be requantised at the doubled scale
+    h = _tile([9.0, 1.0], amax=448.0 * 8)
+    q, s = oracle.block_quant(h, 1, ue8m0=True)
+    assert s[0, 0] == 8.0
+    d = oracle.h_code_ambiguity(h, q, s, True)
+    # 9 = 1.125 * 8 (exact at scale 8); at scale 16, 9/16 = 0.5625 is an e4m3
+    # value too, so 9 stays exact; 1 = 0.125 * 8 and 1/16 = 0.0625 both exact
+    assert d[0, 1] == 0.0 and d[0, 2] == 0.0
+    h2 = _tile([9.5], amax=448.0 * 8)
+    q2, s2 = oracle.block_quant(h2, 1, ue8m0=True)
+    d2 = oracle.h_code_ambiguity(h2, q2, s2, True)
+    # 9.5/8 = 1.1875 rounds to 1.25 (ties to even between 1.125 and 1.25) ->
+    # 10; 9.5/16 = 0.59375 rounds to 0.625 (ties to even) -> 10: same value,
+    # but the midpoint itself is ambiguous at scale 8: 9 or 10
+    assert d2[0, 1] == 1.0
+
+
+def test_layer_allowance_is_zero_in_bf16_and_small_in_fp8():
+    from moe_inputs import CONFIGS, make_inputs
+    import torch
+    u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    for prec in ("bf16", "fp8", "fp8_ue8m0"):
+        cfg = CONFIGS["tiny"].with_(precision=prec, T=8)
+        inp = make_inputs(cfg, seed=2)
+        res = oracle.moe_layer(u16(inp["x"]), u16(inp["w_router"]), inp["bias"].numpy(),
+                               lambda e: (u16(inp["w13"][e]), u16(inp["w2"][e])),
+                               n_experts=cfg.n_experts, top_k=cfg.top_k, n_shared=cfg.n_shared,
+                               precision=prec)
+        out = oracle.bf16_to_f32(res["out"]).astype(np.float64)
+        rms = np.sqrt(np.mean(out ** 2))
+        if prec == "bf16":
+            assert not res["out_allow"].any()
+        else:
+            # a handful of boundary elements per row: well below the output scale
+            assert res["out_allow"].max() < 0.1 * rms
