@@ -60,8 +60,15 @@ constexpr int LAUNCH_REGS = 168;   // 65536 / 384, multiple of 8
 constexpr int EPI_THREADS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_SEG = 1025;
-constexpr int SF_BYTES = 3 * 512;  // block-scaled MMA: A, B-lo and B-hi scale blocks of a stage
+// Block-scaled MMA: a 32-bit TMEM scale column holds four UE8M0 bytes, and an
+// MMA picks one by its scale-factor id; byte j of a scale block belongs to K
+// block 4g + j, so one block serves a group of four stages.
+constexpr int SF_BYTES = 3 * 512;  // scale block: A, B-lo and B-hi (32 lanes x 16 bytes each)
 constexpr int SF_COL = 256;        // TMEM column of the scale factors (A: 4 columns, B: 8)
+constexpr int SF_GROUP = 4;        // K blocks per scale block
+constexpr int SF_BUFS = 2;         // scale blocks in shared memory
+constexpr int SF_STAGING = 4;      // fp32 staging slots (groups) between warps 3 and 2
+constexpr int SF_AHEAD = 2;        // groups whose scale copies warp 3 keeps in flight
 
 // Per-variant roles.  MX (block-scaled MMA): one 256-column accumulator (the
 // scale factors take TMEM columns 256..267), so the epilogue drains it once
@@ -79,7 +86,13 @@ struct Roles {
 struct __align__(1024) GemmSmem {
     uint8_t a[STAGES][A_BYTES];
     uint8_t b[STAGES][B_BYTES];
-    uint8_t sf[STAGES][SF_BYTES];  // MX: UE8M0 scale factors in the tcgen05.cp source layout
+    uint8_t sf[SF_BUFS][SF_BYTES];  // MX: UE8M0 scale blocks in the tcgen05.cp source layout
+    float sf_a[SF_STAGING][SF_GROUP][BM];  // MX: fp32 scales staged by warp 3 for warp 2
+    float sf_b[SF_STAGING][2][SF_GROUP];
+    uint64_t sf_full[SF_STAGING];
+    uint64_t sf_empty[SF_STAGING];
+    uint64_t sf_ready[SF_BUFS];     // scale block written (warp 2 -> MMA issuer)
+    uint64_t sf_free[SF_BUFS];      // scale block copied to TMEM (tcgen05.commit -> warp 2)
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t tfull[2];
@@ -149,10 +162,8 @@ __device__ __forceinline__ void promote32(float2 (&acc)[64], int base, const flo
 }
 
 // E8M0 byte of a power-of-two binary32 scale (2^-127 is the subnormal with
-// exponent field 0, matching E8M0 code 0), repeated in the four bytes.
-__device__ __forceinline__ uint32_t e8m0x4(float sc) {
-    return ((__float_as_uint(sc) >> 23) & 0xffu) * 0x01010101u;
-}
+// exponent field 0, matching E8M0 code 0).
+__device__ __forceinline__ uint32_t e8m0(float sc) { return (__float_as_uint(sc) >> 23) & 0xffu; }
 
 template <bool FP8, bool GATE_UP, bool MX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -176,7 +187,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     // ---------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&s.full[i], MX ? 2 : 1);  // MX: TMA bytes + the scale-factor warp
+            mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -185,6 +196,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&s.xchg[i], EPI_THREADS);
         }
         mbar_init(&s.mma_done, 1);
+        for (int i = 0; i < SF_STAGING; ++i) {
+            mbar_init(&s.sf_full[i], 1);
+            mbar_init(&s.sf_empty[i], 1);
+        }
+        for (int i = 0; i < SF_BUFS; ++i) {
+            mbar_init(&s.sf_ready[i], 1);
+            mbar_init(&s.sf_free[i], 1);
+        }
         s.abort = 0;
         fence_mbar_init();
     }
@@ -277,6 +296,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             uint32_t phase = 0;
             int tb = 0;
             uint32_t tphase = 0;
+            int gq = 0;  // MX: scale blocks consumed
             bool ok = true;
             for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
                 for (int kb = 0; kb < KB; ++kb) {
@@ -288,6 +308,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                             break;
                         }
                     }
+                    const bool group_first = MX && (kb % SF_GROUP) == 0;
+                    if (group_first &&
+                        !mbar_wait(&s.sf_ready[gq % SF_BUFS], (gq / SF_BUFS) & 1, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
                     if (!mbar_wait(&s.full[stage], phase, abort, p.status)) {
                         ok = false;
                         break;
@@ -296,22 +322,31 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const uint32_t d_tmem = tmem_base + tb * BN;
                     const uint64_t adesc = smem_desc_sw128(smem_u32(s.a[stage]));
                     const uint64_t bdesc = smem_desc_sw128(smem_u32(s.b[stage]));
-                    if constexpr (MX) {
-                        // this stage's scale factors into TMEM, ordered before its MMAs
-                        // (and after the previous stage's, which read the same columns)
-                        const uint32_t sf = smem_u32(s.sf[stage]);
+                    if (group_first) {
+                        // the group's scale block into TMEM, ordered before its MMAs
+                        // and after the previous group's, which read the same columns;
+                        // the commit frees the shared-memory block once it is copied
+                        const int buf = gq % SF_BUFS;
+                        const uint32_t sf = smem_u32(s.sf[buf]);
                         tc_cp_32x128b_warpx4(tmem_base + SF_COL, smem_desc_plain(sf, 128));
                         tc_cp_32x128b_warpx4(tmem_base + SF_COL + 4, smem_desc_plain(sf + 512, 128));
                         tc_cp_32x128b_warpx4(tmem_base + SF_COL + 8, smem_desc_plain(sf + 1024, 128));
+                        tc_commit(&s.sf_free[buf]);
+                        ++gq;
                     }
+                    // MX: this K block's scales are byte kb % 4 of each scale column
+                    // (the id in the instruction descriptor and in the TMEM address)
+                    const uint32_t sid = static_cast<uint32_t>(kb % SF_GROUP);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         // +32 bytes of K per instruction: +2 in the >>4 address field;
                         // each K chunk starts a fresh partial sum
                         const uint32_t acc = (chunk_first && kk == 0) ? 0u : 1u;
                         if constexpr (MX)
-                            tc_mma_mx(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                      tmem_base + SF_COL, tmem_base + SF_COL + 4, acc);
+                            tc_mma_mx(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
+                                      idesc | (sid << 29) | (sid << 4),
+                                      (tmem_base + SF_COL) | (sid << 30),
+                                      (tmem_base + SF_COL + 4) | (sid << 30), acc);
                         else
                             tc_mma<FP8>(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc);
                     }
@@ -339,66 +374,112 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
             }
         }
-    } else if (warp == 2) {
+    } else if (warp == 2 || warp == 3) {
         // ------------------------------------- scale factors (block-scaled MMA)
-        // For each stage, in the producer's order: the UE8M0 bytes of A's 128
-        // row scales and of the two B row blocks' scales, written in the
-        // tcgen05.cp source layout (lane l holds rows l, 32+l, 64+l, 96+l of A,
-        // one 32-bit column each, the byte repeated for the four 32-wide K
-        // steps), then an arrive on the stage's full barrier.  Scales are read
-        // from global memory two stages ahead.
+        // Per group of four K blocks (in the producer's order): warp 3 copies
+        // the fp32 scales (A's 128 rows, B's two 128-row blocks, four K blocks
+        // each) from global memory into a staging ring with cp.async, SF_AHEAD
+        // groups ahead; warp 2 writes their UE8M0 bytes in the tcgen05.cp
+        // source layout (lane l holds rows l, 32+l, 64+l, 96+l of A, one 32-bit
+        // column each, byte j for K block 4g + j) and signals the MMA issuer.
+        // The split keeps global loads out of the warp that must fence its
+        // shared-memory writes for the async proxy.
         if constexpr (MX) {
             const int NB = p.b_rows / 128;
+            const int NG = (KB + SF_GROUP - 1) / SF_GROUP;  // groups per tile
             const int my_tiles = total_tiles > static_cast<int>(blockIdx.x)
                                      ? (total_tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
                                      : 0;
-            const int n_steps = my_tiles * KB;
-            auto load = [&](int i, float (&a)[4], float (&b)[2]) {
-                if (i >= n_steps) return;
-                const int tile = blockIdx.x + (i / KB) * gridDim.x, kb = i % KB;
-                int seg, row0, rows_valid, nt;
-                decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int r = row0 + lane + 32 * c;
-                    a[c] = r < p.rows_total ? __ldg(p.a_scales + static_cast<size_t>(r) * KB + kb) : 1.0f;
-                }
-                const int nb_lo = GATE_UP ? nt : 2 * nt;
-                const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
-                b[0] = __ldg(p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * KB + kb);
-                b[1] = __ldg(p.b_scales + (static_cast<size_t>(seg) * NB + nb_hi) * KB + kb);
-            };
-            float a0[4] = {}, a1[4] = {}, a2[4] = {}, b0[2] = {}, b1[2] = {}, b2[2] = {};
-            load(0, a0, b0);
-            load(1, a1, b1);
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int i = 0; i < n_steps; ++i) {
-                load(i + 2, a2, b2);
+            const int n_groups = my_tiles * NG;
+            bool ok = true;
+            // lane 0 waits, the warp follows (bounded; false on timeout/abort)
+            auto warp_wait = [&](uint64_t *bar, uint32_t parity) {
                 int go = 1;
-                if (lane == 0) go = mbar_wait(&s.empty[stage], phase ^ 1, abort, p.status) ? 1 : 0;
-                if (!__shfl_sync(0xffffffffu, go, 0)) break;
-                uint8_t *sf = s.sf[stage];
-                *reinterpret_cast<uint4 *>(sf + 16 * lane) =
-                    make_uint4(e8m0x4(a0[0]), e8m0x4(a0[1]), e8m0x4(a0[2]), e8m0x4(a0[3]));
-                const uint32_t bl = e8m0x4(b0[0]), bh = e8m0x4(b0[1]);
-                *reinterpret_cast<uint4 *>(sf + 512 + 16 * lane) = make_uint4(bl, bl, bl, bl);
-                *reinterpret_cast<uint4 *>(sf + 1024 + 16 * lane) = make_uint4(bh, bh, bh, bh);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.full[stage]);
+                if (lane == 0) go = mbar_wait(bar, parity, abort, p.status) ? 1 : 0;
+                return __shfl_sync(0xffffffffu, go, 0) != 0;
+            };
+            if (warp == 3) {
+                // group i: 4-byte cp.async copies into staging slot i % SF_STAGING
+                // (K blocks past the end and rows past the last: zero fill), one
+                // commit group per group (empty past the last one)
+                auto issue = [&](int i) {
+                    if (i < n_groups) {
+                        const int tile = blockIdx.x + (i / NG) * gridDim.x;
+                        const int kb0 = (i % NG) * SF_GROUP;
+                        int seg, row0, rows_valid, nt;
+                        decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
+                        const int slot = i % SF_STAGING;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    a0[c] = a1[c];
-                    a1[c] = a2[c];
+                        for (int c = 0; c < 4; ++c) {
+                            const int r = row0 + lane + 32 * c;
+#pragma unroll
+                            for (int j = 0; j < SF_GROUP; ++j) {
+                                const bool in = r < p.rows_total && kb0 + j < KB;
+                                cp_async4(&s.sf_a[slot][j][lane + 32 * c],
+                                          p.a_scales + (in ? static_cast<size_t>(r) * KB + kb0 + j : 0),
+                                          in);
+                            }
+                        }
+                        if (lane < 2 * SF_GROUP) {
+                            const int which = lane / SF_GROUP, j = lane % SF_GROUP;
+                            const int nb = which == 0 ? (GATE_UP ? nt : 2 * nt)
+                                                      : (GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1);
+                            const bool in = kb0 + j < KB;
+                            cp_async4(&s.sf_b[slot][which][j],
+                                      p.b_scales + (in ? (static_cast<size_t>(seg) * NB + nb) * KB + kb0 + j : 0),
+                                      in);
+                        }
+                    }
+                    cp_async_commit();
+                };
+                auto claim = [&](int j) {  // staging slot of group j is free again
+                    return j >= n_groups ||
+                           warp_wait(&s.sf_empty[j % SF_STAGING], ((j / SF_STAGING) & 1) ^ 1);
+                };
+                for (int j = 0; j < SF_AHEAD && ok; ++j) {
+                    if (!claim(j)) ok = false;
+                    else issue(j);
                 }
-                b0[0] = b1[0];
-                b0[1] = b1[1];
-                b1[0] = b2[0];
-                b1[1] = b2[1];
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1;
+                for (int i = 0; i < n_groups && ok; ++i) {
+                    if (!claim(i + SF_AHEAD)) break;
+                    issue(i + SF_AHEAD);
+                    cp_async_wait<SF_AHEAD>();  // group i's copies have landed
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.sf_full[i % SF_STAGING]);
+                }
+                cp_async_wait<0>();
+            } else {
+                for (int i = 0; i < n_groups; ++i) {
+                    const int slot = i % SF_STAGING;
+                    if (!warp_wait(&s.sf_full[slot], (i / SF_STAGING) & 1)) break;
+                    uint32_t wa[4], wb[2];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t w = 0;
+#pragma unroll
+                        for (int j = 0; j < SF_GROUP; ++j)
+                            w |= e8m0(s.sf_a[slot][j][lane + 32 * c]) << (8 * j);
+                        wa[c] = w;
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t w = 0;
+#pragma unroll
+                        for (int j = 0; j < SF_GROUP; ++j) w |= e8m0(s.sf_b[slot][h][j]) << (8 * j);
+                        wb[h] = w;
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.sf_empty[slot]);
+                    const int buf = i % SF_BUFS;
+                    // the block's previous contents were copied to TMEM
+                    if (!warp_wait(&s.sf_free[buf], ((i / SF_BUFS) & 1) ^ 1)) break;
+                    uint8_t *sf = s.sf[buf];
+                    *reinterpret_cast<uint4 *>(sf + 16 * lane) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+                    *reinterpret_cast<uint4 *>(sf + 512 + 16 * lane) = make_uint4(wb[0], wb[0], wb[0], wb[0]);
+                    *reinterpret_cast<uint4 *>(sf + 1024 + 16 * lane) = make_uint4(wb[1], wb[1], wb[1], wb[1]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.sf_ready[buf]);
                 }
             }
         }

@@ -191,19 +191,6 @@ constexpr int RS_KC = 256;                 // columns per chunk
 constexpr int RS_WLD = RS_KC + 8;          // padded W_r row, bf16 elements
 constexpr int RS_STAGES = 4;
 
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
-                 "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 template <int BT>
 constexpr size_t router_small_smem() {
     return static_cast<size_t>(RS_STAGES) * (32 * RS_WLD + BT * RS_KC) * 2 +
