@@ -58,10 +58,9 @@ def kernel_traffic(kernel: str, workload: str):
         for pth in rec["sources"]:
             with open(os.path.join(ROOT, pth), "rb") as f:
                 h.update(f.read())
-        k = rec["kernels"][kernel]
-        if h.hexdigest() != rec["source_sha256"] or k["workload"] != workload:
+        if h.hexdigest() != rec["source_sha256"]:
             return None
-        return float(k["traffic_bytes_per_launch"])
+        return float(rec["workloads"][workload][kernel]["traffic_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
         return None
 
