@@ -76,31 +76,31 @@ __device__ __forceinline__ float sigmoid_cw(float l, const ExpConsts &k) {
 }
 
 // ------------------------------------------------------- router_scores ---
-// Larger batches: a CTA of 64 threads owns 64 tokens x 64 experts; thread
-// (ty, tx) owns tokens {4ty..4ty+3, 32+4ty..32+4ty+3} x experts {4tx..4tx+3,
-// 32+4tx..32+4tx+3}, 64 accumulators, each still a sequential FMA chain over
-// d.  Per k step: four 16-byte shared loads (x by broadcast, W_r conflict-
-// free) feed 64 FMAs.  x and W_r chunks of 32 columns are staged transposed
-// ([k][row], binary32) through registers one chunk ahead.
-constexpr int RT_B = 64, RT_KC = 32, RT_THREADS = 64;
+// Larger batches: a CTA of 128 threads owns 64 tokens x 64 experts; thread
+// (ty, tx), ty < 8, tx < 16, owns tokens {4ty..4ty+3, 32+4ty..32+4ty+3} x
+// experts {4tx..4tx+3}, 32 accumulators, each still a sequential FMA chain
+// over d (the paired FMA of sm_100 does two independent correctly rounded
+// FMAs per instruction, on experts (4tx, 4tx+1) and (4tx+2, 4tx+3)).  Per k
+// step: three 16-byte shared loads (x by broadcast, W_r two wavefronts) feed
+// 32 FMAs.  x and W_r chunks of 32 columns are staged transposed ([k][row],
+// binary32) through registers one chunk ahead.
+constexpr int RT_B = 64, RT_KC = 32, RT_THREADS = 128;
 
 __global__ void __launch_bounds__(RT_THREADS)
 router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w, int T, int d,
                      int E, float *__restrict__ scores, PreNorm pn) {
     __shared__ __align__(16) float xs[2][RT_KC][RT_B];  // [k][token]
     __shared__ __align__(16) float ws[2][RT_KC][RT_B];  // [k][expert]
-    const int tid = threadIdx.x, tx = tid & 7, ty = tid >> 3;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int t0 = blockIdx.y * RT_B, e0 = blockIdx.x * RT_B;
     pdl_wait_and_trigger();
 
-    // acc[a][j] holds experts (2j, 2j+1) of the thread's 8: the paired FMA of
-    // sm_100 does two independent correctly rounded FMAs per instruction, so
-    // every output is still its own sequential binary32 FMA chain
-    float2 acc[8][4];
+    // acc[a][j]: token a of the thread's 8, experts (4tx + 2j, 4tx + 2j + 1)
+    float2 acc[8][2];
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = make_float2(0.0f, 0.0f);
+        for (int b = 0; b < 2; ++b) acc[a][b] = make_float2(0.0f, 0.0f);
 
     constexpr int VPR = RT_KC / 8;                 // 16-byte vectors per row per chunk
     constexpr int NV = 2 * RT_B * VPR;             // x rows then W_r rows
@@ -149,15 +149,13 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
             const float4 xa = *reinterpret_cast<const float4 *>(&xs[buf][kk][4 * ty]);
             const float4 xb = *reinterpret_cast<const float4 *>(&xs[buf][kk][32 + 4 * ty]);
             const float4 wa = *reinterpret_cast<const float4 *>(&ws[buf][kk][4 * tx]);
-            const float4 wb = *reinterpret_cast<const float4 *>(&ws[buf][kk][32 + 4 * tx]);
             const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-            const float2 wv[4] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w),
-                                  make_float2(wb.x, wb.y), make_float2(wb.z, wb.w)};
+            const float2 wv[2] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w)};
 #pragma unroll
             for (int a = 0; a < 8; ++a) {
                 const float2 x2 = make_float2(xv[a], xv[a]);
 #pragma unroll
-                for (int b = 0; b < 4; ++b) acc[a][b] = __ffma2_rn(x2, wv[b], acc[a][b]);
+                for (int b = 0; b < 2; ++b) acc[a][b] = __ffma2_rn(x2, wv[b], acc[a][b]);
             }
         }
         if (kc + 1 < nk) store(buf ^ 1);
@@ -170,8 +168,8 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
         const int t = t0 + (a < 4 ? 4 * ty + a : 32 + 4 * ty + a - 4);
         if (t >= T) continue;
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            const int e = e0 + (b < 4 ? 4 * tx + b : 32 + 4 * tx + b - 4);
+        for (int b = 0; b < 4; ++b) {
+            const int e = e0 + 4 * tx + b;
             const float l = (b & 1) ? acc[a][b >> 1].y : acc[a][b >> 1].x;
             if (e < E) scores[static_cast<size_t>(t) * E + e] = sigmoid_cw(l, k);
         }

@@ -379,3 +379,29 @@ def test_prenorm_router_decode_dims_bitexact():
         assert np.array_equal(idx.cpu().numpy(), ridx)
         # zero experts: the block returns the residual stream unchanged
         assert torch.equal(out.cpu().view(torch.int16), h.view(torch.int16))
+
+
+# ------------------------------------------------------ launch records ---
+
+@pytest.mark.parametrize("T,prenorm,precision", [(64, False, "fp8"), (300, False, "fp8"),
+                                                 (64, True, "fp8"), (64, False, "bf16")])
+def test_launch_names_follow_the_path(T, prenorm, precision):
+    """moe_last_launch_name lists the kernels of the last call in launch order:
+    the single-CTA permutation up to 256 tokens, three kernels beyond."""
+    from moe_inputs import make_residual
+    cfg = CONFIGS["tiny"].with_(precision=precision, T=T)
+    inp = _dev(make_inputs(cfg, seed=9))
+    layer = moe.MoELayer(inp["w_router"], inp["bias"], inp["w13"], inp["w2"], top_k=cfg.top_k,
+                         precision=precision)
+    h, gamma = make_residual(cfg, seed=9, device=DEV)
+    run = (lambda: layer.forward_prenorm(h, gamma)) if prenorm else (lambda: layer(inp["x"]))
+    run()
+    assert layer.check_status(T) == 0
+    run()  # the record belongs to the last call on this thread
+    names = moe.moe_last_launch_names()
+    perm = ["perm_small"] if T <= 256 else ["perm_hist", "perm_scan", "perm_scatter"]
+    scatter = "quant_scatter" if precision == "fp8" else "scatter_bf16"
+    want = (["prenorm_rstd"] if prenorm else []) + ["router_scores", "router_topk"] + perm + \
+        [scatter, "grouped_gemm_gate_up", "grouped_gemm_down", "combine"]
+    assert names == want
+    assert moe.moe_last_launch_count() == len(want)
