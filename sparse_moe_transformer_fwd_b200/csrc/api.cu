@@ -189,9 +189,12 @@ PermScratch perm_scratch(void *ws, const Layout &L) {
     return p;
 }
 
+// max_seg_rows: a bound on every segment's rows (T when the segments come
+// from the routing, where a token picks an expert at most once; T*k for
+// caller-given offsets)
 int grouped(const moe_shape *s, const void *a, const float *a_scales, const void *w13,
             const float *w13_scales, const void *w2, const float *w2_scales, uint16_t *y,
-            void *ws, const Layout &L, cudaStream_t st, int *launches) {
+            void *ws, const Layout &L, cudaStream_t st, int *launches, int max_seg_rows) {
     const bool fp8 = is_fp8(s);
     const PermScratch ps = perm_scratch(ws, L);
     const int Rs = s->T * (s->top_k + s->n_shared);
@@ -207,6 +210,7 @@ int grouped(const moe_shape *s, const void *a, const float *a_scales, const void
     g.status = at<int>(ws, L.status);
     g.inject_fault = inject_gemm_fault() ? 1 : 0;
     g.ue8m0 = is_ue8m0(s);
+    g.max_seg_rows = max_seg_rows;
     // gate/up GEMM + SwiGLU
     g.gate_up = true;
     g.a = a;
@@ -383,7 +387,8 @@ int moe_grouped_swiglu(const moe_shape *s, const void *a, const float *a_scales,
     LAUNCH(launch_tile_table(offsets, s->n_experts, s->T, s->top_k, s->n_shared,
                              perm_scratch(ws, L), at<int>(ws, L.status), st, &n),
            "tile table");
-    RETURN_IF(grouped(s, a, a_scales, w13, w13_scales, w2, w2_scales, y, ws, L, st, &n));
+    RETURN_IF(grouped(s, a, a_scales, w13, w13_scales, w2, w2_scales, y, ws, L, st, &n,
+                      s->T * s->top_k));
     mark_launch(st, n);
     g_launches = n;
     return MOE_OK;
@@ -462,7 +467,7 @@ int forward_impl(const moe_shape *s, const uint16_t *x, const uint16_t *gamma, f
                "scatter");
     uint16_t *y = at<uint16_t>(ws, L.y);
     RETURN_IF(grouped(s, at<uint8_t>(ws, L.a), fp8 ? at<float>(ws, L.a_scales) : nullptr, w13,
-                      w13_scales, w2, w2_scales, y, ws, L, st, &n));
+                      w13_scales, w2, w2_scales, y, ws, L, st, &n, s->T));
     LAUNCH(launch_combine(y, row_of, gates, s->T, s->d_model, s->top_k, s->n_shared, out, st, &n,
                           gamma ? x : nullptr),
            "combine");

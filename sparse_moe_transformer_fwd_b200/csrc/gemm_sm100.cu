@@ -165,11 +165,12 @@ __device__ __forceinline__ void promote32(float2 (&acc)[64], int base, const flo
 // exponent field 0, matching E8M0 code 0).
 __device__ __forceinline__ uint32_t e8m0(float sc) { return (__float_as_uint(sc) >> 23) & 0xffu; }
 
-template <bool FP8, bool GATE_UP, bool MX>
+template <bool FP8, bool GATE_UP, bool MX, bool M64>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const KParams p) {
     static_assert(FP8 || !MX, "the block-scaled MMA takes e4m3 operands");
+    static_assert(!M64 || (FP8 && !MX), "64-row tiles: fp8 with software promotion only");
     using R = Roles<MX>;
     extern __shared__ uint8_t smem_raw[];
     GemmSmem &s = *reinterpret_cast<GemmSmem *>(
@@ -178,9 +179,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const int KB = FP8 ? p.K / 128 : p.K / 64;  // stages per tile (128 bytes of K each)
     // stages per promotion chunk: FP8 128 K (the scale block); BF16 256 K;
     // MX: the tensor core applies the scales, so chunks are mx_spc K blocks
-    const int SPC = MX ? p.mx_spc : (FP8 ? 1 : 4);
+    // M64 (batches of at most 64 tokens, so every segment fits 64 rows): the
+    // MMA is M = 64, which fills only lanes 16k..16k+15 of each 32-lane TMEM
+    // quadrant; K steps 2p and 2p + 1 write the two lane halves of one
+    // accumulator buffer, and the epilogue promotes both in one pass (each
+    // thread with its own K step's scales), so the TMEM round trip is paid
+    // once per two K steps.  The halves' sums are added at the tile end.
+    const int SPC = MX ? p.mx_spc : (M64 ? 2 : (FP8 ? 1 : 4));
     // the epilogue multiplies each chunk by s_a * s_w (software promotion)
     constexpr bool SCALED = FP8 && !MX;
+    constexpr int TM = M64 ? 64 : BM;  // rows of an MMA tile
     const int NCH = (KB + SPC - 1) / SPC;        // K chunks per tile (last may be short)
     const int n_seg = p.n_segments;
 
@@ -256,7 +264,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         break;
                     }
                     const bool inject = p.inject_fault && blockIdx.x == 0 && armed == 0;
-                    mbar_arrive_expect_tx(&s.full[stage], STAGE_TX + (inject ? 16 : 0));
+                    mbar_arrive_expect_tx(&s.full[stage],
+                                          TM * 128 + B_BYTES + (inject ? 16 : 0));
                     const int kc = FP8 ? kb * 128 : kb * 64;
                     tma_load_2d(s.a[stage], &tmap_a, kc, row0, &s.full[stage]);
                     // each B box is one contiguous 16 KB weight tile
@@ -291,7 +300,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
-            constexpr uint32_t idesc = MX ? instr_desc_mx(BM, BN) : instr_desc<FP8>(BM, BN);
+            constexpr uint32_t idesc = MX ? instr_desc_mx(BM, BN) : instr_desc<FP8>(TM, BN);
             int stage = 0;
             uint32_t phase = 0;
             int tb = 0;
@@ -319,7 +328,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + tb * BN;
+                    // M64: odd K steps write the upper 16 lanes of each quadrant
+                    const uint32_t d_tmem = tmem_base + tb * BN +
+                                            (M64 ? static_cast<uint32_t>((kb & 1) * 16) << 16 : 0u);
                     const uint64_t adesc = smem_desc_sw128(smem_u32(s.a[stage]));
                     const uint64_t bdesc = smem_desc_sw128(smem_u32(s.b[stage]));
                     if (group_first) {
@@ -340,8 +351,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         // +32 bytes of K per instruction: +2 in the >>4 address field;
-                        // each K chunk starts a fresh partial sum
-                        const uint32_t acc = (chunk_first && kk == 0) ? 0u : 1u;
+                        // each K chunk (M64: each K step) starts a fresh partial sum
+                        const uint32_t acc = ((M64 || chunk_first) && kk == 0) ? 0u : 1u;
                         if constexpr (MX)
                             tc_mma_mx(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
                                       idesc | (sid << 29) | (sid << 4),
@@ -488,7 +499,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(R::EPILOGUE_REGS));
         const int q = warp & 3;            // TMEM lane quadrant = tile rows 32q..32q+31
         const int half = (warp - 4) >> 2;  // column half
-        const int r_in = q * 32 + lane;
+        // M64: lane l holds tile row 16q + l % 16 of K step parity l / 16
+        const int hh = M64 ? (lane >> 4) : 0;
+        const int r_in = M64 ? q * 16 + (lane & 15) : q * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
         const int NB = p.b_rows / 128;
         int tb = 0;
@@ -498,8 +511,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++iter) {
             int seg, row0, rows_valid, nt;
             decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
-            const bool warp_active = q * 32 < rows_valid;
+            const bool warp_active = q * (M64 ? 16 : 32) < rows_valid;
             const bool valid = r_in < rows_valid;
+            const bool store_row = valid && hh == 0;  // M64: one lane of the pair stores
             const size_t row = static_cast<size_t>(row0) + r_in;
             const int col_lo = half * 64, col_hi = 128 + half * 64;
             float2 acc2[64];  // columns (2j, 2j+1) of the thread's 128
@@ -507,22 +521,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
             const int nb_lo = GATE_UP ? nt : 2 * nt;
             const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
-            const float *sw_lo_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * NCH : nullptr;
-            const float *sw_hi_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_hi) * NCH : nullptr;
-            const float *sa_p = SCALED ? p.a_scales + row * NCH : nullptr;
+            const float *sw_lo_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * KB : nullptr;
+            const float *sw_hi_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_hi) * KB : nullptr;
+            const float *sa_p = SCALED ? p.a_scales + row * KB : nullptr;
+            // K block whose partial this thread promotes in chunk c
+            auto kb_of = [&](int c) { return M64 ? 2 * c + hh : c; };
             // scales of chunk c are loaded one chunk ahead (global latency)
             float nsa = 0.0f, nswl = 1.0f, nswh = 1.0f;
-            if (SCALED && warp_active) {
-                nsa = valid ? __ldg(sa_p) : 0.0f;
-                nswl = __ldg(sw_lo_p);
-                nswh = __ldg(sw_hi_p);
+            if (SCALED && warp_active && kb_of(0) < KB) {
+                nsa = valid ? __ldg(sa_p + kb_of(0)) : 0.0f;
+                nswl = __ldg(sw_lo_p + kb_of(0));
+                nswh = __ldg(sw_hi_p + kb_of(0));
             }
             for (int c = 0; c < NCH; ++c) {
                 const float sc_lo = SCALED ? nsa * nswl : 1.0f, sc_hi = SCALED ? nsa * nswh : 1.0f;
-                if (SCALED && warp_active && c + 1 < NCH) {
-                    nsa = valid ? __ldg(sa_p + c + 1) : 0.0f;
-                    nswl = __ldg(sw_lo_p + c + 1);
-                    nswh = __ldg(sw_hi_p + c + 1);
+                const bool kvalid = !M64 || kb_of(c) < KB;  // M64, odd K: no partial in the upper half
+                if (SCALED && warp_active && c + 1 < NCH && kb_of(c + 1) < KB) {
+                    nsa = valid ? __ldg(sa_p + kb_of(c + 1)) : 0.0f;
+                    nswl = __ldg(sw_lo_p + kb_of(c + 1));
+                    nswh = __ldg(sw_hi_p + kb_of(c + 1));
                 }
                 if (!mbar_wait(&s.tfull[tb], tphase, abort, p.status)) {
                     ok = false;
@@ -533,21 +550,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 // buffer is released as soon as the last piece is in registers
                 // (before its FMAs), since the MMA two chunks ahead waits for it
                 float va[32], vb[32];
+                const bool add = warp_active && kvalid;  // the loads below are warp-wide
                 if (warp_active) {
                     const uint32_t base = lane_base + tb * BN;
                     tmem_ld32(base + col_lo, va);
                     tmem_ld32(base + col_lo + 32, vb);
                     tmem_wait_ld(va, vb);
-                    promote32<SCALED>(acc2, 0, va, sc_lo);
+                    if (add) promote32<SCALED>(acc2, 0, va, sc_lo);
                     tmem_ld32(base + col_hi, va);
-                    promote32<SCALED>(acc2, 16, vb, sc_lo);
+                    if (add) promote32<SCALED>(acc2, 16, vb, sc_lo);
                     tmem_ld32(base + col_hi + 32, vb);
                     tmem_wait_ld(va, vb);
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.tempty[tb]);
-                if (warp_active) {
+                if (add) {
                     promote32<SCALED>(acc2, 32, va, sc_hi);
                     promote32<SCALED>(acc2, 48, vb, sc_hi);
                 }
@@ -557,6 +575,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
             }
             if (!ok) break;
+            if constexpr (M64) {
+                // even and odd K steps' sums of the same row meet (both lanes get
+                // the same total)
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    acc2[i].x += __shfl_xor_sync(0xffffffffu, acc2[i].x, 16);
+                    acc2[i].y += __shfl_xor_sync(0xffffffffu, acc2[i].y, 16);
+                }
+            }
             // column c of the thread's 128 (in place, no copy)
             auto acc = [&](int c) -> float & { return (c & 1) ? acc2[c >> 1].y : acc2[c >> 1].x; };
             if constexpr (GATE_UP) {
@@ -579,7 +606,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         break;
                     }
                     const float amax = fmaxf(m, s.amax_x[par][half ^ 1][r_in]);
-                    if (valid) {
+                    if (store_row) {
                         float sc = 1.0f, inv = 0.0f;
                         if (amax != 0.0f) {
                             if (p.ue8m0) {
@@ -605,7 +632,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         }
                         if (half == 0) p.out_scales[row * (p.N_out / 128) + nt] = sc;
                     }
-                } else if (valid) {
+                } else if (store_row) {
                     uint16_t *h = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 128 +
                                   half * 64;
 #pragma unroll
@@ -618,7 +645,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         *reinterpret_cast<uint4 *>(h + c) = o;
                     }
                 }
-            } else if (valid) {
+            } else if (store_row) {
                 uint16_t *y = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 256;
 #pragma unroll
                 for (int c = 0; c < 64; c += 8) {
@@ -667,13 +694,13 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-bool make_map_2d(CUtensorMap *m, const void *base, bool fp8, int K, int rows) {
+bool make_map_2d(CUtensorMap *m, const void *base, bool fp8, int K, int rows, int box_rows = 128) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const int es = fp8 ? 1 : 2;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * es};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), 128};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     return enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -682,7 +709,7 @@ bool make_map_2d(CUtensorMap *m, const void *base, bool fp8, int K, int rows) {
 }
 
 
-template <bool FP8, bool GATE_UP, bool MX>
+template <bool FP8, bool GATE_UP, bool MX, bool M64 = false>
 cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams &kp, int grid,
                      cudaStream_t st) {
     const size_t smem = sizeof(GemmSmem) + 1024;
@@ -692,16 +719,16 @@ cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams
         // refuse to launch a build whose register count differs, as the
         // epilogue's increase would then never be granted.
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, grouped_gemm_kernel<FP8, GATE_UP, MX>);
+        cudaError_t e = cudaFuncGetAttributes(&fa, grouped_gemm_kernel<FP8, GATE_UP, MX, M64>);
         if (e != cudaSuccess) return e;
         if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(grouped_gemm_kernel<FP8, GATE_UP, MX>,
+        e = cudaFuncSetAttribute(grouped_gemm_kernel<FP8, GATE_UP, MX, M64>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    return launch_pdl(grouped_gemm_kernel<FP8, GATE_UP, MX>, dim3(grid), dim3(NUM_THREADS), smem, st,
+    return launch_pdl(grouped_gemm_kernel<FP8, GATE_UP, MX, M64>, dim3(grid), dim3(NUM_THREADS), smem, st,
                       ma, mb, kp);
 }
 
@@ -711,7 +738,11 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     if (g.n_segments > MAX_SEG) return cudaErrorInvalidValue;
     const int b_rows = g.gate_up ? 2 * g.N_out : g.N_out;
     CUtensorMap ma, mb;
-    if (!make_map_2d(&ma, g.a, g.fp8, g.K, g.rows_total)) return cudaErrorInvalidValue;
+    // 64-row MMA tiles when no segment can exceed 64 rows (at most 64 tokens:
+    // a token picks an expert at most once, and the shared segment has T rows)
+    const bool m64 = g.fp8 && !g.ue8m0 && g.max_seg_rows <= 64;
+    if (!make_map_2d(&ma, g.a, g.fp8, g.K, g.rows_total, m64 ? 64 : 128))
+        return cudaErrorInvalidValue;
     // B in the tiled layout: one row of 128 bytes per tile row, tiles stacked
     const long long b_tile_rows = static_cast<long long>(g.n_slots) * b_rows * (g.K * (g.fp8 ? 1 : 2) / 128);
     if (b_tile_rows >= (1LL << 31)) return cudaErrorInvalidValue;
@@ -746,6 +777,9 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     if (g.fp8 && g.ue8m0)
         e = g.gate_up ? launch_t<true, true, true>(ma, mb, kp, grid, st)
                       : launch_t<true, false, true>(ma, mb, kp, grid, st);
+    else if (g.fp8 && m64)
+        e = g.gate_up ? launch_t<true, true, false, true>(ma, mb, kp, grid, st)
+                      : launch_t<true, false, false, true>(ma, mb, kp, grid, st);
     else if (g.fp8)
         e = g.gate_up ? launch_t<true, true, false>(ma, mb, kp, grid, st)
                       : launch_t<true, false, false>(ma, mb, kp, grid, st);

@@ -126,6 +126,7 @@ struct GemmArgs {
     int *status;
     int inject_fault;       // test hook: make one bounded wait run out (see api.cu)
     bool ue8m0;             // fp8 gate/up: H requantised with power-of-two scales
+    int max_seg_rows;       // bound on any segment's rows (T: one row per token and expert)
 };
 cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launches);
 

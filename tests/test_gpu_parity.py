@@ -252,6 +252,10 @@ FWD_CASES = {
     "tiny_k16": dict(top_k=16),
     "tiny_scale2.5": dict(routed_scale=2.5),
     "tiny_wide": dict(d_model=1024, d_expert=512, n_experts=64, top_k=6, T=300),
+    # at most 64 tokens: 64-row MMA tiles in the fp8 GEMMs (full shared
+    # segment; and an odd number of K blocks in the down GEMM, d_expert 384)
+    "tiny_T64": dict(T=64),
+    "tiny_T48_de384": dict(T=48, d_expert=384),
 }
 
 
