@@ -713,8 +713,8 @@ template <bool FP8, bool GATE_UP, bool MX, bool M64 = false>
 cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams &kp, int grid,
                      cudaStream_t st) {
     const size_t smem = sizeof(GemmSmem) + 1024;
-    static bool configured = false;  // per template instance; attribute is per device function
-    if (!configured) {
+    static std::atomic<uint64_t> configured{0};  // per template instance, one bit per device
+    if (first_use_on_device(configured)) {
         // setmaxnreg redistributes exactly NUM_THREADS * LAUNCH_REGS registers:
         // refuse to launch a build whose register count differs, as the
         // epilogue's increase would then never be granted.
@@ -726,7 +726,7 @@ cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem));
         if (e != cudaSuccess) return e;
-        configured = true;
+        mark_used_on_device(configured);
     }
     return launch_pdl(grouped_gemm_kernel<FP8, GATE_UP, MX, M64>, dim3(grid), dim3(NUM_THREADS), smem, st,
                       ma, mb, kp);

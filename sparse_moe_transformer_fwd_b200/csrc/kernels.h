@@ -3,6 +3,8 @@
 // kernels it enqueued to *launches.
 #pragma once
 
+#include <atomic>
+
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
@@ -131,6 +133,22 @@ struct GemmArgs {
 cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launches);
 
 int num_sms();
+
+// Function attributes (dynamic shared memory size) are per device: true once
+// per device for the given per-call-site flag word (devices 0..63; larger
+// device numbers are configured on every call).
+inline bool first_use_on_device(std::atomic<uint64_t> &done) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64) return true;
+    const uint64_t bit = 1ull << dev;
+    return (done.load(std::memory_order_acquire) & bit) == 0;
+}
+inline void mark_used_on_device(std::atomic<uint64_t> &done) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64) done.fetch_or(1ull << dev, std::memory_order_release);
+}
 
 // Error/launch bookkeeping shared by the C entry points (api.cu).
 int record_error(int code, const char *msg);  // sets moe_last_error, returns code

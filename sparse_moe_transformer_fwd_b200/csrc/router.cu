@@ -375,12 +375,12 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
     } else {
         constexpr int BT = 4;
         constexpr size_t smem = router_small_smem<BT>();
-        static bool configured = false;
-        if (!configured) {
+        static std::atomic<uint64_t> configured{0};  // one bit per device
+        if (first_use_on_device(configured)) {
             LAUNCH_OR_RETURN(cudaFuncSetAttribute(router_scores_small_kernel<BT>,
                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                   static_cast<int>(smem)));
-            configured = true;
+            mark_used_on_device(configured);
         }
         dim3 grid((E + 31) / 32, (T + BT - 1) / BT);
         LAUNCH_OR_RETURN(launch_pdl(router_scores_small_kernel<BT>, grid, dim3(BT * 32), smem, st, x, w, T,

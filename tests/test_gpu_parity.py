@@ -256,6 +256,7 @@ FWD_CASES = {
     # segment; and an odd number of K blocks in the down GEMM, d_expert 384)
     "tiny_T64": dict(T=64),
     "tiny_T48_de384": dict(T=48, d_expert=384),
+    "tiny_T64_noshared": dict(T=64, n_shared=0),
 }
 
 
