@@ -7,7 +7,7 @@ batch (T=64 tokens, d_model 7168, 256 routed experts top-8 + 1 shared,
 d_expert 2048, e4m3 blockwise weights and activations, bf16 I/O).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|skew|bf16|tiny]
+                    [--workload decode|prefill|skew|bf16|...|dense_decode|dense_prefill]
 
 N > 1 (launched by torch.distributed.run) runs N independent replicas, one
 per GPU (the layer has no exchange step on one node's replicas): value =
@@ -30,9 +30,11 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from moe_inputs import CONFIGS, make_inputs, make_residual  # noqa: E402
+from moe_inputs import (CONFIGS, DENSE_CONFIGS, make_dense_inputs, make_inputs,  # noqa: E402
+                        make_residual)
 
 METRIC = "MoE-layer tokens/s at DeepSeek-V3 dims"
+DENSE_METRIC = "dense FFN-layer tokens/s at DeepSeek-V3 dims (first layers, d_ff 18432)"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -340,6 +342,164 @@ def run_ours(args, world, rank, local):
     return res, cfg
 
 
+# ------------------------------------------------------ dense layer arm ---
+
+def dense_roofline(cfg, ms: float, peaks, peak_kind: str):
+    """Roofline of the dense gate/up GEMM: its algorithmic bytes (weights,
+    their scales, x codes and scales in, H codes and scales out) and FLOPs;
+    the bound is the roof with the longer floor at the measured peaks (HBM
+    copy bandwidth; tensor: measured bf16 GEMM x 2 for e4m3, the nominal
+    4.5 / 2.25 ratio)."""
+    T, d, f = cfg.T, cfg.d_model, cfg.d_ff
+    es = 2 if cfg.precision == "bf16" else 1
+    sc = 0 if es == 2 else 4
+    nbytes = (2 * f * d * es + sc * (2 * f // 128) * (d // 128) + T * d * es + sc * T * (d // 128)
+              + T * f * es + sc * T * (f // 128))
+    flops = 2.0 * T * d * 2 * f
+    tc_peak = peaks["bf16_tflops"] * (1 if es == 2 else 2)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (tc_peak * 1e12)
+    src = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"
+    if t_tc > t_hbm:
+        ach = flops / (ms * 1e-3) / 1e12
+        return {"kernel": "grouped_gemm_gate_up", "bound": "tensor", "achieved": round(ach, 1),
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": round(ach / tc_peak, 4),
+                "peak_source": src + (" bf16_tflops x 2 (e4m3)" if es == 1 else " bf16_tflops"),
+                "algorithmic_flops": flops, "kernel_ms": round(ms, 4), "traffic": None}
+    ach = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": "grouped_gemm_gate_up", "bound": "hbm", "achieved": round(ach, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+            "peak_source": src + " hbm_gbs", "algorithmic_bytes": nbytes,
+            "kernel_ms": round(ms, 4), "traffic": kernel_traffic("grouped_gemm_gate_up", cfg.name)}
+
+
+def run_dense(args, world, rank, local):
+    import sparse_moe_transformer_fwd_b200 as moe
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = DENSE_CONFIGS[args.workload]
+    inp = make_dense_inputs(cfg, seed=args.seed + rank, device=dev)
+    layer = moe.DenseFFN(inp["w13"], inp["w2"], precision=cfg.precision)
+    del inp["w13"], inp["w2"]
+    torch.cuda.empty_cache()
+    T = cfg.T
+    if args.prenorm:
+        x, gamma = make_residual(cfg, seed=args.seed + rank, device=dev)
+        call = lambda xx, out: layer.forward_prenorm(xx, gamma, 1e-6, out=out)
+    else:
+        x = inp["x"]
+        call = lambda xx, out: layer(xx, out=out)
+    out = torch.empty(T, cfg.d_model, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        call(x, out)
+    torch.cuda.synchronize()
+    if layer.check_status(T) != 0:
+        raise RuntimeError(f"device status: {moe.moe_last_error()}")
+    n_launch = moe.moe_last_launch_count()
+    names = moe.moe_last_launch_names()
+    gi = names.index("grouped_gemm_gate_up")
+    g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for a, b in g_ev:
+        a.record(stream)
+        b.record(stream)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            moe.moe_set_kernel_events([None] * gi + [g_ev[k][0], g_ev[k][1]])
+            call(x, out)
+        moe.moe_set_kernel_events(None)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_step = max_over_ranks(start.elapsed_time(stop), world, dev) / args.steps
+    g1_ms = float(np.mean([a.elapsed_time(b) for a, b in g_ev]))
+    nb = min(args.steps, 10)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)] for _ in range(nb)]
+    for k in range(nb):
+        moe.moe_set_kernel_events(ev[k])
+        call(x, out)
+    moe.moe_set_kernel_events(None)
+    torch.cuda.synchronize()
+    kmean = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(n_launch)]
+                      for k in range(nb)]).mean(0)
+    # end to end with host buffers
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty(T, cfg.d_model, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        call(x_dev, out)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        call(x_dev, out)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    if layer.check_status(T) != 0:
+        raise RuntimeError(f"device status: {moe.moe_last_error()}")
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    res = {
+        "metric": DENSE_METRIC, "value": round(job_throughput(T, world, ms_step), 1),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.precision == "bf16" else "e4m3",
+        "data": "synthetic (seeded; random-init weights of the DeepSeek-V3 dense FFN shape)",
+        "config": {
+            "workload": ("pre-norm block (h + FFN(RMSNorm(h)), fused) " if args.prenorm else "")
+                        + f"{cfg.name}: T={T}, d_model={cfg.d_model}, d_ff={cfg.d_ff}, "
+                        + {"fp8": "e4m3 1x128/128x128 blockwise, fp32 scales, bf16 I/O",
+                           "fp8_ue8m0": "e4m3 blockwise, power-of-two scales, bf16 I/O"}.get(
+                               cfg.precision, "bf16"),
+            "tokens_per_gpu": T,
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "l2": f"inputs larger than L2: {3 * cfg.d_model * cfg.d_ff / 1e6:.0f} MB of weights "
+                  "stream through every step",
+        },
+        "roofline": dense_roofline(cfg, g1_ms, peaks, peak_kind),
+        "kernels_ms": {n: round(float(v), 4) for n, v in zip(names, kmean)},
+        "e2e": {"value": round(T * world / (ms_e2e * 1e-3), 1), "unit": "tokens/s",
+                "ms_per_step": round(ms_e2e, 4),
+                "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                "d2h_bytes_per_step": int(out.numel() * out.element_size())},
+        "gpu_launches": n_launch * args.steps,
+        "clocks": clk.summary(),
+    }
+    return res, cfg
+
+
+def dense_oracle_time(cfg, n_tokens: int, seed: int, reps: int = 1):
+    """Time the oracle's dense layer on n_tokens rows of the batch (rows are
+    independent; the weights' quantisation is part of every call)."""
+    import oracle
+    from threadpoolctl import threadpool_limits
+    inp = make_dense_inputs(cfg, seed=seed)
+    u16 = lambda t: t.detach().contiguous().view(torch.int16).numpy().view(np.uint16)
+    tokens = list(range(0, cfg.T, max(1, cfg.T // n_tokens)))[:n_tokens]
+    x, w13, w2 = u16(inp["x"][tokens]), u16(inp["w13"]), u16(inp["w2"])
+    del inp
+    times = []
+    with threadpool_limits(limits=1):
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            oracle.dense_ffn(x, w13, w2, precision=cfg.precision)
+            times.append(time.perf_counter() - t0)
+    return times, len(tokens)
+
+
 # ----------------------------------------------------- oracle (CPU) arm ---
 
 def oracle_sample_time(cfg, dev, n_tokens: int, seed: int, reps: int = 1):
@@ -382,9 +542,32 @@ def cpu_model():
     return "unknown"
 
 
+def run_reference_dense(args, world):
+    cfg = DENSE_CONFIGS[args.workload]
+    dense_oracle_time(cfg, args.ref_tokens, args.seed, reps=1)
+    times, ntok = dense_oracle_time(cfg, args.ref_tokens, args.seed, reps=args.steps)
+    s_step = statistics.mean(times)
+    value = ntok / s_step
+    sample = (f"{ntok} tokens of the {cfg.name} batch per step through the oracle's dense layer "
+              "(weight quantisation, binary64 GEMMs); C core and numpy on 1 thread")
+    return {
+        "metric": DENSE_METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(s_step * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{cfg.name}: T={cfg.T}, d_model={cfg.d_model}, d_ff={cfg.d_ff}"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": sample, "cpu": cpu_model()},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }, cfg
+
+
 def run_reference(args, world, rank, local):
     if rank != 0:
         return None
+    if args.workload in DENSE_CONFIGS:
+        return run_reference_dense(args, world)
     cfg = CONFIGS[args.workload]
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     n_tok = args.ref_tokens
@@ -417,7 +600,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(CONFIGS), default="decode")
+    ap.add_argument("--workload", choices=list(CONFIGS) + list(DENSE_CONFIGS), default="decode")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-tokens", type=int, default=1,
                     help="tokens of the batch per oracle step (reference arm)")
@@ -435,10 +618,19 @@ def main():
             if r is not None:
                 print(json.dumps(r[0]), flush=True)
             return
-        r = run_ours(args, world, rank, local)
+        dense = args.workload in DENSE_CONFIGS
+        r = (run_dense if dense else run_ours)(args, world, rank, local)
         if r is not None:
             res, cfg = r
-            if world == 1 and not args.no_cpu_baseline:
+            if world == 1 and not args.no_cpu_baseline and dense:
+                times, ntok = dense_oracle_time(cfg, args.cpu_baseline_tokens, args.seed)
+                res["cpu_baseline"] = {
+                    "value": round(ntok / times[0], 4), "unit": "tokens/s", "cores": 1,
+                    "kind": "oracle",
+                    "sample": f"{ntok} tokens of the {cfg.name} batch through the oracle's dense "
+                              f"layer (incl. its weight quantisation), {times[0]:.1f} s, 1 thread",
+                    "cpu": cpu_model()}
+            elif world == 1 and not args.no_cpu_baseline:
                 dev = torch.device("cuda", local)
                 times, ntok, nexp = oracle_sample_time(cfg, dev, args.cpu_baseline_tokens,
                                                        args.seed)

@@ -235,6 +235,48 @@ int moe_forward_prenorm(const moe_shape *shape, const uint16_t *h, const uint16_
                         uint16_t *out, int32_t *topk_idx_out, void *ws, size_t ws_bytes,
                         void *stream);
 
+/* ------------------------------------------------------------------------
+ * Dense FFN layer: the first layers of the model, before the MoE layers
+ * ("DeepSeek-R1" architecture card, "Every architecture field": layout
+ * 3 x dense then 58 x MoE; ffns.dense is a gated MLP with d_ff 18432).
+ *   out = H W2^T,  H = silu(x Wg^T) * (x Wu^T)
+ * computed on the same kernels as the experts, with the same numerics per
+ * precision (x quantised 1x128, weights 128x128, H requantised 1x128 before
+ * the down GEMM; bf16: H rounded to bf16), every row of x in one segment.
+ * Shapes: d_model a multiple of 256, d_ff a multiple of 128, T >= 0. */
+typedef struct {
+    int T;         /* tokens */
+    int d_model;   /* 7168 for DeepSeek-V3 */
+    int d_ff;      /* 18432 for DeepSeek-V3 */
+    int precision; /* enum moe_precision */
+} moe_dense_shape;
+
+/* Bytes of workspace moe_dense_ffn needs (0 on an invalid shape).  It holds
+ * the status word first (read with moe_check_status), the quantised x, H,
+ * and for small batches the split-K partial sums of the down GEMM. */
+size_t moe_dense_workspace_size(const moe_dense_shape *shape);
+
+/* The dense layer.
+ *   x   bf16 [T, d_model]; out bf16 [T, d_model] (written by the down GEMM,
+ *       Y rounded once to bf16)
+ *   w13 [2*d_ff, d_model] (gate rows, then up rows) and w2 [d_model, d_ff]
+ *       in TILED layout, e4m3 with scales [2*d_ff/128, d_model/128] and
+ *       [d_model/128, d_ff/128] (MOE_FP8_BLOCK / MOE_FP8_UE8M0), or bf16
+ *       with NULL scales (MOE_BF16): the layout of one expert slot.
+ *   ws: moe_dense_workspace_size bytes, zero-filled once before first use. */
+int moe_dense_ffn(const moe_dense_shape *shape, const uint16_t *x, const void *w13,
+                  const float *w13_scales, const void *w2, const float *w2_scales,
+                  uint16_t *out, void *ws, size_t ws_bytes, void *stream);
+
+/* The dense FFN block with its pre-norm and residual: out = bf16(h + FFN(x))
+ * with x = bf16((h * rstd) * gamma) as in moe_forward_prenorm; the residual
+ * is added to the binary32 down-GEMM sum before its one rounding (Y is not
+ * stored). */
+int moe_dense_ffn_prenorm(const moe_dense_shape *shape, const uint16_t *h,
+                          const uint16_t *gamma, float eps, const void *w13,
+                          const float *w13_scales, const void *w2, const float *w2_scales,
+                          uint16_t *out, void *ws, size_t ws_bytes, void *stream);
+
 /* Synchronises `stream`, returns the workspace status word (MOE_OK or the
  * first device-recorded MOE_ERR_*), and resets it to MOE_OK.  A workspace must
  * be zero-filled once before first use (or passed here once) so its status

@@ -28,12 +28,13 @@ import os
 import torch
 
 __all__ = ["MoEConfig", "CONFIGS", "make_inputs", "expert_weights", "skew_bias_scale",
-           "make_residual"]
+           "make_residual", "DenseConfig", "DENSE_CONFIGS", "make_dense_inputs"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
 # tensor ids for seeding
 _TID_X, _TID_WR, _TID_BIAS, _TID_W13, _TID_W2, _TID_RANK, _TID_H, _TID_G = 1, 2, 3, 4, 5, 6, 7, 8
+_TID_DW13, _TID_DW2 = 9, 10
 
 
 @dataclasses.dataclass(frozen=True)
@@ -191,3 +192,46 @@ def make_inputs(cfg: MoEConfig, seed: int = 0, device="cpu", identical_experts: 
         w13[e].copy_(a)
         w2[e].copy_(c)
     return dict(x=x, w_router=w_r, bias=b, w13=w13, w2=w2)
+
+
+# ----------------------------------------------------------- dense layers --
+
+@dataclasses.dataclass(frozen=True)
+class DenseConfig:
+    """A dense gated FFN layer: the card's first layers ("Every architecture
+    field": layout 3 x dense then 58 x MoE; ffns.dense gated, d_ff 18432)."""
+    name: str
+    T: int
+    d_model: int
+    d_ff: int
+    precision: str      # "bf16", "fp8" or "fp8_ue8m0", as for the MoE layer
+    w_std: float
+
+    def with_(self, **kw) -> "DenseConfig":
+        return dataclasses.replace(self, **kw)
+
+    def flops_per_token(self) -> float:
+        return 2.0 * 3 * self.d_model * self.d_ff
+
+
+DENSE_CONFIGS = {
+    "dense_tiny": DenseConfig("dense_tiny", T=100, d_model=512, d_ff=768, precision="fp8",
+                              w_std=0.02),
+    # the MoE workloads' batches through a dense first layer (same value recipe)
+    "dense_decode": DenseConfig("dense_decode", T=64, d_model=7168, d_ff=18432,
+                                precision="fp8", w_std=0.006),
+    "dense_prefill": DenseConfig("dense_prefill", T=4096, d_model=7168, d_ff=18432,
+                                 precision="fp8", w_std=0.006),
+}
+
+
+def make_dense_inputs(cfg: DenseConfig, seed: int = 0, device="cpu"):
+    """dict(x [T, d] bf16 (as make_x), w13 [2*d_ff, d] bf16 gate rows then up
+    rows, w2 [d, d_ff] bf16), weights N(0, w_std)."""
+    x = make_x(cfg, seed, device)
+    d, f = cfg.d_model, cfg.d_ff
+    w13 = torch.randn(2 * f, d, generator=_gen(device, seed, _TID_DW13), device=device,
+                      dtype=torch.float32) * cfg.w_std
+    w2 = torch.randn(d, f, generator=_gen(device, seed, _TID_DW2), device=device,
+                     dtype=torch.float32) * cfg.w_std
+    return dict(x=x, w13=w13.to(torch.bfloat16), w2=w2.to(torch.bfloat16))

@@ -29,8 +29,12 @@ What the layer computes, step by step, with the passage each step follows:
     before the down projection; Y is stored as bf16.  In the bf16 scheme H is
     rounded to bf16.
  5. Combine: out[t] = bf16( sum_j g[t,j] * Y[row(t,j)] + Y_shared[t] ) (the
-    shared expert is always active with weight 1: "v3 also inherits the
-    concept of the shared expert, i.e. an always-activated expert").
+    shared expert takes part in every token's output with weight 1: "DeepSeek v3
+    and R1 Model Architecture", section "Structural change").
+
+ 6. Dense gated FFN of the first layers (card, "Every architecture field":
+    layout 3 dense layers then 58 MoE layers; ffns.dense gated, d_ff 18432):
+    one gated MLP as in step 4 over every token, out = bf16(Y).
 
 The oracle mirrors every storage rounding of the layer (bf16 Y, bf16 or e4m3
 H, bf16 out) and otherwise computes in binary64.
@@ -47,7 +51,8 @@ from . import build as _build
 __all__ = [
     "lib", "bf16_to_f32", "bf16_from_f32", "e4m3_decode_table", "e4m3_encode", "sigmoid",
     "router_logits", "route", "permute", "block_quant", "dequant", "expert_forward",
-    "moe_layer", "exp_cw", "rmsnorm", "moe_layer_prenorm",
+    "moe_layer", "exp_cw", "rmsnorm", "moe_layer_prenorm", "dense_ffn", "dense_ffn_prenorm",
+    "h_code_ambiguity", "h_code_alternatives",
 ]
 
 _LIB = None
@@ -291,8 +296,36 @@ def h_code_ambiguity(H, hq, hs, ue8m0: bool, rho: float = H_FLIP_RHO) -> np.ndar
     return delta
 
 
+def h_code_alternatives(H, hq, hs, ue8m0: bool, rho: float = H_FLIP_RHO) -> np.ndarray:
+    """[n, de] binary64, signed: for each element of the fp32 H whose quantiser
+    input lies within rho (relative) of an e4m3 rounding boundary, the change
+    of its dequantised value if it took the code on the other side of that
+    boundary; 0 elsewhere.  These are the other correct H codes; a UE8M0 tile
+    whose scale could double or halve is left to h_code_ambiguity's bound."""
+    global _DEC
+    if _DEC is None:
+        _DEC = e4m3_decode_table()
+    H = np.ascontiguousarray(H, dtype=np.float32)
+    n, de = H.shape
+    base = dequant(hq, hs, 1)
+    sc = np.repeat(np.asarray(hs, dtype=np.float64), 128, axis=1)
+    if ue8m0:
+        x = (H.astype(np.float64) / sc).astype(np.float32)
+    else:
+        amax = np.abs(H).reshape(n, de // 128, 128).max(2)
+        with np.errstate(divide="ignore"):
+            inv = np.where(amax > 0, np.float32(448.0) / amax, np.float32(0.0)).astype(np.float32)
+        x = H * np.repeat(inv, 128, axis=1)
+    alt = np.zeros((n, de))
+    for f in (1.0 + rho, 1.0 - rho):
+        d = _DEC[e4m3_encode(x.astype(np.float64) * f)] * sc - base
+        alt = np.where(alt == 0, d, alt)
+    return alt
+
+
 def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=None,
-                   w2_scales=None, return_h: bool = False, return_allow: bool = False):
+                   w2_scales=None, return_h: bool = False, return_allow: bool = False,
+                   return_f64: bool = False, return_alts: bool = False):
     """One gated expert on a block of rows.
 
     bf16:  a_rows uint16 [n, d], w13 uint16 [2*de, d], w2 uint16 [d, de].
@@ -302,7 +335,10 @@ def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=No
     -> Y as bf16 bits [n, d] (and H: bf16 bits, or (codes, scales) for fp8;
     return_allow: and [n, d] binary64, how far alternative H codes at e4m3
     rounding boundaries could move Y: sum_i h_code_ambiguity_i * |W2[:, i]|;
-    zero for bf16)."""
+    zero for bf16; return_f64: (Y in binary64, before its rounding, and that
+    allowance), with return_alts also, per row, the [m, d] changes of Y that
+    the row's alternative H codes (h_code_alternatives) would make, one row
+    per alternative)."""
     n = a_rows.shape[0]
     if precision == "bf16":
         A = bf16_to_f32(a_rows).astype(np.float64)
@@ -313,6 +349,10 @@ def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=No
         U = A @ W13[de:].T
         H = _bf16_of_f64(_silu_mul(G, U))
         Y = bf16_to_f32(H).astype(np.float64) @ W2.T
+        if return_f64:
+            if return_alts:
+                return Y, np.zeros(Y.shape), [np.zeros((0, Y.shape[1]))] * n
+            return Y, np.zeros(Y.shape)
         y = _bf16_of_f64(Y)
         if return_allow:
             return y, np.zeros(Y.shape)
@@ -328,6 +368,16 @@ def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=No
         ue = precision == "fp8_ue8m0"
         hq, hs = block_quant(H, 1, ue8m0=ue)
         Y = dequant(hq, hs, 1) @ W2.T
+        if return_f64:
+            allow = h_code_ambiguity(H, hq, hs, ue) @ np.abs(W2).T
+            if return_alts:
+                dh = h_code_alternatives(H, hq, hs, ue)
+                alts = []
+                for r in range(n):
+                    cols = np.nonzero(dh[r])[0]
+                    alts.append(dh[r, cols][:, None] * W2[:, cols].T)
+                return Y, allow, alts
+            return Y, allow
         y = _bf16_of_f64(Y)
         if return_allow:
             return y, h_code_ambiguity(H, hq, hs, ue) @ np.abs(W2).T
@@ -429,6 +479,57 @@ def moe_layer_prenorm(h, gamma, eps, w_router, bias, expert, **kw):
     hh = bf16_to_f32(np.asarray(h, dtype=np.uint16)[rows]).astype(np.float64)
     res["moe_out"] = res["out"]
     res["out"] = _bf16_of_f64(hh + res["out_f64"])
+    res["x"] = x
+    res["rstd"] = rstd
+    return res
+
+
+# ------------------------------------------------------------ dense layer --
+
+def dense_ffn(x, w13, w2, *, precision: str, tokens=None):
+    """Dense gated FFN layer (the model's first layers; "DeepSeek-R1" card,
+    "Every architecture field": ffns.dense gated, d_ff 18432): one gated MLP
+    over every token with the expert numerics of the precision (step 4 of the
+    module notes), out = bf16(Y).
+
+    x uint16 [T, d]; w13 uint16 [2*d_ff, d] (gate rows then up rows);
+    w2 uint16 [d, d_ff]; tokens: rows to evaluate (default all; activation
+    tiles are per row, so a subset quantises exactly as the whole batch).
+    Returns dict(out bf16 bits, out_f64, out_allow, tokens, (fp8) xq, xs)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    tokens = np.arange(x.shape[0]) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    res = dict(tokens=tokens)
+    if precision in ("fp8", "fp8_ue8m0"):
+        ue = precision == "fp8_ue8m0"
+        xq, xs = block_quant(x[tokens], 1, ue8m0=ue)
+        w13q, w13s = block_quant(w13, 128, ue8m0=ue)
+        w2q, w2s = block_quant(w2, 128, ue8m0=ue)
+        Y, allow, alts = expert_forward(xq, w13q, w2q, precision, xs, w13s, w2s,
+                                        return_f64=True, return_alts=True)
+        res.update(xq=xq, xs=xs)
+    elif precision == "bf16":
+        Y, allow, alts = expert_forward(x[tokens], w13, w2, "bf16", return_f64=True,
+                                        return_alts=True)
+    else:
+        raise ValueError(precision)
+    res["out_f64"] = Y
+    res["out"] = _bf16_of_f64(Y)
+    res["out_allow"] = allow
+    # per evaluated row: the changes of out_f64 that the row's other correct
+    # H codes would make (h_code_alternatives), one row per alternative
+    res["out_alts"] = alts
+    return res
+
+
+def dense_ffn_prenorm(h, gamma, eps, w13, w2, *, precision: str, tokens=None):
+    """out = bf16(h + FFN(x)), x = RMSNorm(h) * gamma (pre-norm, card "Facts"):
+    the residual is added to the binary64 FFN output, one final rounding."""
+    x, rstd = rmsnorm(h, gamma, eps)
+    res = dense_ffn(x, w13, w2, precision=precision, tokens=tokens)
+    hh = bf16_to_f32(np.asarray(h, dtype=np.uint16)[res["tokens"]]).astype(np.float64)
+    res["ffn_out"] = res["out"]
+    res["out_f64"] = hh + res["out_f64"]
+    res["out"] = _bf16_of_f64(res["out_f64"])
     res["x"] = x
     res["rstd"] = rstd
     return res

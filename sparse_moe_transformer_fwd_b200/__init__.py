@@ -18,7 +18,9 @@ from ._native import (EXPORTS, MOE_BF16, MOE_FP8_BLOCK, MOE_FP8_UE8M0, MOE_LAYOU
                       moe_forward, moe_grouped_swiglu, moe_last_error, moe_last_launch_count,
                       moe_last_launch_names,
                       moe_permute, moe_route, moe_route_noalloc, moe_set_kernel_events,
-                      moe_workspace_size, MOE_ROUTE_NOALLOC_MAX_SCORES)
+                      moe_workspace_size, MOE_ROUTE_NOALLOC_MAX_SCORES, MoeDenseShape,
+                      make_dense_shape, moe_dense_workspace_size, alloc_dense_workspace,
+                      moe_dense_ffn, moe_dense_ffn_prenorm)
 
 __all__ = [
     "MoELayer", "MoeError", "MoeShape", "make_shape", "alloc_workspace", "lib", "EXPORTS",
@@ -27,6 +29,8 @@ __all__ = [
     "quantize_weights", "MOE_BF16", "MOE_FP8_BLOCK", "MOE_FP8_UE8M0", "moe_set_kernel_events",
     "moe_route_noalloc", "MOE_ROUTE_NOALLOC_MAX_SCORES", "moe_pack_tiles", "pack_weights",
     "MOE_LAYOUT_ROWMAJOR", "MOE_LAYOUT_TILED", "moe_forward_prenorm", "moe_last_launch_names",
+    "DenseFFN", "MoeDenseShape", "make_dense_shape", "moe_dense_workspace_size",
+    "alloc_dense_workspace", "moe_dense_ffn", "moe_dense_ffn_prenorm",
 ]
 
 
@@ -113,6 +117,60 @@ class MoELayer:
         moe_forward_prenorm(self.shape(T), h, gamma, eps, self.w_router, self.bias, self.w13,
                             self.w13s, self.w2, self.w2s, out, self.workspace(T),
                             topk_idx_out=topk_idx_out, stream=stream)
+        return out
+
+    def check_status(self, T: int) -> int:
+        return moe_check_status(self.workspace(T))
+
+
+class DenseFFN:
+    """One dense gated FFN layer (the model's first layers) with resident
+    weights, on the expert GEMM kernels.
+
+    w13 bf16 [2*d_ff, d] (gate rows then up rows); w2 bf16 [d, d_ff].
+    precision as for MoELayer ("fp8", "fp8_ue8m0" or "bf16")."""
+
+    def __init__(self, w13, w2, *, precision: str = "fp8"):
+        lib()
+        self.d, self.d_ff = w2.shape
+        self.precision = precision
+        w13, w2 = w13.contiguous().unsqueeze(0), w2.contiguous().unsqueeze(0)
+        if precision in ("fp8", "fp8_ue8m0"):
+            self.w13, self.w13s, self.w2, self.w2s = quantize_weights(
+                w13, w2, ue8m0=precision == "fp8_ue8m0")
+        elif precision == "bf16":
+            self.w13, self.w2 = pack_weights(w13, w2)
+            self.w13s = self.w2s = None
+        else:
+            raise ValueError(precision)
+        self._ws = {}
+
+    def shape(self, T: int) -> MoeDenseShape:
+        return make_dense_shape(T, self.d, self.d_ff, self.precision)
+
+    def workspace(self, T: int) -> torch.Tensor:
+        ws = self._ws.get(T)
+        if ws is None:
+            ws = alloc_dense_workspace(self.shape(T), self.w13.device)
+            self._ws[T] = ws
+        return ws
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty(T, self.d, dtype=torch.bfloat16, device=x.device)
+        moe_dense_ffn(self.shape(T), x, self.w13, self.w13s, self.w2, self.w2s, out,
+                      self.workspace(T), stream=stream)
+        return out
+
+    def forward_prenorm(self, h: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
+                        out: torch.Tensor | None = None, stream=None):
+        """The FFN block: out = h + FFN(RMSNorm(h) * gamma)."""
+        T = h.shape[0]
+        if out is None:
+            out = torch.empty(T, self.d, dtype=torch.bfloat16, device=h.device)
+        moe_dense_ffn_prenorm(self.shape(T), h, gamma, eps, self.w13, self.w13s, self.w2,
+                              self.w2s, out, self.workspace(T), stream=stream)
         return out
 
     def check_status(self, T: int) -> int:

@@ -30,7 +30,8 @@ EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant",
            "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_check_status",
            "moe_last_error", "moe_last_launch_count", "moe_set_kernel_events",
            "moe_route_noalloc", "moe_pack_tiles", "moe_forward_prenorm", "moe_last_launch_name",
-           "fp8_block_quant_ue8m0")
+           "fp8_block_quant_ue8m0", "moe_dense_workspace_size", "moe_dense_ffn",
+           "moe_dense_ffn_prenorm")
 
 # fixed score scratch of moe_route_noalloc, in floats (include/moe_fwd.h)
 MOE_ROUTE_NOALLOC_MAX_SCORES = 1 << 20
@@ -40,6 +41,11 @@ class MoeShape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int), ("d_model", ctypes.c_int), ("n_experts", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("d_expert", ctypes.c_int), ("n_shared", ctypes.c_int),
                 ("routed_scale", ctypes.c_float), ("precision", ctypes.c_int)]
+
+
+class MoeDenseShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("d_model", ctypes.c_int), ("d_ff", ctypes.c_int),
+                ("precision", ctypes.c_int)]
 
 
 class MoeError(RuntimeError):
@@ -73,6 +79,11 @@ def lib() -> ctypes.CDLL:
         L.moe_combine.argtypes = [sp, vp, vp, vp, vp, vp]
         L.moe_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_forward_prenorm.argtypes = [sp, vp, vp, cf, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        dp = ctypes.POINTER(MoeDenseShape)
+        L.moe_dense_workspace_size.argtypes = [dp]
+        L.moe_dense_workspace_size.restype = sz
+        L.moe_dense_ffn.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_dense_ffn_prenorm.argtypes = [dp, vp, vp, cf, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_check_status.argtypes = [vp, vp]
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
@@ -83,7 +94,8 @@ def lib() -> ctypes.CDLL:
         for name in ("moe_route", "moe_route_noalloc", "moe_permute", "fp8_block_quant",
                      "fp8_block_quant_ue8m0", "moe_grouped_swiglu",
                      "moe_combine", "moe_forward", "moe_check_status", "moe_last_launch_count",
-                     "moe_set_kernel_events", "moe_pack_tiles", "moe_forward_prenorm"):
+                     "moe_set_kernel_events", "moe_pack_tiles", "moe_forward_prenorm",
+                     "moe_dense_ffn", "moe_dense_ffn_prenorm"):
             getattr(L, name).restype = ci
         _LIB = L
     return _LIB
@@ -121,6 +133,12 @@ def make_shape(T, d_model, n_experts, top_k, d_expert, n_shared=1, routed_scale=
         else int(precision)
     return MoeShape(int(T), int(d_model), int(n_experts), int(top_k), int(d_expert),
                     int(n_shared), float(routed_scale), prec)
+
+
+def make_dense_shape(T, d_model, d_ff, precision="fp8") -> MoeDenseShape:
+    prec = {"bf16": MOE_BF16, "fp8": MOE_FP8_BLOCK, "fp8_ue8m0": MOE_FP8_UE8M0}[precision] \
+        if isinstance(precision, str) else int(precision)
+    return MoeDenseShape(int(T), int(d_model), int(d_ff), prec)
 
 
 _BF16 = torch.bfloat16
@@ -234,6 +252,39 @@ def moe_forward_prenorm(shape, h, gamma, eps, w_router, bias, w13, w13_scales, w
         _ptr(w2_scales, torch.float32, "w2_scales"), _ptr(out, _BF16, "out"),
         _ptr(topk_idx_out, torch.int32, "topk_idx_out"), _ptr(ws, torch.uint8, "ws"),
         ws.numel(), _stream(stream)))
+
+
+def moe_dense_workspace_size(shape: MoeDenseShape) -> int:
+    n = lib().moe_dense_workspace_size(ctypes.byref(shape))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, lib().moe_last_error().decode())
+    return n
+
+
+def alloc_dense_workspace(shape: MoeDenseShape, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace of moe_dense_workspace_size bytes."""
+    return torch.zeros(moe_dense_workspace_size(shape), dtype=torch.uint8, device=device)
+
+
+def moe_dense_ffn(shape, x, w13, w13_scales, w2, w2_scales, out, ws, stream=None):
+    """Dense gated FFN layer: out = (silu(x Wg^T) * (x Wu^T)) W2^T."""
+    wt = _FP8 if shape.precision in (MOE_FP8_BLOCK, MOE_FP8_UE8M0) else _BF16
+    _check(lib().moe_dense_ffn(
+        ctypes.byref(shape), _ptr(x, _BF16, "x"), _ptr(w13, wt, "w13"),
+        _ptr(w13_scales, torch.float32, "w13_scales"), _ptr(w2, wt, "w2"),
+        _ptr(w2_scales, torch.float32, "w2_scales"), _ptr(out, _BF16, "out"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def moe_dense_ffn_prenorm(shape, h, gamma, eps, w13, w13_scales, w2, w2_scales, out, ws,
+                          stream=None):
+    """out = h + FFN(bf16(RMSNorm(h) * gamma)), one final rounding."""
+    wt = _FP8 if shape.precision in (MOE_FP8_BLOCK, MOE_FP8_UE8M0) else _BF16
+    _check(lib().moe_dense_ffn_prenorm(
+        ctypes.byref(shape), _ptr(h, _BF16, "h"), _ptr(gamma, _BF16, "gamma"), float(eps),
+        _ptr(w13, wt, "w13"), _ptr(w13_scales, torch.float32, "w13_scales"), _ptr(w2, wt, "w2"),
+        _ptr(w2_scales, torch.float32, "w2_scales"), _ptr(out, _BF16, "out"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
 
 
 def moe_check_status(ws, stream=None) -> int:

@@ -3,6 +3,7 @@
 #include "common.cuh"
 #include "kernels.h"
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdlib>
 #include <cstdio>
@@ -498,6 +499,190 @@ int moe_forward_prenorm(const moe_shape *s, const uint16_t *h, const uint16_t *g
     if (!aligned16(gamma)) return fail(MOE_ERR_INVALID_ARG, "gamma is not 16-byte aligned");
     return forward_impl(s, h, gamma, eps, w_router, bias, w13, w13_scales, w2, w2_scales, out,
                         topk_idx_out, ws, ws_bytes, stream);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------- dense FFN layer ---
+namespace moe {
+namespace {
+
+int check_dense_shape(const moe_dense_shape *s) {
+    if (!s) return fail(MOE_ERR_INVALID_ARG, "shape is NULL");
+    if (s->T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+    if (s->d_model <= 0 || s->d_model % 256)
+        return fail(MOE_ERR_INVALID_ARG, "d_model must be a positive multiple of 256");
+    if (s->d_ff <= 0 || s->d_ff % 128)
+        return fail(MOE_ERR_INVALID_ARG, "d_ff must be a positive multiple of 128");
+    if (s->precision != MOE_BF16 && s->precision != MOE_FP8_BLOCK &&
+        s->precision != MOE_FP8_UE8M0)
+        return fail(MOE_ERR_INVALID_ARG, "unknown precision %d", s->precision);
+    if (static_cast<long long>(s->T) * std::max(s->d_model, s->d_ff) > (1LL << 40) ||
+        s->T > (1 << 30))
+        return fail(MOE_ERR_INVALID_ARG, "T too large");
+    return MOE_OK;
+}
+
+// Split K of the dense down GEMM.  Its output has only ceil(T/128) x
+// d_model/256 tiles (28 for a batch of up to 128 tokens at d_model 7168), too
+// few to keep the SMs streaming weights, so small batches split K into up to
+// kDenseMaxSplit ranges.  The workspace reserves the partial sums for batches
+// of at most kDenseSplitRows tokens; the split itself is chosen per launch
+// from the device's SM count.
+constexpr int kDenseMaxSplit = 8;
+constexpr int kDenseSplitRows = 256;
+
+struct DenseLayout {
+    size_t status, rstd, a, a_scales, h, h_scales, partial, counts, total;
+};
+
+DenseLayout dense_layout(const moe_dense_shape *s) {
+    const size_t T = s->T, d = s->d_model, f = s->d_ff;
+    const bool fp8 = s->precision != MOE_BF16;
+    const size_t es = fp8 ? 1 : 2;
+    const bool split = s->T <= kDenseSplitRows && s->precision != MOE_FP8_UE8M0;
+    DenseLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += (bytes + 255) & ~static_cast<size_t>(255);
+        return at;
+    };
+    L.status = take(256);
+    L.rstd = take(T * 4);
+    L.a = take(T * d * es);
+    L.a_scales = take(fp8 ? T * (d / 128) * 4 : 0);
+    L.h = take(T * f * es);
+    L.h_scales = take(fp8 ? T * (f / 128) * 4 : 0);
+    L.partial = take(split ? kDenseMaxSplit * T * d * 4 : 0);
+    L.counts = take(split ? static_cast<size_t>(gemm_output_tiles(s->T, s->d_model)) * 4 : 0);
+    L.total = off;
+    return L;
+}
+
+int dense_ksplit(const moe_dense_shape *s) {
+    if (s->T > kDenseSplitRows || s->precision == MOE_FP8_UE8M0) return 1;
+    const int tiles = gemm_output_tiles(s->T, s->d_model);
+    const int kb = s->precision == MOE_BF16 ? s->d_ff / 64 : s->d_ff / 128;
+    int ks = num_sms() / std::max(tiles, 1);
+    ks = std::min(ks, kDenseMaxSplit);
+    ks = std::min(ks, kb / 2);  // at least two K blocks per range
+    return std::max(ks, 1);
+}
+
+int dense_impl(const moe_dense_shape *s, const uint16_t *x, const uint16_t *gamma, float eps,
+               const void *w13, const float *w13_scales, const void *w2, const float *w2_scales,
+               uint16_t *out, void *ws, size_t ws_bytes, void *stream) {
+    RETURN_IF(check_dense_shape(s));
+    const DenseLayout L = dense_layout(s);
+    if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+    if (reinterpret_cast<uintptr_t>(ws) & 255)
+        return fail(MOE_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (ws_bytes < L.total)
+        return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+    if (s->T == 0) return g_launches = 0, MOE_OK;
+    CHECK_PTR(x);
+    CHECK_PTR(out);
+    CHECK_PTR(w13);
+    CHECK_PTR(w2);
+    const bool fp8 = s->precision != MOE_BF16;
+    const bool ue = s->precision == MOE_FP8_UE8M0;
+    if (fp8) {
+        CHECK_PTR(w13_scales);
+        CHECK_PTR(w2_scales);
+    }
+    if (gamma && !(eps >= 0.0f)) return fail(MOE_ERR_INVALID_ARG, "eps must be >= 0");
+    RETURN_IF(check_device());
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int T = s->T, d = s->d_model;
+    int n = 0;
+    PreNorm pn{};
+    if (gamma) {
+        float *rstd = at<float>(ws, L.rstd);
+        LAUNCH(launch_rstd(x, T, d, eps, rstd, st, &n), "pre-norm statistics");
+        pn.rstd = rstd;
+        pn.gamma = gamma;
+    }
+    // A: x quantised 1x128 (fp8), the normalised copy (bf16 pre-norm), or x itself
+    const void *a = x;
+    if (fp8)
+        LAUNCH(launch_quant_scatter(x, T, d, 0, 1, nullptr, at<uint8_t>(ws, L.a),
+                                    at<float>(ws, L.a_scales), st, &n, pn, ue),
+               "quantise x");
+    else if (gamma)
+        LAUNCH(launch_scatter_bf16(x, T, d, 0, 1, nullptr, at<uint16_t>(ws, L.a), st, &n, pn),
+               "pre-norm x");
+    if (fp8 || gamma) a = at<uint8_t>(ws, L.a);
+    const int ks = dense_ksplit(s);
+    int *counts = at<int>(ws, L.counts);
+    GemmArgs g{};
+    g.fp8 = fp8;
+    g.rows_total = T;
+    g.n_slots = 1;
+    g.n_segments = 1;
+    g.E = 0;
+    g.seg_start = g.seg_rows = g.tile_start = nullptr;  // one segment of all T rows
+    g.status = at<int>(ws, L.status);
+    g.ue8m0 = ue;
+    g.max_seg_rows = T;
+    g.gate_up = true;
+    g.a = a;
+    g.a_scales = fp8 ? at<float>(ws, L.a_scales) : nullptr;
+    g.b = w13;
+    g.b_scales = w13_scales;
+    g.out = at<uint8_t>(ws, L.h);
+    g.out_scales = fp8 ? at<float>(ws, L.h_scales) : nullptr;
+    g.K = d;
+    g.N_out = s->d_ff;
+    if (ks > 1) {
+        g.zero_count = counts;
+        g.n_zero = gemm_output_tiles(T, d);
+    }
+    LAUNCH(launch_grouped_gemm(g, st, &n), "dense gate/up GEMM");
+    g.gate_up = false;
+    g.zero_count = nullptr;
+    g.n_zero = 0;
+    g.a = at<uint8_t>(ws, L.h);
+    g.a_scales = fp8 ? at<float>(ws, L.h_scales) : nullptr;
+    g.b = w2;
+    g.b_scales = w2_scales;
+    g.out = out;
+    g.out_scales = nullptr;
+    g.K = s->d_ff;
+    g.N_out = d;
+    g.ksplit = ks;
+    g.partial = ks > 1 ? at<float>(ws, L.partial) : nullptr;
+    g.tile_count = ks > 1 ? counts : nullptr;
+    g.residual = gamma ? x : nullptr;
+    LAUNCH(launch_grouped_gemm(g, st, &n), "dense down GEMM");
+    mark_launch(st, n);
+    g_launches = n;
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+size_t moe_dense_workspace_size(const moe_dense_shape *shape) {
+    if (check_dense_shape(shape) != MOE_OK) return 0;
+    return dense_layout(shape).total;
+}
+
+int moe_dense_ffn(const moe_dense_shape *s, const uint16_t *x, const void *w13,
+                  const float *w13_scales, const void *w2, const float *w2_scales,
+                  uint16_t *out, void *ws, size_t ws_bytes, void *stream) {
+    return dense_impl(s, x, nullptr, 0.0f, w13, w13_scales, w2, w2_scales, out, ws, ws_bytes,
+                      stream);
+}
+
+int moe_dense_ffn_prenorm(const moe_dense_shape *s, const uint16_t *h, const uint16_t *gamma,
+                          float eps, const void *w13, const float *w13_scales, const void *w2,
+                          const float *w2_scales, uint16_t *out, void *ws, size_t ws_bytes,
+                          void *stream) {
+    if (!gamma) return fail(MOE_ERR_INVALID_ARG, "gamma is NULL");
+    return dense_impl(s, h, gamma, eps, w13, w13_scales, w2, w2_scales, out, ws, ws_bytes, stream);
 }
 
 int moe_check_status(void *ws, void *stream) {

@@ -99,8 +99,10 @@ struct __align__(1024) GemmSmem {
     uint64_t tempty[2];
     uint64_t xchg[2];        // amax exchange between the two column halves
     uint64_t mma_done;
+    uint64_t kready;         // split K: the block's arrival has been counted
     uint32_t tmem_base;
     int abort;
+    int last_arrival;        // split K: this block completes the current output tile
     float amax_x[2][2][BM];  // [iteration parity][column half][row]
     int32_t seg_start[MAX_SEG];
     int32_t seg_rows[MAX_SEG];
@@ -121,6 +123,16 @@ struct KParams {
     int ue8m0;         // H scales: power of two (UE8M0 variant) instead of amax / 448
     int rows_total;
     int mx_spc;        // MX: K blocks accumulated in TMEM per promotion into registers
+    // Split K (down GEMM, software promotion only): each output tile is done
+    // by ksplit work items over consecutive K-block ranges; each writes its
+    // binary32 partial sums to partial[ks], and the last of them to arrive
+    // (tile_count) adds the ksplit partials in index order and stores Y.
+    int ksplit;
+    float *partial;        // [ksplit][rows_total][N_out]
+    int *tile_count;       // [output tiles], zero at launch; reset by the last arrival
+    int *zero_count;       // gate/up GEMM: the following down GEMM's counters, cleared here
+    int n_zero;
+    const uint16_t *residual;  // down GEMM: bf16 [rows_total, N_out] added before rounding Y
 };
 
 __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int tile, int n_tiles_n,
@@ -165,12 +177,16 @@ __device__ __forceinline__ void promote32(float2 (&acc)[64], int base, const flo
 // exponent field 0, matching E8M0 code 0).
 __device__ __forceinline__ uint32_t e8m0(float sc) { return (__float_as_uint(sc) >> 23) & 0xffu; }
 
-template <bool FP8, bool GATE_UP, bool MX, bool M64>
+template <bool FP8, bool GATE_UP, bool MX, bool M64, bool DENSE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const KParams p) {
     static_assert(FP8 || !MX, "the block-scaled MMA takes e4m3 operands");
     static_assert(!M64 || (FP8 && !MX), "64-row tiles: fp8 with software promotion only");
+    // DENSE: the down GEMM of a dense layer, with split K (software promotion
+    // only) and a residual add (a separate instance, so the expert GEMMs keep
+    // their register budget)
+    static_assert(!DENSE || !GATE_UP, "split K and residual: down GEMM only");
     using R = Roles<MX>;
     extern __shared__ uint8_t smem_raw[];
     GemmSmem &s = *reinterpret_cast<GemmSmem *>(
@@ -189,8 +205,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     // the epilogue multiplies each chunk by s_a * s_w (software promotion)
     constexpr bool SCALED = FP8 && !MX;
     constexpr int TM = M64 ? 64 : BM;  // rows of an MMA tile
-    const int NCH = (KB + SPC - 1) / SPC;        // K chunks per tile (last may be short)
     const int n_seg = p.n_segments;
+    // work item = (output tile, K range): K blocks [kb0, kb0 + nk)
+    const int KS = (DENSE && !MX) ? p.ksplit : 1;  // MX: residual only
+    auto k_range = [&](int item, int &tile, int &ks, int &kb0, int &nk) {
+        tile = item / KS;
+        ks = item - tile * KS;
+        kb0 = ks * KB / KS;
+        nk = (ks + 1) * KB / KS - kb0;
+    };
 
     // ---------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
@@ -204,6 +227,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&s.xchg[i], EPI_THREADS);
         }
         mbar_init(&s.mma_done, 1);
+        mbar_init(&s.kready, 1);
         for (int i = 0; i < SF_STAGING; ++i) {
             mbar_init(&s.sf_full[i], 1);
             mbar_init(&s.sf_empty[i], 1);
@@ -225,17 +249,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
     // everything above overlaps the previous kernel; its outputs are read below
     pdl_wait_and_trigger();
-    for (int i = threadIdx.x; i < n_seg; i += NUM_THREADS) {
-        s.seg_start[i] = p.seg_start[i];
-        s.seg_rows[i] = p.seg_rows[i];
-        s.tile_start[i] = p.tile_start[i];
+    if (p.seg_start) {
+        for (int i = threadIdx.x; i < n_seg; i += NUM_THREADS) {
+            s.seg_start[i] = p.seg_start[i];
+            s.seg_rows[i] = p.seg_rows[i];
+            s.tile_start[i] = p.tile_start[i];
+        }
+        if (threadIdx.x == 0) s.tile_start[n_seg] = p.tile_start[n_seg];
+    } else if (threadIdx.x == 0) {
+        // one segment of all rows (a dense layer): no table in memory
+        s.seg_start[0] = 0;
+        s.seg_rows[0] = p.rows_total;
+        s.tile_start[0] = 0;
+        s.tile_start[1] = (p.rows_total + BM - 1) / BM;
     }
-    if (threadIdx.x == 0) s.tile_start[n_seg] = p.tile_start[n_seg];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = s.tmem_base;
     const int total_tiles = s.tile_start[n_seg] * p.n_tiles_n;
+    const int total_items = total_tiles * KS;
     volatile int *abort = &s.abort;
 
     if (warp < 4) {
@@ -249,7 +282,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             int armed = 0;  // bit s: stage s has been armed at least once
             uint32_t armed_phase[STAGES] = {0, 0, 0, 0};
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+            for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
+                int tile, ks, kb0, nk;
+                k_range(item, tile, ks, kb0, nk);
                 int seg, row0, rows_valid, nt;
                 decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
                 // 128-row blocks of B (tile rows of the tiled weight layout)
@@ -258,7 +293,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const int NBq = p.b_rows / 128;
                 const long long t_lo = (static_cast<long long>(seg) * NBq + nb_lo) * KB;
                 const long long t_hi = (static_cast<long long>(seg) * NBq + nb_hi) * KB;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = kb0; kb < kb0 + nk; ++kb) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, p.status)) {
                         ok = false;
                         break;
@@ -307,10 +342,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             uint32_t tphase = 0;
             int gq = 0;  // MX: scale blocks consumed
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-                for (int kb = 0; kb < KB; ++kb) {
+            for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
+                int tile, ks, kb0, nk;
+                k_range(item, tile, ks, kb0, nk);
+                // kb counts the item's K blocks from 0 (MX: the item is all of K)
+                for (int kb = 0; kb < nk; ++kb) {
                     const bool chunk_first = (kb % SPC) == 0;
-                    const bool chunk_last = (kb % SPC) == SPC - 1 || kb == KB - 1;
+                    const bool chunk_last = (kb % SPC) == SPC - 1 || kb == nk - 1;
                     if (chunk_first) {
                         if (!mbar_wait(&s.tempty[tb], tphase ^ 1, abort, p.status)) {
                             ok = false;
@@ -395,6 +433,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         // column each, byte j for K block 4g + j) and signals the MMA issuer.
         // The split keeps global loads out of the warp that must fence its
         // shared-memory writes for the async proxy.
+        if constexpr (!MX) {
+            // idle warps: clear the split-K counters of the down GEMM that
+            // follows (the previous one has finished: griddepcontrol.wait above)
+            for (int i = blockIdx.x * 64 + threadIdx.x - 64; i < p.n_zero; i += gridDim.x * 64)
+                p.zero_count[i] = 0;
+        }
         if constexpr (MX) {
             const int NB = p.b_rows / 128;
             const int NG = (KB + SF_GROUP - 1) / SF_GROUP;  // groups per tile
@@ -508,7 +552,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         uint32_t tphase = 0;
         int iter = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++iter) {
+        for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x, ++iter) {
+            int tile, ks, kb0, nk;
+            k_range(item, tile, ks, kb0, nk);
+            const int nch = (nk + SPC - 1) / SPC;  // K chunks of the item (last may be short)
             int seg, row0, rows_valid, nt;
             decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
             const bool warp_active = q * (M64 ? 16 : 32) < rows_valid;
@@ -521,22 +568,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
             const int nb_lo = GATE_UP ? nt : 2 * nt;
             const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
-            const float *sw_lo_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * KB : nullptr;
-            const float *sw_hi_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_hi) * KB : nullptr;
-            const float *sa_p = SCALED ? p.a_scales + row * KB : nullptr;
-            // K block whose partial this thread promotes in chunk c
+            // scale rows from the item's first K block on
+            const float *sw_lo_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * KB + kb0 : nullptr;
+            const float *sw_hi_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_hi) * KB + kb0 : nullptr;
+            const float *sa_p = SCALED ? p.a_scales + row * KB + kb0 : nullptr;
+            // K block (counted from kb0) whose partial this thread promotes in chunk c
             auto kb_of = [&](int c) { return M64 ? 2 * c + hh : c; };
             // scales of chunk c are loaded one chunk ahead (global latency)
             float nsa = 0.0f, nswl = 1.0f, nswh = 1.0f;
-            if (SCALED && warp_active && kb_of(0) < KB) {
+            if (SCALED && warp_active && kb_of(0) < nk) {
                 nsa = valid ? __ldg(sa_p + kb_of(0)) : 0.0f;
                 nswl = __ldg(sw_lo_p + kb_of(0));
                 nswh = __ldg(sw_hi_p + kb_of(0));
             }
-            for (int c = 0; c < NCH; ++c) {
+            for (int c = 0; c < nch; ++c) {
                 const float sc_lo = SCALED ? nsa * nswl : 1.0f, sc_hi = SCALED ? nsa * nswh : 1.0f;
-                const bool kvalid = !M64 || kb_of(c) < KB;  // M64, odd K: no partial in the upper half
-                if (SCALED && warp_active && c + 1 < NCH && kb_of(c + 1) < KB) {
+                const bool kvalid = !M64 || kb_of(c) < nk;  // M64, odd K: no partial in the upper half
+                if (SCALED && warp_active && c + 1 < nch && kb_of(c + 1) < nk) {
                     nsa = valid ? __ldg(sa_p + kb_of(c + 1)) : 0.0f;
                     nswl = __ldg(sw_lo_p + kb_of(c + 1));
                     nswh = __ldg(sw_hi_p + kb_of(c + 1));
@@ -645,7 +693,99 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         *reinterpret_cast<uint4 *>(h + c) = o;
                     }
                 }
-            } else if (store_row) {
+            } else {
+                if (DENSE && KS > 1) {
+                    // split K: store this K range's partial sums; the last of
+                    // the tile's KS items to arrive adds all KS in K order
+                    // (the same sum whichever block it is) and stores Y
+                    tile = item / KS;  // recomputed: not kept live through the chunk loop
+                    ks = item - tile * KS;
+                    if (store_row) {
+                        float *pp = p.partial + (static_cast<size_t>(ks) * p.rows_total + row) * p.N_out + nt * 256;
+#pragma unroll
+                        for (int c = 0; c < 64; c += 4) {
+                            *reinterpret_cast<float4 *>(pp + col_lo + c) =
+                                make_float4(acc(c), acc(c + 1), acc(c + 2), acc(c + 3));
+                            *reinterpret_cast<float4 *>(pp + col_hi + c) =
+                                make_float4(acc(64 + c), acc(64 + c + 1), acc(64 + c + 2), acc(64 + c + 3));
+                        }
+                    }
+                    // every epilogue thread's stores are fenced before one
+                    // thread counts the block's arrival (bounded waits: a
+                    // block whose peer warps gave up does not hang)
+                    __threadfence();
+                    const int par = iter & 1;
+                    mbar_arrive(&s.xchg[par]);
+                    if (threadIdx.x == NUM_THREADS - EPI_THREADS) {
+                        if (!mbar_wait(&s.xchg[par], (iter >> 1) & 1, abort, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        s.last_arrival = atomicAdd(p.tile_count + tile, 1) == KS - 1;
+                        mbar_arrive(&s.kready);
+                    }
+                    if (!mbar_wait(&s.kready, iter & 1, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!s.last_arrival) continue;
+                    __threadfence();
+                    if (threadIdx.x == NUM_THREADS - EPI_THREADS) p.tile_count[tile] = 0;
+                    if (!store_row) continue;
+                    // 8 columns at a time: the KS partials in K order (+ the
+                    // residual), rounded once to bf16
+                    const uint16_t *rp = p.residual ? p.residual + row * p.N_out + nt * 256 : nullptr;
+                    uint16_t *y = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 256;
+#pragma unroll 1
+                    for (int c = 0; c < 128; c += 8) {
+                        const int col = c < 64 ? col_lo + c : col_hi + (c - 64);
+                        float v[8];
+#pragma unroll 1
+                        for (int k2 = 0; k2 < KS; ++k2) {
+                            const float *qp = p.partial + (static_cast<size_t>(k2) * p.rows_total + row) * p.N_out +
+                                              nt * 256 + col;
+                            const float4 u0 = __ldcg(reinterpret_cast<const float4 *>(qp));
+                            const float4 u1 = __ldcg(reinterpret_cast<const float4 *>(qp + 4));
+                            const float u[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) v[i] = k2 == 0 ? u[i] : __fadd_rn(v[i], u[i]);
+                        }
+                        if (rp) {
+                            const uint4 r = *reinterpret_cast<const uint4 *>(rp + col);
+                            const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                v[2 * i] = __fadd_rn(v[2 * i], bf16_lo(rr[i]));
+                                v[2 * i + 1] = __fadd_rn(v[2 * i + 1], bf16_hi(rr[i]));
+                            }
+                        }
+                        uint4 o;
+                        o.x = pack_bf16x2(v[0], v[1]);
+                        o.y = pack_bf16x2(v[2], v[3]);
+                        o.z = pack_bf16x2(v[4], v[5]);
+                        o.w = pack_bf16x2(v[6], v[7]);
+                        *reinterpret_cast<uint4 *>(y + col) = o;
+                    }
+                    continue;
+                }
+                if (!store_row) continue;
+                if (DENSE && p.residual) {
+                    // the pre-norm block's residual, added before the one rounding
+                    const uint16_t *rp = p.residual + row * p.N_out + nt * 256;
+#pragma unroll
+                    for (int c = 0; c < 64; c += 8) {
+                        const uint4 a = *reinterpret_cast<const uint4 *>(rp + col_lo + c);
+                        const uint4 b = *reinterpret_cast<const uint4 *>(rp + col_hi + c);
+                        const uint32_t ra[4] = {a.x, a.y, a.z, a.w}, rb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            acc(c + 2 * i) = __fadd_rn(acc(c + 2 * i), bf16_lo(ra[i]));
+                            acc(c + 2 * i + 1) = __fadd_rn(acc(c + 2 * i + 1), bf16_hi(ra[i]));
+                            acc(64 + c + 2 * i) = __fadd_rn(acc(64 + c + 2 * i), bf16_lo(rb[i]));
+                            acc(64 + c + 2 * i + 1) = __fadd_rn(acc(64 + c + 2 * i + 1), bf16_hi(rb[i]));
+                        }
+                    }
+                }
                 uint16_t *y = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 256;
 #pragma unroll
                 for (int c = 0; c < 64; c += 8) {
@@ -709,7 +849,7 @@ bool make_map_2d(CUtensorMap *m, const void *base, bool fp8, int K, int rows, in
 }
 
 
-template <bool FP8, bool GATE_UP, bool MX, bool M64 = false>
+template <bool FP8, bool GATE_UP, bool MX, bool M64 = false, bool DENSE = false>
 cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams &kp, int grid,
                      cudaStream_t st) {
     const size_t smem = sizeof(GemmSmem) + 1024;
@@ -719,16 +859,16 @@ cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams
         // refuse to launch a build whose register count differs, as the
         // epilogue's increase would then never be granted.
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, grouped_gemm_kernel<FP8, GATE_UP, MX, M64>);
+        cudaError_t e = cudaFuncGetAttributes(&fa, grouped_gemm_kernel<FP8, GATE_UP, MX, M64, DENSE>);
         if (e != cudaSuccess) return e;
         if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(grouped_gemm_kernel<FP8, GATE_UP, MX, M64>,
+        e = cudaFuncSetAttribute(grouped_gemm_kernel<FP8, GATE_UP, MX, M64, DENSE>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         mark_used_on_device(configured);
     }
-    return launch_pdl(grouped_gemm_kernel<FP8, GATE_UP, MX, M64>, dim3(grid), dim3(NUM_THREADS), smem, st,
+    return launch_pdl(grouped_gemm_kernel<FP8, GATE_UP, MX, M64, DENSE>, dim3(grid), dim3(NUM_THREADS), smem, st,
                       ma, mb, kp);
 }
 
@@ -767,16 +907,35 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     kp.rows_total = g.rows_total;
     // block-scaled MMA (UE8M0 scales): all of K accumulates in TMEM
     kp.mx_spc = g.K / 128;
+    const bool mx = g.fp8 && g.ue8m0;
+    kp.ksplit = (g.gate_up || mx || g.ksplit < 1) ? 1 : g.ksplit;
+    if (kp.ksplit > 1 && (!g.partial || !g.tile_count || kp.ksplit > (g.fp8 ? g.K / 128 : g.K / 64)))
+        return cudaErrorInvalidValue;
+    kp.partial = g.partial;
+    kp.tile_count = g.tile_count;
+    kp.zero_count = g.zero_count;
+    kp.n_zero = g.zero_count ? g.n_zero : 0;
+    kp.residual = g.gate_up ? nullptr : g.residual;
     // upper bound of work items: every segment's tiles, each at most one partial
     const long long max_mtiles = g.rows_total / BM + g.n_segments;
-    const long long max_tiles = max_mtiles * kp.n_tiles_n;
+    const long long max_tiles = max_mtiles * kp.n_tiles_n * kp.ksplit;
     const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
     if (grid <= 0) return cudaSuccess;
     cudaError_t e;
     mark_launch(st, *launches, g.gate_up ? "grouped_gemm_gate_up" : "grouped_gemm_down");
-    if (g.fp8 && g.ue8m0)
+    // the dense layer's down GEMM (split K or a residual) has its own instances
+    const bool dense = !g.gate_up && (kp.ksplit > 1 || kp.residual);
+    if (dense && mx)
+        e = launch_t<true, false, true, false, true>(ma, mb, kp, grid, st);
+    else if (g.fp8 && g.ue8m0)
         e = g.gate_up ? launch_t<true, true, true>(ma, mb, kp, grid, st)
                       : launch_t<true, false, true>(ma, mb, kp, grid, st);
+    else if (dense && g.fp8 && m64)
+        e = launch_t<true, false, false, true, true>(ma, mb, kp, grid, st);
+    else if (dense && g.fp8)
+        e = launch_t<true, false, false, false, true>(ma, mb, kp, grid, st);
+    else if (dense)
+        e = launch_t<false, false, false, false, true>(ma, mb, kp, grid, st);
     else if (g.fp8 && m64)
         e = g.gate_up ? launch_t<true, true, false, true>(ma, mb, kp, grid, st)
                       : launch_t<true, false, false, true>(ma, mb, kp, grid, st);

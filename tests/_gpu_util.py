@@ -12,7 +12,11 @@ allows, per output, the oracle's bound on how far alternative e4m3 codes of H
 could move it (H elements whose quantiser input lies at a rounding boundary,
 oracle.h_code_ambiguity): two correct evaluations of G and U may round such
 an element either way, and one code step of a large H element moves every
-output of its row by up to one step times |W2|."""
+output of its row by up to one step times |W2|.  Where such flips are common
+enough to move the relative L2 as well (the dense layer: all 18432 H elements
+of a row feed each of its outputs with weight 1), the comparison is with the
+correct output nearest to the GPU's: the oracle's, with the row's
+alternative H codes that explain the difference (nearest_correct_output)."""
 from __future__ import annotations
 
 import json
@@ -78,6 +82,40 @@ def assert_out_close(got_bf16, want_u16, what="", allow=None):
     assert rel <= REL_L2 and ex <= MAX_ABS_RMS, \
         f"{what}: rel_l2={rel:.3e} max/rms={mx:.3e} beyond-one-step/rms={ex:.3e}"
     return rel, mx, ex
+
+
+def nearest_correct_output(got_bf16, out_f64, alts):
+    """Several outputs are correct when elements of H sit at e4m3 rounding
+    boundaries: the oracle's, and the oracle's with any of those elements on
+    the other code (oracle.h_code_alternatives; alts[r] lists the changes of
+    row r, one per alternative).  Per row, the alternatives that bring the
+    oracle's binary64 output closer to got are taken (greedy, largest first);
+    -> (bf16 bits of that output, rounded as the oracle rounds, number of
+    alternatives taken)."""
+    got = got_bf16.detach().float().cpu().numpy().astype(np.float64)
+    adj = np.array(out_f64, dtype=np.float64).reshape(got.shape).copy()
+    taken = 0
+    for r, V in enumerate(alts):
+        V = np.asarray(V, dtype=np.float64)
+        if V.size == 0:
+            continue
+        res = got[r] - adj[r]
+        for i in np.argsort(-np.linalg.norm(V, axis=1)):
+            nxt = res - V[i]
+            if nxt @ nxt < res @ res:
+                res = nxt
+                adj[r] += V[i]
+                taken += 1
+    return oracle.bf16_from_f32(adj.astype(np.float32)), taken
+
+
+def assert_close_to_correct(got_bf16, res, what=""):
+    """The output tolerance against the nearest correct output (above), with
+    the max bound's allowance for the alternatives not taken."""
+    want, taken = nearest_correct_output(got_bf16, res["out_f64"], res["out_alts"])
+    _log(what + f" (alternative H codes taken: {taken})", *out_error(got_bf16, want,
+                                                                       res["out_allow"]))
+    return assert_out_close(got_bf16, want, what, allow=res["out_allow"])
 
 
 def oracle_layer(cfg, inp, tokens=None, expert=None):

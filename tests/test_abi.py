@@ -90,3 +90,33 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(4, 256, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         moe.moe_route(s, x, x, x, x, x, torch.zeros(16, dtype=torch.uint8))
+
+
+def _dense(**kw):
+    a = dict(T=64, d_model=7168, d_ff=18432, precision="fp8")
+    a.update(kw)
+    return moe.make_dense_shape(**a)
+
+
+def test_dense_workspace_and_host_errors():
+    """The dense layer's workspace (split-K partials only up to 256 tokens)
+    and its host-side argument checks; nothing here launches a kernel."""
+    L = moe.lib()
+    small, big = moe.moe_dense_workspace_size(_dense()), moe.moe_dense_workspace_size(_dense(T=257))
+    assert small >= 64 * 7168 * 8 * 4 + 64 * (7168 + 18432)   # partials + x and H codes
+    assert big < 257 * (7168 + 18432) * 2 + 257 * 4 * 256      # no partials past 256 tokens
+    for bad in (dict(d_model=7000), dict(d_model=384), dict(d_ff=100), dict(precision=7),
+                dict(T=-1)):
+        assert L.moe_dense_workspace_size(ctypes.byref(_dense(**bad))) == 0, bad
+    s = _dense()
+    need = moe.moe_dense_workspace_size(s)
+    call = lambda shape, nbytes, x=FAKE, w13s=FAKE: L.moe_dense_ffn(
+        ctypes.byref(shape), x, FAKE, w13s, FAKE, FAKE, FAKE, FAKE, nbytes, None)
+    assert call(s, need - 1) == N.MOE_ERR_WORKSPACE
+    assert call(s, need, x=MISALIGNED) == N.MOE_ERR_INVALID_ARG
+    assert call(s, need, w13s=None) == N.MOE_ERR_INVALID_ARG      # e4m3 needs scales
+    assert L.moe_dense_ffn_prenorm(ctypes.byref(s), FAKE, None, ctypes.c_float(1e-6), FAKE, FAKE,
+                                   FAKE, FAKE, FAKE, FAKE, need, None) == N.MOE_ERR_INVALID_ARG
+    e = _dense(T=0)
+    assert call(e, moe.moe_dense_workspace_size(e)) == N.MOE_OK
+    assert moe.moe_last_launch_count() == 0

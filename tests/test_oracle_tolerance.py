@@ -5,6 +5,7 @@ import numpy as np
 import pytest
 
 import oracle
+from moe_inputs import DENSE_CONFIGS, make_dense_inputs
 
 
 def _tile(vals, amax_at=0, amax=448.0):
@@ -74,3 +75,68 @@ def test_layer_allowance_is_zero_in_bf16_and_small_in_fp8():
         else:
             # a handful of boundary elements per row: well below the output scale
             assert res["out_allow"].max() < 0.1 * rms
+
+
+# ------------------------------------------- alternative codes (signed) --
+
+def test_alternatives_are_the_neighbouring_codes():
+    """h_code_alternatives gives, for each element whose quantiser input is
+    within rho of a rounding boundary, the other code's change: it is the
+    adjacent e4m3 value on the far side of that boundary, the boundary lies
+    within rho of the input, and its magnitude is h_code_ambiguity's bound
+    (with fp32 scales that bound has no other source)."""
+    rng = np.random.default_rng(31)
+    H = (rng.standard_normal((16, 256)) * np.exp(rng.uniform(-3, 3, (16, 1)))).astype(np.float32)
+    rho = 2.0 ** -7  # wide, so that many elements have an alternative
+    hq, hs = oracle.block_quant(H, 1)
+    alt = oracle.h_code_alternatives(H, hq, hs, False, rho=rho)
+    amb = oracle.h_code_ambiguity(H, hq, hs, False, rho=rho)
+    assert np.array_equal(np.abs(alt), amb)
+    assert (alt != 0).sum() > 50
+    table = oracle.e4m3_decode_table()
+    finite = np.sort(np.unique(np.abs(table[np.isfinite(table)])))
+    sc = np.repeat(hs, 128, axis=1)
+    cur = table[hq]
+    amax = np.abs(H).reshape(16, 2, 128).max(2)
+    x = H * np.repeat((np.float32(448.0) / amax).astype(np.float32), 128, axis=1)
+    for r, c in zip(*np.nonzero(alt)):
+        other = (cur[r, c] * sc[r, c] + alt[r, c]) / sc[r, c]
+        a, b = sorted((abs(cur[r, c]), abs(other)))
+        i = np.searchsorted(finite, a)
+        assert finite[i] == a and finite[i + 1] == b          # adjacent magnitudes
+        assert np.sign(other) * np.sign(cur[r, c]) >= 0       # same side of zero
+        mid = (a + b) / 2
+        assert abs(abs(float(x[r, c])) - mid) <= rho * abs(float(x[r, c])) * 1.0000001
+
+
+def test_nearest_correct_output_takes_only_explaining_alternatives():
+    """The checker: an output made with the oracle's largest alternative code
+    is recognised (its distance to the nearest correct output drops to the
+    bf16 rounding level); a planted error of the same size that no
+    alternative explains is not absorbed."""
+    import torch
+    from _gpu_util import nearest_correct_output, out_error
+    cfg = DENSE_CONFIGS["dense_tiny"].with_(T=24)
+    inp = make_dense_inputs(cfg, seed=32)
+    u = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    res = oracle.dense_ffn(u(inp["x"]), u(inp["w13"]), u(inp["w2"]), precision="fp8")
+    cand = [(np.linalg.norm(v), r, i) for r, a in enumerate(res["out_alts"]) for i, v in enumerate(a)]
+    assert cand, "no alternative codes in this sample"
+    _, r, i = max(cand)
+    v = res["out_alts"][r][i]
+    as_bf16 = lambda a: torch.from_numpy(
+        oracle.bf16_from_f32(a.astype(np.float32)).view(np.int16)).view(torch.bfloat16)
+    flipped = res["out_f64"].copy()
+    flipped[r] += v
+    got = as_bf16(flipped)
+    want, taken = nearest_correct_output(got, res["out_f64"], res["out_alts"])
+    assert taken >= 1
+    rel_plain = out_error(got, res["out"])[0]
+    rel_near = out_error(got, want)[0]
+    assert rel_near < rel_plain / 4
+    # the same change moved to other columns is no alternative
+    bad = res["out_f64"].copy()
+    bad[r] += np.roll(v, 17)
+    got_bad = as_bf16(bad)
+    want_bad, _ = nearest_correct_output(got_bad, res["out_f64"], res["out_alts"])
+    assert out_error(got_bad, want_bad)[0] > 0.5 * out_error(got_bad, res["out"])[0]
