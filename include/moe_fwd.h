@@ -257,8 +257,10 @@ typedef struct {
 size_t moe_dense_workspace_size(const moe_dense_shape *shape);
 
 /* The dense layer.
- *   x   bf16 [T, d_model]; out bf16 [T, d_model] (written by the down GEMM,
- *       Y rounded once to bf16)
+ *   x   bf16 [T, d_model]; out bf16 [T, d_model]: Y rounded once to bf16,
+ *       stored by the down GEMM, or (batches of at most 256 tokens, whose
+ *       down GEMM splits K over the SMs) by a kernel that adds the K ranges'
+ *       binary32 partial sums in order, so results do not depend on timing
  *   w13 [2*d_ff, d_model] (gate rows, then up rows) and w2 [d_model, d_ff]
  *       in TILED layout, e4m3 with scales [2*d_ff/128, d_model/128] and
  *       [d_model/128, d_ff/128] (MOE_FP8_BLOCK / MOE_FP8_UE8M0), or bf16

@@ -526,14 +526,15 @@ int check_dense_shape(const moe_dense_shape *s) {
 // Split K of the dense down GEMM.  Its output has only ceil(T/128) x
 // d_model/256 tiles (28 for a batch of up to 128 tokens at d_model 7168), too
 // few to keep the SMs streaming weights, so small batches split K into up to
-// kDenseMaxSplit ranges.  The workspace reserves the partial sums for batches
-// of at most kDenseSplitRows tokens; the split itself is chosen per launch
-// from the device's SM count.
-constexpr int kDenseMaxSplit = 8;
+// kDenseMaxSplit ranges, whose binary32 partial sums a reduce kernel adds in
+// order.  The workspace reserves the partial sums for batches of at most
+// kDenseSplitRows tokens; the split itself is chosen per launch from the
+// device's SM count.
+constexpr int kDenseMaxSplit = kMaxSplitK;
 constexpr int kDenseSplitRows = 256;
 
 struct DenseLayout {
-    size_t status, rstd, a, a_scales, h, h_scales, partial, counts, total;
+    size_t status, rstd, a, a_scales, h, h_scales, partial, total;
 };
 
 DenseLayout dense_layout(const moe_dense_shape *s) {
@@ -555,7 +556,6 @@ DenseLayout dense_layout(const moe_dense_shape *s) {
     L.h = take(T * f * es);
     L.h_scales = take(fp8 ? T * (f / 128) * 4 : 0);
     L.partial = take(split ? kDenseMaxSplit * T * d * 4 : 0);
-    L.counts = take(split ? static_cast<size_t>(gemm_output_tiles(s->T, s->d_model)) * 4 : 0);
     L.total = off;
     return L;
 }
@@ -614,7 +614,6 @@ int dense_impl(const moe_dense_shape *s, const uint16_t *x, const uint16_t *gamm
                "pre-norm x");
     if (fp8 || gamma) a = at<uint8_t>(ws, L.a);
     const int ks = dense_ksplit(s);
-    int *counts = at<int>(ws, L.counts);
     GemmArgs g{};
     g.fp8 = fp8;
     g.rows_total = T;
@@ -634,14 +633,8 @@ int dense_impl(const moe_dense_shape *s, const uint16_t *x, const uint16_t *gamm
     g.out_scales = fp8 ? at<float>(ws, L.h_scales) : nullptr;
     g.K = d;
     g.N_out = s->d_ff;
-    if (ks > 1) {
-        g.zero_count = counts;
-        g.n_zero = gemm_output_tiles(T, d);
-    }
     LAUNCH(launch_grouped_gemm(g, st, &n), "dense gate/up GEMM");
     g.gate_up = false;
-    g.zero_count = nullptr;
-    g.n_zero = 0;
     g.a = at<uint8_t>(ws, L.h);
     g.a_scales = fp8 ? at<float>(ws, L.h_scales) : nullptr;
     g.b = w2;
@@ -652,9 +645,12 @@ int dense_impl(const moe_dense_shape *s, const uint16_t *x, const uint16_t *gamm
     g.N_out = d;
     g.ksplit = ks;
     g.partial = ks > 1 ? at<float>(ws, L.partial) : nullptr;
-    g.tile_count = ks > 1 ? counts : nullptr;
     g.residual = gamma ? x : nullptr;
     LAUNCH(launch_grouped_gemm(g, st, &n), "dense down GEMM");
+    if (ks > 1)
+        LAUNCH(launch_splitk_reduce(at<float>(ws, L.partial), ks, T, d, gamma ? x : nullptr, out,
+                                    st, &n),
+               "split-K reduce");
     mark_launch(st, n);
     g_launches = n;
     return MOE_OK;

@@ -99,10 +99,8 @@ struct __align__(1024) GemmSmem {
     uint64_t tempty[2];
     uint64_t xchg[2];        // amax exchange between the two column halves
     uint64_t mma_done;
-    uint64_t kready;         // split K: the block's arrival has been counted
     uint32_t tmem_base;
     int abort;
-    int last_arrival;        // split K: this block completes the current output tile
     float amax_x[2][2][BM];  // [iteration parity][column half][row]
     int32_t seg_start[MAX_SEG];
     int32_t seg_rows[MAX_SEG];
@@ -125,14 +123,10 @@ struct KParams {
     int mx_spc;        // MX: K blocks accumulated in TMEM per promotion into registers
     // Split K (down GEMM, software promotion only): each output tile is done
     // by ksplit work items over consecutive K-block ranges; each writes its
-    // binary32 partial sums to partial[ks], and the last of them to arrive
-    // (tile_count) adds the ksplit partials in index order and stores Y.
+    // binary32 partial sums to partial[ks] (launch_splitk_reduce adds them).
     int ksplit;
     float *partial;        // [ksplit][rows_total][N_out]
-    int *tile_count;       // [output tiles], zero at launch; reset by the last arrival
-    int *zero_count;       // gate/up GEMM: the following down GEMM's counters, cleared here
-    int n_zero;
-    const uint16_t *residual;  // down GEMM: bf16 [rows_total, N_out] added before rounding Y
+    const uint16_t *residual;  // down GEMM without split: bf16 [rows_total, N_out] added before rounding Y
 };
 
 __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int tile, int n_tiles_n,
@@ -227,7 +221,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&s.xchg[i], EPI_THREADS);
         }
         mbar_init(&s.mma_done, 1);
-        mbar_init(&s.kready, 1);
         for (int i = 0; i < SF_STAGING; ++i) {
             mbar_init(&s.sf_full[i], 1);
             mbar_init(&s.sf_empty[i], 1);
@@ -433,12 +426,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         // column each, byte j for K block 4g + j) and signals the MMA issuer.
         // The split keeps global loads out of the warp that must fence its
         // shared-memory writes for the async proxy.
-        if constexpr (!MX) {
-            // idle warps: clear the split-K counters of the down GEMM that
-            // follows (the previous one has finished: griddepcontrol.wait above)
-            for (int i = blockIdx.x * 64 + threadIdx.x - 64; i < p.n_zero; i += gridDim.x * 64)
-                p.zero_count[i] = 0;
-        }
         if constexpr (MX) {
             const int NB = p.b_rows / 128;
             const int NG = (KB + SF_GROUP - 1) / SF_GROUP;  // groups per tile
@@ -695,11 +682,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
             } else {
                 if (DENSE && KS > 1) {
-                    // split K: store this K range's partial sums; the last of
-                    // the tile's KS items to arrive adds all KS in K order
-                    // (the same sum whichever block it is) and stores Y
-                    tile = item / KS;  // recomputed: not kept live through the chunk loop
-                    ks = item - tile * KS;
+                    // split K: store this K range's binary32 partial sums; the
+                    // reduce kernel that follows adds the KS ranges in K order
+                    ks = item - (item / KS) * KS;  // recomputed: not kept live through the chunk loop
                     if (store_row) {
                         float *pp = p.partial + (static_cast<size_t>(ks) * p.rows_total + row) * p.N_out + nt * 256;
 #pragma unroll
@@ -709,62 +694,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                             *reinterpret_cast<float4 *>(pp + col_hi + c) =
                                 make_float4(acc(64 + c), acc(64 + c + 1), acc(64 + c + 2), acc(64 + c + 3));
                         }
-                    }
-                    // every epilogue thread's stores are fenced before one
-                    // thread counts the block's arrival (bounded waits: a
-                    // block whose peer warps gave up does not hang)
-                    __threadfence();
-                    const int par = iter & 1;
-                    mbar_arrive(&s.xchg[par]);
-                    if (threadIdx.x == NUM_THREADS - EPI_THREADS) {
-                        if (!mbar_wait(&s.xchg[par], (iter >> 1) & 1, abort, p.status)) {
-                            ok = false;
-                            break;
-                        }
-                        s.last_arrival = atomicAdd(p.tile_count + tile, 1) == KS - 1;
-                        mbar_arrive(&s.kready);
-                    }
-                    if (!mbar_wait(&s.kready, iter & 1, abort, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    if (!s.last_arrival) continue;
-                    __threadfence();
-                    if (threadIdx.x == NUM_THREADS - EPI_THREADS) p.tile_count[tile] = 0;
-                    if (!store_row) continue;
-                    // 8 columns at a time: the KS partials in K order (+ the
-                    // residual), rounded once to bf16
-                    const uint16_t *rp = p.residual ? p.residual + row * p.N_out + nt * 256 : nullptr;
-                    uint16_t *y = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 256;
-#pragma unroll 1
-                    for (int c = 0; c < 128; c += 8) {
-                        const int col = c < 64 ? col_lo + c : col_hi + (c - 64);
-                        float v[8];
-#pragma unroll 1
-                        for (int k2 = 0; k2 < KS; ++k2) {
-                            const float *qp = p.partial + (static_cast<size_t>(k2) * p.rows_total + row) * p.N_out +
-                                              nt * 256 + col;
-                            const float4 u0 = __ldcg(reinterpret_cast<const float4 *>(qp));
-                            const float4 u1 = __ldcg(reinterpret_cast<const float4 *>(qp + 4));
-                            const float u[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) v[i] = k2 == 0 ? u[i] : __fadd_rn(v[i], u[i]);
-                        }
-                        if (rp) {
-                            const uint4 r = *reinterpret_cast<const uint4 *>(rp + col);
-                            const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                v[2 * i] = __fadd_rn(v[2 * i], bf16_lo(rr[i]));
-                                v[2 * i + 1] = __fadd_rn(v[2 * i + 1], bf16_hi(rr[i]));
-                            }
-                        }
-                        uint4 o;
-                        o.x = pack_bf16x2(v[0], v[1]);
-                        o.y = pack_bf16x2(v[2], v[3]);
-                        o.z = pack_bf16x2(v[4], v[5]);
-                        o.w = pack_bf16x2(v[6], v[7]);
-                        *reinterpret_cast<uint4 *>(y + col) = o;
                     }
                     continue;
                 }
@@ -909,13 +838,11 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     kp.mx_spc = g.K / 128;
     const bool mx = g.fp8 && g.ue8m0;
     kp.ksplit = (g.gate_up || mx || g.ksplit < 1) ? 1 : g.ksplit;
-    if (kp.ksplit > 1 && (!g.partial || !g.tile_count || kp.ksplit > (g.fp8 ? g.K / 128 : g.K / 64)))
+    if (kp.ksplit > 1 && (!g.partial || kp.ksplit > (g.fp8 ? g.K / 128 : g.K / 64)))
         return cudaErrorInvalidValue;
     kp.partial = g.partial;
-    kp.tile_count = g.tile_count;
-    kp.zero_count = g.zero_count;
-    kp.n_zero = g.zero_count ? g.n_zero : 0;
-    kp.residual = g.gate_up ? nullptr : g.residual;
+    // with split K the residual is added by the reduce kernel
+    kp.residual = (g.gate_up || kp.ksplit > 1) ? nullptr : g.residual;
     // upper bound of work items: every segment's tiles, each at most one partial
     const long long max_mtiles = g.rows_total / BM + g.n_segments;
     const long long max_tiles = max_mtiles * kp.n_tiles_n * kp.ksplit;
@@ -947,6 +874,69 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
                       : launch_t<false, false, false>(ma, mb, kp, grid, st);
     ++*launches;
     return e;
+}
+
+// ------------------------------------------------------- split-K reduce ---
+namespace {
+
+// out[r, n] = bf16( ((partial[0][r][n] + partial[1][r][n]) + ...) (+ residual) ),
+// binary32 adds in K-range order; one thread per 8 columns, every K range's
+// loads issued before the adds.
+__global__ void __launch_bounds__(128)
+splitk_reduce_kernel(const float *__restrict__ partial, int ksplit, int rows, int n,
+                     const uint16_t *__restrict__ residual, uint16_t *__restrict__ out) {
+    const int r = blockIdx.x;
+    const int v = blockIdx.y * blockDim.x + threadIdx.x;  // 8-column group
+    pdl_wait_and_trigger();
+    if (v >= n / 8) return;
+    const size_t off = static_cast<size_t>(r) * n + static_cast<size_t>(v) * 8;
+    const size_t kstride = static_cast<size_t>(rows) * n;
+    float4 a[8], b[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        if (k < ksplit) {
+            a[k] = __ldcg(reinterpret_cast<const float4 *>(partial + k * kstride + off));
+            b[k] = __ldcg(reinterpret_cast<const float4 *>(partial + k * kstride + off + 4));
+        }
+    }
+    float f[8] = {a[0].x, a[0].y, a[0].z, a[0].w, b[0].x, b[0].y, b[0].z, b[0].w};
+#pragma unroll
+    for (int k = 1; k < 8; ++k) {
+        if (k < ksplit) {
+            const float g[8] = {a[k].x, a[k].y, a[k].z, a[k].w, b[k].x, b[k].y, b[k].z, b[k].w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = __fadd_rn(f[i], g[i]);
+        }
+    }
+    if (residual) {
+        const uint4 h = *reinterpret_cast<const uint4 *>(residual + off);
+        const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __fadd_rn(f[2 * i], bf16_lo(w[i]));
+            f[2 * i + 1] = __fadd_rn(f[2 * i + 1], bf16_hi(w[i]));
+        }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(f[0], f[1]);
+    o.y = pack_bf16x2(f[2], f[3]);
+    o.z = pack_bf16x2(f[4], f[5]);
+    o.w = pack_bf16x2(f[6], f[7]);
+    *reinterpret_cast<uint4 *>(out + off) = o;
+}
+
+}  // namespace
+
+cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int rows, int n,
+                                 const uint16_t *residual, uint16_t *out, cudaStream_t st,
+                                 int *launches) {
+    if (ksplit < 1 || ksplit > kMaxSplitK || n % 8) return cudaErrorInvalidValue;
+    mark_launch(st, *launches, "splitk_reduce");
+    const dim3 grid(rows, (n / 8 + 127) / 128);
+    LAUNCH_OR_RETURN(launch_pdl(splitk_reduce_kernel, grid, dim3(128), 0, st, partial, ksplit,
+                                rows, n, residual, out));
+    ++*launches;
+    return cudaGetLastError();
 }
 
 }  // namespace moe

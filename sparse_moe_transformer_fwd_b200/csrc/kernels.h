@@ -131,18 +131,20 @@ struct GemmArgs {
     int max_seg_rows;       // bound on any segment's rows (T: one row per token and expert)
     // seg_start == nullptr: one segment of all rows_total rows (no table)
     // Split K of the down GEMM (fp32-scale and bf16 paths): ksplit > 1 work
-    // items per output tile over consecutive K ranges, binary32 partial sums
-    // in partial [ksplit][rows_total][N_out], arrivals counted in tile_count
-    // (one int per 128 x 256 output tile, zero at launch).
+    // items per output tile over consecutive K ranges write binary32 partial
+    // sums to partial [ksplit][rows_total][N_out] instead of Y; the caller
+    // then runs launch_splitk_reduce.
     int ksplit;
     float *partial;
-    int *tile_count;
-    int *zero_count;        // gate/up GEMM: sets n_zero ints here to zero (the
-    int n_zero;             // following down GEMM's tile_count)
-    const uint16_t *residual;  // down GEMM: bf16 [rows_total, N_out] added before rounding
+    const uint16_t *residual;  // down GEMM without split: bf16 [rows_total, N_out] added before rounding
 };
-// Output tiles of a GEMM with one segment of `rows` rows (split-K counters).
+constexpr int kMaxSplitK = 8;
+// Output tiles of a GEMM with one segment of `rows` rows.
 inline int gemm_output_tiles(int rows, int N_out) { return ((rows + 127) / 128) * (N_out / 256); }
+// out [rows, n] = bf16(sum of the ksplit partial sums in order (+ residual)).
+cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int rows, int n,
+                                 const uint16_t *residual, uint16_t *out, cudaStream_t st,
+                                 int *launches);
 cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launches);
 
 int num_sms();

@@ -6,7 +6,7 @@ Small shapes cover the down GEMM's split K (even and uneven K ranges, 64- and
 128-row tiles, bf16), the single-range path past 256 tokens, UE8M0 block
 scales, the pre-norm block with the residual fused into the down GEMM, T = 0,
 the launch record, and bit-identical repeats (the split-K sum has a fixed
-order, and its counters clear themselves).  The DeepSeek-V3 dense layer runs
+order).  The DeepSeek-V3 dense layer runs
 at the decode and prefill batches, compared on sampled rows."""
 import numpy as np
 import pytest
@@ -83,9 +83,8 @@ def test_dense_prenorm_vs_oracle(name, precision):
 
 @pytest.mark.parametrize("name", ["T48_ff640", "T100_ff768", "bf16_T100"])
 def test_dense_split_k_repeats_bitidentical(name):
-    """Three calls give identical bits: each output tile's partial sums are
-    added in K order, whichever block arrives last, and the arrival counters
-    are back at zero after every call."""
+    """Three calls give identical bits: the K ranges' partial sums are added
+    in K order, whatever order the blocks ran in."""
     cfg = CASES[name]
     inp, layer = _layer(cfg, seed=24)
     outs = [layer(inp["x"]).clone() for _ in range(3)]
@@ -112,7 +111,14 @@ def test_dense_launch_names(precision, prenorm):
     names = moe.moe_last_launch_names()
     first = (["prenorm_rstd"] if prenorm else []) + \
         (["quant_scatter"] if precision == "fp8" else (["scatter_bf16"] if prenorm else []))
-    assert names == first + ["grouped_gemm_gate_up", "grouped_gemm_down"]
+    # 100 tokens: the down GEMM splits K, and a reduce kernel adds the ranges
+    assert names == first + ["grouped_gemm_gate_up", "grouped_gemm_down", "splitk_reduce"]
+    # past 256 tokens, no split: the down GEMM stores out (and adds h) itself
+    big = TINY.with_(T=300, precision=precision)
+    inp, layer = _layer(big, seed=26)
+    h, gamma = make_residual(big, seed=26, device=DEV)
+    (layer.forward_prenorm(h, gamma) if prenorm else layer(inp["x"]))
+    assert moe.moe_last_launch_names() == first + ["grouped_gemm_gate_up", "grouped_gemm_down"]
 
 
 def test_dense_rejects_bad_shapes():
