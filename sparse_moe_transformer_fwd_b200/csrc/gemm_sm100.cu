@@ -232,9 +232,35 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         s.abort = 0;
         fence_mbar_init();
     }
+    // One segment (a dense layer): the block's first work item and the weights
+    // it streams depend on no earlier kernel, so thread 0 (which initialised
+    // the barriers) starts the B loads of its first `pre` stages before the
+    // wait below; the producer adds their A loads after it.
+    int pre = 0;
+    const int NBq = p.b_rows / 128;
+    auto b_tile_rows = [&](int seg, int nt, long long &t_lo, long long &t_hi) {
+        const int nb_lo = GATE_UP ? nt : 2 * nt;
+        const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
+        t_lo = (static_cast<long long>(seg) * NBq + nb_lo) * KB;
+        t_hi = (static_cast<long long>(seg) * NBq + nb_hi) * KB;
+    };
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmap_a);
         prefetch_tmap(&tmap_b);
+        const int single_items = ((p.rows_total + BM - 1) / BM) * p.n_tiles_n * KS;
+        if (!p.seg_start && !MX && static_cast<int>(blockIdx.x) < single_items) {
+            int tile, ks, kb0, nk;
+            k_range(blockIdx.x, tile, ks, kb0, nk);
+            long long t_lo, t_hi;
+            b_tile_rows(0, tile % p.n_tiles_n, t_lo, t_hi);
+            pre = min(STAGES, nk);
+            for (int st = 0; st < pre; ++st) {
+                mbar_arrive_expect_tx(&s.full[st], TM * 128 + B_BYTES);
+                tma_load_2d(s.b[st], &tmap_b, 0, static_cast<int>((t_lo + kb0 + st) * 128), &s.full[st]);
+                tma_load_2d(s.b[st] + B_BYTES / 2, &tmap_b, 0, static_cast<int>((t_hi + kb0 + st) * 128),
+                            &s.full[st]);
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(&s.tmem_base, TMEM_COLS);
@@ -281,26 +307,29 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 int seg, row0, rows_valid, nt;
                 decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
                 // 128-row blocks of B (tile rows of the tiled weight layout)
-                const int nb_lo = GATE_UP ? nt : 2 * nt;
-                const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
-                const int NBq = p.b_rows / 128;
-                const long long t_lo = (static_cast<long long>(seg) * NBq + nb_lo) * KB;
-                const long long t_hi = (static_cast<long long>(seg) * NBq + nb_hi) * KB;
+                long long t_lo, t_hi;
+                b_tile_rows(seg, nt, t_lo, t_hi);
+                const bool first = item == static_cast<int>(blockIdx.x);
                 for (int kb = kb0; kb < kb0 + nk; ++kb) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, p.status)) {
                         ok = false;
                         break;
                     }
-                    const bool inject = p.inject_fault && blockIdx.x == 0 && armed == 0;
-                    mbar_arrive_expect_tx(&s.full[stage],
-                                          TM * 128 + B_BYTES + (inject ? 16 : 0));
                     const int kc = FP8 ? kb * 128 : kb * 64;
-                    tma_load_2d(s.a[stage], &tmap_a, kc, row0, &s.full[stage]);
-                    // each B box is one contiguous 16 KB weight tile
-                    tma_load_2d(s.b[stage], &tmap_b, 0, static_cast<int>((t_lo + kb) * 128),
-                                &s.full[stage]);
-                    tma_load_2d(s.b[stage] + B_BYTES / 2, &tmap_b, 0,
-                                static_cast<int>((t_hi + kb) * 128), &s.full[stage]);
+                    if (first && kb - kb0 < pre) {
+                        // armed and its B loads issued before the wait
+                        tma_load_2d(s.a[stage], &tmap_a, kc, row0, &s.full[stage]);
+                    } else {
+                        const bool inject = p.inject_fault && blockIdx.x == 0 && armed == 0;
+                        mbar_arrive_expect_tx(&s.full[stage],
+                                              TM * 128 + B_BYTES + (inject ? 16 : 0));
+                        tma_load_2d(s.a[stage], &tmap_a, kc, row0, &s.full[stage]);
+                        // each B box is one contiguous 16 KB weight tile
+                        tma_load_2d(s.b[stage], &tmap_b, 0, static_cast<int>((t_lo + kb) * 128),
+                                    &s.full[stage]);
+                        tma_load_2d(s.b[stage] + B_BYTES / 2, &tmap_b, 0,
+                                    static_cast<int>((t_hi + kb) * 128), &s.full[stage]);
+                    }
                     armed |= 1 << stage;
                     armed_phase[stage] = phase;
                     if (++stage == STAGES) {
