@@ -35,6 +35,7 @@ from moe_inputs import (CONFIGS, DENSE_CONFIGS, make_dense_inputs, make_inputs, 
 
 METRIC = "MoE-layer tokens/s at DeepSeek-V3 dims"
 DENSE_METRIC = "dense FFN-layer tokens/s at DeepSeek-V3 dims (first layers, d_ff 18432)"
+EVENT_EVERY = 4  # the dominant kernel is bracketed by CUDA events on every 4th timed step
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -289,12 +290,15 @@ def run_ours(args, world, rank, local):
     counts = torch.bincount(idx.reshape(-1).long(), minlength=cfg.n_experts)
 
     # ---- device-timed region: K steps, inputs resident in HBM; the dominant
-    # kernel (gate/up GEMM) is bracketed by CUDA events inside the region
+    # kernel (gate/up GEMM) is bracketed by CUDA events inside the region on
+    # every EVENT_EVERY-th step (an event between two launches stops their
+    # programmatic overlap, so the other steps run as a caller's would)
     gi = names.index("grouped_gemm_gate_up")
-    g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
+    g_steps = list(range(0, args.steps, EVENT_EVERY))
+    g_ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for k in g_steps}
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for a, b in g_ev:  # create the events before timing
+    for a, b in g_ev.values():  # create the events before timing
         a.record(stream)
         b.record(stream)
     barrier(world)
@@ -302,7 +306,7 @@ def run_ours(args, world, rank, local):
     with ClockSampler(local) as clk:
         start.record(stream)
         for k in range(args.steps):
-            moe.moe_set_kernel_events([None] * gi + [g_ev[k][0], g_ev[k][1]])
+            moe.moe_set_kernel_events([None] * gi + list(g_ev[k]) if k in g_ev else None)
             call(x, out=out, topk_idx_out=idx)
         moe.moe_set_kernel_events(None)
         stop.record(stream)
@@ -310,7 +314,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     ms_total = max_over_ranks(start.elapsed_time(stop), world, dev)
     ms_step = ms_total / args.steps
-    g1_ms = float(np.mean([a.elapsed_time(b) for a, b in g_ev]))
+    g1_ms = float(np.mean([a.elapsed_time(b) for a, b in g_ev.values()]))
 
     # ---- per-kernel breakdown (separate pass, every launch bracketed)
     nb = min(args.steps, 10)
@@ -374,6 +378,8 @@ def run_ours(args, world, rank, local):
                            else "fallback",
             "algorithmic_bytes": g1_bytes,
             "kernel_ms": round(g1_ms, 4),
+            "kernel_ms_from": f"CUDA events around this kernel on every {EVENT_EVERY}th step of the "
+                              "timed region",
             "traffic": kernel_traffic("grouped_gemm_gate_up", cfg.name),
             "traffic_source": "profiles/roofline_traffic.json (ncu dram__bytes_read+write, "
                               "one capture of this workload)",
@@ -453,10 +459,10 @@ def run_dense(args, world, rank, local):
     n_launch = moe.moe_last_launch_count()
     names = moe.moe_last_launch_names()
     gi = names.index("grouped_gemm_gate_up")
-    g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
+    g_ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for k in range(0, args.steps, EVENT_EVERY)}
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for a, b in g_ev:
+    for a, b in g_ev.values():
         a.record(stream)
         b.record(stream)
     barrier(world)
@@ -464,14 +470,14 @@ def run_dense(args, world, rank, local):
     with ClockSampler(local) as clk:
         start.record(stream)
         for k in range(args.steps):
-            moe.moe_set_kernel_events([None] * gi + [g_ev[k][0], g_ev[k][1]])
+            moe.moe_set_kernel_events([None] * gi + list(g_ev[k]) if k in g_ev else None)
             call(x, out)
         moe.moe_set_kernel_events(None)
         stop.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     ms_step = max_over_ranks(start.elapsed_time(stop), world, dev) / args.steps
-    g1_ms = float(np.mean([a.elapsed_time(b) for a, b in g_ev]))
+    g1_ms = float(np.mean([a.elapsed_time(b) for a, b in g_ev.values()]))
     nb = min(args.steps, 10)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)] for _ in range(nb)]
     for k in range(nb):

@@ -179,8 +179,9 @@ int check_ws(const moe_shape *s, void *ws, size_t ws_bytes, Layout *L) {
         if (e_ != cudaSuccess) return cuda_fail(e_, what);   \
     } while (0)
 
-PermScratch perm_scratch(void *ws, const Layout &L) {
+PermScratch perm_scratch(void *ws, const Layout &L, int tile_m = kTileM) {
     PermScratch p;
+    p.tile_m = tile_m;
     p.masks = at<uint32_t>(ws, L.masks);
     p.hist = at<int32_t>(ws, L.hist);
     p.blkoff = at<int32_t>(ws, L.blkoff);
@@ -190,14 +191,24 @@ PermScratch perm_scratch(void *ws, const Layout &L) {
     return p;
 }
 
-// max_seg_rows: a bound on every segment's rows (T when the segments come
-// from the routing, where a token picks an expert at most once; T*k for
-// caller-given offsets)
+// Rows per grouped-GEMM tile.  With fp32 scales every 128-wide K block makes
+// a round trip through the epilogue; a 64-row tile carries two K blocks per
+// round trip (M=64 accumulators fill half of each TMEM lane quadrant), so a
+// segment of r rows costs ceil(r/64) * K/256 round trips against
+// ceil(r/128) * K/128 with 128-row tiles.  That wins for batches of at most
+// 64 tokens, whose segments have a few rows each.  At 4096 tokens (~128 rows
+// per expert) 64-row tiles were measured slower (gate/up GEMM 2.68 ms against
+// 2.13): they make fewer round trips but load each weight tile once per 64
+// rows instead of per 128.
+int choose_tile_m(const moe_shape *s) {
+    return (s->precision == MOE_FP8_BLOCK && s->T <= 64) ? 64 : 128;
+}
+
 int grouped(const moe_shape *s, const void *a, const float *a_scales, const void *w13,
             const float *w13_scales, const void *w2, const float *w2_scales, uint16_t *y,
-            void *ws, const Layout &L, cudaStream_t st, int *launches, int max_seg_rows) {
+            void *ws, const Layout &L, cudaStream_t st, int *launches, int tile_m) {
     const bool fp8 = is_fp8(s);
-    const PermScratch ps = perm_scratch(ws, L);
+    const PermScratch ps = perm_scratch(ws, L, tile_m);
     const int Rs = s->T * (s->top_k + s->n_shared);
     GemmArgs g{};
     g.fp8 = fp8;
@@ -211,7 +222,7 @@ int grouped(const moe_shape *s, const void *a, const float *a_scales, const void
     g.status = at<int>(ws, L.status);
     g.inject_fault = inject_gemm_fault() ? 1 : 0;
     g.ue8m0 = is_ue8m0(s);
-    g.max_seg_rows = max_seg_rows;
+    g.tile_m = tile_m;
     // gate/up GEMM + SwiGLU
     g.gate_up = true;
     g.a = a;
@@ -385,11 +396,11 @@ int moe_grouped_swiglu(const moe_shape *s, const void *a, const float *a_scales,
     RETURN_IF(check_device());
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
     int n = 0;
+    const int tile_m = choose_tile_m(s);
     LAUNCH(launch_tile_table(offsets, s->n_experts, s->T, s->top_k, s->n_shared,
-                             perm_scratch(ws, L), at<int>(ws, L.status), st, &n),
+                             perm_scratch(ws, L, tile_m), at<int>(ws, L.status), st, &n),
            "tile table");
-    RETURN_IF(grouped(s, a, a_scales, w13, w13_scales, w2, w2_scales, y, ws, L, st, &n,
-                      s->T * s->top_k));
+    RETURN_IF(grouped(s, a, a_scales, w13, w13_scales, w2, w2_scales, y, ws, L, st, &n, tile_m));
     mark_launch(st, n);
     g_launches = n;
     return MOE_OK;
@@ -453,7 +464,8 @@ int forward_impl(const moe_shape *s, const uint16_t *x, const uint16_t *gamma, f
     LAUNCH(launch_router(x, w_router, bias, s->T, s->d_model, s->n_experts, s->top_k,
                          s->routed_scale, at<float>(ws, L.scores), idx, gates, st, &n, pn),
            "router");
-    LAUNCH(launch_permute(idx, s->T, s->top_k, s->n_experts, s->n_shared, perm_scratch(ws, L),
+    const int tile_m = choose_tile_m(s);
+    LAUNCH(launch_permute(idx, s->T, s->top_k, s->n_experts, s->n_shared, perm_scratch(ws, L, tile_m),
                           at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
                           at<int32_t>(ws, L.row_token), row_of, at<int>(ws, L.status), st, &n),
            "permute");
@@ -468,7 +480,7 @@ int forward_impl(const moe_shape *s, const uint16_t *x, const uint16_t *gamma, f
                "scatter");
     uint16_t *y = at<uint16_t>(ws, L.y);
     RETURN_IF(grouped(s, at<uint8_t>(ws, L.a), fp8 ? at<float>(ws, L.a_scales) : nullptr, w13,
-                      w13_scales, w2, w2_scales, y, ws, L, st, &n, s->T));
+                      w13_scales, w2, w2_scales, y, ws, L, st, &n, tile_m));
     LAUNCH(launch_combine(y, row_of, gates, s->T, s->d_model, s->top_k, s->n_shared, out, st, &n,
                           gamma ? x : nullptr),
            "combine");
@@ -623,7 +635,8 @@ int dense_impl(const moe_dense_shape *s, const uint16_t *x, const uint16_t *gamm
     g.seg_start = g.seg_rows = g.tile_start = nullptr;  // one segment of all T rows
     g.status = at<int>(ws, L.status);
     g.ue8m0 = ue;
-    g.max_seg_rows = T;
+    // one segment of T rows: 64-row tiles only where they save round trips
+    g.tile_m = (s->precision == MOE_FP8_BLOCK && T <= 64) ? 64 : 128;
     g.gate_up = true;
     g.a = a;
     g.a_scales = fp8 ? at<float>(ws, L.a_scales) : nullptr;

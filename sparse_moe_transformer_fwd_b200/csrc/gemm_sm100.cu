@@ -54,7 +54,6 @@ constexpr int BN = 256;                  // tile columns (TMEM columns per buffe
 constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * 128;        // 16 KB per stage
 constexpr int B_BYTES = BN * 128;        // 32 KB per stage
-constexpr int STAGE_TX = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 384;  // 3 warpgroups
 constexpr int LAUNCH_REGS = 168;   // 65536 / 384, multiple of 8
 constexpr int EPI_THREADS = 256;
@@ -129,6 +128,7 @@ struct KParams {
     const uint16_t *residual;  // down GEMM without split: bf16 [rows_total, N_out] added before rounding Y
 };
 
+template <int TM>
 __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int tile, int n_tiles_n,
                                             int &seg, int &row0, int &rows_valid, int &nt) {
     const int mt = tile / n_tiles_n;
@@ -141,8 +141,8 @@ __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int ti
     }
     seg = lo;
     const int mloc = mt - s.tile_start[seg];
-    row0 = s.seg_start[seg] + mloc * BM;
-    rows_valid = min(BM, s.seg_rows[seg] - mloc * BM);
+    row0 = s.seg_start[seg] + mloc * TM;
+    rows_valid = min(TM, s.seg_rows[seg] - mloc * TM);
 }
 
 // silu(g) = g * sigmoid(g) with the fast exponential and reciprocal: H is
@@ -247,7 +247,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmap_a);
         prefetch_tmap(&tmap_b);
-        const int single_items = ((p.rows_total + BM - 1) / BM) * p.n_tiles_n * KS;
+        const int single_items = ((p.rows_total + TM - 1) / TM) * p.n_tiles_n * KS;
         if (!p.seg_start && !MX && static_cast<int>(blockIdx.x) < single_items) {
             int tile, ks, kb0, nk;
             k_range(blockIdx.x, tile, ks, kb0, nk);
@@ -280,7 +280,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         s.seg_start[0] = 0;
         s.seg_rows[0] = p.rows_total;
         s.tile_start[0] = 0;
-        s.tile_start[1] = (p.rows_total + BM - 1) / BM;
+        s.tile_start[1] = (p.rows_total + TM - 1) / TM;
     }
     tc_fence_before();
     __syncthreads();
@@ -305,7 +305,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 int tile, ks, kb0, nk;
                 k_range(item, tile, ks, kb0, nk);
                 int seg, row0, rows_valid, nt;
-                decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
+                decode_tile<TM>(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
                 // 128-row blocks of B (tile rows of the tiled weight layout)
                 long long t_lo, t_hi;
                 b_tile_rows(seg, nt, t_lo, t_hi);
@@ -478,7 +478,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         const int tile = blockIdx.x + (i / NG) * gridDim.x;
                         const int kb0 = (i % NG) * SF_GROUP;
                         int seg, row0, rows_valid, nt;
-                        decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
+                        decode_tile<TM>(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
                         const int slot = i % SF_STAGING;
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
@@ -573,7 +573,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             k_range(item, tile, ks, kb0, nk);
             const int nch = (nk + SPC - 1) / SPC;  // K chunks of the item (last may be short)
             int seg, row0, rows_valid, nt;
-            decode_tile(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
+            decode_tile<TM>(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
             const bool warp_active = q * (M64 ? 16 : 32) < rows_valid;
             const bool valid = r_in < rows_valid;
             const bool store_row = valid && hh == 0;  // M64: one lane of the pair stores
@@ -836,9 +836,10 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     if (g.n_segments > MAX_SEG) return cudaErrorInvalidValue;
     const int b_rows = g.gate_up ? 2 * g.N_out : g.N_out;
     CUtensorMap ma, mb;
-    // 64-row MMA tiles when no segment can exceed 64 rows (at most 64 tokens:
-    // a token picks an expert at most once, and the shared segment has T rows)
-    const bool m64 = g.fp8 && !g.ue8m0 && g.max_seg_rows <= 64;
+    // 64-row MMA tiles: the segment table counts 64-row tiles (fp32 scales)
+    const bool m64 = g.tile_m == 64;
+    if (m64 && (!g.fp8 || g.ue8m0)) return cudaErrorInvalidValue;
+    if (!m64 && g.tile_m != 128) return cudaErrorInvalidValue;
     if (!make_map_2d(&ma, g.a, g.fp8, g.K, g.rows_total, m64 ? 64 : 128))
         return cudaErrorInvalidValue;
     // B in the tiled layout: one row of 128 bytes per tile row, tiles stacked
@@ -873,7 +874,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     // with split K the residual is added by the reduce kernel
     kp.residual = (g.gate_up || kp.ksplit > 1) ? nullptr : g.residual;
     // upper bound of work items: every segment's tiles, each at most one partial
-    const long long max_mtiles = g.rows_total / BM + g.n_segments;
+    const long long max_mtiles = g.rows_total / g.tile_m + g.n_segments;
     const long long max_tiles = max_mtiles * kp.n_tiles_n * kp.ksplit;
     const int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
     if (grid <= 0) return cudaSuccess;

@@ -51,7 +51,8 @@ struct PermScratch {
     int32_t *blkoff;     // [nblk][E]
     int32_t *seg_start;  // [E + 1] first row of segment s (shared segment last)
     int32_t *seg_rows;   // [E + 1] rows of segment s
-    int32_t *tile_start; // [E + 2] prefix of 128-row tiles per segment
+    int32_t *tile_start; // [E + 2] prefix of tile_m-row tiles per segment
+    int tile_m;          // rows per grouped-GEMM tile: 128, or 64 (64-row MMA tiles)
 };
 
 // Pre-norm of the FFN input applied on the fly by the kernels that read it:
@@ -128,7 +129,7 @@ struct GemmArgs {
     int *status;
     int inject_fault;       // test hook: make one bounded wait run out (see api.cu)
     bool ue8m0;             // fp8 gate/up: H requantised with power-of-two scales
-    int max_seg_rows;       // bound on any segment's rows (T: one row per token and expert)
+    int tile_m;             // rows per tile of the segment table (64: M=64 MMA tiles, fp32 scales)
     // seg_start == nullptr: one segment of all rows_total rows (no table)
     // Split K of the down GEMM (fp32-scale and bf16 paths): ksplit > 1 work
     // items per output tile over consecutive K ranges write binary32 partial

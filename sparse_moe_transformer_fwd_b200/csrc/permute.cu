@@ -88,7 +88,7 @@ __device__ int block_exclusive_scan(int v, int *tmp /* [32] */, int *total) {
 // Writes the segment table: seg_start[s], seg_rows[s] for s in [0, S) with
 // S = E + n_shared, and tile_start[s] (S + 1 entries: prefix of m-tiles).
 __device__ void write_tile_table(int count, int start, int e, int E, int T, int R, int n_shared,
-                                 int *tmp, int32_t *seg_start, int32_t *seg_rows,
+                                 int tile_m, int *tmp, int32_t *seg_start, int32_t *seg_rows,
                                  int32_t *tile_start) {
     // routed segments: thread e < E; shared segment: thread E
     int rows = 0, st = 0;
@@ -99,7 +99,7 @@ __device__ void write_tile_table(int count, int start, int e, int E, int T, int 
         rows = T;
         st = R;
     }
-    const int tiles = (rows + kTileM - 1) / kTileM;
+    const int tiles = (rows + tile_m - 1) / tile_m;
     int total;
     const int ts = block_exclusive_scan(tiles, tmp, &total);
     const int S = E + n_shared;
@@ -113,6 +113,7 @@ __device__ void write_tile_table(int count, int start, int e, int E, int T, int 
 
 __global__ void __launch_bounds__(1024)
 perm_scan_kernel(const int32_t *__restrict__ hist, int nblk, int E, int T, int k, int n_shared,
+                 int tile_m,
                  int32_t *__restrict__ blkoff, int32_t *__restrict__ counts,
                  int32_t *__restrict__ offsets, int32_t *seg_start, int32_t *seg_rows,
                  int32_t *tile_start) {
@@ -131,7 +132,7 @@ perm_scan_kernel(const int32_t *__restrict__ hist, int nblk, int E, int T, int k
     const int off = block_exclusive_scan(e < E ? run : 0, tmp, &total);
     if (e < E) offsets[e] = off;
     if (e == 0) offsets[E] = total;
-    write_tile_table(run, off, e, E, T, T * k, n_shared, tmp, seg_start, seg_rows, tile_start);
+    write_tile_table(run, off, e, E, T, T * k, n_shared, tile_m, tmp, seg_start, seg_rows, tile_start);
 }
 
 __global__ void __launch_bounds__(256)
@@ -164,7 +165,7 @@ perm_scatter_kernel(const int32_t *__restrict__ idx, int T, int k, int E,
 // Batches of at most 256 tokens (one bit-matrix block): kernels 1-3 in one
 // CTA of 1024 threads, the bit matrix and the offsets in shared memory.
 __global__ void __launch_bounds__(1024)
-perm_small_kernel(const int32_t *__restrict__ idx, int T, int k, int E, int n_shared,
+perm_small_kernel(const int32_t *__restrict__ idx, int T, int k, int E, int n_shared, int tile_m,
                   int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                   int32_t *__restrict__ row_token, int32_t *__restrict__ row_of,
                   int32_t *seg_start, int32_t *seg_rows, int32_t *tile_start,
@@ -202,7 +203,7 @@ perm_small_kernel(const int32_t *__restrict__ idx, int T, int k, int E, int n_sh
         off_sh[e] = off;
     }
     if (e == 0) offsets[E] = total;
-    write_tile_table(run, off, e, E, T, T * k, n_shared, tmp, seg_start, seg_rows, tile_start);
+    write_tile_table(run, off, e, E, T, T * k, n_shared, tile_m, tmp, seg_start, seg_rows, tile_start);
     __syncthreads();
     for (int i = threadIdx.x; i < np; i += blockDim.x) {
         const int v = idx[i];
@@ -222,7 +223,7 @@ perm_small_kernel(const int32_t *__restrict__ idx, int T, int k, int E, int n_sh
 // [0, T*k) or has a negative size is recorded in the status word and
 // treated as empty, so the GEMMs never touch rows outside the buffers.
 __global__ void __launch_bounds__(1024)
-tile_table_kernel(const int32_t *__restrict__ offsets, int E, int T, int k, int n_shared,
+tile_table_kernel(const int32_t *__restrict__ offsets, int E, int T, int k, int n_shared, int tile_m,
                   int32_t *seg_start, int32_t *seg_rows, int32_t *tile_start,
                   int *status) {
     __shared__ int tmp[32];
@@ -238,7 +239,7 @@ tile_table_kernel(const int32_t *__restrict__ offsets, int E, int T, int k, int 
             count = 0;
         }
     }
-    write_tile_table(count, start, e, E, T, T * k, n_shared, tmp, seg_start, seg_rows, tile_start);
+    write_tile_table(count, start, e, E, T, T * k, n_shared, tile_m, tmp, seg_start, seg_rows, tile_start);
 }
 
 }  // namespace
@@ -251,7 +252,7 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int n_shared
     if (nblk == 1) {
         mark_launch(st, *launches, "perm_small");
         LAUNCH_OR_RETURN(launch_pdl(perm_small_kernel, dim3(1), dim3(1024), 0, st, idx, T, k, E,
-                                    n_shared, counts, offsets, row_token, row_of, s.seg_start,
+                                    n_shared, s.tile_m, counts, offsets, row_token, row_of, s.seg_start,
                                     s.seg_rows, s.tile_start, status));
         ++*launches;
         return cudaGetLastError();
@@ -262,7 +263,7 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int n_shared
     ++*launches;
     mark_launch(st, *launches, "perm_scan");
     LAUNCH_OR_RETURN(launch_pdl(perm_scan_kernel, dim3(1), dim3(1024), 0, st, s.hist, nblk, E, T, k, n_shared,
-                                s.blkoff, counts, offsets, s.seg_start, s.seg_rows, s.tile_start));
+                                s.tile_m, s.blkoff, counts, offsets, s.seg_start, s.seg_rows, s.tile_start));
     ++*launches;
     mark_launch(st, *launches, "perm_scatter");
     LAUNCH_OR_RETURN(launch_pdl(perm_scatter_kernel, dim3(nblk), dim3(256), smem, st, idx, T, k, E, s.masks,
@@ -275,7 +276,7 @@ cudaError_t launch_tile_table(const int32_t *offsets, int E, int T, int k, int n
                               PermScratch s, int *status, cudaStream_t st, int *launches) {
     mark_launch(st, *launches, "tile_table");
     LAUNCH_OR_RETURN(launch_pdl(tile_table_kernel, dim3(1), dim3(1024), 0, st, offsets, E, T, k, n_shared,
-                                s.seg_start, s.seg_rows, s.tile_start, status));
+                                s.tile_m, s.seg_start, s.seg_rows, s.tile_start, status));
     ++*launches;
     return cudaGetLastError();
 }
