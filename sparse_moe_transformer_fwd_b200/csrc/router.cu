@@ -83,8 +83,15 @@ __device__ __forceinline__ float sigmoid_cw(float l, const ExpConsts &k) {
 // FMAs per instruction, on experts (4tx, 4tx+1) and (4tx+2, 4tx+3)).  Per k
 // step: three 16-byte shared loads (x by broadcast, W_r two wavefronts) feed
 // 32 FMAs.  x and W_r chunks of 32 columns are staged transposed ([k][row],
-// binary32) through registers one chunk ahead.
+// binary32) through registers one chunk ahead.  The 16-byte row groups of
+// shared row k are XOR-swizzled by 2 * (k / 8): a thread stores 8 values of
+// one row at k = 8j + c (j = 0..3), and the swizzle spreads a warp's 32
+// stores (8 rows x 4 j) over all 32 banks; the compute reads stay whole
+// 16-byte groups.
 constexpr int RT_B = 64, RT_KC = 32, RT_THREADS = 128;
+__device__ __forceinline__ int rt_swz(int k, int row) {
+    return ((((row >> 2) ^ ((k >> 3) << 1)) & 15) << 2) | (row & 3);
+}
 
 __global__ void __launch_bounds__(RT_THREADS)
 router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w, int T, int d,
@@ -131,8 +138,8 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
             const uint32_t r4[4] = {pre[j].x, pre[j].y, pre[j].z, pre[j].w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                dst[col + 2 * q][r] = bf16_lo(r4[q]);
-                dst[col + 2 * q + 1][r] = bf16_hi(r4[q]);
+                dst[col + 2 * q][rt_swz(col + 2 * q, r)] = bf16_lo(r4[q]);
+                dst[col + 2 * q + 1][rt_swz(col + 2 * q + 1, r)] = bf16_hi(r4[q]);
             }
         }
     };
@@ -146,9 +153,9 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
         if (kc + 1 < nk) load(kc + 1);
 #pragma unroll 4
         for (int kk = 0; kk < RT_KC; ++kk) {
-            const float4 xa = *reinterpret_cast<const float4 *>(&xs[buf][kk][4 * ty]);
-            const float4 xb = *reinterpret_cast<const float4 *>(&xs[buf][kk][32 + 4 * ty]);
-            const float4 wa = *reinterpret_cast<const float4 *>(&ws[buf][kk][4 * tx]);
+            const float4 xa = *reinterpret_cast<const float4 *>(&xs[buf][kk][rt_swz(kk, 4 * ty)]);
+            const float4 xb = *reinterpret_cast<const float4 *>(&xs[buf][kk][rt_swz(kk, 32 + 4 * ty)]);
+            const float4 wa = *reinterpret_cast<const float4 *>(&ws[buf][kk][rt_swz(kk, 4 * tx)]);
             const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
             const float2 wv[2] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w)};
 #pragma unroll
