@@ -11,7 +11,7 @@ import oracle
 import sparse_moe_transformer_fwd_b200 as moe
 from moe_inputs import CONFIGS, make_inputs
 
-from _gpu_util import assert_out_close, from_u16, oracle_layer, u16, untile
+from _gpu_util import assert_close_to_correct, assert_out_close, from_u16, oracle_layer, u16, untile
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0") if torch.cuda.is_available() else None
@@ -237,6 +237,58 @@ def test_grouped_swiglu_and_combine(precision, T):
     assert_out_close(out, ref["out"], "combine", ref["out_allow"])
     # combine alone, fed the oracle's Y: same as the oracle's combine
     assert_out_close(out_ref, ref["out"], "combine of oracle Y")
+
+
+@pytest.mark.parametrize("precision", ["fp8", "bf16"])
+def test_grouped_swiglu_long_caller_segments(precision):
+    """Caller offsets with segments far longer than the batch: at T = 40 the
+    fp32-scale GEMMs take 64-row tiles, so expert 0's 100 rows and expert 5's
+    60 rows span several tiles (a 36-row ragged tile included)."""
+    cfg = CONFIGS["tiny"].with_(precision=precision, T=40)
+    inp = make_inputs(cfg, seed=22)
+    E, k, T = cfg.n_experts, cfg.top_k, cfg.T
+    R = T * k
+    counts = np.zeros(E, np.int64)
+    counts[0], counts[5] = 100, R - 100
+    offsets_np = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    rows = np.concatenate([(np.arange(R) * 7) % T, np.arange(T)])
+    x16 = u16(inp["x"])
+    shape = _shape(cfg)
+    ws = moe.alloc_workspace(shape, DEV)
+    y = torch.empty(cfg.R_s, cfg.d_model, dtype=torch.bfloat16, device=DEV)
+    offsets = torch.from_numpy(offsets_np).to(DEV)
+    w13, w2 = inp["w13"].to(DEV), inp["w2"].to(DEV)
+    if precision == "fp8":
+        xq, xs = oracle.block_quant(x16, 1)
+        w13q, w13s, w2q, w2s = moe.quantize_weights(w13, w2)
+        moe.moe_grouped_swiglu(shape, torch.from_numpy(xq[rows]).to(DEV),
+                               torch.from_numpy(xs[rows]).to(DEV), offsets, w13q, w13s, w2q,
+                               w2s, y, ws)
+    else:
+        w13t, w2t = moe.pack_weights(w13, w2)
+        moe.moe_grouped_swiglu(shape, from_u16(x16[rows], DEV), None, offsets, w13t, None, w2t,
+                               None, y, ws)
+    assert moe.moe_check_status(ws) == 0
+    # the oracle's rows, with their other correct H codes (nearest correct output)
+    seg_of_row = np.concatenate([np.repeat(np.arange(E), counts), np.full(T, E)])
+    res = dict(out_f64=np.zeros((cfg.R_s, cfg.d_model)), out_allow=np.zeros((cfg.R_s, cfg.d_model)),
+               out_alts=[None] * cfg.R_s)
+    for e in (0, 5, E):
+        sel = np.nonzero(seg_of_row == e)[0]
+        w13e, w2e = u16(inp["w13"][e]), u16(inp["w2"][e])
+        if precision == "fp8":
+            q13, s13 = oracle.block_quant(w13e, 128)
+            q2, s2 = oracle.block_quant(w2e, 128)
+            Y, al, alts = oracle.expert_forward(xq[rows[sel]], q13, q2, "fp8", xs[rows[sel]], s13,
+                                                s2, return_f64=True, return_alts=True)
+        else:
+            Y, al, alts = oracle.expert_forward(x16[rows[sel]], w13e, w2e, "bf16",
+                                                return_f64=True, return_alts=True)
+        res["out_f64"][sel] = Y
+        res["out_allow"][sel] = al
+        for i, r in enumerate(sel):
+            res["out_alts"][r] = alts[i]
+    assert_close_to_correct(y, res, f"grouped experts, long caller segments, {precision}")
 
 
 # -------------------------------------------------------- fused forward ---
