@@ -88,3 +88,28 @@ def test_sampled_tokens_vs_oracle(run):
     ref = oracle_layer(cfg, inp, tokens=tokens)
     assert np.array_equal(idx_np[tokens], ref["idx"])
     assert_out_close(out[tokens], ref["out"], cfg.name, ref["out_allow"])
+
+
+def test_prenorm_decode_fullsize_sampled():
+    """The pre-norm block at the decode batch and DeepSeek dims, as the
+    benchmark's --prenorm line runs it: routing of all 64 tokens bit-exact
+    against the oracle's pre-norm, sampled output rows within tolerance."""
+    from moe_inputs import make_residual
+    cfg = CONFIGS["decode"]
+    inp = make_inputs(cfg, seed=0, device=DEV)
+    h, g = make_residual(cfg, seed=0, device=DEV)
+    layer = moe.MoELayer(inp["w_router"], inp["bias"], inp["w13"], inp["w2"], top_k=cfg.top_k,
+                         precision=cfg.precision)
+    idx = torch.empty(cfg.T, cfg.top_k, dtype=torch.int32, device=DEV)
+    out = layer.forward_prenorm(h, g, 1e-6, topk_idx_out=idx)
+    assert layer.check_status(cfg.T) == 0
+    tok = np.array([0, 17, 40, 63])
+    ref = oracle.moe_layer_prenorm(
+        u16(h), u16(g), 1e-6, u16(inp["w_router"]), inp["bias"].cpu().numpy(),
+        lambda e: (u16(inp["w13"][e]), u16(inp["w2"][e])), n_experts=cfg.n_experts,
+        top_k=cfg.top_k, n_shared=cfg.n_shared, precision=cfg.precision, tokens=tok)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    assert_out_close(out[torch.as_tensor(tok, device=DEV)], ref["out"], "prenorm decode sampled",
+                     ref["out_allow"])
+    del layer, inp
+    torch.cuda.empty_cache()

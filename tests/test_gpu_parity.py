@@ -389,6 +389,8 @@ PRENORM_CASES = {
     "tiny_fp8": CONFIGS["tiny"].with_(precision="fp8"),
     "tiny_fp8_T600": CONFIGS["tiny"].with_(precision="fp8", T=600),
     "tiny_bf16_T3": CONFIGS["tiny"].with_(T=3),
+    "tiny_fp8_T40": CONFIGS["tiny"].with_(precision="fp8", T=40),        # 64-row tiles
+    "tiny_ue8m0_T100": CONFIGS["tiny"].with_(precision="fp8_ue8m0", T=100),
 }
 
 
