@@ -249,8 +249,9 @@ router_scores_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__res
         cp_async_commit();
         const uint16_t *ws = ring + (kc % RS_STAGES) * (W_ELEMS + X_ELEMS);
         const uint16_t *xs = ws + W_ELEMS;
-        {   // this warp's token: 8 columns per lane, widened (and pre-normed)
-            const int c = lane * 8;
+        // this warp's token: 8 columns per lane and pass, widened (and pre-normed)
+#pragma unroll
+        for (int c = lane * 8; c < RS_KC; c += 256) {
             const uint4 raw = x_vec(*reinterpret_cast<const uint4 *>(xs + warp * RS_KC + c), pn,
                                     t < T ? t : 0, kc * RS_KC + c);
             *reinterpret_cast<float4 *>(xw + c) =
