@@ -366,6 +366,7 @@ def run_ours(args, world, rank, local):
             "l2": f"inputs larger than L2: {touched} touched experts' weights "
                   f"({g1_bytes / 1e9:.2f} GB in the gate/up GEMM alone) per step",
             "expert_load_max_over_mean": round(float(counts.max()) / (T * cfg.top_k / cfg.n_experts), 2),
+            "experts_empty": int((counts == 0).sum()),
         },
         "roofline": {
             "kernel": "grouped_gemm_gate_up",

@@ -3,6 +3,8 @@
 #include "common.cuh"
 #include "kernels.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <algorithm>
 #include <cstdarg>
 #include <cstdlib>
@@ -24,11 +26,23 @@ thread_local cudaEvent_t *g_events = nullptr;  // profiling hook (moe_set_kernel
 thread_local int g_n_events = 0;
 constexpr int kMaxNamed = 64;
 thread_local const char *g_names[kMaxNamed];  // kernel of each launch of the last call
+thread_local bool g_nvtx_kernel = false;       // a per-kernel NVTX range is open
 }  // namespace
 
 void mark_launch(cudaStream_t st, int index, const char *name) {
     if (g_events && index < g_n_events && g_events[index]) cudaEventRecord(g_events[index], st);
     if (name && index >= 0 && index < kMaxNamed) g_names[index] = name;
+    // NVTX: one host range per kernel launch, inside the call's range
+    if (g_nvtx_kernel) nvtxRangePop();
+    g_nvtx_kernel = name != nullptr;
+    if (name) nvtxRangePushA(name);
+}
+
+CallRange::CallRange(const char *name) { nvtxRangePushA(name); }
+CallRange::~CallRange() {
+    if (g_nvtx_kernel) nvtxRangePop();
+    g_nvtx_kernel = false;
+    nvtxRangePop();
 }
 
 namespace {
@@ -280,6 +294,7 @@ size_t moe_workspace_size(const moe_shape *shape) {
 
 int moe_route(const moe_shape *s, const uint16_t *x, const uint16_t *w_router, const float *bias,
               int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream) {
+    const CallRange nvtx_range("moe_route");
     RETURN_IF(check_shape(s));
     Layout L;
     RETURN_IF(check_ws(s, ws, ws_bytes, &L));
@@ -302,6 +317,7 @@ int moe_route(const moe_shape *s, const uint16_t *x, const uint16_t *w_router, c
 
 int moe_permute(const moe_shape *s, const int32_t *topk_idx, int32_t *counts, int32_t *offsets,
                 int32_t *row_token, int32_t *row_of, void *ws, size_t ws_bytes, void *stream) {
+    const CallRange nvtx_range("moe_permute");
     RETURN_IF(check_shape(s));
     Layout L;
     RETURN_IF(check_ws(s, ws, ws_bytes, &L));
@@ -332,6 +348,7 @@ int moe_permute(const moe_shape *s, const int32_t *topk_idx, int32_t *counts, in
 
 static int block_quant_entry(const uint16_t *in, int rows, int cols, int ld, int block_rows,
                       int out_layout, uint8_t *q, float *scales, void *stream, bool ue8m0) {
+    const CallRange nvtx_range("fp8_block_quant");
     if (rows < 0 || cols <= 0 || cols % 128 || ld < cols || ld % 8)
         return fail(MOE_ERR_INVALID_ARG, "need rows >= 0, cols a positive multiple of 128, "
                                          "ld >= cols, ld % 8 == 0");
@@ -366,6 +383,7 @@ int fp8_block_quant_ue8m0(const uint16_t *in, int rows, int cols, int ld, int bl
 }
 
 int moe_pack_tiles(const void *src, int rows, int row_bytes, void *dst, void *stream) {
+    const CallRange nvtx_range("moe_pack_tiles");
     if (rows < 0 || row_bytes <= 0 || rows % 128 || row_bytes % 128)
         return fail(MOE_ERR_INVALID_ARG, "rows and row_bytes must be multiples of 128");
     if (rows == 0) return g_launches = 0, MOE_OK;
@@ -384,6 +402,7 @@ int moe_grouped_swiglu(const moe_shape *s, const void *a, const float *a_scales,
                        const int32_t *offsets, const void *w13, const float *w13_scales,
                        const void *w2, const float *w2_scales, uint16_t *y, void *ws,
                        size_t ws_bytes, void *stream) {
+    const CallRange nvtx_range("moe_grouped_swiglu");
     RETURN_IF(check_shape(s));
     Layout L;
     RETURN_IF(check_ws(s, ws, ws_bytes, &L));
@@ -408,6 +427,7 @@ int moe_grouped_swiglu(const moe_shape *s, const void *a, const float *a_scales,
 
 int moe_combine(const moe_shape *s, const uint16_t *y, const int32_t *row_of,
                 const float *topk_w, uint16_t *out, void *stream) {
+    const CallRange nvtx_range("moe_combine");
     RETURN_IF(check_shape(s));
     if (s->T == 0) return g_launches = 0, MOE_OK;
     CHECK_PTR(y);
@@ -435,6 +455,7 @@ int forward_impl(const moe_shape *s, const uint16_t *x, const uint16_t *gamma, f
                  const uint16_t *w_router, const float *bias, const void *w13,
                  const float *w13_scales, const void *w2, const float *w2_scales, uint16_t *out,
                  int32_t *topk_idx_out, void *ws, size_t ws_bytes, void *stream) {
+    const CallRange nvtx_range(gamma ? "moe_forward_prenorm" : "moe_forward");
     RETURN_IF(check_shape(s));
     Layout L;
     RETURN_IF(check_ws(s, ws, ws_bytes, &L));
@@ -585,6 +606,7 @@ int dense_ksplit(const moe_dense_shape *s) {
 int dense_impl(const moe_dense_shape *s, const uint16_t *x, const uint16_t *gamma, float eps,
                const void *w13, const float *w13_scales, const void *w2, const float *w2_scales,
                uint16_t *out, void *ws, size_t ws_bytes, void *stream) {
+    const CallRange nvtx_range(gamma ? "moe_dense_ffn_prenorm" : "moe_dense_ffn");
     RETURN_IF(check_dense_shape(s));
     const DenseLayout L = dense_layout(s);
     if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");

@@ -177,4 +177,13 @@ int validate_shape(const moe_shape *s);        // host-side shape checks
 // hook is active, and the name for moe_last_launch_name.
 void mark_launch(cudaStream_t st, int index, const char *name = nullptr);
 
+// NVTX range of one library call on the calling thread (the per-kernel ranges
+// that mark_launch opens nest inside it); closes them on every return path.
+struct CallRange {
+    explicit CallRange(const char *name);
+    ~CallRange();
+    CallRange(const CallRange &) = delete;
+    CallRange &operator=(const CallRange &) = delete;
+};
+
 }  // namespace moe

@@ -47,6 +47,7 @@ extern "C" int moe_route_noalloc(const moe_shape *s, const uint16_t *x, const ui
                                  const float *bias, int32_t *topk_idx, float *topk_w,
                                  void *stream) {
     using namespace moe;
+    const CallRange nvtx_range("moe_route_noalloc");
     if (!s) return record_error(MOE_ERR_INVALID_ARG, "shape is NULL");
     const int rc = validate_shape(s);
     if (rc != MOE_OK) return rc;
