@@ -92,6 +92,8 @@ CONFIGS = {
     # profiling-size stand-in for the large batches: ~1000 rows per expert
     "prefill_small": MoEConfig("prefill_small", T=4096, precision="fp8", bias="zero",
                                **{**_DS, "n_experts": 32}),
+    "prefill_small_ue8m0": MoEConfig("prefill_small_ue8m0", T=4096, precision="fp8_ue8m0",
+                                     bias="zero", **{**_DS, "n_experts": 32}),
 }
 
 
