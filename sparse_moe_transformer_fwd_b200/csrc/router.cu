@@ -186,7 +186,10 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
 // ------------------------------------------------- router_scores (small T)
 // Decode-sized batches: warp w of the CTA owns token t0 + w, lane l owns
 // expert e0 + l; one output per thread, so the kernel is bound by the length
-// of its d-long FMA chain.  Chunks of 256 columns of the CTA's 32 W_r rows
+// of its d-long FMA chain.  Four more warps only issue the ring's cp.async
+// copies: a warp issues one 16-byte-per-lane copy every ~90-160 cycles, and
+// issued by the compute warps the copies took 820 of 2250 cycles per chunk
+// (T = 64: 41 us -> 29 us with the copies moved off the FMA chains).  Chunks of 256 columns of the CTA's 32 W_r rows
 // and BT x rows stream into a 4-stage shared-memory ring with cp.async (W_r
 // rows padded by 16 bytes, so the 32 lanes' 16-byte reads of one column
 // fall in distinct banks), three chunks ahead of the FMAs; each warp widens
@@ -195,6 +198,7 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
 constexpr int RS_KC = 256;                 // columns per chunk
 constexpr int RS_WLD = RS_KC + 8;          // padded W_r row, bf16 elements
 constexpr int RS_STAGES = 4;
+constexpr int RS_PRODUCER_WARPS = 4;       // warps that only issue the ring's copies
 
 template <int BT>
 constexpr size_t router_small_smem() {
@@ -202,11 +206,14 @@ constexpr size_t router_small_smem() {
            static_cast<size_t>(BT) * RS_KC * 4;
 }
 
-template <int BT>
-__global__ void __launch_bounds__(BT * 32)
+template <int BT, int NP>
+__global__ void __launch_bounds__((BT + NP) * 32)
 router_scores_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w, int T,
                            int d, int E, float *__restrict__ scores, PreNorm pn) {
-    constexpr int NT = BT * 32;
+    // warps 0..BT-1 compute (one token each); warps BT..BT+NP-1 only issue the
+    // cp.async copies of the ring, so the compute warps' FMA chains do not
+    // wait behind the copy issue
+    constexpr int NT = NP * 32;  // copy-issuing threads
     constexpr int VPR = RS_KC / 8;                    // 16-byte vectors per row per chunk
     constexpr int W_ELEMS = 32 * RS_WLD, X_ELEMS = BT * RS_KC;
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -215,13 +222,15 @@ router_scores_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__res
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t0 = blockIdx.y * BT, e0 = blockIdx.x * 32;
     const int t = t0 + warp, e = e0 + lane;
+    const bool producer = warp >= BT;
+    const int ptid = tid - BT * 32;  // index among the copy-issuing threads
     pdl_wait_and_trigger();
 
     const int nk = d / RS_KC;
     auto issue = [&](int kc) {
         uint16_t *ws = ring + (kc % RS_STAGES) * (W_ELEMS + X_ELEMS);
         uint16_t *xs = ws + W_ELEMS;
-        for (int v = tid; v < (32 + BT) * VPR; v += NT) {
+        for (int v = ptid; v < (32 + BT) * VPR; v += NT) {
             const int row = v / VPR, col = (v % VPR) * 8;
             if (row < 32) {
                 const bool ok = e0 + row < E;
@@ -235,18 +244,25 @@ router_scores_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__res
             }
         }
     };
+    if (producer) {
 #pragma unroll
-    for (int s = 0; s < RS_STAGES - 1; ++s) {
-        if (s < nk) issue(s);
-        cp_async_commit();
+        for (int s = 0; s < RS_STAGES - 1; ++s) {
+            if (s < nk) issue(s);
+            cp_async_commit();
+        }
+        for (int kc = 0; kc < nk; ++kc) {
+            cp_async_wait<RS_STAGES - 2>();  // this thread's copies of chunk kc landed
+            __syncthreads();  // ... everyone's; and every warp is done with chunk kc - 1
+            if (kc + RS_STAGES - 1 < nk) issue(kc + RS_STAGES - 1);
+            cp_async_commit();
+        }
+        cp_async_wait<0>();
+        return;
     }
     float acc = 0.0f;
     float *xw = xf + warp * RS_KC;
     for (int kc = 0; kc < nk; ++kc) {
-        cp_async_wait<RS_STAGES - 2>();
         __syncthreads();  // chunk kc landed; every warp is done with chunk kc - 1
-        if (kc + RS_STAGES - 1 < nk) issue(kc + RS_STAGES - 1);
-        cp_async_commit();
         const uint16_t *ws = ring + (kc % RS_STAGES) * (W_ELEMS + X_ELEMS);
         const uint16_t *xs = ws + W_ELEMS;
         // this warp's token: 8 columns per lane and pass, widened (and pre-normed)
@@ -293,7 +309,6 @@ router_scores_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__res
         }
         __syncwarp();  // xw is rewritten next chunk
     }
-    cp_async_wait<0>();
     if (t < T && e < E) scores[static_cast<size_t>(t) * E + e] = sigmoid_cw(acc, exp_consts());
 }
 
@@ -381,18 +396,18 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
         LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel, grid, dim3(RT_THREADS), 0, st, x, w, T, d, E, scores,
                                     pn));
     } else {
-        constexpr int BT = 4;
+        constexpr int BT = 4, NP = RS_PRODUCER_WARPS;
         constexpr size_t smem = router_small_smem<BT>();
         static std::atomic<uint64_t> configured{0};  // one bit per device
         if (first_use_on_device(configured)) {
-            LAUNCH_OR_RETURN(cudaFuncSetAttribute(router_scores_small_kernel<BT>,
+            LAUNCH_OR_RETURN(cudaFuncSetAttribute(router_scores_small_kernel<BT, NP>,
                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                   static_cast<int>(smem)));
             mark_used_on_device(configured);
         }
         dim3 grid((E + 31) / 32, (T + BT - 1) / BT);
-        LAUNCH_OR_RETURN(launch_pdl(router_scores_small_kernel<BT>, grid, dim3(BT * 32), smem, st, x, w, T,
-                                    d, E, scores, pn));
+        LAUNCH_OR_RETURN(launch_pdl(router_scores_small_kernel<BT, NP>, grid, dim3((BT + NP) * 32), smem,
+                                    st, x, w, T, d, E, scores, pn));
     }
     ++*launches;
     const int per_lane = (E + 31) / 32;
