@@ -76,7 +76,7 @@ __device__ __forceinline__ float sigmoid_cw(float l, const ExpConsts &k) {
 }
 
 // ------------------------------------------------------- router_scores ---
-// Larger batches: a CTA of 128 threads owns 64 tokens x 64 experts; thread
+// Larger batches: a CTA of 128 threads owns 64 (or 32) tokens x 64 experts; thread
 // (ty, tx), ty < 8, tx < 16, owns tokens {4ty..4ty+3, 32+4ty..32+4ty+3} x
 // experts {4tx..4tx+3}, 32 accumulators, each still a sequential FMA chain
 // over d (the paired FMA of sm_100 does two independent correctly rounded
@@ -93,33 +93,39 @@ __device__ __forceinline__ int rt_swz(int k, int row) {
     return ((((row >> 2) ^ ((k >> 3) << 1)) & 15) << 2) | (row & 3);
 }
 
+// TB tokens per CTA: 64, or 32 for batches whose 64-token tiles would leave
+// SMs idle (fewer tiles than SMs); each thread then owns 4 tokens, not 8.
+template <int TB>
 __global__ void __launch_bounds__(RT_THREADS)
 router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w, int T, int d,
                      int E, float *__restrict__ scores, PreNorm pn) {
-    __shared__ __align__(16) float xs[2][RT_KC][RT_B];  // [k][token]
+    static_assert(TB == 64 || TB == 32, "token tile");
+    constexpr int NTOK = TB / 8;                         // tokens per thread
+    __shared__ __align__(16) float xs[2][RT_KC][TB];    // [k][token]
     __shared__ __align__(16) float ws[2][RT_KC][RT_B];  // [k][expert]
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-    const int t0 = blockIdx.y * RT_B, e0 = blockIdx.x * RT_B;
+    const int t0 = blockIdx.y * TB, e0 = blockIdx.x * RT_B;
     pdl_wait_and_trigger();
 
-    // acc[a][j]: token a of the thread's 8, experts (4tx + 2j, 4tx + 2j + 1)
-    float2 acc[8][2];
+    // acc[a][j]: token a of the thread's NTOK, experts (4tx + 2j, 4tx + 2j + 1)
+    float2 acc[NTOK][2];
 #pragma unroll
-    for (int a = 0; a < 8; ++a)
+    for (int a = 0; a < NTOK; ++a)
 #pragma unroll
         for (int b = 0; b < 2; ++b) acc[a][b] = make_float2(0.0f, 0.0f);
 
     constexpr int VPR = RT_KC / 8;                 // 16-byte vectors per row per chunk
-    constexpr int NV = 2 * RT_B * VPR;             // x rows then W_r rows
+    constexpr int NV = (TB + RT_B) * VPR;          // x rows then W_r rows
     constexpr int PER = NV / RT_THREADS;
+    static_assert(NV % RT_THREADS == 0, "whole vectors per thread");
     uint4 pre[PER];
     auto load = [&](int kc) {
 #pragma unroll
         for (int j = 0; j < PER; ++j) {
             const int v = tid + j * RT_THREADS;
             const int row = v / VPR, col = (v % VPR) * 8;
-            const bool isx = row < RT_B;
-            const int g = isx ? t0 + row : e0 + row - RT_B;
+            const bool isx = row < TB;
+            const int g = isx ? t0 + row : e0 + row - TB;
             pre[j] = make_uint4(0, 0, 0, 0);
             if (g < (isx ? T : E)) {
                 pre[j] = *reinterpret_cast<const uint4 *>((isx ? x : w) + static_cast<size_t>(g) * d +
@@ -133,13 +139,32 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
         for (int j = 0; j < PER; ++j) {
             const int v = tid + j * RT_THREADS;
             const int row = v / VPR, col = (v % VPR) * 8;
-            float(*dst)[RT_B] = row < RT_B ? xs[buf] : ws[buf];
-            const int r = row < RT_B ? row : row - RT_B;
-            const uint32_t r4[4] = {pre[j].x, pre[j].y, pre[j].z, pre[j].w};
+            if constexpr (TB == RT_B) {
+                // x and W_r rows have the same width: one destination pointer
+                float(*dst)[RT_B] = row < RT_B ? xs[buf] : ws[buf];
+                const int r = row < RT_B ? row : row - RT_B;
+                const uint32_t r4[4] = {pre[j].x, pre[j].y, pre[j].z, pre[j].w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                dst[col + 2 * q][rt_swz(col + 2 * q, r)] = bf16_lo(r4[q]);
-                dst[col + 2 * q + 1][rt_swz(col + 2 * q + 1, r)] = bf16_hi(r4[q]);
+                for (int q = 0; q < 4; ++q) {
+                    dst[col + 2 * q][rt_swz(col + 2 * q, r)] = bf16_lo(r4[q]);
+                    dst[col + 2 * q + 1][rt_swz(col + 2 * q + 1, r)] = bf16_hi(r4[q]);
+                }
+                continue;
+            }
+            const uint32_t r4[4] = {pre[j].x, pre[j].y, pre[j].z, pre[j].w};
+            if (row < TB) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    xs[buf][col + 2 * q][rt_swz(col + 2 * q, row)] = bf16_lo(r4[q]);
+                    xs[buf][col + 2 * q + 1][rt_swz(col + 2 * q + 1, row)] = bf16_hi(r4[q]);
+                }
+            } else {
+                const int r = row - TB;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    ws[buf][col + 2 * q][rt_swz(col + 2 * q, r)] = bf16_lo(r4[q]);
+                    ws[buf][col + 2 * q + 1][rt_swz(col + 2 * q + 1, r)] = bf16_hi(r4[q]);
+                }
             }
         }
     };
@@ -154,12 +179,14 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
 #pragma unroll 4
         for (int kk = 0; kk < RT_KC; ++kk) {
             const float4 xa = *reinterpret_cast<const float4 *>(&xs[buf][kk][rt_swz(kk, 4 * ty)]);
-            const float4 xb = *reinterpret_cast<const float4 *>(&xs[buf][kk][rt_swz(kk, 32 + 4 * ty)]);
+            float4 xb = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if constexpr (TB == 64)
+                xb = *reinterpret_cast<const float4 *>(&xs[buf][kk][rt_swz(kk, 32 + 4 * ty)]);
             const float4 wa = *reinterpret_cast<const float4 *>(&ws[buf][kk][rt_swz(kk, 4 * tx)]);
             const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
             const float2 wv[2] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w)};
 #pragma unroll
-            for (int a = 0; a < 8; ++a) {
+            for (int a = 0; a < NTOK; ++a) {
                 const float2 x2 = make_float2(xv[a], xv[a]);
 #pragma unroll
                 for (int b = 0; b < 2; ++b) acc[a][b] = __ffma2_rn(x2, wv[b], acc[a][b]);
@@ -171,7 +198,7 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
 
     const ExpConsts k = exp_consts();
 #pragma unroll
-    for (int a = 0; a < 8; ++a) {
+    for (int a = 0; a < NTOK; ++a) {
         const int t = t0 + (a < 4 ? 4 * ty + a : 32 + 4 * ty + a - 4);
         if (t >= T) continue;
 #pragma unroll
@@ -392,9 +419,18 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
                           float *gates, cudaStream_t st, int *launches, PreNorm pn) {
     mark_launch(st, *launches, "router_scores");
     if (T >= 512) {
-        dim3 grid((E + RT_B - 1) / RT_B, (T + RT_B - 1) / RT_B);
-        LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel, grid, dim3(RT_THREADS), 0, st, x, w, T, d, E, scores,
-                                    pn));
+        // 32-token tiles where 64-token tiles would leave SMs without one
+        const int e_tiles = (E + RT_B - 1) / RT_B;
+        const bool wide = static_cast<long long>((T + RT_B - 1) / RT_B) * e_tiles >= num_sms();
+        if (wide) {
+            dim3 grid(e_tiles, (T + 63) / 64);
+            LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel<64>, grid, dim3(RT_THREADS), 0, st, x, w, T, d,
+                                        E, scores, pn));
+        } else {
+            dim3 grid(e_tiles, (T + 31) / 32);
+            LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel<32>, grid, dim3(RT_THREADS), 0, st, x, w, T, d,
+                                        E, scores, pn));
+        }
     } else {
         constexpr int BT = 4, NP = RS_PRODUCER_WARPS;
         constexpr size_t smem = router_small_smem<BT>();
