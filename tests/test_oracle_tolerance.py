@@ -140,3 +140,41 @@ def test_nearest_correct_output_takes_only_explaining_alternatives():
     got_bad = as_bf16(bad)
     want_bad, _ = nearest_correct_output(got_bad, res["out_f64"], res["out_alts"])
     assert out_error(got_bad, want_bad)[0] > 0.5 * out_error(got_bad, res["out"])[0]
+
+
+def test_nearest_correct_output_without_alternatives_is_the_oracles():
+    """With no alternative codes the nearest correct output is the oracle's
+    own bf16 output, bit for bit (bf16 experts have none)."""
+    import torch
+    from _gpu_util import nearest_correct_output
+    cfg = DENSE_CONFIGS["dense_tiny"].with_(T=12, precision="bf16")
+    inp = make_dense_inputs(cfg, seed=33)
+    u = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    res = oracle.dense_ffn(u(inp["x"]), u(inp["w13"]), u(inp["w2"]), precision="bf16")
+    assert all(len(a) == 0 for a in res["out_alts"])
+    got = torch.from_numpy(res["out"].view(np.int16)).view(torch.bfloat16)
+    want, taken = nearest_correct_output(got, res["out_f64"], res["out_alts"])
+    assert taken == 0 and np.array_equal(want, res["out"])
+
+
+def test_ue8m0_alternatives_are_adjacent_codes_within_the_bound():
+    """With power-of-two scales the code-level alternatives are again the
+    neighbouring e4m3 values across a boundary, and never exceed
+    h_code_ambiguity, which also covers whole-tile scale changes."""
+    rng = np.random.default_rng(34)
+    H = (rng.standard_normal((16, 256)) * np.exp(rng.uniform(-3, 3, (16, 1)))).astype(np.float32)
+    rho = 2.0 ** -7
+    hq, hs = oracle.block_quant(H, 1, ue8m0=True)
+    alt = oracle.h_code_alternatives(H, hq, hs, True, rho=rho)
+    amb = oracle.h_code_ambiguity(H, hq, hs, True, rho=rho)
+    assert (alt != 0).sum() > 50
+    assert np.all(np.abs(alt) <= amb)
+    table = oracle.e4m3_decode_table()
+    finite = np.sort(np.unique(np.abs(table[np.isfinite(table)])))
+    sc = np.repeat(hs, 128, axis=1)
+    cur = table[hq]
+    for r, c in zip(*np.nonzero(alt)):
+        other = (cur[r, c] * sc[r, c] + alt[r, c]) / sc[r, c]
+        a, b = sorted((abs(cur[r, c]), abs(other)))
+        i = np.searchsorted(finite, a)
+        assert finite[i] == a and finite[i + 1] == b
