@@ -2,9 +2,12 @@
 
 One step = one forward pass of the whole layer (router, permutation,
 quantise-and-scatter, grouped gate/up GEMM + SwiGLU, grouped down GEMM,
-combine) over one batch of synthetic tokens.  Default workload: the decode
-batch (T=64 tokens, d_model 7168, 256 routed experts top-8 + 1 shared,
-d_expert 2048, e4m3 blockwise weights and activations, bf16 I/O).
+combine) over one batch of synthetic tokens.  Default workload: the largest
+single-GPU batch, skewed routing (T=16384 tokens, d_model 7168, 256 routed
+experts top-8 + 1 shared, d_expert 2048, e4m3 blockwise weights and
+activations with fp32 scales, bf16 I/O, router bias Zipf-ranked so that the
+hottest expert carries about 10x the mean load).  --workload decode gives the
+T=64 decode batch, whose gate/up GEMM is bound by HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload decode|prefill|skew|bf16|...|dense_decode|dense_prefill]
@@ -35,7 +38,6 @@ from moe_inputs import (CONFIGS, DENSE_CONFIGS, make_dense_inputs, make_inputs, 
 
 METRIC = "MoE-layer tokens/s at DeepSeek-V3 dims"
 DENSE_METRIC = "dense FFN-layer tokens/s at DeepSeek-V3 dims (first layers, d_ff 18432)"
-EVENT_EVERY = 4  # the dominant kernel is bracketed by CUDA events on every 4th timed step
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -189,6 +191,69 @@ def algorithmic_bytes_gemm1(cfg, touched: int) -> float:
     return float(w + a + h)
 
 
+def gemm1_flops(cfg) -> float:
+    """FLOPs of the gate/up GEMM: 2 * R_s rows * 2 d_expert outputs * d_model."""
+    return 2.0 * cfg.R_s * 2 * cfg.d_expert * cfg.d_model
+
+
+def tensor_peak(cfg, peaks) -> float:
+    """Dense tensor-core peak (TFLOP/s) of the GEMMs' operand type: measured
+    bf16 GEMM throughput, times the nominal e4m3 / bf16 ratio (4.5 / 2.25)
+    for the e4m3 precisions."""
+    return peaks["bf16_tflops"] * (1 if cfg.precision == "bf16" else 2)
+
+
+def moe_roofline(cfg, touched: int, ms: float, peaks, peak_kind: str):
+    """Roofline of the gate/up GEMM (the dominant kernel): its algorithmic
+    bytes (algorithmic_bytes_gemm1) and FLOPs (gemm1_flops); the bound is the
+    roof with the longer floor at the measured peaks (HBM copy bandwidth, or
+    the tensor peak of the operand type)."""
+    nbytes = algorithmic_bytes_gemm1(cfg, touched)
+    flops = gemm1_flops(cfg)
+    tc = tensor_peak(cfg, peaks)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (tc * 1e12)
+    src = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"
+    common = {"kernel": "grouped_gemm_gate_up", "algorithmic_bytes": nbytes,
+              "algorithmic_flops": flops, "kernel_ms": round(ms, 4),
+              "floor_ms": {"hbm": round(t_hbm * 1e3, 4), "tensor": round(t_tc * 1e3, 4)}}
+    if t_tc > t_hbm:
+        ach = flops / (ms * 1e-3) / 1e12
+        sus = peaks.get("bf16_tflops_sustained")
+        r = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc, "unit": "TFLOP/s",
+             "frac": round(ach / tc, 4),
+             "peak_source": src + (" bf16_tflops x 2 (e4m3/bf16 nominal ratio)"
+                                   if cfg.precision != "bf16" else " bf16_tflops")}
+        if sus:
+            tcs = sus * (1 if cfg.precision == "bf16" else 2)
+            r["frac_of_sustained"] = round(ach / tcs, 4)
+        return {**common, **r}
+    ach = nbytes / (ms * 1e-3) / 1e9
+    return {**common, "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+            "peak_source": src + " hbm_gbs"}
+
+
+def layer_floor(cfg, touched: int, ms_step: float, peaks):
+    """Floor of the whole layer: the longer of its HBM floor (every touched
+    expert's weights and scales read once, x read and out written once) and
+    its tensor floor (the two grouped GEMMs' FLOPs at the tensor peak); the
+    router's binary32 logits run on the CUDA cores and are not counted in
+    either.  frac = floor / measured step time."""
+    d, de = cfg.d_model, cfg.d_expert
+    es = 2 if cfg.precision == "bf16" else 1
+    sc = 0 if es == 2 else 4 * ((2 * de // 128) * (d // 128) + (d // 128) * (de // 128))
+    w = touched * (3 * de * d * es + sc)
+    io = cfg.T * d * 2 * 2
+    flops = 2.0 * cfg.R_s * 3 * de * d
+    t_hbm = (w + io) / (peaks["hbm_gbs"] * 1e9) * 1e3
+    t_tc = flops / (tensor_peak(cfg, peaks) * 1e12) * 1e3
+    floor = max(t_hbm, t_tc)
+    return {"bound": "tensor" if t_tc > t_hbm else "hbm", "floor_ms": round(floor, 4),
+            "hbm_floor_ms": round(t_hbm, 4), "tensor_floor_ms": round(t_tc, 4),
+            "frac": round(floor / ms_step, 4)}
+
+
 def e2e_host_loop(call, x, d_model, steps, world, dev):
     """End-to-end steps through the public API with pinned host buffers: each
     step copies its x host -> device, runs the layer and copies out device ->
@@ -289,32 +354,33 @@ def run_ours(args, world, rank, local):
     touched = int(torch.unique(idx).numel()) + cfg.n_shared
     counts = torch.bincount(idx.reshape(-1).long(), minlength=cfg.n_experts)
 
-    # ---- device-timed region: K steps, inputs resident in HBM; the dominant
-    # kernel (gate/up GEMM) is bracketed by CUDA events inside the region on
-    # every EVENT_EVERY-th step (an event between two launches stops their
-    # programmatic overlap, so the other steps run as a caller's would)
-    gi = names.index("grouped_gemm_gate_up")
-    g_steps = list(range(0, args.steps, EVENT_EVERY))
-    g_ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for k in g_steps}
+    # ---- device-timed region: K steps, inputs resident in HBM, nothing but the
+    # layer's own launches between the two events
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for a, b in g_ev.values():  # create the events before timing
-        a.record(stream)
-        b.record(stream)
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         start.record(stream)
         for k in range(args.steps):
-            moe.moe_set_kernel_events([None] * gi + list(g_ev[k]) if k in g_ev else None)
             call(x, out=out, topk_idx_out=idx)
-        moe.moe_set_kernel_events(None)
         stop.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     ms_total = max_over_ranks(start.elapsed_time(stop), world, dev)
     ms_step = ms_total / args.steps
-    g1_ms = float(np.mean([a.elapsed_time(b) for a, b in g_ev.values()]))
+
+    # ---- the dominant kernel (gate/up GEMM), bracketed by CUDA events on
+    # every step of a separate pass of K steps (an event between two launches
+    # stops their programmatic overlap, so this pass is not the timed one)
+    gi = names.index("grouped_gemm_gate_up")
+    g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for k in range(args.steps):
+        moe.moe_set_kernel_events([None] * gi + list(g_ev[k]))
+        call(x, out=out, topk_idx_out=idx)
+    moe.moe_set_kernel_events(None)
+    torch.cuda.synchronize()
+    g1_ms = float(np.mean([a.elapsed_time(b) for a, b in g_ev]))
 
     # ---- per-kernel breakdown (separate pass, every launch bracketed)
     nb = min(args.steps, 10)
@@ -338,7 +404,6 @@ def run_ours(args, world, rank, local):
         return None
     peaks, peak_kind = load_peaks()
     g1_bytes = algorithmic_bytes_gemm1(cfg, touched)
-    achieved = g1_bytes / (g1_ms * 1e-3) / 1e9
     tokens_total = T * world
     value = job_throughput(T, world, ms_step)
     res = {
@@ -368,23 +433,13 @@ def run_ours(args, world, rank, local):
             "expert_load_max_over_mean": round(float(counts.max()) / (T * cfg.top_k / cfg.n_experts), 2),
             "experts_empty": int((counts == 0).sum()),
         },
-        "roofline": {
-            "kernel": "grouped_gemm_gate_up",
-            "bound": "hbm",
-            "achieved": round(achieved, 1),
-            "peak": peaks["hbm_gbs"],
-            "unit": "GB/s",
-            "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                           else "fallback",
-            "algorithmic_bytes": g1_bytes,
-            "kernel_ms": round(g1_ms, 4),
-            "kernel_ms_from": f"CUDA events around this kernel on every {EVENT_EVERY}th step of the "
-                              "timed region",
-            "traffic": kernel_traffic("grouped_gemm_gate_up", cfg.name),
-            "traffic_source": "profiles/roofline_traffic.json (ncu dram__bytes_read+write, "
-                              "one capture of this workload)",
-        },
+        "roofline": {**moe_roofline(cfg, touched, g1_ms, peaks, peak_kind),
+                     "kernel_ms_from": "CUDA events around this kernel on every step of a "
+                                       "separate pass of K steps",
+                     "traffic": kernel_traffic("grouped_gemm_gate_up", cfg.name),
+                     "traffic_source": "profiles/roofline_traffic.json (ncu "
+                                       "dram__bytes_read+write per launch)"},
+        "layer_roofline": layer_floor(cfg, touched, ms_step, peaks),
         "kernels_ms": {n: round(float(v), 4) for n, v in zip(names, kmean)},
         "kernels_ms_note": "per-kernel means from a separate pass of the same call with every "
                            "launch bracketed by CUDA events",
@@ -459,26 +514,27 @@ def run_dense(args, world, rank, local):
         raise RuntimeError(f"device status: {moe.moe_last_error()}")
     n_launch = moe.moe_last_launch_count()
     names = moe.moe_last_launch_names()
-    gi = names.index("grouped_gemm_gate_up")
-    g_ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for k in range(0, args.steps, EVENT_EVERY)}
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for a, b in g_ev.values():
-        a.record(stream)
-        b.record(stream)
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         start.record(stream)
         for k in range(args.steps):
-            moe.moe_set_kernel_events([None] * gi + list(g_ev[k]) if k in g_ev else None)
             call(x, out)
-        moe.moe_set_kernel_events(None)
         stop.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     ms_step = max_over_ranks(start.elapsed_time(stop), world, dev) / args.steps
-    g1_ms = float(np.mean([a.elapsed_time(b) for a, b in g_ev.values()]))
+    # the gate/up GEMM bracketed on every step of a separate pass
+    gi = names.index("grouped_gemm_gate_up")
+    g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for k in range(args.steps):
+        moe.moe_set_kernel_events([None] * gi + list(g_ev[k]))
+        call(x, out)
+    moe.moe_set_kernel_events(None)
+    torch.cuda.synchronize()
+    g1_ms = float(np.mean([a.elapsed_time(b) for a, b in g_ev]))
     nb = min(args.steps, 10)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)] for _ in range(nb)]
     for k in range(nb):
@@ -578,6 +634,77 @@ def oracle_sample_time(cfg, dev, n_tokens: int, seed: int, reps: int = 1):
     return times, len(tokens), len(sel)
 
 
+def oracle_sample_time_all_cores(cfg, dev, per_worker: int, seed: int):
+    """The oracle's whole layer on all host cores: one thread per core, each
+    running the oracle (single-threaded per op, BLAS held to one thread) on
+    its own chunk of per_worker tokens of the batch (tokens are independent;
+    the C core and numpy release the interpreter lock).  The workers share
+    the host copies of the experts the sample touches, made before timing.
+    The worker count is the number of usable cores, lowered only if host
+    memory cannot hold the copies plus ~1 GB of temporaries per worker.
+    -> (wall seconds, tokens, workers, experts touched)."""
+    import concurrent.futures as cf
+
+    import psutil
+    from threadpoolctl import threadpool_limits
+
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    inp = make_inputs(cfg, seed=seed, device=dev)
+    u16 = lambda t: t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    wr = u16(inp["w_router"])
+    b = inp["bias"].cpu().numpy()
+    expert_bytes = 3 * cfg.d_expert * cfg.d_model * 2
+    avail = psutil.virtual_memory().available
+    workers = cores
+    while workers > 1:
+        n_tok = workers * per_worker
+        stride = max(1, cfg.T // n_tok)
+        tokens = list(range(0, cfg.T, stride))[:n_tok]
+        x_all = u16(inp["x"][tokens])
+        idx, _, _ = oracle.route(oracle.router_logits(x_all, wr), b, cfg.top_k)
+        sel = sorted(set(int(e) for e in idx.reshape(-1)) | {cfg.n_experts})
+        if len(sel) * expert_bytes + workers * (1 << 30) + (8 << 30) <= avail:
+            break
+        workers //= 2
+    if workers <= 1:
+        return None
+    experts = {e: (u16(inp["w13"][e]), u16(inp["w2"][e])) for e in sel}
+    del inp
+    chunks = [x_all[i * per_worker:(i + 1) * per_worker] for i in range(workers)]
+
+    def one(xc):
+        return oracle.moe_layer(xc, wr, b, lambda e: experts[e], n_experts=cfg.n_experts,
+                                top_k=cfg.top_k, n_shared=cfg.n_shared,
+                                precision=cfg.precision)["out"].shape[0]
+
+    with threadpool_limits(limits=1), cf.ThreadPoolExecutor(workers) as ex:
+        t0 = time.perf_counter()
+        done = sum(ex.map(one, chunks))
+        wall = time.perf_counter() - t0
+    return wall, done, workers, len(sel)
+
+
+def cpu_baseline_ours(cfg, dev, args):
+    """cpu_baseline of the default arm: the oracle on all host cores (one
+    thread per core over token chunks), with the single-threaded form beside it."""
+    times, ntok, nexp = oracle_sample_time(cfg, dev, args.cpu_baseline_tokens, args.seed)
+    single = {"value": round(ntok / times[0], 4), "unit": "tokens/s", "cores": 1,
+              "sample": f"{ntok} tokens of the {cfg.name} batch through the oracle's whole "
+                        f"layer ({nexp} experts incl. their weight quantisation), "
+                        f"{times[0]:.1f} s, 1 thread"}
+    par = oracle_sample_time_all_cores(cfg, dev, args.cpu_baseline_tokens, args.seed)
+    base = {"kind": "oracle", "cpu": cpu_model(), "single_thread": single}
+    if par is None:
+        return {**single, **base, "all_cores": "not run: host memory too small"}
+    wall, ntok_p, workers, nexp_p = par
+    return {"value": round(ntok_p / wall, 4), "unit": "tokens/s", "cores": workers, **base,
+            "sample": f"{ntok_p} tokens of the {cfg.name} batch, {args.cpu_baseline_tokens} per "
+                      f"thread on {workers} threads (one per core), each through the oracle's "
+                      f"whole layer ({nexp_p} experts touched, each thread quantising the "
+                      f"weights of its own experts), {wall:.1f} s wall"}
+
+
 def cpu_model():
     try:
         with open("/proc/cpuinfo") as f:
@@ -647,7 +774,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(CONFIGS) + list(DENSE_CONFIGS), default="decode")
+    ap.add_argument("--workload", choices=list(CONFIGS) + list(DENSE_CONFIGS), default="skew")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-tokens", type=int, default=1,
                     help="tokens of the batch per oracle step (reference arm)")
@@ -678,16 +805,7 @@ def main():
                               f"layer (incl. its weight quantisation), {times[0]:.1f} s, 1 thread",
                     "cpu": cpu_model()}
             elif world == 1 and not args.no_cpu_baseline:
-                dev = torch.device("cuda", local)
-                times, ntok, nexp = oracle_sample_time(cfg, dev, args.cpu_baseline_tokens,
-                                                       args.seed)
-                res["cpu_baseline"] = {
-                    "value": round(ntok / times[0], 4), "unit": "tokens/s", "cores": 1,
-                    "kind": "oracle",
-                    "sample": f"{ntok} tokens of the {cfg.name} batch through the oracle's whole "
-                              f"layer ({nexp} experts incl. their weight quantisation), "
-                              f"{times[0]:.1f} s, 1 thread",
-                    "cpu": cpu_model()}
+                res["cpu_baseline"] = cpu_baseline_ours(cfg, torch.device("cuda", local), args)
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:

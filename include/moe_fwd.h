@@ -68,12 +68,20 @@ enum moe_precision {
                           stored as fp32); see fp8_block_quant_ue8m0 */
 };
 
-/* Weight storage.  The expert GEMMs read their weights in TILED layout: a
- * row-major matrix of R rows x C bytes (R, C multiples of 128) stored as
- * (R/128) x (C/128) tiles of 128 rows x 128 bytes, tile (i, j) at byte
- * offset (i * (C/128) + j) * 16384, row r of a tile at r * 128 inside it.
- * For a stack [n, N, K] of expert matrices, R = n*N.  Each tile is one
- * contiguous 16 KB read (for e4m3 exactly one 128x128 scale block). */
+/* Weight storage (moe_shape.weight_layout, moe_dense_shape.weight_layout).
+ * The expert GEMMs read their weights in either of two layouts:
+ *  - MOE_LAYOUT_ROWMAJOR: each expert matrix [N, K] row-major, contiguous,
+ *    experts stacked ([n, N, K]); the layout of the problem statement.
+ *  - MOE_LAYOUT_TILED: a row-major matrix of R rows x C bytes (R, C
+ *    multiples of 128) stored as (R/128) x (C/128) tiles of 128 rows x 128
+ *    bytes, tile (i, j) at byte offset (i * (C/128) + j) * 16384, row r of a
+ *    tile at r * 128 inside it.  For a stack [n, N, K] of expert matrices,
+ *    R = n*N.  Each tile is one contiguous 16 KB read (for e4m3 exactly one
+ *    128x128 scale block), which the small (weight-streaming) batches read
+ *    at full HBM bandwidth.
+ * The layout of the weights a call reads is the one its shape declares; a
+ * zero-initialised shape declares MOE_LAYOUT_ROWMAJOR.  Scales are [n,
+ * N/128, K/128] row-major in both. */
 enum moe_layout {
     MOE_LAYOUT_ROWMAJOR = 0,
     MOE_LAYOUT_TILED = 1
@@ -81,7 +89,9 @@ enum moe_layout {
 
 /* Layer shape.  T tokens, d_model, n_experts routed experts (E), top_k (k),
  * d_expert, n_shared (0 or 1 shared experts of width d_expert),
- * routed_scale (multiplies every gate), precision (enum moe_precision). */
+ * routed_scale (multiplies every gate), precision (enum moe_precision),
+ * weight_layout (enum moe_layout) of w13 and w2; any other value is
+ * rejected with MOE_ERR_INVALID_ARG. */
 typedef struct moe_shape {
     int T;
     int d_model;
@@ -91,11 +101,31 @@ typedef struct moe_shape {
     int n_shared;
     float routed_scale;
     int precision;
+    int weight_layout;
 } moe_shape;
 
 /* Bytes of device workspace that moe_forward needs for this shape (the other
  * calls need no more).  0 if the shape is invalid (see moe_last_error). */
 size_t moe_workspace_size(const moe_shape *shape);
+
+/* Where moe_forward / moe_forward_prenorm keep their intermediate results
+ * inside the workspace: byte offsets from its start, for inspection (tests,
+ * debugging).  Once the call's kernels have run, the regions hold
+ *   scores    fp32 [T, n_experts]  affinities s = sigmoid(l)
+ *   topk_idx  int32 [T, top_k]     (only when topk_idx_out was NULL)
+ *   topk_w    fp32 [T, top_k]      gates
+ *   counts, offsets, row_token, row_of   the permutation (as moe_permute)
+ *   a         [R_s, d_model] e4m3 (fp8 precisions) or bf16: permuted rows of x
+ *   a_scales  fp32 [R_s, d_model/128] (fp8 precisions)
+ *   h, h_scales   [R_s, d_expert] H (e4m3 + scales, or bf16)
+ *   y         bf16 [R_s, d_model]  expert outputs before the combine
+ * with R_s = T*(top_k + n_shared).  The layout is fixed by the shape.
+ * Returns MOE_OK, or MOE_ERR_INVALID_ARG (invalid shape, NULL out). */
+typedef struct moe_workspace_offsets {
+    size_t status, scores, topk_idx, topk_w, counts, offsets, row_token, row_of;
+    size_t a, a_scales, h, h_scales, y, total;
+} moe_workspace_offsets;
+int moe_workspace_layout(const moe_shape *shape, moe_workspace_offsets *out);
 
 /* Router: logits l = x W_r^T in binary32 (sequential fused multiply-adds over
  * d_model), affinity s = sigmoid(l), selection by s + bias (bias: routing
@@ -124,6 +154,11 @@ int moe_route(const moe_shape *shape, const uint16_t *x, const uint16_t *w_route
  *     nothing enqueued.
  *   - The first call on a device looks up the array's device address (with
  *     that device current), so make that first call before any stream capture.
+ *     The address is looked up again when the device's context has changed
+ *     (after cudaDeviceReset, the library's module is loaded anew), so the
+ *     first call after a reset should also come before any stream capture.
+ *   - Error codes as moe_route (MOE_ERR_UNSUPPORTED on a device that is not
+ *     sm_100).
  *   - Every call shares the one array: calls whose kernels overlap on the GPU
  *     (other streams, other host threads) race and must be serialised by the
  *     caller.  The array keeps the last call's scores; nothing in it needs to
@@ -184,9 +219,9 @@ int moe_pack_tiles(const void *src, int rows, int row_bytes, void *dst, void *st
  *   a_scales   fp32 [R_s, d_model/128] (fp8 precisions) or NULL
  *   offsets    int32 [n_experts + 1] segment starts (as from moe_permute)
  *   w13        [E + n_shared, 2*d_expert, d_model]: gate rows, then up rows,
- *              e4m3 or bf16, in MOE_LAYOUT_TILED
+ *              e4m3 or bf16, in the shape's weight_layout
  *   w13_scales fp32 [E + n_shared, 2*d_expert/128, d_model/128] or NULL
- *   w2         [E + n_shared, d_model, d_expert], MOE_LAYOUT_TILED
+ *   w2         [E + n_shared, d_model, d_expert], in the shape's weight_layout
  *   w2_scales  fp32 [E + n_shared, d_model/128, d_expert/128] or NULL
  *   y          bf16 [R_s, d_model] out
  * In MOE_FP8_BLOCK, H is quantised 1x128 (e4m3) before the down GEMM (with
@@ -209,10 +244,12 @@ int moe_combine(const moe_shape *shape, const uint16_t *y, const int32_t *row_of
 /* The whole layer: route, permute, quantise-and-scatter (or bf16 scatter),
  * grouped gate/up GEMM + SwiGLU, grouped down GEMM, combine.
  *   x [T, d_model] bf16 in; out [T, d_model] bf16 out.
- *   w13/w2 and scales as for moe_grouped_swiglu (tiled; weights are quantised
- *   once, ahead of time, with fp8_block_quant(..., MOE_LAYOUT_TILED, ...) in
- *   MOE_FP8_BLOCK, fp8_block_quant_ue8m0 in MOE_FP8_UE8M0, or repacked with
- *   moe_pack_tiles in MOE_BF16).
+ *   w13/w2 and scales as for moe_grouped_swiglu, in the shape's
+ *   weight_layout (e4m3 weights are quantised once, ahead of time, with
+ *   fp8_block_quant in MOE_FP8_BLOCK or fp8_block_quant_ue8m0 in
+ *   MOE_FP8_UE8M0, with out_layout = the shape's weight_layout; bf16
+ *   weights are used as they are, or repacked once with moe_pack_tiles for
+ *   MOE_LAYOUT_TILED).
  *   topk_idx_out int32 [T, k] or NULL: receives the routing decision. */
 int moe_forward(const moe_shape *shape, const uint16_t *x, const uint16_t *w_router,
                 const float *bias, const void *w13, const float *w13_scales,
@@ -245,10 +282,11 @@ int moe_forward_prenorm(const moe_shape *shape, const uint16_t *h, const uint16_
  * the down GEMM; bf16: H rounded to bf16), every row of x in one segment.
  * Shapes: d_model a multiple of 256, d_ff a multiple of 128, T >= 0. */
 typedef struct {
-    int T;         /* tokens */
-    int d_model;   /* 7168 for DeepSeek-V3 */
-    int d_ff;      /* 18432 for DeepSeek-V3 */
-    int precision; /* enum moe_precision */
+    int T;             /* tokens */
+    int d_model;       /* 7168 for DeepSeek-V3 */
+    int d_ff;          /* 18432 for DeepSeek-V3 */
+    int precision;     /* enum moe_precision */
+    int weight_layout; /* enum moe_layout of w13 and w2 */
 } moe_dense_shape;
 
 /* Bytes of workspace moe_dense_ffn needs (0 on an invalid shape).  It holds
@@ -262,7 +300,7 @@ size_t moe_dense_workspace_size(const moe_dense_shape *shape);
  *       down GEMM splits K over the SMs) by a kernel that adds the K ranges'
  *       binary32 partial sums in order, so results do not depend on timing
  *   w13 [2*d_ff, d_model] (gate rows, then up rows) and w2 [d_model, d_ff]
- *       in TILED layout, e4m3 with scales [2*d_ff/128, d_model/128] and
+ *       in the shape's weight_layout, e4m3 with scales [2*d_ff/128, d_model/128] and
  *       [d_model/128, d_ff/128] (MOE_FP8_BLOCK / MOE_FP8_UE8M0), or bf16
  *       with NULL scales (MOE_BF16): the layout of one expert slot.
  *   ws: moe_dense_workspace_size bytes, zero-filled once before first use. */

@@ -146,15 +146,29 @@ def exp_cw(y: float) -> float:
 
 # ------------------------------------------------------------------ router --
 
-def router_logits(x_bf16, w_router_bf16) -> np.ndarray:
-    """[T, E] binary32 logits, sequential FMA over d_model (C core)."""
+def router_logits(x_bf16, w_router_bf16, workers: int = 1) -> np.ndarray:
+    """[T, E] binary32 logits, sequential FMA over d_model (C core).
+    workers > 1 splits the tokens into that many chunks, each one
+    single-threaded call of the C core on its own thread (every logit is
+    computed on its own, so the result does not depend on the split)."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     w = np.ascontiguousarray(w_router_bf16, dtype=np.uint16)
     T, d = x.shape
     E = w.shape[0]
     out = np.empty((T, E), dtype=np.float32)
-    lib().oracle_router_logits(_p(x, ctypes.c_uint16), _p(w, ctypes.c_uint16), T, d, E,
-                               _p(out, ctypes.c_float))
+
+    def rows(lo, hi):
+        lib().oracle_router_logits(_p(x[lo:hi], ctypes.c_uint16), _p(w, ctypes.c_uint16),
+                                   hi - lo, d, E, _p(out[lo:hi], ctypes.c_float))
+
+    workers = max(1, min(int(workers), T))
+    if workers == 1:
+        rows(0, T)
+    else:
+        import concurrent.futures as cf
+        cuts = np.linspace(0, T, workers + 1).astype(int)
+        with cf.ThreadPoolExecutor(workers) as ex:
+            list(ex.map(lambda i: rows(cuts[i], cuts[i + 1]), range(workers)))
     return out
 
 
@@ -388,7 +402,7 @@ def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=No
 # ------------------------------------------------------------------- layer --
 
 def moe_layer(x, w_router, bias, expert, *, n_experts: int, top_k: int, n_shared: int,
-              precision: str, routed_scale: float = 1.0, tokens=None):
+              precision: str, routed_scale: float = 1.0, tokens=None, workers: int = 1):
     """Forward of one MoE FFN layer.
 
     x uint16 [T, d] (bf16 bits); w_router uint16 [E, d]; bias fp32 [E];
@@ -397,13 +411,16 @@ def moe_layer(x, w_router, bias, expert, *, n_experts: int, top_k: int, n_shared
     touches itself (128x128 blocks).
     tokens: indices of the output rows to evaluate (default: all).  Routing,
     permutation and activation quantisation always cover every token.
+    workers > 1 evaluates the experts (each on its own, unchanged) on that
+    many threads, and the router's logits in as many token chunks; the
+    results do not depend on it.
 
     Returns a dict: logits, scores, idx, gates, counts, offsets, row_token,
     row_of, (fp8) xq, xs, out [len(tokens), d] bf16 bits, tokens."""
     x = np.ascontiguousarray(x, dtype=np.uint16)
     T, d = x.shape
     E, k = n_experts, top_k
-    logits = router_logits(x, w_router)
+    logits = router_logits(x, w_router, workers=workers)
     idx, gates, scores = route(logits, bias, k, routed_scale)
     counts, offsets, row_token, row_of = permute(idx, E)
     res = dict(logits=logits, scores=scores, idx=idx, gates=gates, counts=counts,
@@ -423,10 +440,9 @@ def moe_layer(x, w_router, bias, expert, *, n_experts: int, top_k: int, n_shared
             need.setdefault(E, []).append((ti, k))
     Yt = np.zeros((len(tokens), k + 1, d), dtype=np.float64)
     At = np.zeros((len(tokens), k + 1, d), dtype=np.float64)
-    for e in sorted(need):
+    def one_expert(e):
         w13, w2 = expert(e)
-        pairs = need[e]
-        rows = np.array([tokens[ti] for ti, _ in pairs])
+        rows = np.array([tokens[ti] for ti, _ in need[e]])
         if fp8:
             w13q, w13s = block_quant(w13, 128, ue8m0=ue)
             w2q, w2s = block_quant(w2, 128, ue8m0=ue)
@@ -434,10 +450,21 @@ def moe_layer(x, w_router, bias, expert, *, n_experts: int, top_k: int, n_shared
                                    w13s, w2s, return_allow=True)
         else:
             y, al = expert_forward(x[rows], w13, w2, "bf16", return_allow=True)
-        yf = bf16_to_f32(y).astype(np.float64)
-        for n, (ti, j) in enumerate(pairs):
+        return bf16_to_f32(y).astype(np.float64), al
+
+    def store(e, yf, al):
+        for n, (ti, j) in enumerate(need[e]):
             Yt[ti, j] = yf[n]
             At[ti, j] = al[n]
+
+    if workers > 1:
+        import concurrent.futures as cf
+        with cf.ThreadPoolExecutor(int(workers)) as ex:
+            for e, (yf, al) in zip(sorted(need), ex.map(one_expert, sorted(need))):
+                store(e, yf, al)
+    else:
+        for e in sorted(need):
+            store(e, *one_expert(e))
     g = gates[tokens].astype(np.float64)
     acc = np.einsum("tj,tjd->td", g, Yt[:, :k])
     allow = np.einsum("tj,tjd->td", np.abs(g), At[:, :k])

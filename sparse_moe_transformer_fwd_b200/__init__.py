@@ -20,7 +20,7 @@ from ._native import (EXPORTS, MOE_BF16, MOE_FP8_BLOCK, MOE_FP8_UE8M0, MOE_LAYOU
                       moe_permute, moe_route, moe_route_noalloc, moe_set_kernel_events,
                       moe_workspace_size, MOE_ROUTE_NOALLOC_MAX_SCORES, MoeDenseShape,
                       make_dense_shape, moe_dense_workspace_size, alloc_dense_workspace,
-                      moe_dense_ffn, moe_dense_ffn_prenorm)
+                      moe_dense_ffn, moe_dense_ffn_prenorm, moe_workspace_layout)
 
 __all__ = [
     "MoELayer", "MoeError", "MoeShape", "make_shape", "alloc_workspace", "lib", "EXPORTS",
@@ -30,22 +30,23 @@ __all__ = [
     "moe_route_noalloc", "MOE_ROUTE_NOALLOC_MAX_SCORES", "moe_pack_tiles", "pack_weights",
     "MOE_LAYOUT_ROWMAJOR", "MOE_LAYOUT_TILED", "moe_forward_prenorm", "moe_last_launch_names",
     "DenseFFN", "MoeDenseShape", "make_dense_shape", "moe_dense_workspace_size",
-    "alloc_dense_workspace", "moe_dense_ffn", "moe_dense_ffn_prenorm",
+    "alloc_dense_workspace", "moe_dense_ffn", "moe_dense_ffn_prenorm", "moe_workspace_layout",
 ]
 
 
-def quantize_weights(w13: torch.Tensor, w2: torch.Tensor, stream=None, ue8m0: bool = False):
+def quantize_weights(w13: torch.Tensor, w2: torch.Tensor, stream=None, ue8m0: bool = False,
+                     layout=MOE_LAYOUT_TILED):
     """128x128 e4m3 block quantisation of the stacked expert weights (done
-    once, ahead of the forward passes), codes in the tiled layout the GEMMs
-    read; ue8m0: power-of-two scales.  Returns (w13q, w13s, w2q, w2s)."""
+    once, ahead of the forward passes), codes in `layout` (tiled by default,
+    or row-major); ue8m0: power-of-two scales.  Returns (w13q, w13s, w2q, w2s)."""
     S, n13, d = w13.shape
     _, d2, de = w2.shape
     w13q = torch.empty(S, n13, d, dtype=torch.uint8, device=w13.device)
     w13s = torch.empty(S, n13 // 128, d // 128, dtype=torch.float32, device=w13.device)
     w2q = torch.empty(S, d2, de, dtype=torch.uint8, device=w2.device)
     w2s = torch.empty(S, d2 // 128, de // 128, dtype=torch.float32, device=w2.device)
-    fp8_block_quant(w13, 128, w13q, w13s, layout=MOE_LAYOUT_TILED, stream=stream, ue8m0=ue8m0)
-    fp8_block_quant(w2, 128, w2q, w2s, layout=MOE_LAYOUT_TILED, stream=stream, ue8m0=ue8m0)
+    fp8_block_quant(w13, 128, w13q, w13s, layout=layout, stream=stream, ue8m0=ue8m0)
+    fp8_block_quant(w2, 128, w2q, w2s, layout=layout, stream=stream, ue8m0=ue8m0)
     return w13q, w13s, w2q, w2s
 
 
@@ -65,23 +66,31 @@ class MoELayer:
     expert, if any, is the last slot.  precision "fp8" (fp32 block scales) or
     "fp8_ue8m0" (power-of-two block scales) quantises the expert weights once
     at construction (the bf16 copies are then not needed); "bf16" repacks
-    them."""
+    them.  weight_layout "tiled" (default: 128 x 128-byte tiles, one
+    contiguous 16 KB read per TMA box) or "rowmajor" (the weights as given,
+    e4m3 codes row-major)."""
 
     def __init__(self, w_router, bias, w13, w2, *, top_k: int, n_shared: int = 1,
-                 routed_scale: float = 1.0, precision: str = "fp8", keep_bf16: bool = False):
+                 routed_scale: float = 1.0, precision: str = "fp8", keep_bf16: bool = False,
+                 weight_layout: str = "tiled"):
         lib()  # fail loudly now if the CUDA library is missing
         self.E, self.d = w_router.shape
         self.de = w2.shape[2]
         self.top_k, self.n_shared, self.routed_scale = top_k, n_shared, routed_scale
         self.precision = precision
+        if weight_layout not in ("tiled", "rowmajor"):
+            raise ValueError(weight_layout)
+        self.weight_layout = weight_layout
+        lay = MOE_LAYOUT_TILED if weight_layout == "tiled" else MOE_LAYOUT_ROWMAJOR
         self.w_router, self.bias = w_router.contiguous(), bias.contiguous()
         if precision in ("fp8", "fp8_ue8m0"):
             self.w13, self.w13s, self.w2, self.w2s = quantize_weights(
-                w13.contiguous(), w2.contiguous(), ue8m0=precision == "fp8_ue8m0")
+                w13.contiguous(), w2.contiguous(), ue8m0=precision == "fp8_ue8m0", layout=lay)
             self.w13_bf16 = w13 if keep_bf16 else None
             self.w2_bf16 = w2 if keep_bf16 else None
         elif precision == "bf16":
-            self.w13, self.w2 = pack_weights(w13, w2)
+            self.w13, self.w2 = pack_weights(w13, w2) if lay == MOE_LAYOUT_TILED else \
+                (w13.contiguous(), w2.contiguous())
             self.w13s = self.w2s = None
         else:
             raise ValueError(precision)
@@ -89,7 +98,7 @@ class MoELayer:
 
     def shape(self, T: int) -> MoeShape:
         return make_shape(T, self.d, self.E, self.top_k, self.de, self.n_shared,
-                          self.routed_scale, self.precision)
+                          self.routed_scale, self.precision, self.weight_layout)
 
     def workspace(self, T: int) -> torch.Tensor:
         ws = self._ws.get(T)
@@ -128,25 +137,29 @@ class DenseFFN:
     weights, on the expert GEMM kernels.
 
     w13 bf16 [2*d_ff, d] (gate rows then up rows); w2 bf16 [d, d_ff].
-    precision as for MoELayer ("fp8", "fp8_ue8m0" or "bf16")."""
+    precision and weight_layout as for MoELayer."""
 
-    def __init__(self, w13, w2, *, precision: str = "fp8"):
+    def __init__(self, w13, w2, *, precision: str = "fp8", weight_layout: str = "tiled"):
         lib()
         self.d, self.d_ff = w2.shape
         self.precision = precision
+        if weight_layout not in ("tiled", "rowmajor"):
+            raise ValueError(weight_layout)
+        self.weight_layout = weight_layout
+        lay = MOE_LAYOUT_TILED if weight_layout == "tiled" else MOE_LAYOUT_ROWMAJOR
         w13, w2 = w13.contiguous().unsqueeze(0), w2.contiguous().unsqueeze(0)
         if precision in ("fp8", "fp8_ue8m0"):
             self.w13, self.w13s, self.w2, self.w2s = quantize_weights(
-                w13, w2, ue8m0=precision == "fp8_ue8m0")
+                w13, w2, ue8m0=precision == "fp8_ue8m0", layout=lay)
         elif precision == "bf16":
-            self.w13, self.w2 = pack_weights(w13, w2)
+            self.w13, self.w2 = pack_weights(w13, w2) if lay == MOE_LAYOUT_TILED else (w13, w2)
             self.w13s = self.w2s = None
         else:
             raise ValueError(precision)
         self._ws = {}
 
     def shape(self, T: int) -> MoeDenseShape:
-        return make_dense_shape(T, self.d, self.d_ff, self.precision)
+        return make_dense_shape(T, self.d, self.d_ff, self.precision, self.weight_layout)
 
     def workspace(self, T: int) -> torch.Tensor:
         ws = self._ws.get(T)

@@ -31,7 +31,7 @@ EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant",
            "moe_last_error", "moe_last_launch_count", "moe_set_kernel_events",
            "moe_route_noalloc", "moe_pack_tiles", "moe_forward_prenorm", "moe_last_launch_name",
            "fp8_block_quant_ue8m0", "moe_dense_workspace_size", "moe_dense_ffn",
-           "moe_dense_ffn_prenorm")
+           "moe_dense_ffn_prenorm", "moe_workspace_layout")
 
 # fixed score scratch of moe_route_noalloc, in floats (include/moe_fwd.h)
 MOE_ROUTE_NOALLOC_MAX_SCORES = 1 << 20
@@ -40,12 +40,19 @@ MOE_ROUTE_NOALLOC_MAX_SCORES = 1 << 20
 class MoeShape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int), ("d_model", ctypes.c_int), ("n_experts", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("d_expert", ctypes.c_int), ("n_shared", ctypes.c_int),
-                ("routed_scale", ctypes.c_float), ("precision", ctypes.c_int)]
+                ("routed_scale", ctypes.c_float), ("precision", ctypes.c_int),
+                ("weight_layout", ctypes.c_int)]
 
 
 class MoeDenseShape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int), ("d_model", ctypes.c_int), ("d_ff", ctypes.c_int),
-                ("precision", ctypes.c_int)]
+                ("precision", ctypes.c_int), ("weight_layout", ctypes.c_int)]
+
+
+class MoeWorkspaceOffsets(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "status", "scores", "topk_idx", "topk_w", "counts", "offsets", "row_token", "row_of",
+        "a", "a_scales", "h", "h_scales", "y", "total")]
 
 
 class MoeError(RuntimeError):
@@ -69,6 +76,7 @@ def lib() -> ctypes.CDLL:
         sp = ctypes.POINTER(MoeShape)
         L.moe_workspace_size.argtypes = [sp]
         L.moe_workspace_size.restype = sz
+        L.moe_workspace_layout.argtypes = [sp, ctypes.POINTER(MoeWorkspaceOffsets)]
         L.moe_route.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_permute.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_route_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp]
@@ -95,7 +103,7 @@ def lib() -> ctypes.CDLL:
                      "fp8_block_quant_ue8m0", "moe_grouped_swiglu",
                      "moe_combine", "moe_forward", "moe_check_status", "moe_last_launch_count",
                      "moe_set_kernel_events", "moe_pack_tiles", "moe_forward_prenorm",
-                     "moe_dense_ffn", "moe_dense_ffn_prenorm"):
+                     "moe_dense_ffn", "moe_dense_ffn_prenorm", "moe_workspace_layout"):
             getattr(L, name).restype = ci
         _LIB = L
     return _LIB
@@ -126,19 +134,32 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _layout(weight_layout) -> int:
+    return {"rowmajor": MOE_LAYOUT_ROWMAJOR, "tiled": MOE_LAYOUT_TILED}[weight_layout] \
+        if isinstance(weight_layout, str) else int(weight_layout)
+
+
 def make_shape(T, d_model, n_experts, top_k, d_expert, n_shared=1, routed_scale=1.0,
-               precision="fp8") -> MoeShape:
+               precision="fp8", weight_layout=MOE_LAYOUT_TILED) -> MoeShape:
     prec = {"bf16": MOE_BF16, "fp8": MOE_FP8_BLOCK, "fp8_ue8m0": MOE_FP8_UE8M0}[precision] \
         if isinstance(precision, str) \
         else int(precision)
     return MoeShape(int(T), int(d_model), int(n_experts), int(top_k), int(d_expert),
-                    int(n_shared), float(routed_scale), prec)
+                    int(n_shared), float(routed_scale), prec, _layout(weight_layout))
 
 
-def make_dense_shape(T, d_model, d_ff, precision="fp8") -> MoeDenseShape:
+def make_dense_shape(T, d_model, d_ff, precision="fp8",
+                     weight_layout=MOE_LAYOUT_TILED) -> MoeDenseShape:
     prec = {"bf16": MOE_BF16, "fp8": MOE_FP8_BLOCK, "fp8_ue8m0": MOE_FP8_UE8M0}[precision] \
         if isinstance(precision, str) else int(precision)
-    return MoeDenseShape(int(T), int(d_model), int(d_ff), prec)
+    return MoeDenseShape(int(T), int(d_model), int(d_ff), prec, _layout(weight_layout))
+
+
+def moe_workspace_layout(shape: MoeShape) -> dict:
+    """Byte offsets of moe_forward's intermediate results in its workspace."""
+    o = MoeWorkspaceOffsets()
+    _check(lib().moe_workspace_layout(ctypes.byref(shape), ctypes.byref(o)))
+    return {n: getattr(o, n) for n, _ in MoeWorkspaceOffsets._fields_}
 
 
 _BF16 = torch.bfloat16

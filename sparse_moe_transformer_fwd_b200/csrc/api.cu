@@ -76,6 +76,13 @@ bool inject_gemm_fault() {
     return v && strcmp(v, "gemm_tx") == 0;
 }
 
+// Schedule of the fp32-scale GEMMs' accumulator (see gemm_sm100.cu): two
+// N = 128 halves per K step unless MOE_GEMM_SPLIT_N=0.
+bool gemm_split_n() {
+    const char *v = getenv("MOE_GEMM_SPLIT_N");
+    return !(v && strcmp(v, "0") == 0);
+}
+
 int check_device() {
     int dev = 0, major = 0, minor = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -103,6 +110,8 @@ int check_shape(const moe_shape *s) {
     if (s->precision != MOE_BF16 && s->precision != MOE_FP8_BLOCK &&
         s->precision != MOE_FP8_UE8M0)
         return fail(MOE_ERR_INVALID_ARG, "unknown precision %d", s->precision);
+    if (s->weight_layout != MOE_LAYOUT_ROWMAJOR && s->weight_layout != MOE_LAYOUT_TILED)
+        return fail(MOE_ERR_INVALID_ARG, "unknown weight_layout %d", s->weight_layout);
     const long long R_s = static_cast<long long>(s->T) * (s->top_k + s->n_shared);
     if (R_s * s->d_model > (1LL << 40) || R_s > (1LL << 30))
         return fail(MOE_ERR_INVALID_ARG, "T too large");
@@ -237,6 +246,8 @@ int grouped(const moe_shape *s, const void *a, const float *a_scales, const void
     g.inject_fault = inject_gemm_fault() ? 1 : 0;
     g.ue8m0 = is_ue8m0(s);
     g.tile_m = tile_m;
+    g.b_rowmajor = s->weight_layout == MOE_LAYOUT_ROWMAJOR;
+    g.split_n = gemm_split_n();
     // gate/up GEMM + SwiGLU
     g.gate_up = true;
     g.a = a;
@@ -280,6 +291,7 @@ int check_weights(const moe_shape *s, const void *w13, const float *w13s, const 
 int record_error(int code, const char *msg) { return fail(code, "%s", msg); }
 void record_launches(int n) { g_launches = n; }
 int validate_shape(const moe_shape *s) { return check_shape(s); }
+int validate_device() { return check_device(); }
 
 }  // namespace moe
 
@@ -290,6 +302,27 @@ extern "C" {
 size_t moe_workspace_size(const moe_shape *shape) {
     if (check_shape(shape) != MOE_OK) return 0;
     return layout(shape).total;
+}
+
+int moe_workspace_layout(const moe_shape *shape, moe_workspace_offsets *out) {
+    RETURN_IF(check_shape(shape));
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+    const Layout L = layout(shape);
+    out->status = L.status;
+    out->scores = L.scores;
+    out->topk_idx = L.idx;
+    out->topk_w = L.gates;
+    out->counts = L.counts;
+    out->offsets = L.offsets;
+    out->row_token = L.row_token;
+    out->row_of = L.row_of;
+    out->a = L.a;
+    out->a_scales = L.a_scales;
+    out->h = L.h;
+    out->h_scales = L.h_scales;
+    out->y = L.y;
+    out->total = L.total;
+    return MOE_OK;
 }
 
 int moe_route(const moe_shape *s, const uint16_t *x, const uint16_t *w_router, const float *bias,
@@ -550,6 +583,8 @@ int check_dense_shape(const moe_dense_shape *s) {
     if (s->precision != MOE_BF16 && s->precision != MOE_FP8_BLOCK &&
         s->precision != MOE_FP8_UE8M0)
         return fail(MOE_ERR_INVALID_ARG, "unknown precision %d", s->precision);
+    if (s->weight_layout != MOE_LAYOUT_ROWMAJOR && s->weight_layout != MOE_LAYOUT_TILED)
+        return fail(MOE_ERR_INVALID_ARG, "unknown weight_layout %d", s->weight_layout);
     if (static_cast<long long>(s->T) * std::max(s->d_model, s->d_ff) > (1LL << 40) ||
         s->T > (1 << 30))
         return fail(MOE_ERR_INVALID_ARG, "T too large");
@@ -657,6 +692,8 @@ int dense_impl(const moe_dense_shape *s, const uint16_t *x, const uint16_t *gamm
     g.seg_start = g.seg_rows = g.tile_start = nullptr;  // one segment of all T rows
     g.status = at<int>(ws, L.status);
     g.ue8m0 = ue;
+    g.b_rowmajor = s->weight_layout == MOE_LAYOUT_ROWMAJOR;
+    g.split_n = gemm_split_n();
     // one segment of T rows: 64-row tiles only where they save round trips
     g.tile_m = (s->precision == MOE_FP8_BLOCK && T <= 64) ? 64 : 128;
     g.gate_up = true;

@@ -6,13 +6,15 @@
 //
 // One persistent kernel per GEMM, one CTA per SM, cluster size 1.
 // Work item = (segment, 128-row tile of the segment, 256-column tile of B).
-// Tiles are ordered m-major, n-minor, so the CTAs running at one time share
-// A tiles and the same expert's weights through L2.
+// Within a segment, tiles are ordered column-tile major, row-tile minor, so
+// the CTAs running at one time read the same weight tiles through L2 (each
+// weight byte crosses DRAM once) and re-read the smaller row tiles from L2.
 //   warp 0      TMA producer: A tile 128 x 128 B and two B tiles 128 x 128 B
 //               (gate/up rows, or two halves of the output columns) per
-//               stage, 128-byte swizzle, 4 stages.  The weights are stored in
-//               128 x 128-byte tiles, so each B box is one contiguous 16 KB
-//               read from HBM.
+//               stage, 128-byte swizzle, 4 stages.  Weights stored in the
+//               tiled layout (128 x 128-byte tiles) make each B box one
+//               contiguous 16 KB read from HBM; row-major weights are read
+//               as 128 rows of 128 bytes.
 //   warp 1      TMEM allocator (512 columns) and MMA issuer (one thread):
 //               tcgen05.mma M=128 N=256, K=32 (e4m3) or K=16 (bf16), four per
 //               stage.
@@ -94,8 +96,8 @@ struct __align__(1024) GemmSmem {
     uint64_t sf_free[SF_BUFS];      // scale block copied to TMEM (tcgen05.commit -> warp 2)
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
+    uint64_t tfull[4];   // [2 * buffer + half]: accumulator (half) ready
+    uint64_t tempty[4];  // [2 * buffer + half]: accumulator (half) drained
     uint64_t xchg[2];        // amax exchange between the two column halves
     uint64_t mma_done;
     uint32_t tmem_base;
@@ -126,21 +128,34 @@ struct KParams {
     int ksplit;
     float *partial;        // [ksplit][rows_total][N_out]
     const uint16_t *residual;  // down GEMM without split: bf16 [rows_total, N_out] added before rounding Y
+    int b_rowmajor;        // B row-major [slots * b_rows, K] instead of 128 x 128-byte tiles
+    // fp32 scales, 128-row tiles: each K step's 128 x 256 accumulator is made
+    // by two N = 128 MMAs into two 128-column halves with their own ready and
+    // drained barriers, so the four halves of the two buffers give the
+    // epilogue's TMEM round trip three half steps of MMA work to hide in
+    int split_n;
 };
 
+// Output tile `tile` -> (segment, first row, valid rows, column tile).  The
+// tiles of segment s are numbered tile_start[s] * n_tiles_n on, column tile
+// major and row tile minor: consecutive tiles (run side by side by
+// neighbouring CTAs) read the same weight tile for different row tiles, so
+// each weight tile crosses DRAM once while its row tiles are in flight.
 template <int TM>
 __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int tile, int n_tiles_n,
                                             int &seg, int &row0, int &rows_valid, int &nt) {
-    const int mt = tile / n_tiles_n;
-    nt = tile - mt * n_tiles_n;
-    int lo = 0, hi = n_seg - 1;  // last segment whose first tile is <= mt
+    const int mt = tile / n_tiles_n;  // tile_start[s] * n_tiles_n <= tile  <=>  tile_start[s] <= mt
+    int lo = 0, hi = n_seg - 1;       // last segment whose first tile is <= mt
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (s.tile_start[mid] <= mt) lo = mid;
         else hi = mid - 1;
     }
     seg = lo;
-    const int mloc = mt - s.tile_start[seg];
+    const int m_s = s.tile_start[seg + 1] - s.tile_start[seg];  // row tiles of the segment
+    const int local = tile - s.tile_start[seg] * n_tiles_n;
+    nt = local / m_s;
+    const int mloc = local - nt * m_s;
     row0 = s.seg_start[seg] + mloc * TM;
     rows_valid = min(TM, s.seg_rows[seg] - mloc * TM);
 }
@@ -216,14 +231,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&s.empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s.tfull[i], 1);
-            mbar_init(&s.tempty[i], EPI_THREADS / 32);
+            mbar_init(&s.tfull[2 * i], 1);
+            mbar_init(&s.tempty[2 * i], EPI_THREADS / 32);
+            mbar_init(&s.tfull[2 * i + 1], 1);
+            mbar_init(&s.tempty[2 * i + 1], EPI_THREADS / 32);
             mbar_init(&s.xchg[i], EPI_THREADS);
         }
         mbar_init(&s.mma_done, 1);
         for (int i = 0; i < SF_STAGING; ++i) {
             mbar_init(&s.sf_full[i], 1);
-            mbar_init(&s.sf_empty[i], 1);
+            // freed by warp 2 (block-scaled MMA) or by every epilogue warp (fp32 scales)
+            mbar_init(&s.sf_empty[i], MX ? 1 : EPI_THREADS / 32);
         }
         for (int i = 0; i < SF_BUFS; ++i) {
             mbar_init(&s.sf_ready[i], 1);
@@ -238,11 +256,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     // wait below; the producer adds their A loads after it.
     int pre = 0;
     const int NBq = p.b_rows / 128;
-    auto b_tile_rows = [&](int seg, int nt, long long &t_lo, long long &t_hi) {
+    // The two 128-row blocks of B a work item reads (gate and up rows, or
+    // the two halves of the output columns), as 128-row block indices of the
+    // stacked weights: t_lo, t_hi = slot * NBq + block.
+    auto b_blocks = [&](int seg, int nt, long long &t_lo, long long &t_hi) {
         const int nb_lo = GATE_UP ? nt : 2 * nt;
         const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
-        t_lo = (static_cast<long long>(seg) * NBq + nb_lo) * KB;
-        t_hi = (static_cast<long long>(seg) * NBq + nb_hi) * KB;
+        t_lo = static_cast<long long>(seg) * NBq + nb_lo;
+        t_hi = static_cast<long long>(seg) * NBq + nb_hi;
+    };
+    // TMA box (128 rows x 128 bytes) of block t at K block kb: tiled layout,
+    // tile row (t * KB + kb) * 128 of a 128-byte-wide map; row-major, rows
+    // t * 128.. at K offset kb * 128 bytes.
+    auto load_b = [&](void *dst, long long t, int kb, uint64_t *bar) {
+        if (p.b_rowmajor)
+            tma_load_2d(dst, &tmap_b, FP8 ? kb * 128 : kb * 64, static_cast<int>(t * 128), bar);
+        else
+            tma_load_2d(dst, &tmap_b, 0, static_cast<int>((t * KB + kb) * 128), bar);
     };
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmap_a);
@@ -252,13 +282,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             int tile, ks, kb0, nk;
             k_range(blockIdx.x, tile, ks, kb0, nk);
             long long t_lo, t_hi;
-            b_tile_rows(0, tile % p.n_tiles_n, t_lo, t_hi);
+            // one segment of ceil(rows / TM) row tiles: column tile = tile / row tiles
+            b_blocks(0, tile / ((p.rows_total + TM - 1) / TM), t_lo, t_hi);
             pre = min(STAGES, nk);
             for (int st = 0; st < pre; ++st) {
                 mbar_arrive_expect_tx(&s.full[st], TM * 128 + B_BYTES);
-                tma_load_2d(s.b[st], &tmap_b, 0, static_cast<int>((t_lo + kb0 + st) * 128), &s.full[st]);
-                tma_load_2d(s.b[st] + B_BYTES / 2, &tmap_b, 0, static_cast<int>((t_hi + kb0 + st) * 128),
-                            &s.full[st]);
+                load_b(s.b[st], t_lo, kb0 + st, &s.full[st]);
+                load_b(s.b[st] + B_BYTES / 2, t_hi, kb0 + st, &s.full[st]);
             }
         }
     }
@@ -306,9 +336,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 k_range(item, tile, ks, kb0, nk);
                 int seg, row0, rows_valid, nt;
                 decode_tile<TM>(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
-                // 128-row blocks of B (tile rows of the tiled weight layout)
                 long long t_lo, t_hi;
-                b_tile_rows(seg, nt, t_lo, t_hi);
+                b_blocks(seg, nt, t_lo, t_hi);
                 const bool first = item == static_cast<int>(blockIdx.x);
                 for (int kb = kb0; kb < kb0 + nk; ++kb) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, p.status)) {
@@ -324,11 +353,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         mbar_arrive_expect_tx(&s.full[stage],
                                               TM * 128 + B_BYTES + (inject ? 16 : 0));
                         tma_load_2d(s.a[stage], &tmap_a, kc, row0, &s.full[stage]);
-                        // each B box is one contiguous 16 KB weight tile
-                        tma_load_2d(s.b[stage], &tmap_b, 0, static_cast<int>((t_lo + kb) * 128),
-                                    &s.full[stage]);
-                        tma_load_2d(s.b[stage] + B_BYTES / 2, &tmap_b, 0,
-                                    static_cast<int>((t_hi + kb) * 128), &s.full[stage]);
+                        load_b(s.b[stage], t_lo, kb, &s.full[stage]);
+                        load_b(s.b[stage] + B_BYTES / 2, t_hi, kb, &s.full[stage]);
                     }
                     armed |= 1 << stage;
                     armed_phase[stage] = phase;
@@ -358,6 +384,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
             constexpr uint32_t idesc = MX ? instr_desc_mx(BM, BN) : instr_desc<FP8>(TM, BN);
+            constexpr uint32_t idesc_half = instr_desc<FP8>(TM, BN / 2);
+            const bool split = SCALED && !M64 && p.split_n;
             int stage = 0;
             uint32_t phase = 0;
             int tb = 0;
@@ -372,7 +400,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const bool chunk_first = (kb % SPC) == 0;
                     const bool chunk_last = (kb % SPC) == SPC - 1 || kb == nk - 1;
                     if (chunk_first) {
-                        if (!mbar_wait(&s.tempty[tb], tphase ^ 1, abort, p.status)) {
+                        if (!mbar_wait(&s.tempty[2 * tb], tphase ^ 1, abort, p.status)) {
                             ok = false;
                             break;
                         }
@@ -408,25 +436,50 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     // MX: this K block's scales are byte kb % 4 of each scale column
                     // (the id in the instruction descriptor and in the TMEM address)
                     const uint32_t sid = static_cast<uint32_t>(kb % SF_GROUP);
+                    if (split) {
+                        // columns 0..127 (B rows 0..127), then 128..255; each half
+                        // is one K step (SPC = 1): a fresh partial sum
+                        const uint64_t bdesc_hi = smem_desc_sw128(smem_u32(s.b[stage] + B_BYTES / 2));
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        // +32 bytes of K per instruction: +2 in the >>4 address field;
-                        // each K chunk (M64: each K step) starts a fresh partial sum
-                        const uint32_t acc = ((M64 || chunk_first) && kk == 0) ? 0u : 1u;
-                        if constexpr (MX)
-                            tc_mma_mx(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
-                                      idesc | (sid << 29) | (sid << 4),
-                                      (tmem_base + SF_COL) | (sid << 30),
-                                      (tmem_base + SF_COL + 4) | (sid << 30), acc);
-                        else
-                            tc_mma<FP8>(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc);
-                    }
-                    tc_commit(&s.empty[stage]);
-                    if (chunk_last) {
-                        tc_commit(&s.tfull[tb]);
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma<FP8>(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc_half, kk ? 1u : 0u);
+                        tc_commit(&s.tfull[2 * tb]);
+                        if (!mbar_wait(&s.tempty[2 * tb + 1], tphase ^ 1, abort, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma<FP8>(d_tmem + BN / 2, adesc + 2 * kk, bdesc_hi + 2 * kk, idesc_half,
+                                        kk ? 1u : 0u);
+                        tc_commit(&s.empty[stage]);
+                        tc_commit(&s.tfull[2 * tb + 1]);
                         if (++tb == R::NBUF) {
                             tb = 0;
                             tphase ^= 1;
+                        }
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            // +32 bytes of K per instruction: +2 in the >>4 address field;
+                            // each K chunk (M64: each K step) starts a fresh partial sum
+                            const uint32_t acc = ((M64 || chunk_first) && kk == 0) ? 0u : 1u;
+                            if constexpr (MX)
+                                tc_mma_mx(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
+                                          idesc | (sid << 29) | (sid << 4),
+                                          (tmem_base + SF_COL) | (sid << 30),
+                                          (tmem_base + SF_COL + 4) | (sid << 30), acc);
+                            else
+                                tc_mma<FP8>(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc);
+                        }
+                        tc_commit(&s.empty[stage]);
+                        if (chunk_last) {
+                            tc_commit(&s.tfull[2 * tb]);
+                            if (++tb == R::NBUF) {
+                                tb = 0;
+                                tphase ^= 1;
+                            }
                         }
                     }
                     if (++stage == STAGES) {
@@ -446,22 +499,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             }
         }
     } else if (warp == 2 || warp == 3) {
-        // ------------------------------------- scale factors (block-scaled MMA)
-        // Per group of four K blocks (in the producer's order): warp 3 copies
-        // the fp32 scales (A's 128 rows, B's two 128-row blocks, four K blocks
-        // each) from global memory into a staging ring with cp.async, SF_AHEAD
-        // groups ahead; warp 2 writes their UE8M0 bytes in the tcgen05.cp
-        // source layout (lane l holds rows l, 32+l, 64+l, 96+l of A, one 32-bit
-        // column each, byte j for K block 4g + j) and signals the MMA issuer.
-        // The split keeps global loads out of the warp that must fence its
-        // shared-memory writes for the async proxy.
-        if constexpr (MX) {
+        // ------------------------------------------------------ block scales
+        // Per group of four K blocks of each work item, in the producer's
+        // order: warp 3 copies the fp32 scales (A's rows of the tile, B's two
+        // 128-row blocks, four K blocks each) from global memory into a
+        // staging ring with cp.async, SF_AHEAD groups ahead.
+        //  - fp32 scales (software promotion): the epilogue reads them there,
+        //    so no global load sits in its per-K-block loop.
+        //  - block-scaled MMA: warp 2 writes their UE8M0 bytes in the
+        //    tcgen05.cp source layout (lane l holds rows l, 32+l, 64+l, 96+l
+        //    of A, one 32-bit column each, byte j for K block 4g + j) and
+        //    signals the MMA issuer.  The split keeps global loads out of the
+        //    warp that must fence its shared-memory writes for the async proxy.
+        if constexpr (MX || SCALED) {
             const int NB = p.b_rows / 128;
-            const int NG = (KB + SF_GROUP - 1) / SF_GROUP;  // groups per tile
-            const int my_tiles = total_tiles > static_cast<int>(blockIdx.x)
-                                     ? (total_tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
-                                     : 0;
-            const int n_groups = my_tiles * NG;
+            auto groups_of = [&](int item) {
+                int tile, ks, kb0, nk;
+                k_range(item, tile, ks, kb0, nk);
+                return (nk + SF_GROUP - 1) / SF_GROUP;
+            };
+            int n_groups = 0;  // groups of all of this block's work items
+            for (int item = blockIdx.x; item < total_items; item += gridDim.x)
+                n_groups += groups_of(item);
             bool ok = true;
             // lane 0 waits, the warp follows (bounded; false on timeout/abort)
             auto warp_wait = [&](uint64_t *bar, uint32_t parity) {
@@ -470,24 +529,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 return __shfl_sync(0xffffffffu, go, 0) != 0;
             };
             if (warp == 3) {
-                // group i: 4-byte cp.async copies into staging slot i % SF_STAGING
-                // (K blocks past the end and rows past the last: zero fill), one
-                // commit group per group (empty past the last one)
+                // group i (in order): 4-byte cp.async copies into staging slot
+                // i % SF_STAGING (K blocks past the item's range and rows past
+                // the last: zero fill), one commit group per group (empty past
+                // the last one); (cur_item, cur_g) is the next group to issue
+                int cur_item = blockIdx.x, cur_g = 0;
                 auto issue = [&](int i) {
                     if (i < n_groups) {
-                        const int tile = blockIdx.x + (i / NG) * gridDim.x;
-                        const int kb0 = (i % NG) * SF_GROUP;
+                        int tile, ks, kb0, nk;
+                        k_range(cur_item, tile, ks, kb0, nk);
+                        const int kbs = kb0 + cur_g * SF_GROUP;
+                        const int jn = min(SF_GROUP, nk - cur_g * SF_GROUP);
                         int seg, row0, rows_valid, nt;
                         decode_tile<TM>(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
                         const int slot = i % SF_STAGING;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
+                        for (int c = 0; c < TM / 32; ++c) {
                             const int r = row0 + lane + 32 * c;
 #pragma unroll
                             for (int j = 0; j < SF_GROUP; ++j) {
-                                const bool in = r < p.rows_total && kb0 + j < KB;
+                                const bool in = r < p.rows_total && j < jn;
                                 cp_async4(&s.sf_a[slot][j][lane + 32 * c],
-                                          p.a_scales + (in ? static_cast<size_t>(r) * KB + kb0 + j : 0),
+                                          p.a_scales + (in ? static_cast<size_t>(r) * KB + kbs + j : 0),
                                           in);
                             }
                         }
@@ -495,10 +558,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                             const int which = lane / SF_GROUP, j = lane % SF_GROUP;
                             const int nb = which == 0 ? (GATE_UP ? nt : 2 * nt)
                                                       : (GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1);
-                            const bool in = kb0 + j < KB;
+                            const bool in = j < jn;
                             cp_async4(&s.sf_b[slot][which][j],
-                                      p.b_scales + (in ? (static_cast<size_t>(seg) * NB + nb) * KB + kb0 + j : 0),
+                                      p.b_scales + (in ? (static_cast<size_t>(seg) * NB + nb) * KB + kbs + j : 0),
                                       in);
+                        }
+                        if (++cur_g == groups_of(cur_item)) {
+                            cur_g = 0;
+                            cur_item += gridDim.x;
                         }
                     }
                     cp_async_commit();
@@ -519,7 +586,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     if (lane == 0) mbar_arrive(&s.sf_full[i % SF_STAGING]);
                 }
                 cp_async_wait<0>();
-            } else {
+            } else if constexpr (MX) {
                 for (int i = 0; i < n_groups; ++i) {
                     const int slot = i % SF_STAGING;
                     if (!warp_wait(&s.sf_full[slot], (i / SF_STAGING) & 1)) break;
@@ -563,10 +630,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const int hh = M64 ? (lane >> 4) : 0;
         const int r_in = M64 ? q * 16 + (lane & 15) : q * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-        const int NB = p.b_rows / 128;
+        const bool split = SCALED && !M64 && p.split_n;
         int tb = 0;
         uint32_t tphase = 0;
         int iter = 0;
+        int gq = 0;  // scale groups consumed (fp32 scales)
         bool ok = true;
         for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x, ++iter) {
             int tile, ks, kb0, nk;
@@ -582,30 +650,32 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             float2 acc2[64];  // columns (2j, 2j+1) of the thread's 128
 #pragma unroll
             for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
-            const int nb_lo = GATE_UP ? nt : 2 * nt;
-            const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
-            // scale rows from the item's first K block on
-            const float *sw_lo_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_lo) * KB + kb0 : nullptr;
-            const float *sw_hi_p = SCALED ? p.b_scales + (static_cast<size_t>(seg) * NB + nb_hi) * KB + kb0 : nullptr;
-            const float *sa_p = SCALED ? p.a_scales + row * KB + kb0 : nullptr;
             // K block (counted from kb0) whose partial this thread promotes in chunk c
             auto kb_of = [&](int c) { return M64 ? 2 * c + hh : c; };
-            // scales of chunk c are loaded one chunk ahead (global latency)
-            float nsa = 0.0f, nswl = 1.0f, nswh = 1.0f;
-            if (SCALED && warp_active && kb_of(0) < nk) {
-                nsa = valid ? __ldg(sa_p + kb_of(0)) : 0.0f;
-                nswl = __ldg(sw_lo_p + kb_of(0));
-                nswh = __ldg(sw_hi_p + kb_of(0));
-            }
             for (int c = 0; c < nch; ++c) {
-                const float sc_lo = SCALED ? nsa * nswl : 1.0f, sc_hi = SCALED ? nsa * nswh : 1.0f;
                 const bool kvalid = !M64 || kb_of(c) < nk;  // M64, odd K: no partial in the upper half
-                if (SCALED && warp_active && c + 1 < nch && kb_of(c + 1) < nk) {
-                    nsa = valid ? __ldg(sa_p + kb_of(c + 1)) : 0.0f;
-                    nswl = __ldg(sw_lo_p + kb_of(c + 1));
-                    nswh = __ldg(sw_hi_p + kb_of(c + 1));
+                float sc_lo = 1.0f, sc_hi = 1.0f;
+                if constexpr (SCALED) {
+                    // this chunk's scales, staged by warp 3 in groups of four K
+                    // blocks (M64: a chunk is two K blocks of one group)
+                    const int kba = M64 ? 2 * c : c;
+                    const int slot = gq % SF_STAGING;
+                    if (kba % SF_GROUP == 0 &&
+                        !mbar_wait(&s.sf_full[slot], (gq / SF_STAGING) & 1, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const int j = kb_of(c) % SF_GROUP;
+                    const float sa = valid ? s.sf_a[slot][j][r_in] : 0.0f;
+                    sc_lo = sa * s.sf_b[slot][0][j];
+                    sc_hi = sa * s.sf_b[slot][1][j];
+                    if (kba % SF_GROUP == SF_GROUP - (M64 ? 2 : 1) || c == nch - 1) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&s.sf_empty[slot]);
+                        ++gq;
+                    }
                 }
-                if (!mbar_wait(&s.tfull[tb], tphase, abort, p.status)) {
+                if (!mbar_wait(&s.tfull[2 * tb], tphase, abort, p.status)) {
                     ok = false;
                     break;
                 }
@@ -615,6 +685,44 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 // (before its FMAs), since the MMA two chunks ahead waits for it
                 float va[32], vb[32];
                 const bool add = warp_active && kvalid;  // the loads below are warp-wide
+                if (split) {
+                    // each half is released as soon as its pieces are in registers
+                    const uint32_t base = lane_base + tb * BN;
+                    if (warp_active) {
+                        tmem_ld32(base + col_lo, va);
+                        tmem_ld32(base + col_lo + 32, vb);
+                        tmem_wait_ld(va, vb);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.tempty[2 * tb]);
+                    if (add) {
+                        promote32<SCALED>(acc2, 0, va, sc_lo);
+                        promote32<SCALED>(acc2, 16, vb, sc_lo);
+                    }
+                    if (!mbar_wait(&s.tfull[2 * tb + 1], tphase, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (warp_active) {
+                        tmem_ld32(base + col_hi, va);
+                        tmem_ld32(base + col_hi + 32, vb);
+                        tmem_wait_ld(va, vb);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.tempty[2 * tb + 1]);
+                    if (add) {
+                        promote32<SCALED>(acc2, 32, va, sc_hi);
+                        promote32<SCALED>(acc2, 48, vb, sc_hi);
+                    }
+                    if (++tb == R::NBUF) {
+                        tb = 0;
+                        tphase ^= 1;
+                    }
+                    continue;
+                }
                 if (warp_active) {
                     const uint32_t base = lane_base + tb * BN;
                     tmem_ld32(base + col_lo, va);
@@ -628,7 +736,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s.tempty[tb]);
+                if (lane == 0) mbar_arrive(&s.tempty[2 * tb]);
                 if (add) {
                     promote32<SCALED>(acc2, 32, va, sc_hi);
                     promote32<SCALED>(acc2, 48, vb, sc_hi);
@@ -842,11 +950,18 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     if (!m64 && g.tile_m != 128) return cudaErrorInvalidValue;
     if (!make_map_2d(&ma, g.a, g.fp8, g.K, g.rows_total, m64 ? 64 : 128))
         return cudaErrorInvalidValue;
-    // B in the tiled layout: one row of 128 bytes per tile row, tiles stacked
-    const long long b_tile_rows = static_cast<long long>(g.n_slots) * b_rows * (g.K * (g.fp8 ? 1 : 2) / 128);
-    if (b_tile_rows >= (1LL << 31)) return cudaErrorInvalidValue;
-    if (!make_map_2d(&mb, g.b, g.fp8, g.fp8 ? 128 : 64, static_cast<int>(b_tile_rows)))
-        return cudaErrorInvalidValue;
+    if (g.b_rowmajor) {
+        // B row-major [n_slots * b_rows, K], the same map shape as A
+        const long long rows = static_cast<long long>(g.n_slots) * b_rows;
+        if (rows >= (1LL << 31)) return cudaErrorInvalidValue;
+        if (!make_map_2d(&mb, g.b, g.fp8, g.K, static_cast<int>(rows))) return cudaErrorInvalidValue;
+    } else {
+        // B in the tiled layout: one row of 128 bytes per tile row, tiles stacked
+        const long long b_tile_rows = static_cast<long long>(g.n_slots) * b_rows * (g.K * (g.fp8 ? 1 : 2) / 128);
+        if (b_tile_rows >= (1LL << 31)) return cudaErrorInvalidValue;
+        if (!make_map_2d(&mb, g.b, g.fp8, g.fp8 ? 128 : 64, static_cast<int>(b_tile_rows)))
+            return cudaErrorInvalidValue;
+    }
     KParams kp;
     kp.a_scales = g.a_scales;
     kp.b_scales = g.b_scales;
@@ -864,6 +979,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     kp.inject_fault = g.inject_fault;
     kp.ue8m0 = g.ue8m0 ? 1 : 0;
     kp.rows_total = g.rows_total;
+    kp.b_rowmajor = g.b_rowmajor ? 1 : 0;
+    kp.split_n = g.split_n ? 1 : 0;
     // block-scaled MMA (UE8M0 scales): all of K accumulates in TMEM
     kp.mx_spc = g.K / 128;
     const bool mx = g.fp8 && g.ue8m0;

@@ -115,7 +115,9 @@ struct GemmArgs {
     bool gate_up;
     const void *a;          // [rows_total, K]
     const float *a_scales;  // [rows_total, K/128] (fp8)
-    const void *b;          // [n_slots, B rows, K] in 128 x 128-byte tiles
+    const void *b;          // [n_slots, B rows, K]: 128 x 128-byte tiles, or row-major
+    bool b_rowmajor;        // b (and its layout) row-major instead of tiled
+    bool split_n;           // fp32 scales, 128-row tiles: two N = 128 MMAs per K step
     const float *b_scales;  // [n_slots, B rows/128, K/128] (fp8)
     void *out;              // H or Y
     float *out_scales;      // H scales (fp8 gate_up)
@@ -170,6 +172,7 @@ inline void mark_used_on_device(std::atomic<uint64_t> &done) {
 int record_error(int code, const char *msg);  // sets moe_last_error, returns code
 void record_launches(int n);                   // sets moe_last_launch_count
 int validate_shape(const moe_shape *s);        // host-side shape checks
+int validate_device();                         // MOE_ERR_UNSUPPORTED unless the device is sm_100
 
 // Called just before the call's kernel launch number `index` with that
 // kernel's name (and once more after the last launch, without a name):

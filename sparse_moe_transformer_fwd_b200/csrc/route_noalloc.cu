@@ -19,22 +19,48 @@ static __device__ __align__(256) float g_noalloc_scores[MOE_ROUTE_NOALLOC_MAX_SC
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 float *g_addr[kMaxDevices] = {};
+void *g_ctx[kMaxDevices] = {};  // the context g_addr[dev] was looked up in
 
 thread_local char g_msg[256];
 
-// Device address of the scratch on the current device, looked up once per
-// device (in host code the symbol is only a host-side stand-in).
+// The calling thread's current CUDA context (driver API, fetched through the
+// runtime so the library needs no link-time driver dependency), or NULL.
+void *current_context() {
+    using GetCurrentFn = int (*)(void **);
+    static GetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<GetCurrentFn>(p);
+    });
+    void *ctx = nullptr;
+    if (!fn || fn(&ctx) != 0) return nullptr;
+    return ctx;
+}
+
+// Device address of the scratch on the current device.  In host code the
+// symbol is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress, once per device and context: a device whose primary
+// context was destroyed (cudaDeviceReset) and created again loads the
+// library's module anew, possibly at another address, so a change of context
+// repeats the lookup.
 cudaError_t scratch_address(float **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    void *ctx = current_context();
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev]) {
+    if (!g_addr[dev] || !ctx || ctx != g_ctx[dev]) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scores);
         if (e != cudaSuccess) return e;
         g_addr[dev] = static_cast<float *>(p);
+        // the lookup made the device's primary context current if none was
+        g_ctx[dev] = current_context();
     }
     *out = g_addr[dev];
     return cudaSuccess;
@@ -70,6 +96,9 @@ extern "C" int moe_route_noalloc(const moe_shape *s, const uint16_t *x, const ui
             return record_error(MOE_ERR_INVALID_ARG, g_msg);
         }
     }
+    // the same device check (and error code) as moe_route
+    const int dc = validate_device();
+    if (dc != MOE_OK) return dc;
     float *scores = nullptr;
     cudaError_t e = scratch_address(&scores);
     if (e != cudaSuccess) {

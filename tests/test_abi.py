@@ -120,3 +120,47 @@ def test_dense_workspace_and_host_errors():
     e = _dense(T=0)
     assert call(e, moe.moe_dense_workspace_size(e)) == N.MOE_OK
     assert moe.moe_last_launch_count() == 0
+
+
+def test_weight_layout_is_declared_and_checked():
+    """The shape declares the weights' layout: row-major (0, the value of a
+    zero-initialised shape) or tiled (1); any other value is rejected on the
+    host before anything is enqueued, for the MoE and the dense layer."""
+    assert N.MOE_LAYOUT_ROWMAJOR == 0 and N.MOE_LAYOUT_TILED == 1
+    assert moe.make_shape(64, 7168, 256, 8, 2048).weight_layout == N.MOE_LAYOUT_TILED
+    zero = N.MoeShape()
+    assert zero.weight_layout == N.MOE_LAYOUT_ROWMAJOR
+    for lay in (N.MOE_LAYOUT_ROWMAJOR, N.MOE_LAYOUT_TILED):
+        assert moe.moe_workspace_size(_shape(weight_layout=lay)) > 0
+        assert moe.moe_dense_workspace_size(_dense(weight_layout=lay)) > 0
+    for bad in (2, -1, 7):
+        s = _shape(weight_layout=bad)
+        assert moe.lib().moe_workspace_size(ctypes.byref(s)) == 0
+        assert "weight_layout" in moe.moe_last_error()
+        assert _call_forward(s, 1 << 30) == N.MOE_ERR_INVALID_ARG
+        assert moe.lib().moe_dense_workspace_size(ctypes.byref(_dense(weight_layout=bad))) == 0
+
+
+def test_workspace_layout_regions():
+    """moe_workspace_layout: every region starts on a 256-byte boundary,
+    regions follow one another without overlap in the order listed, sized
+    for the shape, and the total is moe_workspace_size."""
+    for kw in (dict(), dict(precision="bf16"), dict(T=16384), dict(T=1, n_experts=16, top_k=4,
+                                                                    d_model=512, d_expert=256)):
+        s = _shape(**kw)
+        o = moe.moe_workspace_layout(s)
+        assert o["total"] == moe.moe_workspace_size(s)
+        T, E, k, d, de = s.T, s.n_experts, s.top_k, s.d_model, s.d_expert
+        Rs = T * (k + s.n_shared)
+        es = 2 if s.precision == N.MOE_BF16 else 1
+        need = {"scores": T * E * 4, "topk_idx": T * k * 4, "topk_w": T * k * 4,
+                "counts": E * 4, "offsets": (E + 1) * 4, "row_token": T * k * 4,
+                "row_of": T * k * 4, "a": Rs * d * es, "h": Rs * de * es, "y": Rs * d * 2}
+        if es == 1:
+            need.update(a_scales=Rs * (d // 128) * 4, h_scales=Rs * (de // 128) * 4)
+        names = sorted(need, key=lambda n: o[n])
+        for a, b in zip(names, names[1:]):
+            assert o[a] % 256 == 0 and o[a] + need[a] <= o[b], (a, b)
+        assert o[names[-1]] + need[names[-1]] <= o["total"]
+    with pytest.raises(moe.MoeError):
+        moe.moe_workspace_layout(_shape(d_model=100))

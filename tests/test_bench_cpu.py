@@ -20,12 +20,50 @@ PEAKS = {"hbm_gbs": 6545.3, "bf16_tflops": 1667.2, "bf16_tflops_sustained": 1396
 
 
 def test_gate_up_algorithmic_bytes_match_measured_dram():
-    """Decode: 155 routed experts were touched plus the shared one; ncu read
-    the gate/up GEMM's weights once, so the two counts agree within 0.5 %."""
+    """Decode: 154 routed experts were touched (102 of 256 got no token) plus
+    the shared one; ncu read the gate/up GEMM's weights once, so the two
+    counts agree within 0.5 %.  155 touched experts give the bench's
+    4,557,405,184 algorithmic bytes exactly."""
     rec = json.load(open(RECORD))
     measured = rec["workloads"]["decode"]["grouped_gemm_gate_up"]["traffic_bytes_per_launch"]
-    alg = bench.algorithmic_bytes_gemm1(CONFIGS["decode"], touched=156)
+    alg = bench.algorithmic_bytes_gemm1(CONFIGS["decode"], touched=155)
+    assert alg == 4557405184
     assert abs(alg - measured) / measured < 0.005
+
+
+def test_moe_roofline_bound_follows_the_longer_floor():
+    """The MoE arm's bound is the roof with the longer floor at the measured
+    peaks: HBM for decode and prefill (weights dominate), tensor for the
+    skewed T=16384 batch (8.66 TFLOP of gate/up against ~8.9 GB) and for the
+    bf16 T=8192 batch; frac = achieved / peak, recomputable from the line."""
+    dec = bench.moe_roofline(CONFIGS["decode"], 155, 0.6664, PEAKS, "measured")
+    assert dec["bound"] == "hbm" and dec["unit"] == "GB/s"
+    assert dec["achieved"] == pytest.approx(4557405184 / 0.6664e-3 / 1e9, rel=1e-4)
+    pre = bench.moe_roofline(CONFIGS["prefill"], 257, 2.15, PEAKS, "measured")
+    assert pre["bound"] == "hbm"
+    skew = bench.moe_roofline(CONFIGS["skew"], 257, 6.37, PEAKS, "measured")
+    assert skew["bound"] == "tensor" and skew["unit"] == "TFLOP/s"
+    flops = 2.0 * 16384 * 9 * 4096 * 7168
+    assert skew["algorithmic_flops"] == flops
+    assert skew["peak"] == pytest.approx(2 * PEAKS["bf16_tflops"])
+    assert skew["achieved"] == pytest.approx(flops / 6.37e-3 / 1e12, rel=1e-4)
+    assert skew["frac"] == pytest.approx(skew["achieved"] / skew["peak"], rel=1e-3)
+    b16 = bench.moe_roofline(CONFIGS["bf16"], 257, 5.6, PEAKS, "measured")
+    assert b16["bound"] == "tensor" and b16["peak"] == pytest.approx(PEAKS["bf16_tflops"])
+
+
+def test_layer_floor():
+    """Whole-layer floor: the longer of (touched experts' three matrices and
+    scales + x in + out) / HBM and (both GEMMs' FLOPs) / tensor peak."""
+    c = CONFIGS["skew"]
+    f = bench.layer_floor(c, 257, 12.3, PEAKS)
+    w = 257 * (3 * 2048 * 7168 + 4 * (32 * 56 + 56 * 16))
+    t_hbm = (w + 16384 * 7168 * 4) / (PEAKS["hbm_gbs"] * 1e9) * 1e3
+    t_tc = 2.0 * 16384 * 9 * 3 * 2048 * 7168 / (2 * PEAKS["bf16_tflops"] * 1e12) * 1e3
+    assert f["bound"] == "tensor"
+    assert f["floor_ms"] == pytest.approx(max(t_hbm, t_tc), abs=1e-4)
+    assert f["frac"] == pytest.approx(max(t_hbm, t_tc) / 12.3, abs=1e-4)
+    assert bench.layer_floor(CONFIGS["decode"], 155, 1.05, PEAKS)["bound"] == "hbm"
 
 
 def test_dense_roofline_bounds_and_bytes():

@@ -352,6 +352,40 @@ def test_forward_all_tokens_on_few_experts(precision):
     assert_out_close(out, ref["out"], "few experts", ref["out_allow"])
 
 
+@pytest.mark.parametrize("precision", ["bf16", "fp8", "fp8_ue8m0"])
+@pytest.mark.parametrize("T", [200, 40])
+def test_rowmajor_weights_match_tiled(precision, T):
+    """Expert weights in the problem statement's row-major layout, declared so
+    in the shape (weight_layout MOE_LAYOUT_ROWMAJOR), give the tiled layer's
+    routing and output bit for bit: the codes and the arithmetic are the
+    same, only the coordinates of the weights' TMA boxes differ.  T=40 runs
+    64-row tiles (fp32 scales), T=200 128-row tiles.  The same for the dense
+    layer (split-K down GEMM at T=40)."""
+    cfg = CONFIGS["tiny"].with_(precision=precision, T=T)
+    d = _dev(make_inputs(cfg, seed=5))
+    kw = dict(top_k=cfg.top_k, n_shared=cfg.n_shared, precision=precision)
+    lt = moe.MoELayer(d["w_router"], d["bias"], d["w13"], d["w2"], weight_layout="tiled", **kw)
+    lr = moe.MoELayer(d["w_router"], d["bias"], d["w13"], d["w2"], weight_layout="rowmajor", **kw)
+    assert lr.shape(T).weight_layout == moe.MOE_LAYOUT_ROWMAJOR
+    it = torch.empty(T, cfg.top_k, dtype=torch.int32, device=DEV)
+    ir = torch.empty_like(it)
+    ot, orr = lt(d["x"], topk_idx_out=it), lr(d["x"], topk_idx_out=ir)
+    assert lt.check_status(T) == 0 and lr.check_status(T) == 0, moe.moe_last_error()
+    assert torch.equal(it, ir)
+    assert torch.equal(ot.view(torch.int16), orr.view(torch.int16))
+    if precision != "bf16":
+        n13, dm = lr.w13.shape[1:]
+        assert np.array_equal(untile(lt.w13[3].cpu().numpy(), n13, dm), lr.w13[3].cpu().numpy())
+    from moe_inputs import DENSE_CONFIGS, make_dense_inputs
+    dc = DENSE_CONFIGS["dense_tiny"].with_(T=T, precision=precision)
+    di = {k: v.to(DEV) for k, v in make_dense_inputs(dc, seed=5).items()}
+    dt = moe.DenseFFN(di["w13"], di["w2"], precision=precision, weight_layout="tiled")
+    dr = moe.DenseFFN(di["w13"], di["w2"], precision=precision, weight_layout="rowmajor")
+    a, b = dt(di["x"]), dr(di["x"])
+    assert dt.check_status(T) == 0 and dr.check_status(T) == 0, moe.moe_last_error()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 def test_forward_empty_batch():
     cfg = CONFIGS["tiny"]
     inp = _dev(make_inputs(cfg, seed=1))

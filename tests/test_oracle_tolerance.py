@@ -129,8 +129,8 @@ def test_nearest_correct_output_takes_only_explaining_alternatives():
     flipped = res["out_f64"].copy()
     flipped[r] += v
     got = as_bf16(flipped)
-    want, taken = nearest_correct_output(got, res["out_f64"], res["out_alts"])
-    assert taken >= 1
+    want, taken, cands = nearest_correct_output(got, res["out_f64"], res["out_alts"])
+    assert taken >= 1 and cands >= taken
     rel_plain = out_error(got, res["out"])[0]
     rel_near = out_error(got, want)[0]
     assert rel_near < rel_plain / 4
@@ -138,7 +138,7 @@ def test_nearest_correct_output_takes_only_explaining_alternatives():
     bad = res["out_f64"].copy()
     bad[r] += np.roll(v, 17)
     got_bad = as_bf16(bad)
-    want_bad, _ = nearest_correct_output(got_bad, res["out_f64"], res["out_alts"])
+    want_bad, _, _ = nearest_correct_output(got_bad, res["out_f64"], res["out_alts"])
     assert out_error(got_bad, want_bad)[0] > 0.5 * out_error(got_bad, res["out"])[0]
 
 
@@ -153,8 +153,8 @@ def test_nearest_correct_output_without_alternatives_is_the_oracles():
     res = oracle.dense_ffn(u(inp["x"]), u(inp["w13"]), u(inp["w2"]), precision="bf16")
     assert all(len(a) == 0 for a in res["out_alts"])
     got = torch.from_numpy(res["out"].view(np.int16)).view(torch.bfloat16)
-    want, taken = nearest_correct_output(got, res["out_f64"], res["out_alts"])
-    assert taken == 0 and np.array_equal(want, res["out"])
+    want, taken, cands = nearest_correct_output(got, res["out_f64"], res["out_alts"])
+    assert taken == 0 and cands == 0 and np.array_equal(want, res["out"])
 
 
 def test_ue8m0_alternatives_are_adjacent_codes_within_the_bound():

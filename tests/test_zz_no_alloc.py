@@ -40,7 +40,9 @@ def _route_both(cfg, seed):
     return (idx_ref.cpu(), g_ref.cpu()), outs
 
 
-@pytest.mark.parametrize("name,T", [("decode", 64), ("tiny", 128), ("decode", 4096)])
+# T=64: the small-batch router; T=600: 32-token tiles; T=4096: 64-token tiles
+@pytest.mark.parametrize("name,T", [("decode", 64), ("tiny", 128), ("decode", 600),
+                                    ("decode", 4096)])
 def test_noalloc_route_matches_moe_route(name, T):
     cfg = CONFIGS[name].with_(T=T)
     (idx_ref, g_ref), outs = _route_both(cfg, seed=5)
@@ -58,3 +60,72 @@ def test_noalloc_route_rejects_oversize():
                               t.float(), t, t.float())
     assert ei.value.code == moe._native.MOE_ERR_INVALID_ARG
     assert "exceeds" in moe.moe_last_error()
+
+
+_RESET_CHILD = r"""
+import ctypes, sys
+import numpy as np
+sys.path.insert(0, sys.argv[1])
+import sparse_moe_transformer_fwd_b200 as moe
+rt = ctypes.CDLL(sys.argv[2])
+vp, sz = ctypes.c_void_p, ctypes.c_size_t
+rt.cudaMalloc.argtypes = [ctypes.POINTER(vp), sz]
+rt.cudaMemcpy.argtypes = [vp, vp, sz, ctypes.c_int]
+rt.cudaFree.argtypes = [vp]
+T, d, E, k = 600, 7168, 256, 8
+rng = np.random.default_rng(7)
+bf = lambda a: (a.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+x = bf(rng.standard_normal((T, d)))
+w = bf(rng.standard_normal((E, d)) * 0.006)
+b = (rng.random(E) * 0.2 - 0.1).astype(np.float32)
+shape = moe.make_shape(T, d, E, k, 2048)
+L = moe.lib()
+
+def dev(a):
+    p = vp()
+    assert rt.cudaMalloc(ctypes.byref(p), a.nbytes) == 0
+    assert rt.cudaMemcpy(p, a.ctypes.data, a.nbytes, 1) == 0
+    return p
+
+def route(noalloc):
+    xp, wp, bp = dev(x), dev(w), dev(b)
+    idx, g = np.zeros((T, k), np.int32), np.zeros((T, k), np.float32)
+    ip, gp = dev(idx), dev(g)
+    if noalloc:
+        rc = L.moe_route_noalloc(ctypes.byref(shape), xp, wp, bp, ip, gp, None)
+    else:
+        n = L.moe_workspace_size(ctypes.byref(shape))
+        ws = dev(np.zeros(n, np.uint8))
+        rc = L.moe_route(ctypes.byref(shape), xp, wp, bp, ip, gp, ws, n, None)
+    assert rc == 0, L.moe_last_error()
+    assert rt.cudaMemcpy(idx.ctypes.data, ip, idx.nbytes, 2) == 0
+    assert rt.cudaMemcpy(g.ctypes.data, gp, g.nbytes, 2) == 0
+    for p in (xp, wp, bp, ip, gp):
+        rt.cudaFree(p)
+    return idx, g
+
+ref = route(False)
+first = route(True)
+assert rt.cudaDeviceReset() == 0          # ends this process's context only
+after = route(True)                       # a new context: the scratch is looked up again
+for got in (first, after):
+    assert np.array_equal(got[0], ref[0])
+    assert np.array_equal(got[1].view(np.uint32), ref[1].view(np.uint32))
+print("reset ok")
+"""
+
+
+def test_noalloc_route_after_device_reset():
+    """A process that resets its device (cudaDeviceReset) and routes again gets
+    the same bits as moe_route: the library looks the scratch address up again
+    in the new context.  Run in a child process, which owns the only context
+    it resets; buffers come from the CUDA runtime directly."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cudart = next(p for p in ("/usr/local/cuda/lib64/libcudart.so.12",
+                              "/usr/local/cuda/lib64/libcudart.so") if os.path.exists(p))
+    r = subprocess.run([sys.executable, "-c", _RESET_CHILD, root, cudart], capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0 and "reset ok" in r.stdout, r.stdout + r.stderr
