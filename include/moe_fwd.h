@@ -232,6 +232,19 @@ int moe_grouped_swiglu(const moe_shape *shape, const void *a, const float *a_sca
                        const void *w2, const float *w2_scales, uint16_t *y,
                        void *ws, size_t ws_bytes, void *stream);
 
+/* Quantise-and-scatter, the step between moe_permute and the grouped GEMMs
+ * ("DeepSeek-R1", "Quantization": blockwise FP8 with 1x128 activation
+ * tiles): row row_of[t, j] of `a` receives token t's codes for its j-th
+ * expert, and row T*k + t the shared expert's copy (n_shared = 1); in the
+ * fp8 precisions each row is x[t] quantised 1x128 (scale amax/448, or the
+ * power-of-two scale in MOE_FP8_UE8M0), in MOE_BF16 it is x[t] itself.
+ *   x        bf16 [T, d_model]; row_of int32 [T, top_k] (from moe_permute)
+ *   a        [R_s, d_model] e4m3 codes (fp8 precisions) or bf16 out
+ *   a_scales fp32 [R_s, d_model/128] out (fp8 precisions; NULL in MOE_BF16)
+ * R_s = T*(top_k + n_shared).  The same kernel moe_forward runs. */
+int moe_quant_scatter(const moe_shape *shape, const uint16_t *x, const int32_t *row_of, void *a,
+                      float *a_scales, void *stream);
+
 /* Weighted un-permute plus the always-on shared expert ("Structural change":
  * an always-activated expert): out[t] = bf16( sum_j topk_w[t,j] *
  * y[row_of[t,j]] + y[T*k + t] ), binary32 accumulation in rank order (the
@@ -316,6 +329,85 @@ int moe_dense_ffn_prenorm(const moe_dense_shape *shape, const uint16_t *h,
                           const uint16_t *gamma, float eps, const void *w13,
                           const float *w13_scales, const void *w2, const float *w2_scales,
                           uint16_t *out, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Expert parallelism ("DeepSeek v3 and R1 Model Architecture", "Local
+ * Balanced Routing to Experts": routed experts are spread over devices,
+ * tokens travel to the devices that hold their experts, and the routing
+ * keeps the load of devices and of communication balanced).
+ * G ranks; rank r owns routed experts r*P .. r*P + P - 1 (P = n_experts / G);
+ * every rank holds the shared expert.  One layer call:
+ *  1. every rank, on its own tokens: moe_route, moe_permute,
+ *     moe_quant_scatter.  Its routed rows are in global expert order, so its
+ *     rows for owner o form one contiguous block;
+ *  2. the ranks exchange their per-expert counts and derive the exchange
+ *     plan (which block goes where; the segments of each owner's receive
+ *     buffer; where results return);
+ *  3. every rank (a source): moe_ep_dispatch copies its block for each owner
+ *     into that owner's receive buffer;
+ *  4. every rank (an owner): moe_ep_grouped_swiglu over its received rows,
+ *     one segment per (source, local expert); the down GEMM's epilogue
+ *     stores each Y row straight into its source's Y buffer, at the row's
+ *     place in the source's permuted order;
+ *  5. every rank: moe_ep_grouped_swiglu over its own shared rows (one
+ *     segment, the shared expert's weights, returning into its own Y
+ *     buffer), then moe_combine.
+ * Destination pointers may be other GPUs' memory (peer mappings) or, for
+ * ranks emulated on one GPU, buffers of this one; the kernels only load this
+ * GPU's memory (no TMA multicast) and store with plain stores. */
+#define MOE_EP_MAX_RANKS 64
+
+/* One contiguous block of a source's rows for one owner. */
+typedef struct moe_ep_block {
+    int src_row;  /* first row in the source's permuted buffer `a` */
+    int rows;     /* rows in the block (0: nothing to send) */
+    int dst;      /* owner rank (index into recv_a / recv_scales) */
+    int dst_row;  /* first row in the owner's receive buffer */
+} moe_ep_block;
+
+/* Dispatch (step 3): copies each block's rows of `a` (and their fp32 block
+ * scales in the fp8 precisions) into recv_a[dst] / recv_scales[dst].
+ *   a          [a_rows, d_model] e4m3 or bf16 (from moe_quant_scatter)
+ *   a_scales   fp32 [a_rows, d_model/128] (fp8 precisions) or NULL
+ *   blocks     host array of n_blocks (0..MOE_EP_MAX_RANKS) blocks
+ *   recv_a, recv_scales, recv_capacity  host arrays of `world` entries:
+ *              device pointers of each owner's receive buffer ([capacity,
+ *              d_model] codes, [capacity, d_model/128] scales) and its rows
+ * Every block is checked on the host against a_rows and the destination's
+ * capacity (MOE_ERR_INVALID_ARG otherwise, nothing enqueued).  Blocks must
+ * not overlap in a destination.  Reads only shape->d_model and precision. */
+int moe_ep_dispatch(const moe_shape *shape, const void *a, const float *a_scales, int a_rows,
+                    int n_blocks, const moe_ep_block *blocks, int world, void *const *recv_a,
+                    float *const *recv_scales, const int *recv_capacity, void *stream);
+
+/* Bytes of workspace moe_ep_grouped_swiglu needs for `rows` received rows in
+ * n_segments (1..1024) segments (0 if invalid): the status word first, the
+ * checked segment table, H and its scales. */
+size_t moe_ep_workspace_size(const moe_shape *shape, int rows, int n_segments);
+
+/* The owner's grouped gated MLP over received rows (step 4), or a rank's
+ * shared expert over its own shared rows (step 5): for segment i (rows
+ * seg_start[i] .. + seg_rows[i] of `a`, weight slot seg_slot[i], or i when
+ * seg_slot is NULL)  H = silu(A W_gate^T) * (A W_up^T),  Y = H W_down^T,
+ * numerics as moe_grouped_swiglu (H requantised 1x128 in the fp8
+ * precisions).  Row j of segment i is stored in ret_y[seg_src[i]] at row
+ * seg_ret[i] + (j - seg_start[i]) (bf16 [.., d_model]).
+ *   a, a_scales     [rows, d_model] received rows (e4m3 + fp32 scales, or bf16)
+ *   seg_*           int32 device arrays [n_segments]
+ *   w13, w2, scales n_slots weight slots laid out as for moe_grouped_swiglu
+ *                   (gate rows then up rows), in the shape's weight_layout
+ *   ret_y, ret_capacity  host arrays of `world` entries: each source's Y
+ *                   buffer (device pointer) and its rows
+ * Segments that reach outside `a`, name a slot or source that does not
+ * exist, or would store past a source's capacity are recorded in the
+ * status word (MOE_ERR_DEVICE_INDEX, read with moe_check_status) and
+ * skipped.  Reads shape->d_model, d_expert, precision and weight_layout. */
+int moe_ep_grouped_swiglu(const moe_shape *shape, int rows, const void *a, const float *a_scales,
+                          int n_segments, const int32_t *seg_start, const int32_t *seg_rows,
+                          const int32_t *seg_slot, const int32_t *seg_src, const int32_t *seg_ret,
+                          int n_slots, const void *w13, const float *w13_scales, const void *w2,
+                          const float *w2_scales, int world, uint16_t *const *ret_y,
+                          const int *ret_capacity, void *ws, size_t ws_bytes, void *stream);
 
 /* Synchronises `stream`, returns the workspace status word (MOE_OK or the
  * first device-recorded MOE_ERR_*), and resets it to MOE_OK.  A workspace must

@@ -52,7 +52,7 @@ __all__ = [
     "lib", "bf16_to_f32", "bf16_from_f32", "e4m3_decode_table", "e4m3_encode", "sigmoid",
     "router_logits", "route", "permute", "block_quant", "dequant", "expert_forward",
     "moe_layer", "exp_cw", "rmsnorm", "moe_layer_prenorm", "dense_ffn", "dense_ffn_prenorm",
-    "h_code_ambiguity", "h_code_alternatives",
+    "h_code_ambiguity", "h_code_alternatives", "h_bf16_ambiguity", "h_bf16_alternatives",
 ]
 
 _LIB = None
@@ -267,6 +267,36 @@ def _bf16_of_f64(v) -> np.ndarray:
 H_FLIP_RHO = 2.0 ** -14
 
 
+def h_bf16_ambiguity(Hf, rho: float = H_FLIP_RHO) -> np.ndarray:
+    """[n, de] binary64: per element of H in the bf16 precision (Hf: its
+    binary64 value before the rounding to bf16), the largest change of its
+    bf16 value that a relative perturbation of at most rho could cause: 0
+    unless Hf lies within rho of a bf16 rounding boundary, else the gap to
+    the bf16 neighbour across that boundary.  Two correct evaluations of G
+    and U (accumulated in different orders) may round such an element either
+    way, as with the e4m3 codes of the fp8 precisions."""
+    Hf = np.asarray(Hf, dtype=np.float64)
+    base = bf16_to_f32(_bf16_of_f64(Hf)).astype(np.float64)
+    delta = np.zeros_like(base)
+    for f in (1.0 + rho, 1.0 - rho):
+        alt = bf16_to_f32(_bf16_of_f64(Hf * f)).astype(np.float64)
+        delta = np.maximum(delta, np.abs(alt - base))
+    return delta
+
+
+def h_bf16_alternatives(Hf, rho: float = H_FLIP_RHO) -> np.ndarray:
+    """[n, de] binary64, signed: for each element of bf16 H within rho of a
+    bf16 rounding boundary, the change of its value if it rounded to the
+    neighbour across that boundary; 0 elsewhere."""
+    Hf = np.asarray(Hf, dtype=np.float64)
+    base = bf16_to_f32(_bf16_of_f64(Hf)).astype(np.float64)
+    alt = np.zeros_like(base)
+    for f in (1.0 + rho, 1.0 - rho):
+        d = bf16_to_f32(_bf16_of_f64(Hf * f)).astype(np.float64) - base
+        alt = np.where(alt == 0, d, alt)
+    return alt
+
+
 def _ue8m0_exponent(amax):
     m, e = np.frexp(np.asarray(amax, dtype=np.float64))
     return np.maximum(np.where(m > 0.875, e - 8, e - 9), -127)
@@ -348,8 +378,8 @@ def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=No
     fp8_ue8m0: as fp8, every scale a power of two; H is requantised the same way.
     -> Y as bf16 bits [n, d] (and H: bf16 bits, or (codes, scales) for fp8;
     return_allow: and [n, d] binary64, how far alternative H codes at e4m3
-    rounding boundaries could move Y: sum_i h_code_ambiguity_i * |W2[:, i]|;
-    zero for bf16; return_f64: (Y in binary64, before its rounding, and that
+    rounding boundaries (bf16: alternative bf16 roundings, h_bf16_ambiguity)
+    could move Y: sum_i ambiguity_i * |W2[:, i]|; return_f64: (Y in binary64, before its rounding, and that
     allowance), with return_alts also, per row, the [m, d] changes of Y that
     the row's alternative H codes (h_code_alternatives) would make, one row
     per alternative)."""
@@ -361,15 +391,22 @@ def expert_forward(a_rows, w13, w2, precision: str, a_scales=None, w13_scales=No
         de = W13.shape[0] // 2
         G = A @ W13[:de].T
         U = A @ W13[de:].T
-        H = _bf16_of_f64(_silu_mul(G, U))
+        Hf = _silu_mul(G, U)
+        H = _bf16_of_f64(Hf)
         Y = bf16_to_f32(H).astype(np.float64) @ W2.T
         if return_f64:
+            allow = h_bf16_ambiguity(Hf) @ np.abs(W2).T
             if return_alts:
-                return Y, np.zeros(Y.shape), [np.zeros((0, Y.shape[1]))] * n
-            return Y, np.zeros(Y.shape)
+                dh = h_bf16_alternatives(Hf)
+                alts = []
+                for r in range(n):
+                    cols = np.nonzero(dh[r])[0]
+                    alts.append(dh[r, cols][:, None] * W2[:, cols].T)
+                return Y, allow, alts
+            return Y, allow
         y = _bf16_of_f64(Y)
         if return_allow:
-            return y, np.zeros(Y.shape)
+            return y, h_bf16_ambiguity(Hf) @ np.abs(W2).T
         return (y, H) if return_h else y
     if precision in ("fp8", "fp8_ue8m0"):
         A = dequant(a_rows, a_scales, 1)

@@ -20,7 +20,9 @@ from ._native import (EXPORTS, MOE_BF16, MOE_FP8_BLOCK, MOE_FP8_UE8M0, MOE_LAYOU
                       moe_permute, moe_route, moe_route_noalloc, moe_set_kernel_events,
                       moe_workspace_size, MOE_ROUTE_NOALLOC_MAX_SCORES, MoeDenseShape,
                       make_dense_shape, moe_dense_workspace_size, alloc_dense_workspace,
-                      moe_dense_ffn, moe_dense_ffn_prenorm, moe_workspace_layout)
+                      moe_dense_ffn, moe_dense_ffn_prenorm, moe_workspace_layout,
+                      moe_quant_scatter, moe_ep_dispatch, moe_ep_workspace_size,
+                      moe_ep_grouped_swiglu, MOE_EP_MAX_RANKS)
 
 __all__ = [
     "MoELayer", "MoeError", "MoeShape", "make_shape", "alloc_workspace", "lib", "EXPORTS",
@@ -31,6 +33,8 @@ __all__ = [
     "MOE_LAYOUT_ROWMAJOR", "MOE_LAYOUT_TILED", "moe_forward_prenorm", "moe_last_launch_names",
     "DenseFFN", "MoeDenseShape", "make_dense_shape", "moe_dense_workspace_size",
     "alloc_dense_workspace", "moe_dense_ffn", "moe_dense_ffn_prenorm", "moe_workspace_layout",
+    "moe_quant_scatter", "moe_ep_dispatch", "moe_ep_workspace_size", "moe_ep_grouped_swiglu",
+    "MOE_EP_MAX_RANKS",
 ]
 
 

@@ -31,7 +31,10 @@ EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "fp8_block_quant",
            "moe_last_error", "moe_last_launch_count", "moe_set_kernel_events",
            "moe_route_noalloc", "moe_pack_tiles", "moe_forward_prenorm", "moe_last_launch_name",
            "fp8_block_quant_ue8m0", "moe_dense_workspace_size", "moe_dense_ffn",
-           "moe_dense_ffn_prenorm", "moe_workspace_layout")
+           "moe_dense_ffn_prenorm", "moe_workspace_layout", "moe_quant_scatter",
+           "moe_ep_dispatch", "moe_ep_workspace_size", "moe_ep_grouped_swiglu")
+
+MOE_EP_MAX_RANKS = 64
 
 # fixed score scratch of moe_route_noalloc, in floats (include/moe_fwd.h)
 MOE_ROUTE_NOALLOC_MAX_SCORES = 1 << 20
@@ -47,6 +50,11 @@ class MoeShape(ctypes.Structure):
 class MoeDenseShape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int), ("d_model", ctypes.c_int), ("d_ff", ctypes.c_int),
                 ("precision", ctypes.c_int), ("weight_layout", ctypes.c_int)]
+
+
+class MoeEpBlock(ctypes.Structure):
+    _fields_ = [("src_row", ctypes.c_int), ("rows", ctypes.c_int), ("dst", ctypes.c_int),
+                ("dst_row", ctypes.c_int)]
 
 
 class MoeWorkspaceOffsets(ctypes.Structure):
@@ -77,6 +85,15 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_size.argtypes = [sp]
         L.moe_workspace_size.restype = sz
         L.moe_workspace_layout.argtypes = [sp, ctypes.POINTER(MoeWorkspaceOffsets)]
+        L.moe_quant_scatter.argtypes = [sp, vp, vp, vp, vp, vp]
+        pp = ctypes.POINTER(ctypes.c_void_p)
+        ip = ctypes.POINTER(ctypes.c_int)
+        L.moe_ep_dispatch.argtypes = [sp, vp, vp, ci, ci, ctypes.POINTER(MoeEpBlock), ci, pp, pp,
+                                      ip, vp]
+        L.moe_ep_workspace_size.argtypes = [sp, ci, ci]
+        L.moe_ep_workspace_size.restype = sz
+        L.moe_ep_grouped_swiglu.argtypes = [sp, ci, vp, vp, ci, vp, vp, vp, vp, vp, ci, vp, vp, vp,
+                                            vp, ci, pp, ip, vp, sz, vp]
         L.moe_route.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_permute.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_route_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp]
@@ -103,7 +120,8 @@ def lib() -> ctypes.CDLL:
                      "fp8_block_quant_ue8m0", "moe_grouped_swiglu",
                      "moe_combine", "moe_forward", "moe_check_status", "moe_last_launch_count",
                      "moe_set_kernel_events", "moe_pack_tiles", "moe_forward_prenorm",
-                     "moe_dense_ffn", "moe_dense_ffn_prenorm", "moe_workspace_layout"):
+                     "moe_dense_ffn", "moe_dense_ffn_prenorm", "moe_workspace_layout",
+                     "moe_quant_scatter", "moe_ep_dispatch", "moe_ep_grouped_swiglu"):
             getattr(L, name).restype = ci
         _LIB = L
     return _LIB
@@ -306,6 +324,63 @@ def moe_dense_ffn_prenorm(shape, h, gamma, eps, w13, w13_scales, w2, w2_scales, 
         _ptr(w13, wt, "w13"), _ptr(w13_scales, torch.float32, "w13_scales"), _ptr(w2, wt, "w2"),
         _ptr(w2_scales, torch.float32, "w2_scales"), _ptr(out, _BF16, "out"),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def moe_quant_scatter(shape, x, row_of, a, a_scales, stream=None):
+    """x quantised 1x128 (or copied, bf16) into the permuted rows of `a`."""
+    fp8 = shape.precision in (MOE_FP8_BLOCK, MOE_FP8_UE8M0)
+    _check(lib().moe_quant_scatter(ctypes.byref(shape), _ptr(x, _BF16, "x"),
+                                   _ptr(row_of, torch.int32, "row_of"),
+                                   _ptr(a, _FP8 if fp8 else _BF16, "a"),
+                                   _ptr(a_scales, torch.float32, "a_scales"), _stream(stream)))
+
+
+def _ptr_array(tensors, dtype=None, name="tensor"):
+    arr = (ctypes.c_void_p * len(tensors))()
+    for i, t in enumerate(tensors):
+        arr[i] = _ptr(t, dtype, f"{name}[{i}]").value if t is not None else None
+    return arr
+
+
+def moe_ep_dispatch(shape, a, a_scales, blocks, recv_a, recv_scales=None, stream=None):
+    """Copies blocks [(src_row, rows, dst, dst_row)] of the source's permuted
+    rows `a` (and scales) into the owners' receive buffers recv_a[dst]."""
+    fp8 = shape.precision in (MOE_FP8_BLOCK, MOE_FP8_UE8M0)
+    world = len(recv_a)
+    blk = (MoeEpBlock * max(1, len(blocks)))(*[MoeEpBlock(*map(int, b)) for b in blocks])
+    cap = (ctypes.c_int * world)(*[int(t.shape[0]) for t in recv_a])
+    ra = _ptr_array(recv_a, _FP8 if fp8 else _BF16, "recv_a")
+    rs = _ptr_array(recv_scales, torch.float32, "recv_scales") if recv_scales is not None else None
+    _check(lib().moe_ep_dispatch(ctypes.byref(shape), _ptr(a, _FP8 if fp8 else _BF16, "a"),
+                                 _ptr(a_scales, torch.float32, "a_scales"), int(a.shape[0]),
+                                 len(blocks), blk, world, ra, rs, cap, _stream(stream)))
+
+
+def moe_ep_workspace_size(shape, rows: int, n_segments: int) -> int:
+    n = lib().moe_ep_workspace_size(ctypes.byref(shape), int(rows), int(n_segments))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, lib().moe_last_error().decode())
+    return n
+
+
+def moe_ep_grouped_swiglu(shape, a, a_scales, seg_start, seg_rows, seg_slot, seg_src, seg_ret,
+                          n_slots, w13, w13_scales, w2, w2_scales, ret_y, ws, stream=None):
+    """Grouped gated MLP over the segments of `a`; row j of segment i is
+    stored in ret_y[seg_src[i]] at row seg_ret[i] + (j - seg_start[i])."""
+    fp8 = shape.precision in (MOE_FP8_BLOCK, MOE_FP8_UE8M0)
+    wt = _FP8 if fp8 else _BF16
+    world = len(ret_y)
+    cap = (ctypes.c_int * world)(*[int(t.shape[0]) for t in ret_y])
+    i32 = torch.int32
+    _check(lib().moe_ep_grouped_swiglu(
+        ctypes.byref(shape), int(a.shape[0]), _ptr(a, wt, "a"),
+        _ptr(a_scales, torch.float32, "a_scales"), int(seg_start.numel()),
+        _ptr(seg_start, i32, "seg_start"), _ptr(seg_rows, i32, "seg_rows"),
+        _ptr(seg_slot, i32, "seg_slot"), _ptr(seg_src, i32, "seg_src"),
+        _ptr(seg_ret, i32, "seg_ret"), int(n_slots), _ptr(w13, wt, "w13"),
+        _ptr(w13_scales, torch.float32, "w13_scales"), _ptr(w2, wt, "w2"),
+        _ptr(w2_scales, torch.float32, "w2_scales"), world, _ptr_array(ret_y, _BF16, "ret_y"),
+        cap, _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
 
 
 def moe_check_status(ws, stream=None) -> int:

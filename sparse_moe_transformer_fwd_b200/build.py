@@ -16,7 +16,7 @@ CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoe_fwd.so")
 SOURCES = ["api.cu", "router.cu", "permute.cu", "quant.cu", "combine.cu", "gemm_sm100.cu",
-           "route_noalloc.cu"]
+           "route_noalloc.cu", "ep.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]

@@ -76,13 +76,6 @@ bool inject_gemm_fault() {
     return v && strcmp(v, "gemm_tx") == 0;
 }
 
-// Schedule of the fp32-scale GEMMs' accumulator (see gemm_sm100.cu): two
-// N = 128 halves per K step unless MOE_GEMM_SPLIT_N=0.
-bool gemm_split_n() {
-    const char *v = getenv("MOE_GEMM_SPLIT_N");
-    return !(v && strcmp(v, "0") == 0);
-}
-
 int check_device() {
     int dev = 0, major = 0, minor = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -247,7 +240,6 @@ int grouped(const moe_shape *s, const void *a, const float *a_scales, const void
     g.ue8m0 = is_ue8m0(s);
     g.tile_m = tile_m;
     g.b_rowmajor = s->weight_layout == MOE_LAYOUT_ROWMAJOR;
-    g.split_n = gemm_split_n();
     // gate/up GEMM + SwiGLU
     g.gate_up = true;
     g.a = a;
@@ -458,6 +450,90 @@ int moe_grouped_swiglu(const moe_shape *s, const void *a, const float *a_scales,
     return MOE_OK;
 }
 
+int moe_quant_scatter(const moe_shape *s, const uint16_t *x, const int32_t *row_of, void *a,
+                      float *a_scales, void *stream) {
+    const CallRange nvtx_range("moe_quant_scatter");
+    RETURN_IF(check_shape(s));
+    if (s->T == 0) return g_launches = 0, MOE_OK;
+    CHECK_PTR(x);
+    CHECK_PTR(row_of);
+    CHECK_PTR(a);
+    const bool fp8 = is_fp8(s);
+    if (fp8) CHECK_PTR(a_scales);
+    RETURN_IF(check_device());
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int n = 0;
+    if (fp8)
+        LAUNCH(launch_quant_scatter(x, s->T, s->d_model, s->top_k, s->n_shared, row_of,
+                                    static_cast<uint8_t *>(a), a_scales, st, &n, PreNorm{},
+                                    is_ue8m0(s)),
+               "quant_scatter");
+    else
+        LAUNCH(launch_scatter_bf16(x, s->T, s->d_model, s->top_k, s->n_shared, row_of,
+                                   static_cast<uint16_t *>(a), st, &n, PreNorm{}),
+               "scatter");
+    mark_launch(st, n);
+    g_launches = n;
+    return MOE_OK;
+}
+
+int moe_ep_dispatch(const moe_shape *s, const void *a, const float *a_scales, int a_rows,
+                    int n_blocks, const moe_ep_block *blocks, int world, void *const *recv_a,
+                    float *const *recv_scales, const int *recv_capacity, void *stream) {
+    const CallRange nvtx_range("moe_ep_dispatch");
+    RETURN_IF(check_shape(s));
+    if (world < 1 || world > MOE_EP_MAX_RANKS)
+        return fail(MOE_ERR_INVALID_ARG, "world must be in 1..%d", MOE_EP_MAX_RANKS);
+    if (n_blocks < 0 || n_blocks > MOE_EP_MAX_RANKS)
+        return fail(MOE_ERR_INVALID_ARG, "n_blocks must be in 0..%d", MOE_EP_MAX_RANKS);
+    if (a_rows < 0) return fail(MOE_ERR_INVALID_ARG, "a_rows < 0");
+    if (n_blocks > 0 && (!blocks || !recv_a || !recv_capacity))
+        return fail(MOE_ERR_INVALID_ARG, "blocks, recv_a and recv_capacity must not be NULL");
+    const bool fp8 = is_fp8(s);
+    EpDispatchArgs g{};
+    g.n_blocks = n_blocks;
+    g.row_bytes = s->d_model * (fp8 ? 1 : 2);
+    g.n_scales = fp8 ? s->d_model / 128 : 0;
+    int total = 0;
+    for (int b = 0; b < n_blocks; ++b) {
+        const moe_ep_block &k = blocks[b];
+        if (k.rows < 0 || k.src_row < 0 || static_cast<long long>(k.src_row) + k.rows > a_rows)
+            return fail(MOE_ERR_INVALID_ARG, "block %d: source rows outside the buffer", b);
+        if (k.dst < 0 || k.dst >= world)
+            return fail(MOE_ERR_INVALID_ARG, "block %d: destination rank %d out of range", b, k.dst);
+        if (k.dst_row < 0 || static_cast<long long>(k.dst_row) + k.rows > recv_capacity[k.dst])
+            return fail(MOE_ERR_INVALID_ARG, "block %d: receive rows outside rank %d's buffer", b,
+                        k.dst);
+        if (k.rows > 0) {
+            if (!recv_a[k.dst] || !aligned16(recv_a[k.dst]))
+                return fail(MOE_ERR_INVALID_ARG, "recv_a[%d] is NULL or not 16-byte aligned", k.dst);
+            if (fp8 && (!recv_scales || !recv_scales[k.dst] ||
+                        (reinterpret_cast<uintptr_t>(recv_scales[k.dst]) & 3)))
+                return fail(MOE_ERR_INVALID_ARG, "recv_scales[%d] is NULL or misaligned", k.dst);
+        }
+        g.src_row[b] = k.src_row;
+        g.dst[b] = k.dst;
+        g.dst_row[b] = k.dst_row;
+        g.prefix[b] = total;
+        total += k.rows;
+    }
+    g.prefix[n_blocks] = total;
+    for (int r = 0; r < world; ++r) {
+        g.dst_a[r] = recv_a ? static_cast<uint8_t *>(recv_a[r]) : nullptr;
+        g.dst_s[r] = (fp8 && recv_scales) ? recv_scales[r] : nullptr;
+    }
+    if (total == 0) return g_launches = 0, MOE_OK;
+    CHECK_PTR(a);
+    if (fp8) CHECK_PTR(a_scales);
+    RETURN_IF(check_device());
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int n = 0;
+    LAUNCH(launch_ep_dispatch(a, fp8 ? a_scales : nullptr, g, st, &n), "ep dispatch");
+    mark_launch(st, n);
+    g_launches = n;
+    return MOE_OK;
+}
+
 int moe_combine(const moe_shape *s, const uint16_t *y, const int32_t *row_of,
                 const float *topk_w, uint16_t *out, void *stream) {
     const CallRange nvtx_range("moe_combine");
@@ -628,6 +704,30 @@ DenseLayout dense_layout(const moe_dense_shape *s) {
     return L;
 }
 
+// Workspace of moe_ep_grouped_swiglu: status word, the checked segment table
+// (start, rows, tile prefix, slot, source, return row), H and its scales.
+struct EpLayout {
+    size_t status, table, h, h_scales, total;
+};
+
+EpLayout ep_layout(const moe_shape *s, int rows, int n_seg) {
+    const bool fp8 = is_fp8(s);
+    const size_t de = s->d_expert, R = rows;
+    EpLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += (bytes + 255) & ~static_cast<size_t>(255);
+        return at;
+    };
+    L.status = take(256);
+    L.table = take(6 * (static_cast<size_t>(n_seg) + 1) * 4);
+    L.h = take(R * de * (fp8 ? 1 : 2));
+    L.h_scales = take(fp8 ? R * (de / 128) * 4 : 0);
+    L.total = off;
+    return L;
+}
+
 int dense_ksplit(const moe_dense_shape *s) {
     if (s->T > kDenseSplitRows || s->precision == MOE_FP8_UE8M0) return 1;
     const int tiles = gemm_output_tiles(s->T, s->d_model);
@@ -693,7 +793,6 @@ int dense_impl(const moe_dense_shape *s, const uint16_t *x, const uint16_t *gamm
     g.status = at<int>(ws, L.status);
     g.ue8m0 = ue;
     g.b_rowmajor = s->weight_layout == MOE_LAYOUT_ROWMAJOR;
-    g.split_n = gemm_split_n();
     // one segment of T rows: 64-row tiles only where they save round trips
     g.tile_m = (s->precision == MOE_FP8_BLOCK && T <= 64) ? 64 : 128;
     g.gate_up = true;
@@ -751,6 +850,119 @@ int moe_dense_ffn_prenorm(const moe_dense_shape *s, const uint16_t *h, const uin
                           void *stream) {
     if (!gamma) return fail(MOE_ERR_INVALID_ARG, "gamma is NULL");
     return dense_impl(s, h, gamma, eps, w13, w13_scales, w2, w2_scales, out, ws, ws_bytes, stream);
+}
+
+size_t moe_ep_workspace_size(const moe_shape *s, int rows, int n_segments) {
+    if (check_shape(s) != MOE_OK) return 0;
+    if (rows < 0 || n_segments < 1 || n_segments > 1024) {
+        fail(MOE_ERR_INVALID_ARG, "need rows >= 0 and 1 <= n_segments <= 1024");
+        return 0;
+    }
+    return ep_layout(s, rows, n_segments).total;
+}
+
+int moe_ep_grouped_swiglu(const moe_shape *s, int rows, const void *a, const float *a_scales,
+                          int n_segments, const int32_t *seg_start, const int32_t *seg_rows,
+                          const int32_t *seg_slot, const int32_t *seg_src, const int32_t *seg_ret,
+                          int n_slots, const void *w13, const float *w13_scales, const void *w2,
+                          const float *w2_scales, int world, uint16_t *const *ret_y,
+                          const int *ret_capacity, void *ws, size_t ws_bytes, void *stream) {
+    const CallRange nvtx_range("moe_ep_grouped_swiglu");
+    RETURN_IF(check_shape(s));
+    if (rows < 0) return fail(MOE_ERR_INVALID_ARG, "rows < 0");
+    if (n_segments < 1 || n_segments > 1024)
+        return fail(MOE_ERR_INVALID_ARG, "n_segments must be in 1..1024");
+    if (n_slots < 1 || n_slots > 1024) return fail(MOE_ERR_INVALID_ARG, "n_slots must be in 1..1024");
+    if (world < 1 || world > MOE_EP_MAX_RANKS)
+        return fail(MOE_ERR_INVALID_ARG, "world must be in 1..%d", MOE_EP_MAX_RANKS);
+    const EpLayout L = ep_layout(s, rows, n_segments);
+    if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+    if (reinterpret_cast<uintptr_t>(ws) & 255)
+        return fail(MOE_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (ws_bytes < L.total)
+        return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+    if (rows == 0) return g_launches = 0, MOE_OK;
+    CHECK_PTR(a);
+    if (is_fp8(s)) CHECK_PTR(a_scales);
+    CHECK_PTR(seg_start);
+    CHECK_PTR(seg_rows);
+    CHECK_PTR(seg_src);
+    CHECK_PTR(seg_ret);
+    if (seg_slot && !aligned16(seg_slot))
+        return fail(MOE_ERR_INVALID_ARG, "seg_slot is not 16-byte aligned");
+    if (!ret_y || !ret_capacity) return fail(MOE_ERR_INVALID_ARG, "ret_y and ret_capacity are NULL");
+    for (int r = 0; r < world; ++r) {
+        if (!ret_y[r] || !aligned16(ret_y[r]))
+            return fail(MOE_ERR_INVALID_ARG, "ret_y[%d] is NULL or not 16-byte aligned", r);
+        if (ret_capacity[r] < 0) return fail(MOE_ERR_INVALID_ARG, "ret_capacity[%d] < 0", r);
+    }
+    RETURN_IF(check_weights(s, w13, w13_scales, w2, w2_scales));
+    RETURN_IF(check_device());
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool fp8 = is_fp8(s);
+    int n = 0;
+    EpTableArgs t{};
+    t.start = seg_start;
+    t.rows = seg_rows;
+    t.slot = seg_slot;
+    t.src = seg_src;
+    t.ret = seg_ret;
+    t.n_seg = n_segments;
+    t.rows_total = rows;
+    t.n_slots = n_slots;
+    t.world = world;
+    t.tile_m = kTileM;
+    for (int r = 0; r < world; ++r) t.ret_capacity[r] = ret_capacity[r];
+    int32_t *tab = at<int32_t>(ws, L.table);
+    const size_t S = static_cast<size_t>(n_segments) + 1;
+    int32_t *v_start = tab, *v_rows = tab + S, *v_tiles = tab + 2 * S, *v_slot = tab + 3 * S,
+            *v_src = tab + 4 * S, *v_ret = tab + 5 * S;
+    LAUNCH(launch_ep_table(t, v_start, v_rows, v_tiles, v_slot, v_src, v_ret, at<int>(ws, L.status),
+                           st, &n),
+           "ep segment table");
+    GemmArgs g{};
+    g.fp8 = fp8;
+    g.rows_total = rows;
+    g.n_slots = n_slots;
+    g.n_segments = n_segments;
+    g.E = n_segments;
+    g.seg_start = v_start;
+    g.seg_rows = v_rows;
+    g.tile_start = v_tiles;
+    g.seg_slot = v_slot;
+    g.status = at<int>(ws, L.status);
+    g.inject_fault = 0;
+    g.ue8m0 = is_ue8m0(s);
+    g.tile_m = kTileM;
+    g.b_rowmajor = s->weight_layout == MOE_LAYOUT_ROWMAJOR;
+    g.gate_up = true;
+    g.a = a;
+    g.a_scales = a_scales;
+    g.b = w13;
+    g.b_scales = w13_scales;
+    g.out = at<uint8_t>(ws, L.h);
+    g.out_scales = fp8 ? at<float>(ws, L.h_scales) : nullptr;
+    g.K = s->d_model;
+    g.N_out = s->d_expert;
+    LAUNCH(launch_grouped_gemm(g, st, &n), "EP gate/up GEMM");
+    // down GEMM: Y rows straight into the source ranks' buffers
+    g.gate_up = false;
+    g.a = at<uint8_t>(ws, L.h);
+    g.a_scales = fp8 ? at<float>(ws, L.h_scales) : nullptr;
+    g.b = w2;
+    g.b_scales = w2_scales;
+    g.out = ret_y[0];
+    g.out_scales = nullptr;
+    g.K = s->d_expert;
+    g.N_out = s->d_model;
+    g.seg_src = v_src;
+    g.seg_ret = v_ret;
+    g.ep_world = world;
+    g.ret_y = ret_y;
+    LAUNCH(launch_grouped_gemm(g, st, &n), "EP down GEMM");
+    mark_launch(st, n);
+    g_launches = n;
+    return MOE_OK;
 }
 
 int moe_check_status(void *ws, void *stream) {

@@ -96,8 +96,8 @@ struct __align__(1024) GemmSmem {
     uint64_t sf_free[SF_BUFS];      // scale block copied to TMEM (tcgen05.commit -> warp 2)
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
-    uint64_t tfull[4];   // [2 * buffer + half]: accumulator (half) ready
-    uint64_t tempty[4];  // [2 * buffer + half]: accumulator (half) drained
+    uint64_t tfull[2];   // accumulator buffer ready
+    uint64_t tempty[2];  // accumulator buffer drained
     uint64_t xchg[2];        // amax exchange between the two column halves
     uint64_t mma_done;
     uint32_t tmem_base;
@@ -129,11 +129,12 @@ struct KParams {
     float *partial;        // [ksplit][rows_total][N_out]
     const uint16_t *residual;  // down GEMM without split: bf16 [rows_total, N_out] added before rounding Y
     int b_rowmajor;        // B row-major [slots * b_rows, K] instead of 128 x 128-byte tiles
-    // fp32 scales, 128-row tiles: each K step's 128 x 256 accumulator is made
-    // by two N = 128 MMAs into two 128-column halves with their own ready and
-    // drained barriers, so the four halves of the two buffers give the
-    // epilogue's TMEM round trip three half steps of MMA work to hide in
-    int split_n;
+    // Expert parallelism.  seg_slot (NULL: segment s uses weight slot s):
+    // the weight slot of each segment.  seg_ret (NULL: Y stays in out): the
+    // down GEMM stores row j of segment s into ret_y[seg_src[s]] at row
+    // seg_ret[s] + (j - seg_start[s]), the source rank's own Y buffer.
+    const int32_t *seg_slot, *seg_src, *seg_ret;
+    uint16_t *ret_y[kMaxEpRanks];
 };
 
 // Output tile `tile` -> (segment, first row, valid rows, column tile).  The
@@ -231,10 +232,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&s.empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s.tfull[2 * i], 1);
-            mbar_init(&s.tempty[2 * i], EPI_THREADS / 32);
-            mbar_init(&s.tfull[2 * i + 1], 1);
-            mbar_init(&s.tempty[2 * i + 1], EPI_THREADS / 32);
+            mbar_init(&s.tfull[i], 1);
+            mbar_init(&s.tempty[i], EPI_THREADS / 32);
             mbar_init(&s.xchg[i], EPI_THREADS);
         }
         mbar_init(&s.mma_done, 1);
@@ -337,7 +336,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 int seg, row0, rows_valid, nt;
                 decode_tile<TM>(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
                 long long t_lo, t_hi;
-                b_blocks(seg, nt, t_lo, t_hi);
+                b_blocks(p.seg_slot ? __ldg(p.seg_slot + seg) : seg, nt, t_lo, t_hi);
                 const bool first = item == static_cast<int>(blockIdx.x);
                 for (int kb = kb0; kb < kb0 + nk; ++kb) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, p.status)) {
@@ -384,8 +383,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
             constexpr uint32_t idesc = MX ? instr_desc_mx(BM, BN) : instr_desc<FP8>(TM, BN);
-            constexpr uint32_t idesc_half = instr_desc<FP8>(TM, BN / 2);
-            const bool split = SCALED && !M64 && p.split_n;
             int stage = 0;
             uint32_t phase = 0;
             int tb = 0;
@@ -400,7 +397,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const bool chunk_first = (kb % SPC) == 0;
                     const bool chunk_last = (kb % SPC) == SPC - 1 || kb == nk - 1;
                     if (chunk_first) {
-                        if (!mbar_wait(&s.tempty[2 * tb], tphase ^ 1, abort, p.status)) {
+                        if (!mbar_wait(&s.tempty[tb], tphase ^ 1, abort, p.status)) {
                             ok = false;
                             break;
                         }
@@ -436,50 +433,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     // MX: this K block's scales are byte kb % 4 of each scale column
                     // (the id in the instruction descriptor and in the TMEM address)
                     const uint32_t sid = static_cast<uint32_t>(kb % SF_GROUP);
-                    if (split) {
-                        // columns 0..127 (B rows 0..127), then 128..255; each half
-                        // is one K step (SPC = 1): a fresh partial sum
-                        const uint64_t bdesc_hi = smem_desc_sw128(smem_u32(s.b[stage] + B_BYTES / 2));
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc_mma<FP8>(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc_half, kk ? 1u : 0u);
-                        tc_commit(&s.tfull[2 * tb]);
-                        if (!mbar_wait(&s.tempty[2 * tb + 1], tphase ^ 1, abort, p.status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc_mma<FP8>(d_tmem + BN / 2, adesc + 2 * kk, bdesc_hi + 2 * kk, idesc_half,
-                                        kk ? 1u : 0u);
-                        tc_commit(&s.empty[stage]);
-                        tc_commit(&s.tfull[2 * tb + 1]);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        // +32 bytes of K per instruction: +2 in the >>4 address field;
+                        // each K chunk (M64: each K step) starts a fresh partial sum
+                        const uint32_t acc = ((M64 || chunk_first) && kk == 0) ? 0u : 1u;
+                        if constexpr (MX)
+                            tc_mma_mx(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
+                                      idesc | (sid << 29) | (sid << 4),
+                                      (tmem_base + SF_COL) | (sid << 30),
+                                      (tmem_base + SF_COL + 4) | (sid << 30), acc);
+                        else
+                            tc_mma<FP8>(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc);
+                    }
+                    tc_commit(&s.empty[stage]);
+                    if (chunk_last) {
+                        tc_commit(&s.tfull[tb]);
                         if (++tb == R::NBUF) {
                             tb = 0;
                             tphase ^= 1;
-                        }
-                    } else {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            // +32 bytes of K per instruction: +2 in the >>4 address field;
-                            // each K chunk (M64: each K step) starts a fresh partial sum
-                            const uint32_t acc = ((M64 || chunk_first) && kk == 0) ? 0u : 1u;
-                            if constexpr (MX)
-                                tc_mma_mx(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
-                                          idesc | (sid << 29) | (sid << 4),
-                                          (tmem_base + SF_COL) | (sid << 30),
-                                          (tmem_base + SF_COL + 4) | (sid << 30), acc);
-                            else
-                                tc_mma<FP8>(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc);
-                        }
-                        tc_commit(&s.empty[stage]);
-                        if (chunk_last) {
-                            tc_commit(&s.tfull[2 * tb]);
-                            if (++tb == R::NBUF) {
-                                tb = 0;
-                                tphase ^= 1;
-                            }
                         }
                     }
                     if (++stage == STAGES) {
@@ -555,12 +527,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                             }
                         }
                         if (lane < 2 * SF_GROUP) {
+                            const int slot_w = p.seg_slot ? __ldg(p.seg_slot + seg) : seg;
                             const int which = lane / SF_GROUP, j = lane % SF_GROUP;
                             const int nb = which == 0 ? (GATE_UP ? nt : 2 * nt)
                                                       : (GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1);
                             const bool in = j < jn;
                             cp_async4(&s.sf_b[slot][which][j],
-                                      p.b_scales + (in ? (static_cast<size_t>(seg) * NB + nb) * KB + kbs + j : 0),
+                                      p.b_scales + (in ? (static_cast<size_t>(slot_w) * NB + nb) * KB + kbs + j : 0),
                                       in);
                         }
                         if (++cur_g == groups_of(cur_item)) {
@@ -630,7 +603,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const int hh = M64 ? (lane >> 4) : 0;
         const int r_in = M64 ? q * 16 + (lane & 15) : q * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-        const bool split = SCALED && !M64 && p.split_n;
         int tb = 0;
         uint32_t tphase = 0;
         int iter = 0;
@@ -675,7 +647,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         ++gq;
                     }
                 }
-                if (!mbar_wait(&s.tfull[2 * tb], tphase, abort, p.status)) {
+                if (!mbar_wait(&s.tfull[tb], tphase, abort, p.status)) {
                     ok = false;
                     break;
                 }
@@ -685,44 +657,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 // (before its FMAs), since the MMA two chunks ahead waits for it
                 float va[32], vb[32];
                 const bool add = warp_active && kvalid;  // the loads below are warp-wide
-                if (split) {
-                    // each half is released as soon as its pieces are in registers
-                    const uint32_t base = lane_base + tb * BN;
-                    if (warp_active) {
-                        tmem_ld32(base + col_lo, va);
-                        tmem_ld32(base + col_lo + 32, vb);
-                        tmem_wait_ld(va, vb);
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s.tempty[2 * tb]);
-                    if (add) {
-                        promote32<SCALED>(acc2, 0, va, sc_lo);
-                        promote32<SCALED>(acc2, 16, vb, sc_lo);
-                    }
-                    if (!mbar_wait(&s.tfull[2 * tb + 1], tphase, abort, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (warp_active) {
-                        tmem_ld32(base + col_hi, va);
-                        tmem_ld32(base + col_hi + 32, vb);
-                        tmem_wait_ld(va, vb);
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s.tempty[2 * tb + 1]);
-                    if (add) {
-                        promote32<SCALED>(acc2, 32, va, sc_hi);
-                        promote32<SCALED>(acc2, 48, vb, sc_hi);
-                    }
-                    if (++tb == R::NBUF) {
-                        tb = 0;
-                        tphase ^= 1;
-                    }
-                    continue;
-                }
                 if (warp_active) {
                     const uint32_t base = lane_base + tb * BN;
                     tmem_ld32(base + col_lo, va);
@@ -736,7 +670,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s.tempty[2 * tb]);
+                if (lane == 0) mbar_arrive(&s.tempty[tb]);
                 if (add) {
                     promote32<SCALED>(acc2, 32, va, sc_hi);
                     promote32<SCALED>(acc2, 48, vb, sc_hi);
@@ -853,6 +787,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     }
                 }
                 uint16_t *y = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 256;
+                if (p.seg_ret) {
+                    // expert parallelism: straight into the source rank's Y buffer
+                    const size_t r_src = static_cast<size_t>(__ldg(p.seg_ret + seg)) + (row - s.seg_start[seg]);
+                    y = p.ret_y[__ldg(p.seg_src + seg)] + r_src * p.N_out + nt * 256;
+                }
 #pragma unroll
                 for (int c = 0; c < 64; c += 8) {
                     uint4 o;
@@ -962,7 +901,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
         if (!make_map_2d(&mb, g.b, g.fp8, g.fp8 ? 128 : 64, static_cast<int>(b_tile_rows)))
             return cudaErrorInvalidValue;
     }
-    KParams kp;
+    KParams kp{};
     kp.a_scales = g.a_scales;
     kp.b_scales = g.b_scales;
     kp.out = g.out;
@@ -980,7 +919,13 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     kp.ue8m0 = g.ue8m0 ? 1 : 0;
     kp.rows_total = g.rows_total;
     kp.b_rowmajor = g.b_rowmajor ? 1 : 0;
-    kp.split_n = g.split_n ? 1 : 0;
+    kp.seg_slot = g.seg_slot;
+    kp.seg_src = g.seg_src;
+    kp.seg_ret = g.seg_ret;
+    if (g.seg_ret) {
+        if (g.ep_world < 1 || g.ep_world > kMaxEpRanks || !g.ret_y) return cudaErrorInvalidValue;
+        for (int i = 0; i < g.ep_world; ++i) kp.ret_y[i] = g.ret_y[i];
+    }
     // block-scaled MMA (UE8M0 scales): all of K accumulates in TMEM
     kp.mx_spc = g.K / 128;
     const bool mx = g.fp8 && g.ue8m0;

@@ -117,7 +117,11 @@ struct GemmArgs {
     const float *a_scales;  // [rows_total, K/128] (fp8)
     const void *b;          // [n_slots, B rows, K]: 128 x 128-byte tiles, or row-major
     bool b_rowmajor;        // b (and its layout) row-major instead of tiled
-    bool split_n;           // fp32 scales, 128-row tiles: two N = 128 MMAs per K step
+    // expert parallelism (see KParams): per-segment weight slot, and the
+    // return of Y rows to the source ranks' buffers (seg_ret NULL: none)
+    const int32_t *seg_slot = nullptr, *seg_src = nullptr, *seg_ret = nullptr;
+    int ep_world = 0;
+    uint16_t *const *ret_y = nullptr;  // host array of ep_world device pointers
     const float *b_scales;  // [n_slots, B rows/128, K/128] (fp8)
     void *out;              // H or Y
     float *out_scales;      // H scales (fp8 gate_up)
@@ -142,6 +146,7 @@ struct GemmArgs {
     const uint16_t *residual;  // down GEMM without split: bf16 [rows_total, N_out] added before rounding
 };
 constexpr int kMaxSplitK = 8;
+constexpr int kMaxEpRanks = MOE_EP_MAX_RANKS;  // ranks of an expert-parallel group
 // Output tiles of a GEMM with one segment of `rows` rows.
 inline int gemm_output_tiles(int rows, int N_out) { return ((rows + 127) / 128) * (N_out / 256); }
 // out [rows, n] = bf16(sum of the ksplit partial sums in order (+ residual)).
@@ -169,6 +174,28 @@ inline void mark_used_on_device(std::atomic<uint64_t> &done) {
 }
 
 // Error/launch bookkeeping shared by the C entry points (api.cu).
+// Expert parallelism: the segment table of a grouped GEMM over received rows.
+struct EpTableArgs {
+    const int32_t *start, *rows, *slot, *src, *ret;  // device arrays [n_seg]; slot may be NULL
+    int n_seg, rows_total, n_slots, world, tile_m;
+    int ret_capacity[kMaxEpRanks];  // rows of each source rank's Y buffer
+};
+cudaError_t launch_ep_table(const EpTableArgs &a, int32_t *seg_start, int32_t *seg_rows,
+                            int32_t *tile_start, int32_t *seg_slot, int32_t *seg_src,
+                            int32_t *seg_ret, int *status, cudaStream_t st, int *launches);
+
+// Expert parallelism: rows of one source rank's permuted buffer copied into
+// the owners' receive buffers, one contiguous block per owner.
+struct EpDispatchArgs {
+    int n_blocks, row_bytes, n_scales;
+    int src_row[kMaxEpRanks], dst[kMaxEpRanks], dst_row[kMaxEpRanks];
+    int prefix[kMaxEpRanks + 1];  // rows of blocks before block b
+    uint8_t *dst_a[kMaxEpRanks];
+    float *dst_s[kMaxEpRanks];
+};
+cudaError_t launch_ep_dispatch(const void *a, const float *a_scales, const EpDispatchArgs &g,
+                               cudaStream_t st, int *launches);
+
 int record_error(int code, const char *msg);  // sets moe_last_error, returns code
 void record_launches(int n);                   // sets moe_last_launch_count
 int validate_shape(const moe_shape *s);        // host-side shape checks

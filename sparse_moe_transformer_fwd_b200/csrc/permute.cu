@@ -242,6 +242,48 @@ tile_table_kernel(const int32_t *__restrict__ offsets, int E, int T, int k, int 
     write_tile_table(count, start, e, E, T, T * k, n_shared, tile_m, tmp, seg_start, seg_rows, tile_start);
 }
 
+// Segment table of an expert-parallel grouped GEMM from caller segments
+// (any row ranges of the receive buffer): checked copies of start, rows,
+// weight slot, source rank and return row, and the prefix of tile_m-row
+// tiles.  A segment that reaches outside the buffer, names a slot or a source
+// that does not exist, or would return rows past its source's buffer is
+// recorded in the status word and emptied.
+__global__ void __launch_bounds__(1024)
+ep_table_kernel(EpTableArgs a, int32_t *seg_start, int32_t *seg_rows, int32_t *tile_start,
+                int32_t *seg_slot, int32_t *seg_src, int32_t *seg_ret, int *status) {
+    __shared__ int tmp[32];
+    const int i = threadIdx.x;
+    pdl_wait_and_trigger();
+    int start = 0, rows = 0, slot = 0, src = 0, ret = 0;
+    if (i < a.n_seg) {
+        start = a.start[i];
+        rows = a.rows[i];
+        slot = a.slot ? a.slot[i] : i;
+        src = a.src[i];
+        ret = a.ret[i];
+        const bool ok = start >= 0 && rows >= 0 &&
+                        static_cast<long long>(start) + rows <= a.rows_total && slot >= 0 &&
+                        slot < a.n_slots && src >= 0 && src < a.world && ret >= 0 &&
+                        static_cast<long long>(ret) + rows <= a.ret_capacity[src < 0 || src >= a.world ? 0 : src];
+        if (!ok) {
+            set_status(status, MOE_ERR_DEVICE_INDEX);
+            start = rows = slot = src = ret = 0;
+        }
+    }
+    const int tiles = (rows + a.tile_m - 1) / a.tile_m;
+    int total;
+    const int ts = block_exclusive_scan(tiles, tmp, &total);
+    if (i < a.n_seg) {
+        seg_start[i] = start;
+        seg_rows[i] = rows;
+        tile_start[i] = ts;
+        seg_slot[i] = slot;
+        seg_src[i] = src;
+        seg_ret[i] = ret;
+    }
+    if (i == 0) tile_start[a.n_seg] = total;
+}
+
 }  // namespace
 
 cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int n_shared, PermScratch s,
@@ -277,6 +319,18 @@ cudaError_t launch_tile_table(const int32_t *offsets, int E, int T, int k, int n
     mark_launch(st, *launches, "tile_table");
     LAUNCH_OR_RETURN(launch_pdl(tile_table_kernel, dim3(1), dim3(1024), 0, st, offsets, E, T, k, n_shared,
                                 s.tile_m, s.seg_start, s.seg_rows, s.tile_start, status));
+    ++*launches;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_table(const EpTableArgs &a, int32_t *seg_start, int32_t *seg_rows,
+                            int32_t *tile_start, int32_t *seg_slot, int32_t *seg_src,
+                            int32_t *seg_ret, int *status, cudaStream_t st, int *launches) {
+    if (a.n_seg < 1 || a.n_seg > 1024 || a.world < 1 || a.world > kMaxEpRanks)
+        return cudaErrorInvalidValue;
+    mark_launch(st, *launches, "ep_table");
+    LAUNCH_OR_RETURN(launch_pdl(ep_table_kernel, dim3(1), dim3(1024), 0, st, a, seg_start, seg_rows,
+                                tile_start, seg_slot, seg_src, seg_ret, status));
     ++*launches;
     return cudaGetLastError();
 }

@@ -16,10 +16,12 @@ per-expert row counts this module derives, for one rank:
             back (or the dispatch all-to-all run in reverse).
 
 Only the counts are exchanged here (one all_gather, NCCL on GPUs or gloo on
-the CPU).  The data path that would use the plan (rows pushed into the
-owners' receive buffers through peer pointers, the grouped GEMM over
-(source, expert) segments, Y stored back from the down GEMM's epilogue) is
-not part of the library: it needs several GPUs.
+the CPU).  The data path that uses the plan is the library's
+moe_ep_dispatch (rows pushed into the owners' receive buffers),
+moe_ep_grouped_swiglu (the grouped GEMM over (source, expert) segments, Y
+stored back from the down GEMM's epilogue into the source's buffer) and
+moe_combine; dispatch_blocks and gemm_segments turn a plan into their
+arguments.
 """
 from __future__ import annotations
 
@@ -27,7 +29,7 @@ import dataclasses
 
 import numpy as np
 
-__all__ = ["EPPlan", "ep_plan", "exchange_counts"]
+__all__ = ["EPPlan", "ep_plan", "exchange_counts", "dispatch_blocks", "gemm_segments"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -95,3 +97,39 @@ def exchange_counts(counts_local, group=None):
     parts = [torch.empty_like(counts_local) for _ in range(world)]
     dist.all_gather(parts, counts_local, group=group)
     return torch.stack(parts)
+
+
+def dispatch_blocks(counts_all, source: int):
+    """The moe_ep_dispatch blocks of one source rank: for every owner o with
+    rows from it, (first row in the source's permuted order, rows, o, first
+    row in o's receive buffer)."""
+    c = np.asarray(counts_all, dtype=np.int64)
+    G = c.shape[0]
+    mine = ep_plan(c, source)
+    out = []
+    for o in range(G):
+        if mine.send_rows[o] == 0:
+            continue
+        dst_row = ep_plan(c, o).recv_start[source]
+        out.append((int(mine.send_start[o]), int(mine.send_rows[o]), o, int(dst_row)))
+    return out
+
+
+def gemm_segments(plan: EPPlan, order: str = "slot"):
+    """Segments of the owner's grouped GEMM as int32 arrays (start, rows,
+    slot, source, return row): one per (source, local expert), the return
+    row being where the segment's first row sits in its source's permuted
+    order (return_base of the source plus its offset inside the source's
+    block).  order "slot" lists them weight slot major (an expert's segments
+    from all sources one after the other, so its weights are read while
+    they are in L2), "source" in buffer order.  Empty segments are left out
+    (at least one segment is kept)."""
+    start = plan.seg_start.astype(np.int64)
+    src = plan.seg_source.astype(np.int64)
+    ret = plan.return_base[src] + (start - plan.recv_start[src])
+    keys = np.lexsort((src, plan.seg_slot)) if order == "slot" else np.arange(len(start))
+    keep = [i for i in keys if plan.seg_rows[i] > 0] or [int(keys[0])]
+    idx = np.array(keep, dtype=np.int64)
+    i32 = lambda a: np.ascontiguousarray(a[idx], dtype=np.int32)
+    return {"seg_start": i32(start), "seg_rows": i32(plan.seg_rows), "seg_slot": i32(plan.seg_slot),
+            "seg_src": i32(src), "seg_ret": i32(ret)}

@@ -227,3 +227,42 @@ def test_gloo_expert_parallel_forward_matches_the_layer():
     # row batches: within one bf16 step, almost every bit equal
     assert all(ok for _, ok, _ in res)
     assert all(frac < 0.01 for _, _, frac in res)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_dispatch_blocks_and_gemm_segments_follow_every_row(G):
+    """dispatch_blocks and gemm_segments, the arguments of moe_ep_dispatch and
+    moe_ep_grouped_swiglu: every routed row of every source is sent once,
+    lands in its owner's receive buffer inside exactly one segment whose slot
+    is its expert, and returns to the row it came from in its source's
+    permuted order."""
+    from sparse_moe_transformer_fwd_b200.ep_plan import dispatch_blocks, gemm_segments
+    rng = np.random.default_rng(40 + G)
+    E, k = 16, 4
+    idxs = [_idx(rng, 20 + 13 * s, E, k, skew=bool(s % 2)) for s in range(G)]
+    perm = [_row_ids(idx, E, s) for s, idx in enumerate(idxs)]
+    counts = np.stack([c for _, c in perm])
+    P = E // G
+    recv = [np.full(ep_plan(counts, o).total_recv, -1, dtype=np.int64) for o in range(G)]
+    for s in range(G):
+        ids = perm[s][0]
+        for src_row, rows, o, dst_row in dispatch_blocks(counts, s):
+            assert np.all(recv[o][dst_row:dst_row + rows] == -1)      # no overlap
+            recv[o][dst_row:dst_row + rows] = ids[src_row:src_row + rows]
+    returned = [np.full(len(perm[s][0]), -1, dtype=np.int64) for s in range(G)]
+    for o in range(G):
+        assert np.all(recv[o] >= 0)                                  # every row filled
+        segs = gemm_segments(ep_plan(counts, o))
+        covered = np.zeros(len(recv[o]), dtype=int)
+        for st, n, slot, src, ret in zip(*(segs[k] for k in ("seg_start", "seg_rows", "seg_slot",
+                                                                 "seg_src", "seg_ret"))):
+            rows = recv[o][st:st + n]
+            covered[st:st + n] += 1
+            assert np.all(rows // 1_000_000 == src)                   # from that source
+            assert np.all((rows // 1000) % 1000 == o * P + slot)      # of that expert
+            returned[src][ret:ret + n] = rows
+        assert np.all(covered == 1)
+        # weight-slot-major order
+        assert np.all(np.diff(segs["seg_slot"]) >= 0)
+    for s in range(G):
+        assert np.array_equal(returned[s], perm[s][0])                # back where it came from

@@ -57,7 +57,9 @@ def test_scale_boundary_of_power_of_two_tiles():
     assert d2[0, 1] == 1.0
 
 
-def test_layer_allowance_is_zero_in_bf16_and_small_in_fp8():
+def test_layer_allowance_is_small_in_every_precision():
+    """A handful of H elements per row sit near a rounding boundary (bf16 or
+    e4m3), so the allowance stays well below the output scale."""
     from moe_inputs import CONFIGS, make_inputs
     import torch
     u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
@@ -70,11 +72,8 @@ def test_layer_allowance_is_zero_in_bf16_and_small_in_fp8():
                                precision=prec)
         out = oracle.bf16_to_f32(res["out"]).astype(np.float64)
         rms = np.sqrt(np.mean(out ** 2))
-        if prec == "bf16":
-            assert not res["out_allow"].any()
-        else:
-            # a handful of boundary elements per row: well below the output scale
-            assert res["out_allow"].max() < 0.1 * rms
+        # a handful of boundary elements per row: well below the output scale
+        assert res["out_allow"].max() < 0.1 * rms
 
 
 # ------------------------------------------- alternative codes (signed) --
@@ -143,20 +142,69 @@ def test_nearest_correct_output_takes_only_explaining_alternatives():
 
 
 def test_nearest_correct_output_without_alternatives_is_the_oracles():
-    """With no alternative codes the nearest correct output is the oracle's
-    own bf16 output, bit for bit (bf16 experts have none)."""
+    """With no alternatives the nearest correct output is the oracle's own
+    bf16 output, bit for bit."""
     import torch
     from _gpu_util import nearest_correct_output
     cfg = DENSE_CONFIGS["dense_tiny"].with_(T=12, precision="bf16")
     inp = make_dense_inputs(cfg, seed=33)
     u = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
     res = oracle.dense_ffn(u(inp["x"]), u(inp["w13"]), u(inp["w2"]), precision="bf16")
-    assert all(len(a) == 0 for a in res["out_alts"])
+    none = [np.zeros((0, cfg.d_model))] * cfg.T
     got = torch.from_numpy(res["out"].view(np.int16)).view(torch.bfloat16)
-    want, taken, cands = nearest_correct_output(got, res["out_f64"], res["out_alts"])
+    want, taken, cands = nearest_correct_output(got, res["out_f64"], none)
     assert taken == 0 and cands == 0 and np.array_equal(want, res["out"])
 
 
+def _bf16_round_torch(v):
+    """bf16 value of binary64 v via torch (binary32 first, as the oracle and
+    the GPU round): an implementation independent of the oracle's codec."""
+    import torch
+    return torch.from_numpy(np.asarray(v, dtype=np.float64).astype(np.float32)).to(
+        torch.bfloat16).to(torch.float64).numpy()
+
+
+def test_bf16_h_ambiguity_is_the_neighbour_gap_at_boundaries():
+    """h_bf16_ambiguity: exactly the gap to the bf16 neighbour for values
+    within rho of a rounding boundary (midpoints of adjacent bf16 values),
+    0 for values well inside a rounding interval; checked against torch's
+    bf16 rounding of the perturbed values.  h_bf16_alternatives gives the
+    signed change to that neighbour."""
+    rng = np.random.default_rng(35)
+    rho = 2.0 ** -14
+    lo = _bf16_round_torch(np.exp(rng.uniform(-6, 6, 400)) * rng.choice([-1, 1], 400))
+    step = 2.0 ** (np.floor(np.log2(np.abs(lo))) - 7)
+    hi = lo + np.sign(lo) * step                        # the next bf16 magnitude
+    mid = (lo + hi) / 2                                  # rounding boundary
+    near = mid * (1 + rng.uniform(-0.5, 0.5, 400) * rho)   # within rho of it
+    inside = lo + np.sign(lo) * step / 4                 # a quarter step from lo
+    H = np.stack([near, inside])
+    amb = oracle.h_bf16_ambiguity(H, rho)
+    alt = oracle.h_bf16_alternatives(H, rho)
+    base = _bf16_round_torch(H)
+    brute = np.maximum(np.abs(_bf16_round_torch(H * (1 + rho)) - base),
+                       np.abs(_bf16_round_torch(H * (1 - rho)) - base))
+    assert np.array_equal(amb, brute)
+    assert np.allclose(amb[0], step, rtol=0, atol=0)     # every boundary value: one step
+    assert np.all(amb[1] == 0) and np.all(alt[1] == 0)
+    other = base[0] + alt[0]                             # the neighbour across the boundary
+    assert np.all(np.isin(other, np.stack([lo, hi]))) and np.all(other != base[0])
+
+
+def test_bf16_layer_allowance_covers_a_planted_flip():
+    """The bf16 expert's allowance bounds the output change of any one H
+    element taking its other rounding: plant the flip of the in-band element
+    with the largest effect and compare row by row."""
+    cfg = DENSE_CONFIGS["dense_tiny"].with_(T=16, precision="bf16")
+    inp = make_dense_inputs(cfg, seed=36)
+    import torch
+    u = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    x, w13, w2 = u(inp["x"]), u(inp["w13"]), u(inp["w2"])
+    Y, allow, alts = oracle.expert_forward(x, w13, w2, "bf16", return_f64=True, return_alts=True)
+    assert sum(len(a) for a in alts) > 0, "no element near a bf16 boundary in this sample"
+    for r, a in enumerate(alts):
+        for v in a:
+            assert np.all(np.abs(v) <= allow[r] * (1 + 1e-12))
 def test_ue8m0_alternatives_are_adjacent_codes_within_the_bound():
     """With power-of-two scales the code-level alternatives are again the
     neighbouring e4m3 values across a boundary, and never exceed
