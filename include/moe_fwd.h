@@ -36,6 +36,10 @@
  *    are recorded in a status word at the start of the workspace; read and
  *    clear it with moe_check_status().  A kernel that records an error skips
  *    the offending access and finishes, so the CUDA context stays usable.
+ *  - The library keeps per-device state (kernel attributes, the no-alloc
+ *    router's scratch address) keyed by the device's current context, so it
+ *    keeps working after the device is reset (cudaDeviceReset) and its
+ *    context created again.
  *  - Shapes: d_model a multiple of 256, d_expert a multiple of 128;
  *    1 <= top_k <= min(n_experts, 32); n_shared 0 or 1; n_experts + n_shared
  *    <= 1024; T >= 0 (T = 0 enqueues nothing).
@@ -397,7 +401,8 @@ size_t moe_ep_workspace_size(const moe_shape *shape, int rows, int n_segments);
  *   w13, w2, scales n_slots weight slots laid out as for moe_grouped_swiglu
  *                   (gate rows then up rows), in the shape's weight_layout
  *   ret_y, ret_capacity  host arrays of `world` entries: each source's Y
- *                   buffer (device pointer) and its rows
+ *                   buffer (device pointer; may be NULL when its capacity is
+ *                   0) and its rows
  * Segments that reach outside `a`, name a slot or source that does not
  * exist, or would store past a source's capacity are recorded in the
  * status word (MOE_ERR_DEVICE_INDEX, read with moe_check_status) and

@@ -10,9 +10,38 @@
 #include <cstdlib>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 namespace moe {
+
+// Unique id of the calling thread's current CUDA context (driver API, fetched
+// through the runtime so the library needs no link-time driver dependency),
+// or 0 if there is none or the driver cannot tell.  Ids are never reused in a
+// process, unlike context handles: after cudaDeviceReset the new primary
+// context may get the old handle.
+unsigned long long current_context_id() {
+    using GetCurrentFn = int (*)(void **);
+    using GetIdFn = int (*)(void *, unsigned long long *);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    void *ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0) return 0;
+    return id;
+}
 
 int num_sms() {
     int dev = 0, n = 148;
@@ -707,7 +736,7 @@ DenseLayout dense_layout(const moe_dense_shape *s) {
 // Workspace of moe_ep_grouped_swiglu: status word, the checked segment table
 // (start, rows, tile prefix, slot, source, return row), H and its scales.
 struct EpLayout {
-    size_t status, table, h, h_scales, total;
+    size_t status, table, ret_y, h, h_scales, total;
 };
 
 EpLayout ep_layout(const moe_shape *s, int rows, int n_seg) {
@@ -722,6 +751,7 @@ EpLayout ep_layout(const moe_shape *s, int rows, int n_seg) {
     };
     L.status = take(256);
     L.table = take(6 * (static_cast<size_t>(n_seg) + 1) * 4);
+    L.ret_y = take(MOE_EP_MAX_RANKS * sizeof(void *));
     L.h = take(R * de * (fp8 ? 1 : 2));
     L.h_scales = take(fp8 ? R * (de / 128) * 4 : 0);
     L.total = off;
@@ -892,9 +922,10 @@ int moe_ep_grouped_swiglu(const moe_shape *s, int rows, const void *a, const flo
         return fail(MOE_ERR_INVALID_ARG, "seg_slot is not 16-byte aligned");
     if (!ret_y || !ret_capacity) return fail(MOE_ERR_INVALID_ARG, "ret_y and ret_capacity are NULL");
     for (int r = 0; r < world; ++r) {
-        if (!ret_y[r] || !aligned16(ret_y[r]))
-            return fail(MOE_ERR_INVALID_ARG, "ret_y[%d] is NULL or not 16-byte aligned", r);
         if (ret_capacity[r] < 0) return fail(MOE_ERR_INVALID_ARG, "ret_capacity[%d] < 0", r);
+        // a source with no rows (capacity 0) may pass NULL; nothing returns to it
+        if (ret_capacity[r] > 0 && (!ret_y[r] || !aligned16(ret_y[r])))
+            return fail(MOE_ERR_INVALID_ARG, "ret_y[%d] is NULL or not 16-byte aligned", r);
     }
     RETURN_IF(check_weights(s, w13, w13_scales, w2, w2_scales));
     RETURN_IF(check_device());
@@ -912,13 +943,17 @@ int moe_ep_grouped_swiglu(const moe_shape *s, int rows, const void *a, const flo
     t.n_slots = n_slots;
     t.world = world;
     t.tile_m = kTileM;
-    for (int r = 0; r < world; ++r) t.ret_capacity[r] = ret_capacity[r];
+    for (int r = 0; r < world; ++r) {
+        t.ret_capacity[r] = ret_capacity[r];
+        t.ret_y[r] = ret_y[r];
+    }
     int32_t *tab = at<int32_t>(ws, L.table);
     const size_t S = static_cast<size_t>(n_segments) + 1;
     int32_t *v_start = tab, *v_rows = tab + S, *v_tiles = tab + 2 * S, *v_slot = tab + 3 * S,
             *v_src = tab + 4 * S, *v_ret = tab + 5 * S;
-    LAUNCH(launch_ep_table(t, v_start, v_rows, v_tiles, v_slot, v_src, v_ret, at<int>(ws, L.status),
-                           st, &n),
+    uint16_t **ret_dev = at<uint16_t *>(ws, L.ret_y);
+    LAUNCH(launch_ep_table(t, v_start, v_rows, v_tiles, v_slot, v_src, v_ret, ret_dev,
+                           at<int>(ws, L.status), st, &n),
            "ep segment table");
     GemmArgs g{};
     g.fp8 = fp8;
@@ -957,8 +992,7 @@ int moe_ep_grouped_swiglu(const moe_shape *s, int rows, const void *a, const flo
     g.N_out = s->d_model;
     g.seg_src = v_src;
     g.seg_ret = v_ret;
-    g.ep_world = world;
-    g.ret_y = ret_y;
+    g.ret_y_dev = ret_dev;
     LAUNCH(launch_grouped_gemm(g, st, &n), "EP down GEMM");
     mark_launch(st, n);
     g_launches = n;

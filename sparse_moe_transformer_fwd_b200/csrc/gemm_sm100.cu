@@ -6,15 +6,13 @@
 //
 // One persistent kernel per GEMM, one CTA per SM, cluster size 1.
 // Work item = (segment, 128-row tile of the segment, 256-column tile of B).
-// Within a segment, tiles are ordered column-tile major, row-tile minor, so
-// the CTAs running at one time read the same weight tiles through L2 (each
-// weight byte crosses DRAM once) and re-read the smaller row tiles from L2.
+// Tiles are ordered m-major, n-minor, so the CTAs running at one time share
+// A tiles and the same expert's weights through L2.
 //   warp 0      TMA producer: A tile 128 x 128 B and two B tiles 128 x 128 B
 //               (gate/up rows, or two halves of the output columns) per
-//               stage, 128-byte swizzle, 4 stages.  Weights stored in the
-//               tiled layout (128 x 128-byte tiles) make each B box one
-//               contiguous 16 KB read from HBM; row-major weights are read
-//               as 128 rows of 128 bytes.
+//               stage, 128-byte swizzle, 4 stages.  The weights are stored in
+//               128 x 128-byte tiles, so each B box is one contiguous 16 KB
+//               read from HBM.
 //   warp 1      TMEM allocator (512 columns) and MMA issuer (one thread):
 //               tcgen05.mma M=128 N=256, K=32 (e4m3) or K=16 (bf16), four per
 //               stage.
@@ -96,8 +94,8 @@ struct __align__(1024) GemmSmem {
     uint64_t sf_free[SF_BUFS];      // scale block copied to TMEM (tcgen05.commit -> warp 2)
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
-    uint64_t tfull[2];   // accumulator buffer ready
-    uint64_t tempty[2];  // accumulator buffer drained
+    uint64_t tfull[2];
+    uint64_t tempty[2];
     uint64_t xchg[2];        // amax exchange between the two column halves
     uint64_t mma_done;
     uint32_t tmem_base;
@@ -129,34 +127,23 @@ struct KParams {
     float *partial;        // [ksplit][rows_total][N_out]
     const uint16_t *residual;  // down GEMM without split: bf16 [rows_total, N_out] added before rounding Y
     int b_rowmajor;        // B row-major [slots * b_rows, K] instead of 128 x 128-byte tiles
-    // Expert parallelism.  seg_slot (NULL: segment s uses weight slot s):
-    // the weight slot of each segment.  seg_ret (NULL: Y stays in out): the
-    // down GEMM stores row j of segment s into ret_y[seg_src[s]] at row
-    // seg_ret[s] + (j - seg_start[s]), the source rank's own Y buffer.
     const int32_t *seg_slot, *seg_src, *seg_ret;
-    uint16_t *ret_y[kMaxEpRanks];
+    uint16_t *const *ret_y;  // device array [world]
 };
 
-// Output tile `tile` -> (segment, first row, valid rows, column tile).  The
-// tiles of segment s are numbered tile_start[s] * n_tiles_n on, column tile
-// major and row tile minor: consecutive tiles (run side by side by
-// neighbouring CTAs) read the same weight tile for different row tiles, so
-// each weight tile crosses DRAM once while its row tiles are in flight.
 template <int TM>
 __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int tile, int n_tiles_n,
                                             int &seg, int &row0, int &rows_valid, int &nt) {
-    const int mt = tile / n_tiles_n;  // tile_start[s] * n_tiles_n <= tile  <=>  tile_start[s] <= mt
-    int lo = 0, hi = n_seg - 1;       // last segment whose first tile is <= mt
+    const int mt = tile / n_tiles_n;
+    nt = tile - mt * n_tiles_n;
+    int lo = 0, hi = n_seg - 1;  // last segment whose first tile is <= mt
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (s.tile_start[mid] <= mt) lo = mid;
         else hi = mid - 1;
     }
     seg = lo;
-    const int m_s = s.tile_start[seg + 1] - s.tile_start[seg];  // row tiles of the segment
-    const int local = tile - s.tile_start[seg] * n_tiles_n;
-    nt = local / m_s;
-    const int mloc = local - nt * m_s;
+    const int mloc = mt - s.tile_start[seg];
     row0 = s.seg_start[seg] + mloc * TM;
     rows_valid = min(TM, s.seg_rows[seg] - mloc * TM);
 }
@@ -166,7 +153,7 @@ __device__ __forceinline__ void decode_tile(const GemmSmem &s, int n_seg, int ti
 // and the accurate versions made the end of every tile a long latency chain
 // that stalled the tensor core (the next tile's third chunk waits for it).
 // exp(-g) overflows to +inf for g < -88 and rcp(inf) = 0, so silu -> 0.
-__device__ __forceinline__ float silu(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // acc[base..base+15] (column pairs) += partial * scale (FP8 promotion) or
 // += partial (BF16 chunk sum), with the paired binary32 FMA / add of sm_100
@@ -239,8 +226,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         mbar_init(&s.mma_done, 1);
         for (int i = 0; i < SF_STAGING; ++i) {
             mbar_init(&s.sf_full[i], 1);
-            // freed by warp 2 (block-scaled MMA) or by every epilogue warp (fp32 scales)
-            mbar_init(&s.sf_empty[i], MX ? 1 : EPI_THREADS / 32);
+            mbar_init(&s.sf_empty[i], 1);
         }
         for (int i = 0; i < SF_BUFS; ++i) {
             mbar_init(&s.sf_ready[i], 1);
@@ -255,23 +241,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     // wait below; the producer adds their A loads after it.
     int pre = 0;
     const int NBq = p.b_rows / 128;
-    // The two 128-row blocks of B a work item reads (gate and up rows, or
-    // the two halves of the output columns), as 128-row block indices of the
-    // stacked weights: t_lo, t_hi = slot * NBq + block.
-    auto b_blocks = [&](int seg, int nt, long long &t_lo, long long &t_hi) {
+    auto b_blocks = [&](int slot, int nt, long long &t_lo, long long &t_hi) {
         const int nb_lo = GATE_UP ? nt : 2 * nt;
         const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
-        t_lo = static_cast<long long>(seg) * NBq + nb_lo;
-        t_hi = static_cast<long long>(seg) * NBq + nb_hi;
+        t_lo = static_cast<long long>(slot) * NBq + nb_lo;
+        t_hi = static_cast<long long>(slot) * NBq + nb_hi;
     };
-    // TMA box (128 rows x 128 bytes) of block t at K block kb: tiled layout,
-    // tile row (t * KB + kb) * 128 of a 128-byte-wide map; row-major, rows
-    // t * 128.. at K offset kb * 128 bytes.
+    const int rm = p.b_rowmajor;
     auto load_b = [&](void *dst, long long t, int kb, uint64_t *bar) {
-        if (p.b_rowmajor)
-            tma_load_2d(dst, &tmap_b, FP8 ? kb * 128 : kb * 64, static_cast<int>(t * 128), bar);
-        else
-            tma_load_2d(dst, &tmap_b, 0, static_cast<int>((t * KB + kb) * 128), bar);
+        const int x = rm ? (FP8 ? kb * 128 : kb * 64) : 0;
+        const int y = static_cast<int>(rm ? t * 128 : (t * KB + kb) * 128);
+        tma_load_2d(dst, &tmap_b, x, y, bar);
     };
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmap_a);
@@ -281,8 +261,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             int tile, ks, kb0, nk;
             k_range(blockIdx.x, tile, ks, kb0, nk);
             long long t_lo, t_hi;
-            // one segment of ceil(rows / TM) row tiles: column tile = tile / row tiles
-            b_blocks(0, tile / ((p.rows_total + TM - 1) / TM), t_lo, t_hi);
+            b_blocks(0, tile % p.n_tiles_n, t_lo, t_hi);
             pre = min(STAGES, nk);
             for (int st = 0; st < pre; ++st) {
                 mbar_arrive_expect_tx(&s.full[st], TM * 128 + B_BYTES);
@@ -471,28 +450,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             }
         }
     } else if (warp == 2 || warp == 3) {
-        // ------------------------------------------------------ block scales
-        // Per group of four K blocks of each work item, in the producer's
-        // order: warp 3 copies the fp32 scales (A's rows of the tile, B's two
-        // 128-row blocks, four K blocks each) from global memory into a
-        // staging ring with cp.async, SF_AHEAD groups ahead.
-        //  - fp32 scales (software promotion): the epilogue reads them there,
-        //    so no global load sits in its per-K-block loop.
-        //  - block-scaled MMA: warp 2 writes their UE8M0 bytes in the
-        //    tcgen05.cp source layout (lane l holds rows l, 32+l, 64+l, 96+l
-        //    of A, one 32-bit column each, byte j for K block 4g + j) and
-        //    signals the MMA issuer.  The split keeps global loads out of the
-        //    warp that must fence its shared-memory writes for the async proxy.
-        if constexpr (MX || SCALED) {
+        // ------------------------------------- scale factors (block-scaled MMA)
+        // Per group of four K blocks (in the producer's order): warp 3 copies
+        // the fp32 scales (A's 128 rows, B's two 128-row blocks, four K blocks
+        // each) from global memory into a staging ring with cp.async, SF_AHEAD
+        // groups ahead; warp 2 writes their UE8M0 bytes in the tcgen05.cp
+        // source layout (lane l holds rows l, 32+l, 64+l, 96+l of A, one 32-bit
+        // column each, byte j for K block 4g + j) and signals the MMA issuer.
+        // The split keeps global loads out of the warp that must fence its
+        // shared-memory writes for the async proxy.
+        if constexpr (MX) {
             const int NB = p.b_rows / 128;
-            auto groups_of = [&](int item) {
-                int tile, ks, kb0, nk;
-                k_range(item, tile, ks, kb0, nk);
-                return (nk + SF_GROUP - 1) / SF_GROUP;
-            };
-            int n_groups = 0;  // groups of all of this block's work items
-            for (int item = blockIdx.x; item < total_items; item += gridDim.x)
-                n_groups += groups_of(item);
+            const int NG = (KB + SF_GROUP - 1) / SF_GROUP;  // groups per tile
+            const int my_tiles = total_tiles > static_cast<int>(blockIdx.x)
+                                     ? (total_tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
+                                     : 0;
+            const int n_groups = my_tiles * NG;
             bool ok = true;
             // lane 0 waits, the warp follows (bounded; false on timeout/abort)
             auto warp_wait = [&](uint64_t *bar, uint32_t parity) {
@@ -501,44 +474,36 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 return __shfl_sync(0xffffffffu, go, 0) != 0;
             };
             if (warp == 3) {
-                // group i (in order): 4-byte cp.async copies into staging slot
-                // i % SF_STAGING (K blocks past the item's range and rows past
-                // the last: zero fill), one commit group per group (empty past
-                // the last one); (cur_item, cur_g) is the next group to issue
-                int cur_item = blockIdx.x, cur_g = 0;
+                // group i: 4-byte cp.async copies into staging slot i % SF_STAGING
+                // (K blocks past the end and rows past the last: zero fill), one
+                // commit group per group (empty past the last one)
                 auto issue = [&](int i) {
                     if (i < n_groups) {
-                        int tile, ks, kb0, nk;
-                        k_range(cur_item, tile, ks, kb0, nk);
-                        const int kbs = kb0 + cur_g * SF_GROUP;
-                        const int jn = min(SF_GROUP, nk - cur_g * SF_GROUP);
+                        const int tile = blockIdx.x + (i / NG) * gridDim.x;
+                        const int kb0 = (i % NG) * SF_GROUP;
                         int seg, row0, rows_valid, nt;
                         decode_tile<TM>(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
                         const int slot = i % SF_STAGING;
 #pragma unroll
-                        for (int c = 0; c < TM / 32; ++c) {
+                        for (int c = 0; c < 4; ++c) {
                             const int r = row0 + lane + 32 * c;
 #pragma unroll
                             for (int j = 0; j < SF_GROUP; ++j) {
-                                const bool in = r < p.rows_total && j < jn;
+                                const bool in = r < p.rows_total && kb0 + j < KB;
                                 cp_async4(&s.sf_a[slot][j][lane + 32 * c],
-                                          p.a_scales + (in ? static_cast<size_t>(r) * KB + kbs + j : 0),
+                                          p.a_scales + (in ? static_cast<size_t>(r) * KB + kb0 + j : 0),
                                           in);
                             }
                         }
                         if (lane < 2 * SF_GROUP) {
-                            const int slot_w = p.seg_slot ? __ldg(p.seg_slot + seg) : seg;
                             const int which = lane / SF_GROUP, j = lane % SF_GROUP;
                             const int nb = which == 0 ? (GATE_UP ? nt : 2 * nt)
                                                       : (GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1);
-                            const bool in = j < jn;
+                            const bool in = kb0 + j < KB;
+                            const int slot_w = p.seg_slot ? __ldg(p.seg_slot + seg) : seg;
                             cp_async4(&s.sf_b[slot][which][j],
-                                      p.b_scales + (in ? (static_cast<size_t>(slot_w) * NB + nb) * KB + kbs + j : 0),
+                                      p.b_scales + (in ? (static_cast<size_t>(slot_w) * NB + nb) * KB + kb0 + j : 0),
                                       in);
-                        }
-                        if (++cur_g == groups_of(cur_item)) {
-                            cur_g = 0;
-                            cur_item += gridDim.x;
                         }
                     }
                     cp_async_commit();
@@ -559,7 +524,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     if (lane == 0) mbar_arrive(&s.sf_full[i % SF_STAGING]);
                 }
                 cp_async_wait<0>();
-            } else if constexpr (MX) {
+            } else {
                 for (int i = 0; i < n_groups; ++i) {
                     const int slot = i % SF_STAGING;
                     if (!warp_wait(&s.sf_full[slot], (i / SF_STAGING) & 1)) break;
@@ -603,10 +568,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const int hh = M64 ? (lane >> 4) : 0;
         const int r_in = M64 ? q * 16 + (lane & 15) : q * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+        const int NB = p.b_rows / 128;
         int tb = 0;
         uint32_t tphase = 0;
         int iter = 0;
-        int gq = 0;  // scale groups consumed (fp32 scales)
         bool ok = true;
         for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x, ++iter) {
             int tile, ks, kb0, nk;
@@ -622,30 +587,29 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             float2 acc2[64];  // columns (2j, 2j+1) of the thread's 128
 #pragma unroll
             for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
+            const int nb_lo = GATE_UP ? nt : 2 * nt;
+            const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
+            // scale rows from the item's first K block on
+            const int slot_w = (SCALED && p.seg_slot) ? __ldg(p.seg_slot + seg) : seg;
+            const float *sw_lo_p = SCALED ? p.b_scales + (static_cast<size_t>(slot_w) * NB + nb_lo) * KB + kb0 : nullptr;
+            const float *sw_hi_p = SCALED ? p.b_scales + (static_cast<size_t>(slot_w) * NB + nb_hi) * KB + kb0 : nullptr;
+            const float *sa_p = SCALED ? p.a_scales + row * KB + kb0 : nullptr;
             // K block (counted from kb0) whose partial this thread promotes in chunk c
             auto kb_of = [&](int c) { return M64 ? 2 * c + hh : c; };
+            // scales of chunk c are loaded one chunk ahead (global latency)
+            float nsa = 0.0f, nswl = 1.0f, nswh = 1.0f;
+            if (SCALED && warp_active && kb_of(0) < nk) {
+                nsa = valid ? __ldg(sa_p + kb_of(0)) : 0.0f;
+                nswl = __ldg(sw_lo_p + kb_of(0));
+                nswh = __ldg(sw_hi_p + kb_of(0));
+            }
             for (int c = 0; c < nch; ++c) {
+                const float sc_lo = SCALED ? nsa * nswl : 1.0f, sc_hi = SCALED ? nsa * nswh : 1.0f;
                 const bool kvalid = !M64 || kb_of(c) < nk;  // M64, odd K: no partial in the upper half
-                float sc_lo = 1.0f, sc_hi = 1.0f;
-                if constexpr (SCALED) {
-                    // this chunk's scales, staged by warp 3 in groups of four K
-                    // blocks (M64: a chunk is two K blocks of one group)
-                    const int kba = M64 ? 2 * c : c;
-                    const int slot = gq % SF_STAGING;
-                    if (kba % SF_GROUP == 0 &&
-                        !mbar_wait(&s.sf_full[slot], (gq / SF_STAGING) & 1, abort, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    const int j = kb_of(c) % SF_GROUP;
-                    const float sa = valid ? s.sf_a[slot][j][r_in] : 0.0f;
-                    sc_lo = sa * s.sf_b[slot][0][j];
-                    sc_hi = sa * s.sf_b[slot][1][j];
-                    if (kba % SF_GROUP == SF_GROUP - (M64 ? 2 : 1) || c == nch - 1) {
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&s.sf_empty[slot]);
-                        ++gq;
-                    }
+                if (SCALED && warp_active && c + 1 < nch && kb_of(c + 1) < nk) {
+                    nsa = valid ? __ldg(sa_p + kb_of(c + 1)) : 0.0f;
+                    nswl = __ldg(sw_lo_p + kb_of(c + 1));
+                    nswh = __ldg(sw_hi_p + kb_of(c + 1));
                 }
                 if (!mbar_wait(&s.tfull[tb], tphase, abort, p.status)) {
                     ok = false;
@@ -788,7 +752,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
                 uint16_t *y = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 256;
                 if (p.seg_ret) {
-                    // expert parallelism: straight into the source rank's Y buffer
                     const size_t r_src = static_cast<size_t>(__ldg(p.seg_ret + seg)) + (row - s.seg_start[seg]);
                     y = p.ret_y[__ldg(p.seg_src + seg)] + r_src * p.N_out + nt * 256;
                 }
@@ -858,7 +821,7 @@ template <bool FP8, bool GATE_UP, bool MX, bool M64 = false, bool DENSE = false>
 cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams &kp, int grid,
                      cudaStream_t st) {
     const size_t smem = sizeof(GemmSmem) + 1024;
-    static std::atomic<uint64_t> configured{0};  // per template instance, one bit per device
+    static DeviceConfigured configured{};  // per template instance
     if (first_use_on_device(configured)) {
         // setmaxnreg redistributes exactly NUM_THREADS * LAUNCH_REGS registers:
         // refuse to launch a build whose register count differs, as the
@@ -890,12 +853,10 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     if (!make_map_2d(&ma, g.a, g.fp8, g.K, g.rows_total, m64 ? 64 : 128))
         return cudaErrorInvalidValue;
     if (g.b_rowmajor) {
-        // B row-major [n_slots * b_rows, K], the same map shape as A
         const long long rows = static_cast<long long>(g.n_slots) * b_rows;
         if (rows >= (1LL << 31)) return cudaErrorInvalidValue;
         if (!make_map_2d(&mb, g.b, g.fp8, g.K, static_cast<int>(rows))) return cudaErrorInvalidValue;
     } else {
-        // B in the tiled layout: one row of 128 bytes per tile row, tiles stacked
         const long long b_tile_rows = static_cast<long long>(g.n_slots) * b_rows * (g.K * (g.fp8 ? 1 : 2) / 128);
         if (b_tile_rows >= (1LL << 31)) return cudaErrorInvalidValue;
         if (!make_map_2d(&mb, g.b, g.fp8, g.fp8 ? 128 : 64, static_cast<int>(b_tile_rows)))
@@ -922,10 +883,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     kp.seg_slot = g.seg_slot;
     kp.seg_src = g.seg_src;
     kp.seg_ret = g.seg_ret;
-    if (g.seg_ret) {
-        if (g.ep_world < 1 || g.ep_world > kMaxEpRanks || !g.ret_y) return cudaErrorInvalidValue;
-        for (int i = 0; i < g.ep_world; ++i) kp.ret_y[i] = g.ret_y[i];
-    }
+    kp.ret_y = g.ret_y_dev;
+    if (g.seg_ret && !g.ret_y_dev) return cudaErrorInvalidValue;
     // block-scaled MMA (UE8M0 scales): all of K accumulates in TMEM
     kp.mx_spc = g.K / 128;
     const bool mx = g.fp8 && g.ue8m0;

@@ -120,8 +120,7 @@ struct GemmArgs {
     // expert parallelism (see KParams): per-segment weight slot, and the
     // return of Y rows to the source ranks' buffers (seg_ret NULL: none)
     const int32_t *seg_slot = nullptr, *seg_src = nullptr, *seg_ret = nullptr;
-    int ep_world = 0;
-    uint16_t *const *ret_y = nullptr;  // host array of ep_world device pointers
+    uint16_t *const *ret_y_dev = nullptr;  // device array: each source rank's Y buffer
     const float *b_scales;  // [n_slots, B rows/128, K/128] (fp8)
     void *out;              // H or Y
     float *out_scales;      // H scales (fp8 gate_up)
@@ -157,20 +156,31 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
 
 int num_sms();
 
-// Function attributes (dynamic shared memory size) are per device: true once
-// per device for the given per-call-site flag word (devices 0..63; larger
-// device numbers are configured on every call).
-inline bool first_use_on_device(std::atomic<uint64_t> &done) {
+// Unique id of the calling thread's current CUDA context, or 0 if there is
+// none or the driver cannot tell (api.cu).  Ids are never reused within a
+// process, unlike context handles.
+unsigned long long current_context_id();
+
+// Function attributes (dynamic shared memory size) belong to the module
+// loaded in a device's context, so they are set again whenever the context
+// changes (a device reset destroys the primary context and its modules).
+// One flag word per call site: the context id each device was configured in
+// (devices 0..63; larger device numbers, and a driver that reports no ids,
+// are configured on every call).
+struct DeviceConfigured {
+    std::atomic<unsigned long long> ctx[64];
+};
+inline bool first_use_on_device(DeviceConfigured &done) {
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 64) return true;
-    const uint64_t bit = 1ull << dev;
-    return (done.load(std::memory_order_acquire) & bit) == 0;
+    const unsigned long long id = current_context_id();
+    if (dev < 0 || dev >= 64 || id == 0) return true;
+    return done.ctx[dev].load(std::memory_order_acquire) != id;
 }
-inline void mark_used_on_device(std::atomic<uint64_t> &done) {
+inline void mark_used_on_device(DeviceConfigured &done) {
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64) done.fetch_or(1ull << dev, std::memory_order_release);
+    if (dev >= 0 && dev < 64) done.ctx[dev].store(current_context_id(), std::memory_order_release);
 }
 
 // Error/launch bookkeeping shared by the C entry points (api.cu).
@@ -179,10 +189,13 @@ struct EpTableArgs {
     const int32_t *start, *rows, *slot, *src, *ret;  // device arrays [n_seg]; slot may be NULL
     int n_seg, rows_total, n_slots, world, tile_m;
     int ret_capacity[kMaxEpRanks];  // rows of each source rank's Y buffer
+    uint16_t *ret_y[kMaxEpRanks];   // each source rank's Y buffer
 };
+// Also writes a.ret_y to ret_y_dev [world] (device memory the GEMM reads).
 cudaError_t launch_ep_table(const EpTableArgs &a, int32_t *seg_start, int32_t *seg_rows,
                             int32_t *tile_start, int32_t *seg_slot, int32_t *seg_src,
-                            int32_t *seg_ret, int *status, cudaStream_t st, int *launches);
+                            int32_t *seg_ret, uint16_t **ret_y_dev, int *status, cudaStream_t st,
+                            int *launches);
 
 // Expert parallelism: rows of one source rank's permuted buffer copied into
 // the owners' receive buffers, one contiguous block per owner.

@@ -250,10 +250,12 @@ tile_table_kernel(const int32_t *__restrict__ offsets, int E, int T, int k, int 
 // recorded in the status word and emptied.
 __global__ void __launch_bounds__(1024)
 ep_table_kernel(EpTableArgs a, int32_t *seg_start, int32_t *seg_rows, int32_t *tile_start,
-                int32_t *seg_slot, int32_t *seg_src, int32_t *seg_ret, int *status) {
+                int32_t *seg_slot, int32_t *seg_src, int32_t *seg_ret, uint16_t **ret_y_dev,
+                int *status) {
     __shared__ int tmp[32];
     const int i = threadIdx.x;
     pdl_wait_and_trigger();
+    if (i < a.world) ret_y_dev[i] = a.ret_y[i];
     int start = 0, rows = 0, slot = 0, src = 0, ret = 0;
     if (i < a.n_seg) {
         start = a.start[i];
@@ -325,12 +327,13 @@ cudaError_t launch_tile_table(const int32_t *offsets, int E, int T, int k, int n
 
 cudaError_t launch_ep_table(const EpTableArgs &a, int32_t *seg_start, int32_t *seg_rows,
                             int32_t *tile_start, int32_t *seg_slot, int32_t *seg_src,
-                            int32_t *seg_ret, int *status, cudaStream_t st, int *launches) {
+                            int32_t *seg_ret, uint16_t **ret_y_dev, int *status, cudaStream_t st,
+                            int *launches) {
     if (a.n_seg < 1 || a.n_seg > 1024 || a.world < 1 || a.world > kMaxEpRanks)
         return cudaErrorInvalidValue;
     mark_launch(st, *launches, "ep_table");
     LAUNCH_OR_RETURN(launch_pdl(ep_table_kernel, dim3(1), dim3(1024), 0, st, a, seg_start, seg_rows,
-                                tile_start, seg_slot, seg_src, seg_ret, status));
+                                tile_start, seg_slot, seg_src, seg_ret, ret_y_dev, status));
     ++*launches;
     return cudaGetLastError();
 }

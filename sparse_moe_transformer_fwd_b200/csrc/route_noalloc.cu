@@ -19,48 +19,30 @@ static __device__ __align__(256) float g_noalloc_scores[MOE_ROUTE_NOALLOC_MAX_SC
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 float *g_addr[kMaxDevices] = {};
-void *g_ctx[kMaxDevices] = {};  // the context g_addr[dev] was looked up in
+unsigned long long g_ctx_id[kMaxDevices] = {};  // context the address was looked up in
 
 thread_local char g_msg[256];
-
-// The calling thread's current CUDA context (driver API, fetched through the
-// runtime so the library needs no link-time driver dependency), or NULL.
-void *current_context() {
-    using GetCurrentFn = int (*)(void **);
-    static GetCurrentFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
-                cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<GetCurrentFn>(p);
-    });
-    void *ctx = nullptr;
-    if (!fn || fn(&ctx) != 0) return nullptr;
-    return ctx;
-}
 
 // Device address of the scratch on the current device.  In host code the
 // symbol is only a host-side stand-in, so the address is looked up with
 // cudaGetSymbolAddress, once per device and context: a device whose primary
 // context was destroyed (cudaDeviceReset) and created again loads the
-// library's module anew, possibly at another address, so a change of context
-// repeats the lookup.
+// library's module anew, possibly at another address, so a new context id
+// repeats the lookup (as does a driver that cannot report ids: id 0).
 cudaError_t scratch_address(float **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    void *ctx = current_context();
+    const unsigned long long id = current_context_id();
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev] || !ctx || ctx != g_ctx[dev]) {
+    if (!g_addr[dev] || id == 0 || id != g_ctx_id[dev]) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scores);
         if (e != cudaSuccess) return e;
         g_addr[dev] = static_cast<float *>(p);
         // the lookup made the device's primary context current if none was
-        g_ctx[dev] = current_context();
+        g_ctx_id[dev] = current_context_id();
     }
     *out = g_addr[dev];
     return cudaSuccess;

@@ -434,7 +434,7 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
     } else {
         constexpr int BT = 4, NP = RS_PRODUCER_WARPS;
         constexpr size_t smem = router_small_smem<BT>();
-        static std::atomic<uint64_t> configured{0};  // one bit per device
+        static DeviceConfigured configured{};
         if (first_use_on_device(configured)) {
             LAUNCH_OR_RETURN(cudaFuncSetAttribute(router_scores_small_kernel<BT, NP>,
                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,

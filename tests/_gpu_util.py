@@ -143,7 +143,9 @@ def assert_close_to_correct(got_bf16, res, what=""):
     the max bound's allowance for the alternatives not taken; the number of
     alternatives taken stays within max_alternatives of the candidates."""
     want, taken, cands = nearest_correct_output(got_bf16, res["out_f64"], res["out_alts"])
-    plain = out_error(got_bf16, res["out"], res["out_allow"])
+    oracle_out = res["out"] if "out" in res else oracle.bf16_from_f32(
+        np.asarray(res["out_f64"], dtype=np.float64).astype(np.float32))
+    plain = out_error(got_bf16, oracle_out, res["out_allow"])
     out = assert_out_close(got_bf16, want, what, allow=res["out_allow"],
                            alternatives_taken=taken, alternatives_in_band=cands,
                            rel_l2_before_alternatives=plain[0])
@@ -151,13 +153,20 @@ def assert_close_to_correct(got_bf16, res, what=""):
     return out
 
 
-def oracle_layer(cfg, inp, tokens=None, expert=None):
+# host threads the oracle may use for its independent experts (each expert's
+# evaluation stays single-threaded; results do not depend on the count)
+ORACLE_WORKERS = max(1, min(len(os.sched_getaffinity(0)), 16))
+
+
+def oracle_layer(cfg, inp, tokens=None, expert=None, workers=ORACLE_WORKERS):
     """Oracle forward of the layer on the tokens listed (default all).  Tokens
     of an MoE layer are independent, so a subset is evaluated as its own batch."""
     x = inp["x"] if tokens is None else inp["x"][torch.as_tensor(tokens, device=inp["x"].device)]
     if expert is None:
         expert = lambda e: (u16(inp["w13"][e]), u16(inp["w2"][e]))
-    return oracle.moe_layer(u16(x), u16(inp["w_router"]), inp["bias"].detach().cpu().numpy(),
-                            expert, n_experts=cfg.n_experts, top_k=cfg.top_k,
-                            n_shared=cfg.n_shared, precision=cfg.precision,
-                            routed_scale=cfg.routed_scale)
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        return oracle.moe_layer(u16(x), u16(inp["w_router"]), inp["bias"].detach().cpu().numpy(),
+                                expert, n_experts=cfg.n_experts, top_k=cfg.top_k,
+                                n_shared=cfg.n_shared, precision=cfg.precision,
+                                routed_scale=cfg.routed_scale, workers=workers)

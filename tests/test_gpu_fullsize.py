@@ -204,10 +204,12 @@ def test_prenorm_decode_fullsize():
     assert layer.check_status(T) == 0
     off = moe.moe_workspace_layout(layer.shape(T))
     ws = layer.workspace(T)
-    ref = oracle.moe_layer_prenorm(
-        u16(h), u16(g), 1e-6, u16(inp["w_router"]), inp["bias"].cpu().numpy(),
-        lambda e: (u16(inp["w13"][e]), u16(inp["w2"][e])), n_experts=E,
-        top_k=k, n_shared=cfg.n_shared, precision=cfg.precision)
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        ref = oracle.moe_layer_prenorm(
+            u16(h), u16(g), 1e-6, u16(inp["w_router"]), inp["bias"].cpu().numpy(),
+            lambda e: (u16(inp["w13"][e]), u16(inp["w2"][e])), n_experts=E,
+            top_k=k, n_shared=cfg.n_shared, precision=cfg.precision, workers=min(WORKERS, 16))
     s = _ws_region(ws, off, "scores", T * E, torch.float32).reshape(T, E)
     assert np.array_equal(s.view(np.uint32), ref["scores"].view(np.uint32))
     assert np.array_equal(_ws_region(ws, off, "topk_idx", T * k, torch.int32).reshape(T, k),

@@ -104,22 +104,26 @@ def route(noalloc):
         rt.cudaFree(p)
     return idx, g
 
+def same(a, b):
+    return np.array_equal(a[0], b[0]) and np.array_equal(a[1].view(np.uint32), b[1].view(np.uint32))
+
 ref = route(False)
 first = route(True)
+assert same(first, ref), "before the reset"
 assert rt.cudaDeviceReset() == 0          # ends this process's context only
 after = route(True)                       # a new context: the scratch is looked up again
-for got in (first, after):
-    assert np.array_equal(got[0], ref[0])
-    assert np.array_equal(got[1].view(np.uint32), ref[1].view(np.uint32))
+assert same(after, ref), "no-alloc router after the reset"
+assert same(route(False), ref), "workspace router after the reset"
 print("reset ok")
 """
 
 
 def test_noalloc_route_after_device_reset():
     """A process that resets its device (cudaDeviceReset) and routes again gets
-    the same bits as moe_route: the library looks the scratch address up again
-    in the new context.  Run in a child process, which owns the only context
-    it resets; buffers come from the CUDA runtime directly."""
+    the same bits as before: the library looks the scratch address up again
+    in the new context (whose handle may equal the old one; its id does not),
+    and re-applies its kernel attributes.  Run in a child process, which owns
+    the only context it resets; buffers come from the CUDA runtime directly."""
     import os
     import subprocess
     import sys
