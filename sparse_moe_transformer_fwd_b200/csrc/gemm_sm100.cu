@@ -170,6 +170,42 @@ __device__ __forceinline__ void promote32(float2 (&acc)[64], int base, const flo
     }
 }
 
+// Transpose of an N x N block of 16-byte chunks held by a group of N lanes
+// (lanes N*g .. N*g + N-1, li = lane % N): on entry lane li holds chunks
+// c[0..N-1] of its own row; on exit it holds chunk li of the group's rows
+// 0..N-1 in c[0..N-1].  Each stage swaps bit m of the lane with bit m of the
+// chunk index (log2 N stages of paired shuffles).  Used so that a store
+// instruction writes whole row segments (N lanes x 16 bytes of one row)
+// instead of 16 bytes of 32 different rows.
+template <int N>
+__device__ __forceinline__ void transpose_chunks(uint4 (&c)[N], int li) {
+#pragma unroll
+    for (int m = 1; m < N; m <<= 1) {
+        const bool up = (li & m) != 0;
+#pragma unroll
+        for (int e = 0; e < N; ++e) {
+            if (e & m) continue;
+            const uint4 send = up ? c[e] : c[e | m];
+            uint4 r;
+            r.x = __shfl_xor_sync(0xffffffffu, send.x, m);
+            r.y = __shfl_xor_sync(0xffffffffu, send.y, m);
+            r.z = __shfl_xor_sync(0xffffffffu, send.z, m);
+            r.w = __shfl_xor_sync(0xffffffffu, send.w, m);
+            if (up) c[e] = r;
+            else c[e | m] = r;
+        }
+    }
+}
+
+// Tile row whose output lane `l` of an epilogue warp of quadrant q stores,
+// or -1 if that lane stores none (past the tile's valid rows; with 64-row
+// tiles, lanes 16-31 hold the odd K steps' sums of lanes 0-15's rows).
+template <bool M64>
+__device__ __forceinline__ int stored_row_of_lane(int l, int q, int rows_valid) {
+    const int r = M64 ? q * 16 + (l & 15) : q * 32 + l;
+    return (r < rows_valid && (!M64 || l < 16)) ? r : -1;
+}
+
 // E8M0 byte of a power-of-two binary32 scale (2^-127 is the subnormal with
 // exponent field 0, matching E8M0 code 0).
 __device__ __forceinline__ uint32_t e8m0(float sc) { return (__float_as_uint(sc) >> 23) & 0xffu; }
@@ -676,43 +712,60 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         break;
                     }
                     const float amax = fmaxf(m, s.amax_x[par][half ^ 1][r_in]);
-                    if (store_row) {
-                        float sc = 1.0f, inv = 0.0f;
-                        if (amax != 0.0f) {
-                            if (p.ue8m0) {
-                                sc = ue8m0_scale(amax, &inv);
-                            } else {
-                                sc = __fdiv_rn(amax, 448.0f);
-                                inv = __fdiv_rn(448.0f, amax);
-                            }
+                    float sc = 1.0f, inv = 0.0f;
+                    if (amax != 0.0f) {
+                        if (p.ue8m0) {
+                            sc = ue8m0_scale(amax, &inv);
+                        } else {
+                            sc = __fdiv_rn(amax, 448.0f);
+                            inv = __fdiv_rn(448.0f, amax);
                         }
-                        uint8_t *hq = static_cast<uint8_t *>(p.out) + row * p.N_out + nt * 128 +
-                                      half * 64;
+                    }
+                    if (warp_active) {  // uniform over the warp
+                        // 64 codes = four 16-byte chunks; transposed across
+                        // groups of 4 lanes so each store writes 64 contiguous
+                        // bytes of a row
+                        uint4 ch[4];
 #pragma unroll
-                        for (int c = 0; c < 64; c += 16) {
+                        for (int c = 0; c < 4; ++c) {
                             uint32_t w[4];
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
-                                const int b = c + 4 * i;
+                                const int b = 16 * c + 4 * i;
                                 const uint32_t lo = e4m3x2(__fmul_rn(acc(b), inv), __fmul_rn(acc(b + 1), inv));
                                 const uint32_t hi = e4m3x2(__fmul_rn(acc(b + 2), inv), __fmul_rn(acc(b + 3), inv));
                                 w[i] = amax != 0.0f ? (lo | (hi << 16)) : 0u;
                             }
-                            *reinterpret_cast<uint4 *>(hq + c) = make_uint4(w[0], w[1], w[2], w[3]);
+                            ch[c] = make_uint4(w[0], w[1], w[2], w[3]);
                         }
-                        if (half == 0) p.out_scales[row * (p.N_out / 128) + nt] = sc;
-                    }
-                } else if (store_row) {
-                    uint16_t *h = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 128 +
-                                  half * 64;
+                        const int li = lane & 3;
+                        transpose_chunks<4>(ch, li);
+                        uint8_t *h0 = static_cast<uint8_t *>(p.out) + static_cast<size_t>(row0) * p.N_out +
+                                      nt * 128 + half * 64 + 16 * li;
 #pragma unroll
-                    for (int c = 0; c < 64; c += 8) {
-                        uint4 o;
-                        o.x = pack_bf16x2(acc(c), acc(c + 1));
-                        o.y = pack_bf16x2(acc(c + 2), acc(c + 3));
-                        o.z = pack_bf16x2(acc(c + 4), acc(c + 5));
-                        o.w = pack_bf16x2(acc(c + 6), acc(c + 7));
-                        *reinterpret_cast<uint4 *>(h + c) = o;
+                        for (int j = 0; j < 4; ++j) {
+                            const int o = stored_row_of_lane<M64>((lane & ~3) | j, q, rows_valid);
+                            if (o >= 0) *reinterpret_cast<uint4 *>(h0 + static_cast<size_t>(o) * p.N_out) = ch[j];
+                        }
+                    }
+                    if (store_row && half == 0) p.out_scales[row * (p.N_out / 128) + nt] = sc;
+                } else if (warp_active) {
+                    // bf16 H: 64 values = eight 16-byte chunks, transposed as Y
+                    uint4 ch[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int c = 8 * j;
+                        ch[j] = make_uint4(pack_bf16x2(acc(c), acc(c + 1)), pack_bf16x2(acc(c + 2), acc(c + 3)),
+                                           pack_bf16x2(acc(c + 4), acc(c + 5)), pack_bf16x2(acc(c + 6), acc(c + 7)));
+                    }
+                    const int li = lane & 7;
+                    transpose_chunks<8>(ch, li);
+                    uint16_t *h0 = static_cast<uint16_t *>(p.out) + static_cast<size_t>(row0) * p.N_out +
+                                   nt * 128 + half * 64 + 8 * li;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int o = stored_row_of_lane<M64>((lane & ~7) | j, q, rows_valid);
+                        if (o >= 0) *reinterpret_cast<uint4 *>(h0 + static_cast<size_t>(o) * p.N_out) = ch[j];
                     }
                 }
             } else {
@@ -732,8 +785,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     }
                     continue;
                 }
-                if (!store_row) continue;
-                if (DENSE && p.residual) {
+                if (!warp_active) continue;  // uniform over the warp
+                if (DENSE && p.residual && store_row) {
                     // the pre-norm block's residual, added before the one rounding
                     const uint16_t *rp = p.residual + row * p.N_out + nt * 256;
 #pragma unroll
@@ -750,24 +803,38 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         }
                     }
                 }
-                uint16_t *y = static_cast<uint16_t *>(p.out) + row * p.N_out + nt * 256;
+                // Y rows of the tile: one segment, so the base is uniform over
+                // the warp and each lane's row differs by its index
+                uint16_t *ybase = static_cast<uint16_t *>(p.out) + nt * 256;
+                long long yr = static_cast<long long>(row);
                 if (p.seg_ret) {
-                    const size_t r_src = static_cast<size_t>(__ldg(p.seg_ret + seg)) + (row - s.seg_start[seg]);
-                    y = p.ret_y[__ldg(p.seg_src + seg)] + r_src * p.N_out + nt * 256;
+                    // expert parallelism: straight into the source rank's Y buffer
+                    ybase = p.ret_y[__ldg(p.seg_src + seg)] + nt * 256;
+                    yr = static_cast<long long>(__ldg(p.seg_ret + seg)) + (yr - s.seg_start[seg]);
                 }
+                // bf16 chunks of 8 columns; transposed across groups of 8
+                // lanes so each store writes 128 contiguous bytes of a row
+                // (one 64-column half at a time, to bound the live registers)
+                const long long yr0 = yr - r_in;
+                const int li = lane & 7;
+                int yoff[8];  // tile row held by lane (lane & ~7) | j, -1: not stored
 #pragma unroll
-                for (int c = 0; c < 64; c += 8) {
-                    uint4 o;
-                    o.x = pack_bf16x2(acc(c), acc(c + 1));
-                    o.y = pack_bf16x2(acc(c + 2), acc(c + 3));
-                    o.z = pack_bf16x2(acc(c + 4), acc(c + 5));
-                    o.w = pack_bf16x2(acc(c + 6), acc(c + 7));
-                    *reinterpret_cast<uint4 *>(y + col_lo + c) = o;
-                    o.x = pack_bf16x2(acc(64 + c), acc(64 + c + 1));
-                    o.y = pack_bf16x2(acc(64 + c + 2), acc(64 + c + 3));
-                    o.z = pack_bf16x2(acc(64 + c + 4), acc(64 + c + 5));
-                    o.w = pack_bf16x2(acc(64 + c + 6), acc(64 + c + 7));
-                    *reinterpret_cast<uint4 *>(y + col_hi + c) = o;
+                for (int j = 0; j < 8; ++j) yoff[j] = stored_row_of_lane<M64>((lane & ~7) | j, q, rows_valid);
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint4 ch[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int c = 64 * hf + 8 * j;
+                        ch[j] = make_uint4(pack_bf16x2(acc(c), acc(c + 1)), pack_bf16x2(acc(c + 2), acc(c + 3)),
+                                           pack_bf16x2(acc(c + 4), acc(c + 5)), pack_bf16x2(acc(c + 6), acc(c + 7)));
+                    }
+                    transpose_chunks<8>(ch, li);
+                    const int col = (hf ? col_hi : col_lo) + 8 * li;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (yoff[j] >= 0)
+                            *reinterpret_cast<uint4 *>(ybase + (yr0 + yoff[j]) * p.N_out + col) = ch[j];
                 }
             }
         }
