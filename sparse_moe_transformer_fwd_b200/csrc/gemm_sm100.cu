@@ -43,7 +43,9 @@
 #include "common.cuh"
 #include "kernels.h"
 
+#include <cstddef>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 
 namespace moe {
@@ -67,6 +69,17 @@ constexpr int SF_COL = 256;        // TMEM column of the scale factors (A: 4 col
 constexpr int SF_GROUP = 4;        // K blocks per scale block
 constexpr int SF_BUFS = 2;         // scale blocks in shared memory
 constexpr int SF_STAGING = 4;      // fp32 staging slots (groups) between warps 3 and 2
+constexpr int SC_GROUPS = 3;       // fp32 promotion: scale groups of four K blocks in shared memory
+
+// Scales of the K blocks kb0 + 4g .. kb0 + 4g + 3 of one work item (K blocks
+// kb0 .. kb0 + nk - 1), for the fp32 promotion: written by TMA (or by warps 2
+// and 3 where the scale rows cannot be tensor-mapped), read by the epilogue.
+// Row-major boxes of the [rows, K/128] and [weight rows / 128, K/128] arrays.
+// Each TMA destination starts on a 128-byte boundary.
+struct alignas(128) ScaleGroup {
+    float a[BM][SF_GROUP];                  // activation scale: [tile row][K block % 4] (16 bytes a row)
+    alignas(128) float w[2][32];            // weight scale: [column half][K block % 4] (rows 128 bytes apart)
+};
 constexpr int SF_AHEAD = 2;        // groups whose scale copies warp 3 keeps in flight
 
 // Per-variant roles.  MX (block-scaled MMA): one 256-column accumulator (the
@@ -86,7 +99,12 @@ struct __align__(1024) GemmSmem {
     uint8_t a[STAGES][A_BYTES];
     uint8_t b[STAGES][B_BYTES];
     uint8_t sf[SF_BUFS][SF_BYTES];  // MX: UE8M0 scale blocks in the tcgen05.cp source layout
-    float sf_a[SF_STAGING][SF_GROUP][BM];  // MX: fp32 scales staged by warp 3 for warp 2
+    union {
+        float sf_a[SF_STAGING][SF_GROUP][BM];  // MX: fp32 scales staged by warp 3 for warp 2
+        ScaleGroup scg[SC_GROUPS];             // fp32 promotion: ring of scale groups
+    };
+    uint64_t sc_full[SC_GROUPS];   // group written (warps 2 and 3 arrive)
+    uint64_t sc_empty[SC_GROUPS];  // group read (one arrive per epilogue warp)
     float sf_b[SF_STAGING][2][SF_GROUP];
     uint64_t sf_full[SF_STAGING];
     uint64_t sf_empty[SF_STAGING];
@@ -107,6 +125,10 @@ struct __align__(1024) GemmSmem {
 };
 
 static_assert(sizeof(GemmSmem) + 1024 <= 227 * 1024, "shared memory budget of one CTA");
+// TMA destinations of the scale ring: 128-byte boundaries
+static_assert(offsetof(GemmSmem, scg) % 128 == 0 && sizeof(ScaleGroup) % 128 == 0 &&
+                  offsetof(ScaleGroup, w) % 128 == 0 && sizeof(ScaleGroup::w[0]) == 128,
+              "scale-group TMA destinations must start on 128-byte boundaries");
 
 struct KParams {
     const float *a_scales;
@@ -129,6 +151,7 @@ struct KParams {
     int b_rowmajor;        // B row-major [slots * b_rows, K] instead of 128 x 128-byte tiles
     const int32_t *seg_slot, *seg_src, *seg_ret;
     uint16_t *const *ret_y;  // device array [world]
+    int sc_tma;            // fp32 promotion: the scale groups are loaded by TMA (tmap_sa, tmap_sw)
 };
 
 template <int TM>
@@ -213,7 +236,9 @@ __device__ __forceinline__ uint32_t e8m0(float sc) { return (__float_as_uint(sc)
 template <bool FP8, bool GATE_UP, bool MX, bool M64, bool DENSE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                    const __grid_constant__ CUtensorMap tmap_b, const KParams p) {
+                    const __grid_constant__ CUtensorMap tmap_b,
+                    const __grid_constant__ CUtensorMap tmap_sa,
+                    const __grid_constant__ CUtensorMap tmap_sw, const KParams p) {
     static_assert(FP8 || !MX, "the block-scaled MMA takes e4m3 operands");
     static_assert(!M64 || (FP8 && !MX), "64-row tiles: fp8 with software promotion only");
     // DENSE: the down GEMM of a dense layer, with split K (software promotion
@@ -263,6 +288,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         for (int i = 0; i < SF_STAGING; ++i) {
             mbar_init(&s.sf_full[i], 1);
             mbar_init(&s.sf_empty[i], 1);
+        }
+        for (int i = 0; i < SC_GROUPS; ++i) {
+            mbar_init(&s.sc_full[i], p.sc_tma ? 1 : 2);
+            mbar_init(&s.sc_empty[i], EPI_THREADS / 32);
         }
         for (int i = 0; i < SF_BUFS; ++i) {
             mbar_init(&s.sf_ready[i], 1);
@@ -594,6 +623,93 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     if (lane == 0) mbar_arrive(&s.sf_ready[buf]);
                 }
             }
+        } else if constexpr (SCALED) {
+            // ------------------------------------ scales of the fp32 promotion
+            // The epilogue's per-chunk promotion reads its scales from a ring
+            // of SC_GROUPS groups in shared memory (four K blocks of the item
+            // each), so the epilogue warps issue no global load.  With tensor
+            // maps of the scale arrays (rows of K/128 scales a multiple of 16
+            // bytes, every item's first K block a multiple of 4), one thread of
+            // warp 2 fills each group with three TMA loads that complete on the
+            // group's barrier: it never waits for data.
+            // Otherwise warps 2 and 3 load and store the group (warp 2: rows
+            // 0-63, warp 3: rows 64-127).  Either way a group is written once
+            // the epilogue has released its slot.
+            const int lw = warp - 2;
+            const int NB = p.b_rows / 128;
+            int gall = 0;  // groups written, over all items (ring position)
+            bool ok = true;
+            if (p.sc_tma && !(lw == 0 && lane == 0)) ok = false;  // one thread issues the loads
+            for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
+                int tile, ks, kb0, nk;
+                k_range(item, tile, ks, kb0, nk);
+                int seg, row0, rows_valid, nt;
+                decode_tile<TM>(s, n_seg, tile, p.n_tiles_n, seg, row0, rows_valid, nt);
+                const int slot_w = p.seg_slot ? __ldg(p.seg_slot + seg) : seg;
+                const int nb_lo = GATE_UP ? nt : 2 * nt;
+                const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
+                for (int kbg = kb0; kbg < kb0 + nk; kbg += SF_GROUP, ++gall) {
+                    const int slot = gall % SC_GROUPS;
+                    const uint32_t par = ((gall / SC_GROUPS) & 1) ^ 1;
+                    ScaleGroup &sg = s.scg[slot];
+                    if (p.sc_tma) {
+                        if (!mbar_wait(&s.sc_empty[slot], par, abort, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&s.sc_full[slot], TM * 16 + 32);
+                        tma_load_2d(sg.a, &tmap_sa, kbg, row0, &s.sc_full[slot]);
+                        tma_load_2d(sg.w[0], &tmap_sw, kbg, slot_w * NB + nb_lo, &s.sc_full[slot]);
+                        tma_load_2d(sg.w[1], &tmap_sw, kbg, slot_w * NB + nb_hi, &s.sc_full[slot]);
+                        continue;
+                    }
+                    // lane l: rows 64 lw + l and 64 lw + 32 + l; lanes 0-7 the weight
+                    // scales (lanes 0-3 the low column half, 4-7 the high)
+                    const int r0 = 64 * lw + lane, r1 = r0 + 32;
+                    const int wj = lane & 3, wh = (lane >> 2) & 1;
+                    float a0[SF_GROUP], a1[SF_GROUP];
+                    float wv = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < SF_GROUP; ++j) {
+                        const int kb = kbg + j;
+                        const bool in = kb < kb0 + nk;
+                        a0[j] = (in && r0 < rows_valid) ? __ldg(p.a_scales + (static_cast<size_t>(row0) + r0) * KB + kb) : 0.0f;
+                        a1[j] = (in && r1 < rows_valid) ? __ldg(p.a_scales + (static_cast<size_t>(row0) + r1) * KB + kb) : 0.0f;
+                    }
+                    if (lane < 8 && kbg + wj < kb0 + nk)
+                        wv = __ldg(p.b_scales + (static_cast<size_t>(slot_w) * NB + (wh ? nb_hi : nb_lo)) * KB + kbg + wj);
+                    int go = 1;
+                    if (lane == 0) go = mbar_wait(&s.sc_empty[slot], par, abort, p.status) ? 1 : 0;
+                    if (__shfl_sync(0xffffffffu, go, 0) == 0) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int j = 0; j < SF_GROUP; ++j) {
+                        sg.a[r0][j] = a0[j];
+                        sg.a[r1][j] = a1[j];
+                    }
+                    if (lane < 8) sg.w[wh][wj] = wv;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.sc_full[slot]);
+                }
+            }
+            if (p.sc_tma && lw == 0 && lane == 0) {
+                // drain: the TMA loads of the last groups have landed before the
+                // block exits (one budget for all)
+                const long long t0 = clock64();
+                for (int i = gall > SC_GROUPS ? gall - SC_GROUPS : 0; i < gall; ++i) {
+                    bool late = false;
+                    while (!mbar_try_wait(&s.sc_full[i % SC_GROUPS], (i / SC_GROUPS) & 1)) {
+                        if (clock64() - t0 > kWaitBudgetCycles) {
+                            set_status(p.status, MOE_ERR_TIMEOUT);
+                            late = true;
+                            break;
+                        }
+                    }
+                    if (late) break;
+                }
+            }
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------- epilogue
@@ -604,10 +720,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const int hh = M64 ? (lane >> 4) : 0;
         const int r_in = M64 ? q * 16 + (lane & 15) : q * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-        const int NB = p.b_rows / 128;
         int tb = 0;
         uint32_t tphase = 0;
         int iter = 0;
+        int sgrp = 0;  // scale groups of earlier items (ring position)
         bool ok = true;
         for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x, ++iter) {
             int tile, ks, kb0, nk;
@@ -623,30 +739,38 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             float2 acc2[64];  // columns (2j, 2j+1) of the thread's 128
 #pragma unroll
             for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
-            const int nb_lo = GATE_UP ? nt : 2 * nt;
-            const int nb_hi = GATE_UP ? p.N_out / 128 + nt : 2 * nt + 1;
-            // scale rows from the item's first K block on
-            const int slot_w = (SCALED && p.seg_slot) ? __ldg(p.seg_slot + seg) : seg;
-            const float *sw_lo_p = SCALED ? p.b_scales + (static_cast<size_t>(slot_w) * NB + nb_lo) * KB + kb0 : nullptr;
-            const float *sw_hi_p = SCALED ? p.b_scales + (static_cast<size_t>(slot_w) * NB + nb_hi) * KB + kb0 : nullptr;
-            const float *sa_p = SCALED ? p.a_scales + row * KB + kb0 : nullptr;
             // K block (counted from kb0) whose partial this thread promotes in chunk c
             auto kb_of = [&](int c) { return M64 ? 2 * c + hh : c; };
-            // scales of chunk c are loaded one chunk ahead (global latency)
-            float nsa = 0.0f, nswl = 1.0f, nswh = 1.0f;
-            if (SCALED && warp_active && kb_of(0) < nk) {
-                nsa = valid ? __ldg(sa_p + kb_of(0)) : 0.0f;
-                nswl = __ldg(sw_lo_p + kb_of(0));
-                nswh = __ldg(sw_hi_p + kb_of(0));
-            }
-            for (int c = 0; c < nch; ++c) {
-                const float sc_lo = SCALED ? nsa * nswl : 1.0f, sc_hi = SCALED ? nsa * nswh : 1.0f;
-                const bool kvalid = !M64 || kb_of(c) < nk;  // M64, odd K: no partial in the upper half
-                if (SCALED && warp_active && c + 1 < nch && kb_of(c + 1) < nk) {
-                    nsa = valid ? __ldg(sa_p + kb_of(c + 1)) : 0.0f;
-                    nswl = __ldg(sw_lo_p + kb_of(c + 1));
-                    nswh = __ldg(sw_hi_p + kb_of(c + 1));
+            // chunks per scale group of four K blocks (M64: K steps 2c and
+            // 2c + 1 share a chunk, so a group is two chunks)
+            constexpr int GPC = M64 ? 2 : 4;
+            // Scales from the ring in shared memory, read a group (four K
+            // blocks) at a time with three 16-byte shared-memory loads: at the
+            // end of the chunk before the group's first (after that chunk's
+            // buffer release) and consumed only after the next TMEM loads have
+            // landed, so shared-memory latency stays off the accumulator round
+            // trip.  The previous group's slot is released at that read (its
+            // values were consumed a chunk earlier), the item's last group
+            // after the item.
+            float4 g_a = make_float4(0.0f, 0.0f, 0.0f, 0.0f), g_wl = g_a, g_wh = g_a;
+            auto fetch_scales = [&](int cc) {
+                if (cc % GPC != 0) return true;
+                const int gi = sgrp + cc / GPC;
+                const int slot = gi % SC_GROUPS;
+                if (cc > 0) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.sc_empty[(gi - 1) % SC_GROUPS]);
                 }
+                if (!mbar_wait(&s.sc_full[slot], (gi / SC_GROUPS) & 1, abort, p.status)) return false;
+                g_a = *reinterpret_cast<const float4 *>(s.scg[slot].a[r_in]);
+                g_wl = *reinterpret_cast<const float4 *>(s.scg[slot].w[0]);
+                g_wh = *reinterpret_cast<const float4 *>(s.scg[slot].w[1]);
+                return true;
+            };
+            auto pick = [](const float4 &v, int j) { return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w)); };
+            if constexpr (SCALED) ok = fetch_scales(0);
+            for (int c = 0; c < nch && ok; ++c) {
+                const bool kvalid = !M64 || kb_of(c) < nk;  // M64, odd K: no partial in the upper half
                 if (!mbar_wait(&s.tfull[tb], tphase, abort, p.status)) {
                     ok = false;
                     break;
@@ -656,12 +780,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 // buffer is released as soon as the last piece is in registers
                 // (before its FMAs), since the MMA two chunks ahead waits for it
                 float va[32], vb[32];
+                float sc_lo = 1.0f, sc_hi = 1.0f;
                 const bool add = warp_active && kvalid;  // the loads below are warp-wide
                 if (warp_active) {
                     const uint32_t base = lane_base + tb * BN;
                     tmem_ld32(base + col_lo, va);
                     tmem_ld32(base + col_lo + 32, vb);
                     tmem_wait_ld(va, vb);
+                    if constexpr (SCALED) {
+                        // the group's scale loads are consumed here, not earlier
+                        asm volatile("" : "+f"(g_a.x), "+f"(g_a.y), "+f"(g_a.z), "+f"(g_a.w));
+                        const int j = kb_of(c) & 3;
+                        const float sa = pick(g_a, j);
+                        sc_lo = sa * pick(g_wl, j);
+                        sc_hi = sa * pick(g_wh, j);
+                    }
                     if (add) promote32<SCALED>(acc2, 0, va, sc_lo);
                     tmem_ld32(base + col_hi, va);
                     if (add) promote32<SCALED>(acc2, 16, vb, sc_lo);
@@ -675,10 +808,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     promote32<SCALED>(acc2, 32, va, sc_hi);
                     promote32<SCALED>(acc2, 48, vb, sc_hi);
                 }
+                if (SCALED && c + 1 < nch && !fetch_scales(c + 1)) ok = false;
                 if (++tb == R::NBUF) {
                     tb = 0;
                     tphase ^= 1;
                 }
+            }
+            if constexpr (SCALED) {
+                // the item's last scale group has been consumed
+                __syncwarp();
+                const int n_groups = (nk + SF_GROUP - 1) / SF_GROUP;
+                if (ok && lane == 0) mbar_arrive(&s.sc_empty[(sgrp + n_groups - 1) % SC_GROUPS]);
+                sgrp += n_groups;
             }
             if (!ok) break;
             if constexpr (M64) {
@@ -884,9 +1025,25 @@ bool make_map_2d(CUtensorMap *m, const void *base, bool fp8, int K, int rows, in
 }
 
 
+// binary32 [rows, cols] row-major, boxes of box_rows x 4 (16 bytes a row, no
+// swizzle; reads past the array give 0)
+bool make_map_scales(CUtensorMap *m, const float *base, int cols, long long rows, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || cols % 4 != 0 || (reinterpret_cast<uintptr_t>(base) & 15) != 0 || rows < 1 ||
+        rows >= (1LL << 31))
+        return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
+    cuuint32_t box[2] = {4, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool FP8, bool GATE_UP, bool MX, bool M64 = false, bool DENSE = false>
-cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams &kp, int grid,
-                     cudaStream_t st) {
+cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &msa,
+                     const CUtensorMap &msw, const KParams &kp, int grid, cudaStream_t st) {
     const size_t smem = sizeof(GemmSmem) + 1024;
     static DeviceConfigured configured{};  // per template instance
     if (first_use_on_device(configured)) {
@@ -904,7 +1061,7 @@ cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const KParams
         mark_used_on_device(configured);
     }
     return launch_pdl(grouped_gemm_kernel<FP8, GATE_UP, MX, M64, DENSE>, dim3(grid), dim3(NUM_THREADS), smem, st,
-                      ma, mb, kp);
+                      ma, mb, msa, msw, kp);
 }
 
 }  // namespace
@@ -952,6 +1109,21 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     kp.seg_ret = g.seg_ret;
     kp.ret_y = g.ret_y_dev;
     if (g.seg_ret && !g.ret_y_dev) return cudaErrorInvalidValue;
+    // fp32 promotion: tensor maps of the two scale arrays when their rows are
+    // whole 16-byte units (else warps 2 and 3 load the scale groups)
+    CUtensorMap msa, msw;
+    std::memset(&msa, 0, sizeof(msa));
+    std::memset(&msw, 0, sizeof(msw));
+    if (g.fp8 && !g.ue8m0) {
+        const int kbn = g.K / 128;
+        const int ksp = (g.gate_up || g.ksplit < 1) ? 1 : g.ksplit;
+        bool aligned = true;  // every work item's first K block a multiple of 4 (16-byte x)
+        for (int ks = 0; ks < ksp; ++ks) aligned = aligned && (ks * kbn / ksp) % 4 == 0;
+        kp.sc_tma = aligned &&
+                    make_map_scales(&msa, g.a_scales, kbn, g.rows_total, m64 ? 64 : 128) &&
+                    make_map_scales(&msw, g.b_scales, kbn, static_cast<long long>(g.n_slots) * (b_rows / 128), 1)
+                        ? 1 : 0;
+    }
     // block-scaled MMA (UE8M0 scales): all of K accumulates in TMEM
     kp.mx_spc = g.K / 128;
     const bool mx = g.fp8 && g.ue8m0;
@@ -971,25 +1143,25 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t st, int *launche
     // the dense layer's down GEMM (split K or a residual) has its own instances
     const bool dense = !g.gate_up && (kp.ksplit > 1 || kp.residual);
     if (dense && mx)
-        e = launch_t<true, false, true, false, true>(ma, mb, kp, grid, st);
+        e = launch_t<true, false, true, false, true>(ma, mb, msa, msw, kp, grid, st);
     else if (g.fp8 && g.ue8m0)
-        e = g.gate_up ? launch_t<true, true, true>(ma, mb, kp, grid, st)
-                      : launch_t<true, false, true>(ma, mb, kp, grid, st);
+        e = g.gate_up ? launch_t<true, true, true>(ma, mb, msa, msw, kp, grid, st)
+                      : launch_t<true, false, true>(ma, mb, msa, msw, kp, grid, st);
     else if (dense && g.fp8 && m64)
-        e = launch_t<true, false, false, true, true>(ma, mb, kp, grid, st);
+        e = launch_t<true, false, false, true, true>(ma, mb, msa, msw, kp, grid, st);
     else if (dense && g.fp8)
-        e = launch_t<true, false, false, false, true>(ma, mb, kp, grid, st);
+        e = launch_t<true, false, false, false, true>(ma, mb, msa, msw, kp, grid, st);
     else if (dense)
-        e = launch_t<false, false, false, false, true>(ma, mb, kp, grid, st);
+        e = launch_t<false, false, false, false, true>(ma, mb, msa, msw, kp, grid, st);
     else if (g.fp8 && m64)
-        e = g.gate_up ? launch_t<true, true, false, true>(ma, mb, kp, grid, st)
-                      : launch_t<true, false, false, true>(ma, mb, kp, grid, st);
+        e = g.gate_up ? launch_t<true, true, false, true>(ma, mb, msa, msw, kp, grid, st)
+                      : launch_t<true, false, false, true>(ma, mb, msa, msw, kp, grid, st);
     else if (g.fp8)
-        e = g.gate_up ? launch_t<true, true, false>(ma, mb, kp, grid, st)
-                      : launch_t<true, false, false>(ma, mb, kp, grid, st);
+        e = g.gate_up ? launch_t<true, true, false>(ma, mb, msa, msw, kp, grid, st)
+                      : launch_t<true, false, false>(ma, mb, msa, msw, kp, grid, st);
     else
-        e = g.gate_up ? launch_t<false, true, false>(ma, mb, kp, grid, st)
-                      : launch_t<false, false, false>(ma, mb, kp, grid, st);
+        e = g.gate_up ? launch_t<false, true, false>(ma, mb, msa, msw, kp, grid, st)
+                      : launch_t<false, false, false>(ma, mb, msa, msw, kp, grid, st);
     ++*launches;
     return e;
 }
