@@ -16,7 +16,11 @@
 //   warp 1      TMEM allocator (512 columns) and MMA issuer (one thread):
 //               tcgen05.mma M=128 N=256, K=32 (e4m3) or K=16 (bf16), four per
 //               stage.
-//   warps 2-3   idle (warpgroup 0 gives its registers to the epilogue)
+//   warps 2-3   fp32 scales: one thread fills a ring of three scale groups
+//               (four K blocks of the tile's activation and weight scales)
+//               in shared memory by TMA, or both warps load them where the
+//               scale rows cannot be tensor-mapped; block-scaled MMA: the
+//               UE8M0 scale factors for tcgen05.cp; bf16: idle
 //   warps 4-11  epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (tile rows);
 //               warps 4-7 take columns [0,64) and [128,192), warps 8-11 take
 //               [64,128) and [192,256).
@@ -32,12 +36,17 @@
 //   accumulation of K = 7168 put the layer output 1.25e-3 (relative L2) away
 //   from the binary64 oracle), and chunks added in binary32 registers bring
 //   it back.
+//   The epilogue takes each chunk's two scale products from the scale
+//   ring (three 16-byte shared-memory loads per four K blocks) and issues no
+//   global load in its K loop.
 // Epilogue: gate/up GEMM -> H = silu(G) * U, then (FP8) 1x128 e4m3
 //   quantisation of H (one 128-feature tile per row per work item; the two
 //   column halves exchange their amax through shared memory; power-of-two
 //   scales in the UE8M0 variant) or (BF16) bf16
 //   rounding; down GEMM -> Y in bf16.  Rows past the segment end are computed
-//   from neighbouring rows and never stored.
+//   from neighbouring rows and never stored.  The stores transpose 16-byte
+//   chunks across groups of lanes so each instruction writes whole row
+//   segments.
 // Every wait is bounded; on expiry the block records MOE_ERR_TIMEOUT, drains
 // its own TMA loads and MMAs, frees its TMEM and exits.
 #include "common.cuh"
