@@ -176,20 +176,29 @@ router_scores_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
     for (int kc = 0; kc < nk; ++kc) {
         const int buf = kc & 1;
         if (kc + 1 < nk) load(kc + 1);
-#pragma unroll 4
-        for (int kk = 0; kk < RT_KC; ++kk) {
-            const float4 xa = *reinterpret_cast<const float4 *>(&xs[buf][kk][rt_swz(kk, 4 * ty)]);
-            float4 xb = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            if constexpr (TB == 64)
-                xb = *reinterpret_cast<const float4 *>(&xs[buf][kk][rt_swz(kk, 32 + 4 * ty)]);
-            const float4 wa = *reinterpret_cast<const float4 *>(&ws[buf][kk][rt_swz(kk, 4 * tx)]);
-            const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-            const float2 wv[2] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w)};
+        // the swizzle changes every 8 rows of k (rt_swz): per 8-row phase one
+        // base address per operand, and constant offsets for its 8 rows
 #pragma unroll
-            for (int a = 0; a < NTOK; ++a) {
-                const float2 x2 = make_float2(xv[a], xv[a]);
+        for (int ph = 0; ph < RT_KC / 8; ++ph) {
+            const int sw = (ph << 1) & 15;
+            const float *xa_p = &xs[buf][8 * ph][((ty ^ sw) & 15) << 2];                  // tokens 4ty..
+            const float *xb_p = TB == 64 ? &xs[buf][8 * ph][(((8 + ty) ^ sw) & 15) << 2]  // 32+4ty..
+                                         : xa_p;
+            const float *wa_p = &ws[buf][8 * ph][((tx ^ sw) & 15) << 2];                  // experts 4tx..
 #pragma unroll
-                for (int b = 0; b < 2; ++b) acc[a][b] = __ffma2_rn(x2, wv[b], acc[a][b]);
+            for (int u = 0; u < 8; ++u) {
+                const float4 xa = *reinterpret_cast<const float4 *>(xa_p + u * TB);
+                float4 xb = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if constexpr (TB == 64) xb = *reinterpret_cast<const float4 *>(xb_p + u * TB);
+                const float4 wa = *reinterpret_cast<const float4 *>(wa_p + u * RT_B);
+                const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+                const float2 wv[2] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w)};
+#pragma unroll
+                for (int a = 0; a < NTOK; ++a) {
+                    const float2 x2 = make_float2(xv[a], xv[a]);
+#pragma unroll
+                    for (int b = 0; b < 2; ++b) acc[a][b] = __ffma2_rn(x2, wv[b], acc[a][b]);
+                }
             }
         }
         if (kc + 1 < nk) store(buf ^ 1);
@@ -419,9 +428,15 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
                           float *gates, cudaStream_t st, int *launches, PreNorm pn) {
     mark_launch(st, *launches, "router_scores");
     if (T >= 512) {
-        // 32-token tiles where 64-token tiles would leave SMs without one
+        // 64-token tiles, except where they would leave SMs without one, or
+        // put 3 or 4 on the busiest SM: measured at E = 256, d = 7168, 32-token
+        // tiles win there (T = 6144: 0.72 against 0.83 ms; T = 8192: 0.82
+        // against 0.86) and lose elsewhere (T = 4096: 0.57 against 0.39 ms;
+        // T = 12288: 1.27 against 1.05)
         const int e_tiles = (E + RT_B - 1) / RT_B;
-        const bool wide = static_cast<long long>((T + RT_B - 1) / RT_B) * e_tiles >= num_sms();
+        const long long tiles64 = static_cast<long long>((T + RT_B - 1) / RT_B) * e_tiles;
+        const int sms = num_sms();
+        const bool wide = tiles64 >= sms && !(tiles64 > 2LL * sms && tiles64 <= 4LL * sms);
         if (wide) {
             dim3 grid(e_tiles, (T + 63) / 64);
             LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel<64>, grid, dim3(RT_THREADS), 0, st, x, w, T, d,

@@ -95,5 +95,6 @@ def test_traffic_record_used_only_where_it_applies():
         assert got == rec["workloads"]["decode"]["grouped_gemm_gate_up"]["traffic_bytes_per_launch"]
     else:
         assert got is None
-    assert bench.kernel_traffic("grouped_gemm_gate_up", "skew") is None
+    assert "bf16" not in rec["workloads"]
+    assert bench.kernel_traffic("grouped_gemm_gate_up", "bf16") is None
     assert bench.kernel_traffic("no_such_kernel", "decode") is None
