@@ -320,6 +320,37 @@ def e2e_host_loop(call, x, d_model, steps, world, dev):
     return times[0], times[1]
 
 
+def moe_config(cfg, T: int, world: int, prenorm: bool) -> dict:
+    """The line's `config`: the workload only, identical in both arms."""
+    return {
+        "workload": ("pre-norm block (h + MoE(RMSNorm(h)), fused) " if prenorm else "")
+                    + f"{cfg.name}: T={T}, d_model={cfg.d_model}, {cfg.n_experts} experts "
+                    f"top-{cfg.top_k} + {cfg.n_shared} shared, d_expert={cfg.d_expert}, "
+                    + ({"fp8": "e4m3 1x128/128x128 blockwise, fp32 scales, bf16 I/O",
+                        "fp8_ue8m0": "e4m3 1x128/128x128 blockwise, power-of-two (UE8M0) "
+                                     "scales, bf16 I/O"}.get(cfg.precision, "bf16")),
+        "tokens_per_gpu": T,
+        "parallelism": "replicas" if world > 1 else "single GPU",
+        "l2": "inputs larger than L2: the touched experts' weights (GB per step) stream through "
+              "every step",
+    }
+
+
+def dense_config(cfg, T: int, world: int, prenorm: bool) -> dict:
+    """The dense line's `config`, identical in both arms."""
+    return {
+        "workload": ("pre-norm block (h + FFN(RMSNorm(h)), fused) " if prenorm else "")
+                    + f"{cfg.name}: T={T}, d_model={cfg.d_model}, d_ff={cfg.d_ff}, "
+                    + {"fp8": "e4m3 1x128/128x128 blockwise, fp32 scales, bf16 I/O",
+                       "fp8_ue8m0": "e4m3 blockwise, power-of-two scales, bf16 I/O"}.get(
+                           cfg.precision, "bf16"),
+        "tokens_per_gpu": T,
+        "parallelism": "replicas" if world > 1 else "single GPU",
+        "l2": f"inputs larger than L2: {3 * cfg.d_model * cfg.d_ff / 1e6:.0f} MB of weights "
+              "stream through every step",
+    }
+
+
 def run_ours(args, world, rank, local):
     import sparse_moe_transformer_fwd_b200 as moe
     dev = torch.device("cuda", local)
@@ -419,20 +450,11 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16" if cfg.precision == "bf16" else "e4m3",
         "data": "synthetic (seeded; random-init weights of the DeepSeek-V3 MoE layer shape)",
-        "config": {
-            "workload": ("pre-norm block (h + MoE(RMSNorm(h)), fused) " if args.prenorm else "")
-                        + f"{cfg.name}: T={T}, d_model={cfg.d_model}, {cfg.n_experts} experts "
-                        f"top-{cfg.top_k} + {cfg.n_shared} shared, d_expert={cfg.d_expert}, "
-                        + ({"fp8": "e4m3 1x128/128x128 blockwise, fp32 scales, bf16 I/O",
-                            "fp8_ue8m0": "e4m3 1x128/128x128 blockwise, power-of-two (UE8M0) "
-                                         "scales, bf16 I/O"}.get(cfg.precision, "bf16")),
-            "tokens_per_gpu": T,
-            "parallelism": "replicas" if world > 1 else "single GPU",
-            "l2": f"inputs larger than L2: {touched} touched experts' weights "
-                  f"({g1_bytes / 1e9:.2f} GB in the gate/up GEMM alone) per step",
-            "expert_load_max_over_mean": round(float(counts.max()) / (T * cfg.top_k / cfg.n_experts), 2),
-            "experts_empty": int((counts == 0).sum()),
-        },
+        "config": moe_config(cfg, T, world, args.prenorm),
+        "routing": {"touched_experts": touched,
+                    "gate_up_algorithmic_bytes": int(g1_bytes),
+                    "expert_load_max_over_mean": round(float(counts.max()) / (T * cfg.top_k / cfg.n_experts), 2),
+                    "experts_empty": int((counts == 0).sum())},
         "roofline": {**moe_roofline(cfg, touched, g1_ms, peaks, peak_kind),
                      "kernel_ms_from": "CUDA events around this kernel on every step of a "
                                        "separate pass of K steps",
@@ -557,17 +579,7 @@ def run_dense(args, world, rank, local):
         "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if cfg.precision == "bf16" else "e4m3",
         "data": "synthetic (seeded; random-init weights of the DeepSeek-V3 dense FFN shape)",
-        "config": {
-            "workload": ("pre-norm block (h + FFN(RMSNorm(h)), fused) " if args.prenorm else "")
-                        + f"{cfg.name}: T={T}, d_model={cfg.d_model}, d_ff={cfg.d_ff}, "
-                        + {"fp8": "e4m3 1x128/128x128 blockwise, fp32 scales, bf16 I/O",
-                           "fp8_ue8m0": "e4m3 blockwise, power-of-two scales, bf16 I/O"}.get(
-                               cfg.precision, "bf16"),
-            "tokens_per_gpu": T,
-            "parallelism": "replicas" if world > 1 else "single GPU",
-            "l2": f"inputs larger than L2: {3 * cfg.d_model * cfg.d_ff / 1e6:.0f} MB of weights "
-                  "stream through every step",
-        },
+        "config": dense_config(cfg, T, world, args.prenorm),
         "roofline": dense_roofline(cfg, g1_ms, peaks, peak_kind),
         "kernels_ms": {n: round(float(v), 4) for n, v in zip(names, kmean)},
         "e2e": {"value": round(T * world / (ms_e2e * 1e-3), 1), "unit": "tokens/s",
@@ -729,7 +741,7 @@ def run_reference_dense(args, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(s_step * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": f"{cfg.name}: T={cfg.T}, d_model={cfg.d_model}, d_ff={cfg.d_ff}"},
+        "config": dense_config(cfg, cfg.T, world, args.prenorm),
         "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": sample, "cpu": cpu_model()},
         "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -759,8 +771,7 @@ def run_reference(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(s_step * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": f"{cfg.name}: T={cfg.T}, d_model={cfg.d_model}, "
-                               f"{cfg.n_experts} experts top-{cfg.top_k} + {cfg.n_shared} shared"},
+        "config": moe_config(cfg, cfg.T, world, args.prenorm),
         "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": sample, "cpu": cpu_model()},
         "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,

@@ -98,3 +98,15 @@ def test_traffic_record_used_only_where_it_applies():
     assert "bf16" not in rec["workloads"]
     assert bench.kernel_traffic("grouped_gemm_gate_up", "bf16") is None
     assert bench.kernel_traffic("no_such_kernel", "decode") is None
+
+
+def test_reference_arm_reports_the_same_config():
+    """Both arms name the workload with the same `config` (the driver compares
+    them); the reference arm runs the oracle on a bounded sample."""
+    import argparse
+    args = argparse.Namespace(steps=1, warmup=3, workload="tiny", ref_tokens=1, seed=0,
+                              prenorm=False)
+    res, cfg = bench.run_reference(args, 1, 0, 0)
+    assert res["config"] == bench.moe_config(CONFIGS["tiny"], CONFIGS["tiny"].T, 1, False)
+    assert res["impl"] == "reference" and res["metric"] == bench.METRIC
+    assert res["e2e"]["value"] == res["value"] and res["cpu_baseline"]["value"] == res["value"]
