@@ -17,6 +17,7 @@
 //   warp arg-max under (sel desc, expert asc); gates g_j = s_j / S *
 //   routed_scale with S the binary32 sum of the selected s in rank order.
 #include "common.cuh"
+#include <algorithm>
 #include "kernels.h"
 
 namespace moe {
@@ -421,6 +422,51 @@ router_topk_kernel(const float *__restrict__ scores, const float *__restrict__ b
     }
 }
 
+// Unused dynamic shared memory that caps the CTAs of a router_scores launch
+// resident on one SM at `cap` (0 or 5 and more: no cap).  When the tiles of a
+// launch fit in one wave, the block scheduler may stack up to five CTAs (the
+// register limit) on some SMs and leave others with few; the cap spreads
+// them out.  Measured at E = 256, d = 7168, 64-token tiles: T = 6144 (384
+// tiles, cap 3) 0.83 -> 0.56 ms, T = 8192 (512 tiles, cap 4) 0.86 -> 0.72
+// ms, T = 4096 (cap 2) unchanged; 64-token tiles so capped beat 32-token
+// tiles at every T from 4096 to 16384.  Returns the padding in bytes,
+// checked with the occupancy calculator (0 where the cap cannot be met), and
+// remembers it per device context.
+template <int TB>
+int router_residency_pad(int cap) {
+    if (cap <= 0 || cap >= 5) return 0;
+    static DeviceConfigured configured[5]{};
+    static std::atomic<int> cached[5][64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const bool slot = dev >= 0 && dev < 64;
+    if (slot && !first_use_on_device(configured[cap])) return cached[cap][dev].load(std::memory_order_relaxed);
+    int per_sm = 0, reserved = 0, opt_in = 0;
+    cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    cudaDeviceGetAttribute(&opt_in, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    constexpr int kStatic = 2 * RT_KC * (TB + RT_B) * 4;  // xs and ws
+    int pad = (per_sm / cap - reserved - kStatic) & ~1023;
+    int n = 0;
+    // the largest padding any cap uses, so a launch never exceeds the attribute
+    if (pad <= 0 || kStatic + pad > opt_in) {
+        pad = 0;
+    } else if (cudaFuncSetAttribute(router_scores_kernel<TB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    opt_in - kStatic) != cudaSuccess ||
+               cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, router_scores_kernel<TB>, RT_THREADS,
+                                                             pad) != cudaSuccess) {
+        cudaGetLastError();  // a refused attribute or query: launch without the cap
+        pad = 0;
+    } else if (n != cap) {
+        pad = 0;
+    }
+    if (slot) {
+        cached[cap][dev].store(pad, std::memory_order_relaxed);
+        mark_used_on_device(configured[cap]);
+    }
+    return pad;
+}
+
 }  // namespace
 
 cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bias, int T, int d,
@@ -428,23 +474,25 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
                           float *gates, cudaStream_t st, int *launches, PreNorm pn) {
     mark_launch(st, *launches, "router_scores");
     if (T >= 512) {
-        // 64-token tiles, except where they would leave SMs without one, or
-        // put 3 or 4 on the busiest SM: measured at E = 256, d = 7168, 32-token
-        // tiles win there (T = 6144: 0.72 against 0.83 ms; T = 8192: 0.82
-        // against 0.86) and lose elsewhere (T = 4096: 0.57 against 0.39 ms;
-        // T = 12288: 1.27 against 1.05)
+        // 64-token tiles, or 32-token tiles where 64-token tiles would leave
+        // SMs without one; the CTAs resident per SM are capped at the fewest
+        // that hold the whole launch in one wave (router_residency_pad)
         const int e_tiles = (E + RT_B - 1) / RT_B;
         const long long tiles64 = static_cast<long long>((T + RT_B - 1) / RT_B) * e_tiles;
         const int sms = num_sms();
-        const bool wide = tiles64 >= sms && !(tiles64 > 2LL * sms && tiles64 <= 4LL * sms);
+        const bool wide = tiles64 >= sms;
+        const long long tiles = wide ? tiles64 : static_cast<long long>((T + 31) / 32) * e_tiles;
+        const int cap = static_cast<int>(std::min<long long>((tiles + sms - 1) / sms, 5));
         if (wide) {
+            const int pad = router_residency_pad<64>(cap);
             dim3 grid(e_tiles, (T + 63) / 64);
-            LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel<64>, grid, dim3(RT_THREADS), 0, st, x, w, T, d,
-                                        E, scores, pn));
+            LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel<64>, grid, dim3(RT_THREADS), pad, st, x, w, T,
+                                        d, E, scores, pn));
         } else {
+            const int pad = router_residency_pad<32>(cap);
             dim3 grid(e_tiles, (T + 31) / 32);
-            LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel<32>, grid, dim3(RT_THREADS), 0, st, x, w, T, d,
-                                        E, scores, pn));
+            LAUNCH_OR_RETURN(launch_pdl(router_scores_kernel<32>, grid, dim3(RT_THREADS), pad, st, x, w, T,
+                                        d, E, scores, pn));
         }
     } else {
         constexpr int BT = 4, NP = RS_PRODUCER_WARPS;

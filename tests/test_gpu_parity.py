@@ -40,6 +40,11 @@ ROUTE_CASES = {
     "tiny_scale2.5": CONFIGS["tiny"].with_(routed_scale=2.5),
     "decode": CONFIGS["decode"],
     "ds_T600_bigtile": CONFIGS["decode"].with_(T=600),
+    # 64-token tiles launched with 2, 3 and 4 CTAs per SM at most (the
+    # residency cap of launches that fit in one wave on 148 SMs)
+    "tiny_T12000_cap2": CONFIGS["tiny"].with_(T=12000),
+    "tiny_T24000_cap3": CONFIGS["tiny"].with_(T=24000),
+    "tiny_T32000_cap4": CONFIGS["tiny"].with_(T=32000),
 }
 
 
