@@ -467,6 +467,49 @@ int router_residency_pad(int cap) {
     return pad;
 }
 
+// Dynamic shared memory of a router_scores_small_kernel launch: the ring it
+// needs, or (cap 1: no more CTAs than SMs) enough to keep a second CTA off
+// each SM, so the block scheduler cannot stack two CTAs on one SM while
+// others idle.  Sets the kernel's shared-memory attribute once per device
+// context; -1 if even the ring cannot be granted.
+int router_small_smem_for(int cap) {
+    constexpr int BT = 4, NP = RS_PRODUCER_WARPS;
+    constexpr int need = static_cast<int>(router_small_smem<BT>());
+    static DeviceConfigured configured{};
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const bool slot = dev >= 0 && dev < 64;
+    int one = 0;  // dynamic shared memory that leaves room for one CTA per SM (0: none found)
+    if (slot && !first_use_on_device(configured)) {
+        one = cached[dev].load(std::memory_order_relaxed);
+    } else {
+        int per_sm = 0, reserved = 0, opt_in = 0, n = 0;
+        cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+        cudaDeviceGetAttribute(&opt_in, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (opt_in < need ||
+            cudaFuncSetAttribute(router_scores_small_kernel<BT, NP>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, opt_in) != cudaSuccess) {
+            cudaGetLastError();
+            return -1;
+        }
+        const int big = std::min(opt_in, per_sm - reserved) & ~1023;
+        if (big >= need) {
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, router_scores_small_kernel<BT, NP>,
+                                                              (BT + NP) * 32, big) != cudaSuccess)
+                cudaGetLastError();  // no cap: the query is not the caller's error
+            else if (n == 1)
+                one = big;
+        }
+        if (slot) {
+            cached[dev].store(one, std::memory_order_relaxed);
+            mark_used_on_device(configured);
+        }
+    }
+    return (cap <= 1 && one > 0) ? one : need;
+}
+
 }  // namespace
 
 cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bias, int T, int d,
@@ -496,15 +539,10 @@ cudaError_t launch_router(const uint16_t *x, const uint16_t *w, const float *bia
         }
     } else {
         constexpr int BT = 4, NP = RS_PRODUCER_WARPS;
-        constexpr size_t smem = router_small_smem<BT>();
-        static DeviceConfigured configured{};
-        if (first_use_on_device(configured)) {
-            LAUNCH_OR_RETURN(cudaFuncSetAttribute(router_scores_small_kernel<BT, NP>,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  static_cast<int>(smem)));
-            mark_used_on_device(configured);
-        }
         dim3 grid((E + 31) / 32, (T + BT - 1) / BT);
+        const int ctas = static_cast<int>(grid.x * grid.y);
+        const int smem = router_small_smem_for((ctas + num_sms() - 1) / num_sms());
+        if (smem < 0) return cudaErrorInvalidConfiguration;
         LAUNCH_OR_RETURN(launch_pdl(router_scores_small_kernel<BT, NP>, grid, dim3((BT + NP) * 32), smem,
                                     st, x, w, T, d, E, scores, pn));
     }
