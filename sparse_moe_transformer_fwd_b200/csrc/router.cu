@@ -9,10 +9,10 @@
 //   degree-7 Taylor polynomial (W. J. Cody, W. Waite, "Software Manual for
 //   the Elementary Functions", 1980).  Every operation is a correctly rounded
 //   binary32 operation, so the results are reproducible bit for bit.
-//   Tiling (large batches): a CTA owns 64 tokens x 64 experts, each thread an
-//   8 x 8 register tile; decode-size batches use one output per thread (see
-//   router_scores_small_kernel).  x and W_r chunks are staged in shared memory
-//   as binary32 (bf16 widening is exact).
+//   Tiling (large batches): a CTA owns 64 (or 32) tokens x 64 experts, each
+//   thread 8 (or 4) tokens x 4 experts; decode-size batches use one output
+//   per thread (see router_scores_small_kernel).  x and W_r chunks are staged
+//   in shared memory as binary32 (bf16 widening is exact).
 // Kernel 2 (router_topk): one warp per token.  sel = s + b; k rounds of a
 //   warp arg-max under (sel desc, expert asc); gates g_j = s_j / S *
 //   routed_scale with S the binary32 sum of the selected s in rank order.
