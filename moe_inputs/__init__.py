@@ -94,6 +94,10 @@ CONFIGS = {
                                **{**_DS, "n_experts": 32}),
     "prefill_small_ue8m0": MoEConfig("prefill_small_ue8m0", T=4096, precision="fp8_ue8m0",
                                      bias="zero", **{**_DS, "n_experts": 32}),
+    # profiling-size stand-in for the skew batch: the same Zipf-ranked bias
+    # over 32 routed experts, so one expert carries several times the mean
+    "skew_small": MoEConfig("skew_small", T=4096, precision="fp8", bias="zipf",
+                            **{**_DS, "n_experts": 32}),
 }
 
 
