@@ -140,7 +140,11 @@ int moe_workspace_layout(const moe_shape *shape, moe_workspace_offsets *out);
  *   bias     fp32 [n_experts]
  *   topk_idx int32 [T, top_k] out: expert ids, best first
  *   topk_w   fp32 [T, top_k]  out: gates in the same order
- *   ws       workspace (>= moe_workspace_size bytes): holds the [T, E] scores */
+ *   ws       workspace (>= moe_workspace_size bytes): holds the [T, E] scores
+ * When the scores kernel's grid fits in one wave, its blocks ask for unused
+ * shared memory so that no SM holds more of them than the wave needs; a
+ * kernel that the caller runs concurrently on another stream then finds less
+ * shared memory free on those SMs for the scores kernel's duration. */
 int moe_route(const moe_shape *shape, const uint16_t *x, const uint16_t *w_router,
               const float *bias, int32_t *topk_idx, float *topk_w,
               void *ws, size_t ws_bytes, void *stream);
